@@ -1,0 +1,345 @@
+"""Pins of the fp64 CPU oracle against things other than itself.
+
+Each test checks one oracle routine against a library routine, a closed form,
+an invariant, a hand-worked fixture or brute force, chosen so that a dropped
+term, a wrong sign or index or a transposed operand fails one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _planted(rng, T, d, sig, noise=0.0):
+    m = len(sig)
+    U, _ = np.linalg.qr(rng.standard_normal((T, m)))
+    V, _ = np.linalg.qr(rng.standard_normal((d, m)))
+    X = (U * np.asarray(sig)[None, :]) @ V.T
+    E = noise * rng.standard_normal((T, d))
+    return X + E, E
+
+
+# ---------------------------------------------------------------- SVD
+@pytest.mark.parametrize("T,d", [(96, 32), (40, 40), (24, 48)])
+def test_svd_matches_lapack(oracle_mod, T, d):
+    rng = np.random.default_rng(T * 7 + d)
+    X = rng.standard_normal((T, d)) * np.exp(-np.arange(d) / 5.0)[None, :]
+    s, Vr, US, sweeps = oracle_mod.svd(X)
+    s_ref = scipy.linalg.svd(X, compute_uv=False, lapack_driver="gesvd")
+    m = min(T, d)
+    assert np.all(np.abs(s[:m] - s_ref) <= 1e-12 * s_ref[0])
+    assert np.all(s[m:] == 0.0)
+    assert np.all(np.diff(s) <= 0.0)
+    # V orthonormal; X = (U Sigma) V^T exactly up to rounding
+    assert np.allclose(Vr.T @ Vr, np.eye(d), atol=1e-13)
+    assert np.abs(US @ Vr.T - X).max() <= 1e-12 * np.abs(X).max()
+    # the columns of U Sigma have norms sigma and are mutually orthogonal
+    G = US.T @ US
+    assert np.allclose(np.sqrt(np.diag(G))[:m], s[:m], rtol=0, atol=1e-12 * s[0])
+    off = G - np.diag(np.diag(G))
+    assert np.abs(off).max() <= 1e-11 * s[0] ** 2
+
+
+def test_svd_planted_closed_form(oracle_mod):
+    rng = np.random.default_rng(11)
+    tau = 9.0
+    sig = np.exp(-np.arange(64) / tau)
+    X, _ = _planted(rng, 256, 64, sig)
+    s, _, _, _ = oracle_mod.svd(X)
+    assert np.abs(s - sig).max() <= 1e-13
+
+
+def test_svd_weyl_with_noise(oracle_mod):
+    rng = np.random.default_rng(12)
+    sig = np.exp(-np.arange(32) / 6.0)
+    X, E = _planted(rng, 128, 32, sig, noise=1e-3)
+    s, _, _, _ = oracle_mod.svd(X)
+    bound = np.linalg.norm(E, 2)
+    assert np.all(np.abs(s - sig) <= bound * (1 + 1e-9))
+
+
+@pytest.mark.parametrize("T,d", [(80, 24), (16, 24)])
+def test_eckart_young(oracle_mod, T, d):
+    rng = np.random.default_rng(T + d)
+    X = rng.standard_normal((T, d)) @ np.diag(np.exp(-np.arange(d) / 4.0))
+    s, Vr, US, _ = oracle_mod.svd(X)
+    m = min(T, d)
+    for r in range(0, m + 1):
+        A = US[:, :r]
+        B = Vr[:, :r].T
+        Xh = oracle_mod.reconstruct(A, B) if r else np.zeros_like(X)
+        err = np.sum((X - Xh) ** 2)
+        tail = np.sum(s[r:] ** 2)
+        assert abs(err - tail) <= 1e-10 * max(tail, 1e-300) + 1e-24 * np.sum(X ** 2)
+    Xfull = oracle_mod.reconstruct(US[:, :m], Vr[:, :m].T)
+    assert np.abs(Xfull - X).max() <= 1e-12 * np.abs(X).max()
+
+
+def test_reconstruct_matches_matmul(oracle_mod):
+    rng = np.random.default_rng(3)
+    A = rng.standard_normal((17, 5))
+    B = rng.standard_normal((5, 9))
+    assert np.allclose(oracle_mod.reconstruct(A, B), A @ B, rtol=0, atol=1e-13)
+    # a non-square case where a transposed operand could not match
+    assert oracle_mod.reconstruct(A, B).shape == (17, 9)
+
+
+# ---------------------------------------------------------------- allocation
+def test_alloc_golden(oracle_mod):
+    cases = json.load(open(os.path.join(GOLDEN, "alloc_tiny.json")))["cases"]
+    for c in cases:
+        sigma = np.asarray(c["sigma"], dtype=np.float64)
+        nb, d = sigma.shape
+        key = oracle_mod.keys(sigma, np.array([c["eps"]]), np.zeros(nb, dtype=np.int32))
+        caps = np.full(nb, d, dtype=np.int32)
+        g = oracle_mod.allocate_greedy(key, caps, c["R"])
+        s = oracle_mod.allocate_sort(key, caps, c["R"])
+        assert list(g) == c["ranks"], c["why"]
+        assert list(s) == c["ranks"], c["why"]
+
+
+def _brute(sigma, eps, caps, R, r_min):
+    """Max of sum log(1 + sigma^2/eps^2) over all rank vectors with sum R."""
+    nb, d = sigma.shape
+    gain = np.log1p(sigma ** 2 / eps ** 2)
+    cums = [np.concatenate([[0.0], np.cumsum(gain[b])]) for b in range(nb)]
+    best, arg = -1.0, None
+    ranges = [range(min(r_min, caps[b]), caps[b] + 1) for b in range(nb)]
+    for r in itertools.product(*ranges):
+        if sum(r) != R:
+            continue
+        f = sum(cums[b][r[b]] for b in range(nb))
+        if f > best + 1e-12 * abs(best):
+            best, arg = f, r
+    return best, arg
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_alloc_brute_force(oracle_mod, seed):
+    rng = np.random.default_rng(100 + seed)
+    nb = int(rng.integers(1, 5))
+    d = int(rng.integers(2, 7))
+    sigma = -np.sort(-rng.exponential(1.0, size=(nb, d)), axis=1)
+    if seed % 3 == 0:   # plant exact ties across blocks
+        sigma[:, :] = sigma[0:1, :]
+    eps = float(rng.uniform(0.05, 2.0))
+    caps = np.array([int(rng.integers(1, d + 1)) for _ in range(nb)], dtype=np.int32)
+    r_min = int(rng.integers(0, 2))
+    lo = sum(min(r_min, c) for c in caps)
+    R = int(rng.integers(lo, int(caps.sum()) + 1))
+    key = oracle_mod.keys(sigma, np.array([eps]), np.zeros(nb, dtype=np.int32))
+    g = oracle_mod.allocate_greedy(key, caps, R, r_min)
+    s = oracle_mod.allocate_sort(key, caps, R, r_min)
+    assert np.array_equal(g, s)
+    assert g.sum() == R
+    assert np.all(g <= caps) and np.all(g >= np.minimum(r_min, caps))
+    best, _ = _brute(sigma, eps, caps, R, r_min)
+    f = float(np.sum([np.sum(np.log1p(sigma[b, :g[b]] ** 2 / eps ** 2)) for b in range(nb)]))
+    assert f >= best - 1e-12 * max(abs(best), 1.0)
+    assert abs(oracle_mod.objective(key, g) - f) <= 1e-12 * max(abs(f), 1.0)
+
+
+def test_alloc_special_cases(oracle_mod):
+    rng = np.random.default_rng(5)
+    d = 8
+    one = -np.sort(-rng.exponential(1.0, size=(1, d)), axis=1)
+    k1 = oracle_mod.keys(one, np.array([0.1]), np.zeros(1, dtype=np.int32))
+    for R in range(0, d + 1):
+        assert list(oracle_mod.allocate_greedy(k1, np.array([d], np.int32), R)) == [R]
+    # identical spectra in every block: ranks differ by at most one, lower blocks first
+    nb = 5
+    same = np.repeat(one, nb, axis=0)
+    ks = oracle_mod.keys(same, np.array([0.1]), np.zeros(nb, dtype=np.int32))
+    caps = np.full(nb, d, np.int32)
+    for R in range(0, nb * d + 1):
+        r = oracle_mod.allocate_greedy(ks, caps, R)
+        assert r.max() - r.min() <= 1
+        assert np.all(np.diff(r) <= 0)
+        assert r.sum() == R
+    # budget 0 and budget 100%
+    rand = -np.sort(-rng.exponential(1.0, size=(4, d)), axis=1)
+    kr = oracle_mod.keys(rand, np.array([0.3]), np.zeros(4, dtype=np.int32))
+    caps = np.array([8, 3, 8, 5], np.int32)
+    assert list(oracle_mod.allocate_sort(kr, caps, 0)) == [0, 0, 0, 0]
+    assert list(oracle_mod.allocate_sort(kr, caps, int(caps.sum()))) == list(caps)
+    with pytest.raises(ValueError):
+        oracle_mod.allocate_sort(kr, caps, int(caps.sum()) + 1)
+
+
+def test_keys_groups_and_zero_eps(oracle_mod):
+    sigma = np.array([[2.0, 1.0], [2.0, 1.0], [0.0, 0.0]])
+    key = oracle_mod.keys(sigma, np.array([1.0, 2.0, 0.0]), np.array([0, 1, 2], np.int32))
+    assert key.tolist() == [[4.0, 1.0], [1.0, 0.25], [0.0, 0.0]]
+
+
+def test_budget_and_blocking(oracle_mod):
+    assert oracle_mod.block_lengths(2048, 256) == [256] * 8
+    assert oracle_mod.block_lengths(1000, 256) == [256, 256, 256, 232]
+    assert oracle_mod.budget(1, 1, 2048, 256, 128, 0.5) == 512
+    assert oracle_mod.budget(28, 4, 131072, 512, 128, 0.75) == 2752512
+    assert oracle_mod.budget(1, 1, 100, 64, 128, 0.5) == 50     # min(64,128) + min(36,128) = 100
+    assert oracle_mod.rank_caps(100, 64, 128) == [64, 36]
+    assert oracle_mod.rank_caps(100, 64, 128, r_max=40) == [40, 36]
+
+
+# ---------------------------------------------------------------- INT8
+def test_int8_bound_and_zero_column(oracle_mod):
+    rng = np.random.default_rng(9)
+    X = (rng.standard_normal((50, 7)) * np.array([1, 1e-3, 10, 0, 3, 1e-6, 1])).astype(np.float32)
+    Q, s = oracle_mod.quant_int8_cols(X)
+    assert s[3] == 0.0 and np.all(Q[:, 3] == 0)
+    for j in range(7):
+        if s[j] == 0:
+            continue
+        err = np.abs(X[:, j].astype(np.float64) - s[j] * Q[:, j].astype(np.float64))
+        assert np.all(err <= s[j] * (0.5 + 1e-5))
+        assert np.abs(Q[:, j]).max() == 127
+    assert np.abs(Q.astype(int)).max() <= 127
+
+
+def test_int8_round_half_even(oracle_mod):
+    # column absmax 127 -> scale exactly 1.0; 2.5 -> 2, 3.5 -> 4, -2.5 -> -2
+    X = np.array([[127.0], [2.5], [3.5], [-2.5], [-127.0]], dtype=np.float32)
+    Q, s = oracle_mod.quant_int8_cols(X)
+    assert s[0] == 1.0
+    assert Q[:, 0].tolist() == [127, 2, 4, -2, -127]
+
+
+# ---------------------------------------------------------------- RoPE / attention
+def test_rope_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "rope_d4.json")))
+    for c in g["cases"]:
+        out = oracle_mod.rope(np.array(c["x"], float), c["pos"], g["base"])
+        assert np.allclose(out, c["out"], rtol=0, atol=1e-15), c["why"]
+
+
+def test_rope_properties(oracle_mod):
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal(128)
+    base = 1e6
+    assert np.array_equal(oracle_mod.rope(x, 0, base), x)
+    for p in [1, 77, 4095, 131071]:
+        y = oracle_mod.rope(x, p, base)
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) <= 1e-13 * np.linalg.norm(x)
+    # composition: R(a) R(b) = R(a + b)
+    a, b = 1234, 567
+    assert np.allclose(oracle_mod.rope(oracle_mod.rope(x, a, base), b, base),
+                       oracle_mod.rope(x, a + b, base), rtol=0, atol=1e-11)
+    # inner products depend only on the position difference
+    y = rng.standard_normal(128)
+    d1 = oracle_mod.rope(x, 1000, base) @ oracle_mod.rope(y, 900, base)
+    d2 = oracle_mod.rope(x, 100, base) @ oracle_mod.rope(y, 0, base)
+    assert abs(d1 - d2) <= 1e-11
+
+
+def test_attention_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "attention_2tok.json")))
+    out = oracle_mod.attention(np.array(g["q"], float), np.array(g["K"], float), np.array(g["V"], float))[0]
+    assert np.allclose(out, g["out"], rtol=0, atol=1e-15)
+
+
+def test_attention_special_cases_and_library(oracle_mod):
+    rng = np.random.default_rng(8)
+    K = rng.standard_normal((33, 16))
+    V = rng.standard_normal((33, 16))
+    # one token: output is its value
+    assert np.allclose(oracle_mod.attention(rng.standard_normal(16), K[:1], V[:1])[0], V[0], atol=1e-15)
+    # q = 0: uniform weights, output is the mean value
+    assert np.allclose(oracle_mod.attention(np.zeros(16), K, V)[0], V.mean(axis=0), atol=1e-14)
+    # scipy softmax as an independent library route
+    q = rng.standard_normal((3, 16)) * 3
+    ref = scipy.special.softmax(q @ K.T / 4.0, axis=1) @ V
+    assert np.allclose(oracle_mod.attention(q, K, V), ref, rtol=0, atol=1e-13)
+    # large scores do not overflow (max subtraction)
+    big = oracle_mod.attention(q * 1e3, K, V)
+    assert np.all(np.isfinite(big))
+
+
+def _full_rank_factors(oracle_mod, X, block_len):
+    A, B = [], []
+    T = X.shape[0]
+    for b in range(math.ceil(T / block_len)):
+        Xb = X[b * block_len:min((b + 1) * block_len, T)]
+        s, Vr, US, _ = oracle_mod.svd(Xb)
+        m = min(Xb.shape)
+        A.append(US[:, :m])
+        B.append(Vr[:, :m].T)
+    return A, B
+
+
+def test_full_rank_compressed_attention_equals_dense(oracle_mod):
+    rng = np.random.default_rng(21)
+    T, d, bl, base = 200, 16, 64, 1e4
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    AK, BK = _full_rank_factors(oracle_mod, K, bl)
+    AV, BV = _full_rank_factors(oracle_mod, V, bl)
+    q = rng.standard_normal(d)
+    blocks = [0, 1, 2, 3]
+    pos = [b * bl for b in blocks]
+    out = oracle_mod.decode_one(lambda b: AK[b], lambda b: BK[b], lambda b: AV[b], lambda b: BV[b],
+                                q, blocks, pos, base)
+    Kr = np.stack([oracle_mod.rope(K[t], t, base) for t in range(T)])
+    ref = scipy.special.softmax(Kr @ q / math.sqrt(d)) @ V
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+    # a subset of blocks equals dense attention over exactly those tokens
+    sub = [1, 3]
+    out2 = oracle_mod.decode_one(lambda b: AK[b], lambda b: BK[b], lambda b: AV[b], lambda b: BV[b],
+                                 q, sub, [b * bl for b in sub], base)
+    idx = np.r_[64:128, 192:200]
+    ref2 = scipy.special.softmax(Kr[idx] @ q / math.sqrt(d)) @ V[idx]
+    assert np.abs(out2 - ref2).max() <= 1e-12 * np.abs(ref2).max()
+
+
+def test_decode_invariances(oracle_mod):
+    rng = np.random.default_rng(22)
+    d, base = 16, 1e6
+    AK = [rng.standard_normal((40, 5)) for _ in range(3)]
+    BK = [np.linalg.qr(rng.standard_normal((d, 5)))[0].T for _ in range(3)]
+    AV = [rng.standard_normal((40, 4)) for _ in range(3)]
+    BV = [np.linalg.qr(rng.standard_normal((d, 4)))[0].T for _ in range(3)]
+    f = dict(AK=lambda b: AK[b], BK=lambda b: BK[b], AV=lambda b: AV[b], BV=lambda b: BV[b])
+    q = rng.standard_normal(d)
+    o = oracle_mod.decode_one(f["AK"], f["BK"], f["AV"], f["BV"], q, [0, 1, 2], [0, 40, 80], base)
+    # block order does not matter
+    o_perm = oracle_mod.decode_one(f["AK"], f["BK"], f["AV"], f["BV"], q, [2, 0, 1], [80, 0, 40], base)
+    assert np.abs(o - o_perm).max() <= 1e-14
+    # shifting every key position by m and rotating q by m leaves o unchanged
+    m = 100000
+    o_shift = oracle_mod.decode_one(f["AK"], f["BK"], f["AV"], f["BV"], oracle_mod.rope(q, m, base),
+                                    [0, 1, 2], [m, m + 40, m + 80], base)
+    assert np.abs(o - o_shift).max() <= 1e-10
+    # a rank-0 key block keeps its tokens in the softmax with score 0
+    z = np.zeros((40, 0))
+    o_zero = oracle_mod.decode_one(lambda b: z, lambda b: np.zeros((0, d)), f["AV"], f["BV"],
+                                   q, [0], [0], base)
+    assert np.allclose(o_zero, AV[0].mean(axis=0) @ BV[0], atol=1e-14)
+
+
+def test_compress_end_to_end_small(oracle_mod):
+    from block_wise_rank_b200 import synth
+    import torch
+    K = synth.planted_cache(1, 2, 300, 32, 64, (2.0, 10.0), seed=1, out_dtype=torch.float64)
+    V = synth.planted_cache(1, 2, 300, 32, 64, (4.0, 12.0), seed=2, out_dtype=torch.float64)
+    res = oracle_mod.compress(K.numpy(), V.numpy(), 64, budget_frac=0.5, eps_rel=1e-2)
+    for kind, X in enumerate((K.numpy(), V.numpy())):
+        r = res[kind]
+        R = oracle_mod.budget(1, 2, 300, 64, 32, 0.5)
+        assert r["ranks"].sum() == R == r["R"]
+        assert np.allclose(r["eps"], 1e-2 * r["sigma"][..., 0].max(axis=-1), rtol=0, atol=0)
+        for h in range(2):
+            for b in range(5):
+                tb = min(64, 300 - 64 * b)
+                Xb = X[0, h, 64 * b:64 * b + tb]
+                rb = r["ranks"][0, h, b]
+                assert rb <= min(tb, 32)
+                Xh = oracle_mod.reconstruct(r["A"][0][h][b], r["B"][0][h][b]) if rb else np.zeros_like(Xb)
+                tail = np.sum(r["sigma"][0, h, b, rb:] ** 2)
+                assert abs(np.sum((Xb - Xh) ** 2) - tail) <= 1e-9 * tail + 1e-20
