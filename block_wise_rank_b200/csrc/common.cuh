@@ -1,0 +1,72 @@
+// common.cuh -- shared device helpers of libmilo (one translation unit).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "milo.h"
+
+namespace milo {
+
+constexpr int D = 128;          // head dimension served by every kernel
+constexpr int HALF = D / 2;     // RoPE pairs (i, i + 64)
+
+// Device status word (one per device that loads the library).  Kernels OR
+// bits into it; milo_get_status reads and clears it.
+enum : unsigned {
+    ST_NOT_CONVERGED = 1u,
+    ST_NONFINITE = 2u,
+    ST_BOUNDS = 4u,
+    ST_UNSORTED = 8u,
+    ST_TIMEOUT = 16u,
+};
+__device__ unsigned g_status;
+
+__device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
+
+__host__ __device__ __forceinline__ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// tokens in block b of a (layer, head) row of T tokens
+__host__ __device__ __forceinline__ int block_tokens(int T, int block_len, int b) {
+    int r = T - b * block_len;
+    return r < block_len ? r : block_len;
+}
+
+// largest admissible rank of a block: min(T_b, d, r_max if > 0)
+__host__ __device__ __forceinline__ int block_cap(int Tb, int r_max) {
+    int c = Tb < D ? Tb : D;
+    if (r_max > 0 && r_max < c) c = r_max;
+    return c;
+}
+
+// element loads of a factor / cache in any supported dtype, as fp32
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f32<int8_t>(int8_t v) { return (float)v; }
+
+__device__ __forceinline__ float load_elem(const void *base, int64_t i, int dtype) {
+    switch (dtype) {
+    case MILO_F32: return ((const float *)base)[i];
+    case MILO_BF16: return __bfloat162float(((const __nv_bfloat16 *)base)[i]);
+    default: return (float)((const int8_t *)base)[i];
+    }
+}
+
+__host__ __device__ __forceinline__ int dtype_bytes(int dtype) {
+    return dtype == MILO_F32 ? 4 : (dtype == MILO_BF16 ? 2 : 1);
+}
+
+// One kind's section of the factor arena (device pointers).
+struct KindView {
+    int32_t *ranks;
+    int64_t *offsets;
+    float *sigma;
+    double *eps;
+    float *scaleA;
+    float *scaleB;
+    void *data;
+};
+
+}  // namespace milo

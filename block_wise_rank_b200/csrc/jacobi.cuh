@@ -1,0 +1,172 @@
+// jacobi.cuh -- batched one-sided Jacobi on the d x d Gram tile, one CTA per
+// (block, kind), the tile held in shared memory.
+//
+// Step "SVD of K and of V per block" (evolve.pub review of MILO, Summary).
+// One-sided (Hestenes) Jacobi orthogonalises the columns of X_b by plane
+// rotations; the rotation for the column pair (p, q) is decided by the three
+// inner products a_p.a_p, a_q.a_q and a_p.a_q, which are the entries of the
+// rotated Gram matrix G' = W^T G W.  Keeping G' (d x d) in shared memory
+// instead of X_b (T_b x d) turns each column rotation into the symmetric
+// update G' <- J^T G' J and the accumulation W <- W J; X_b itself is rotated
+// once, at the end, by the projection A_b = X_b W (project.cuh).  The
+// converged diagonal holds sigma_k^2 and W the right singular vectors.
+//
+// Parallel order: the round-robin ("circle") tournament -- 127 rounds of 64
+// disjoint pairs per sweep; pairs of one round commute, so all 64 rotations
+// of a round are applied at once.  A sweep with no rotation ends the solve;
+// the sweep cap raises ST_NOT_CONVERGED and still writes the current result.
+#pragma once
+#include "common.cuh"
+
+namespace milo {
+
+constexpr int JAC_THREADS = 512;
+constexpr int JAC_NPAIR = D / 2;                       // 64 pairs per round
+constexpr int JAC_NTRI = JAC_NPAIR * (JAC_NPAIR + 1) / 2;  // 2080 pair blocks (i <= i2)
+constexpr int JAC_LD = D + 1;                          // padded row stride of G and W
+
+struct JacobiSmem {
+    float G[D * JAC_LD];
+    float W[D * JAC_LD];
+    float c[JAC_NPAIR], s[JAC_NPAIR], t[JAC_NPAIR];
+    int p[JAC_NPAIR], q[JAC_NPAIR];
+    unsigned short tri[JAC_NTRI][2];
+    float lam[D];
+    int rank[D];
+    float floor_abs;
+};
+
+// G_io: [2][n_blk][128][128] fp32.  In: the Gram matrices.  Out: the
+// eigenvectors, columns sorted by descending eigenvalue (W[j][k] = v_k[j]).
+// sigma_K/sigma_V: [n_blk][128] singular values, descending; entries past
+// min(T_b, d) are set to 0 (the rank of a T_b x d block).
+__global__ void __launch_bounds__(JAC_THREADS, 1)
+k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restrict__ sigma_V,
+         int64_t n_blk, int Tn, int block_len, int n_b, int max_sweeps, float tol) {
+    extern __shared__ __align__(16) unsigned char jac_raw[];
+    JacobiSmem &sm = *reinterpret_cast<JacobiSmem *>(jac_raw);
+    const int tid = threadIdx.x;
+    const int blk = blockIdx.x, kind = blockIdx.y;
+    float *Gg = G_io + ((int64_t)kind * n_blk + blk) * D * D;
+
+    for (int e = tid; e < D * D; e += JAC_THREADS) {
+        int i = e / D, j = e % D;
+        sm.G[i * JAC_LD + j] = Gg[e];
+        sm.W[i * JAC_LD + j] = (i == j) ? 1.f : 0.f;
+    }
+    for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
+        // enumerate pair blocks (i, i2) with i <= i2
+        int i = 0, rem = e;
+        while (rem >= JAC_NPAIR - i) { rem -= JAC_NPAIR - i; ++i; }
+        sm.tri[e][0] = (unsigned short)i;
+        sm.tri[e][1] = (unsigned short)(i + rem);
+    }
+    __syncthreads();
+    if (tid < 32) {
+        float tr = 0.f;
+        for (int k = tid; k < D; k += 32) tr += fabsf(sm.G[k * JAC_LD + k]);
+        for (int o = 16; o; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
+        if (tid == 0) sm.floor_abs = 1e-10f * tr;
+    }
+    __syncthreads();
+    const float floor_abs = sm.floor_abs;
+
+    bool converged = false;
+    for (int sweep = 0; sweep < max_sweeps && !converged; ++sweep) {
+        int any = 0;
+        for (int r = 0; r < D - 1; ++r) {
+            int rot = 0;
+            if (tid < JAC_NPAIR) {
+                int a, b;
+                if (tid == 0) { a = r; b = D - 1; }
+                else { a = (r + tid) % (D - 1); b = (r - tid + (D - 1)) % (D - 1); }
+                int p = min(a, b), q = max(a, b);
+                float app = sm.G[p * JAC_LD + p], aqq = sm.G[q * JAC_LD + q], apq = sm.G[p * JAC_LD + q];
+                float c = 1.f, s = 0.f, tn = 0.f;
+                if (fabsf(apq) > floor_abs && fabsf(apq) > tol * sqrtf(fabsf(app)) * sqrtf(fabsf(aqq))) {
+                    float zeta = (aqq - app) / (2.f * apq);
+                    tn = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
+                    c = rsqrtf(1.f + tn * tn);
+                    s = c * tn;
+                    rot = 1;
+                }
+                sm.p[tid] = p; sm.q[tid] = q;
+                sm.c[tid] = c; sm.s[tid] = s; sm.t[tid] = tn;
+            }
+            rot = __syncthreads_or(rot);
+            any |= rot;
+            if (!rot) continue;   // uniform across the CTA
+            // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2, mirrored
+            for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
+                const int i = sm.tri[e][0], i2 = sm.tri[e][1];
+                const int p = sm.p[i], q = sm.q[i];
+                const float c1 = sm.c[i], s1 = sm.s[i];
+                if (i == i2) {
+                    if (s1 != 0.f) {
+                        const float tn = sm.t[i];
+                        const float apq = sm.G[p * JAC_LD + q];
+                        sm.G[p * JAC_LD + p] -= tn * apq;
+                        sm.G[q * JAC_LD + q] += tn * apq;
+                        sm.G[p * JAC_LD + q] = 0.f;
+                        sm.G[q * JAC_LD + p] = 0.f;
+                    }
+                    continue;
+                }
+                const int p2 = sm.p[i2], q2 = sm.q[i2];
+                const float c2 = sm.c[i2], s2 = sm.s[i2];
+                const float a = sm.G[p * JAC_LD + p2], bb = sm.G[p * JAC_LD + q2];
+                const float cc = sm.G[q * JAC_LD + p2], ee = sm.G[q * JAC_LD + q2];
+                // columns (p2, q2) by J2, then rows (p, q) by J1^T
+                const float a1 = c2 * a - s2 * bb, b1 = s2 * a + c2 * bb;
+                const float c1_ = c2 * cc - s2 * ee, e1 = s2 * cc + c2 * ee;
+                const float na = c1 * a1 - s1 * c1_, nc = s1 * a1 + c1 * c1_;
+                const float nb = c1 * b1 - s1 * e1, ne = s1 * b1 + c1 * e1;
+                sm.G[p * JAC_LD + p2] = na; sm.G[p2 * JAC_LD + p] = na;
+                sm.G[p * JAC_LD + q2] = nb; sm.G[q2 * JAC_LD + p] = nb;
+                sm.G[q * JAC_LD + p2] = nc; sm.G[p2 * JAC_LD + q] = nc;
+                sm.G[q * JAC_LD + q2] = ne; sm.G[q2 * JAC_LD + q] = ne;
+            }
+            // W <- W J: columns (p_i, q_i) of every row
+            for (int e = tid; e < D * JAC_NPAIR; e += JAC_THREADS) {
+                const int i = e % JAC_NPAIR, j = e / JAC_NPAIR;
+                const float s1 = sm.s[i];
+                if (s1 == 0.f) continue;
+                const float c1 = sm.c[i];
+                const int p = sm.p[i], q = sm.q[i];
+                const float wp = sm.W[j * JAC_LD + p], wq = sm.W[j * JAC_LD + q];
+                sm.W[j * JAC_LD + p] = c1 * wp - s1 * wq;
+                sm.W[j * JAC_LD + q] = s1 * wp + c1 * wq;
+            }
+            __syncthreads();
+        }
+        if (!any) converged = true;
+    }
+    if (!converged && tid == 0) raise_status(ST_NOT_CONVERGED);
+
+    // eigenvalues, stable descending order
+    if (tid < D) sm.lam[tid] = sm.G[tid * JAC_LD + tid];
+    __syncthreads();
+    if (tid < D) {
+        const float lk = sm.lam[tid];
+        int rk = 0;
+        for (int j = 0; j < D; ++j) {
+            const float lj = sm.lam[j];
+            rk += (lj > lk) || (lj == lk && j < tid);
+        }
+        sm.rank[tid] = rk;
+        if (!isfinite(lk)) raise_status(ST_NONFINITE);
+        float *sig = (kind == 0 ? sigma_K : sigma_V) + (int64_t)blk * D;
+        // X_b has rank <= T_b: singular values past min(T_b, d) are exactly 0
+        const int Tb = block_tokens(Tn, block_len, blk % n_b);
+        sig[rk] = rk < Tb ? sqrtf(fmaxf(lk, 0.f)) : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < D * D; e += JAC_THREADS) {
+        const int j = e / D, k = e % D;
+        Gg[j * D + sm.rank[k]] = sm.W[j * JAC_LD + k];
+    }
+}
+
+inline size_t jacobi_smem_bytes() { return sizeof(JacobiSmem); }
+
+}  // namespace milo

@@ -1,0 +1,580 @@
+// milo.cu -- libmilo: the C ABI (include/milo.h) and its launch sequences.
+//
+// One translation unit: the kernel headers below are included here so that
+// the library has one device status word and needs no relocatable device
+// code.  Every step of the path runs in these kernels; the host code only
+// validates arguments, lays out caller-owned buffers and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+#include "gram_simt.cuh"
+#include "gram_tc.cuh"
+#include "jacobi.cuh"
+#include "alloc.cuh"
+#include "project_simt.cuh"
+#include "decode_simt.cuh"
+#include "decode_tc.cuh"
+
+using namespace milo;
+
+struct milo_factors {
+    milo_cache_shape shape;
+    milo_compress_params params;
+    void *arena;
+    size_t arena_bytes;
+    int n_b;
+    int64_t n_blk;
+    int64_t R;
+    KindView kv[2];
+};
+
+namespace {
+
+constexpr int kLdPad = 16;     // token stride rounding of packed A^T rows
+constexpr size_t kAlign = 256;
+
+bool g_log = false;
+
+void log_msg(const char *what) {
+    if (g_log) fprintf(stderr, "[milo] %s\n", what);
+}
+
+struct Init {
+    Init() {
+        const char *e = getenv("MILO_LOG");
+        g_log = e && e[0] == '1';
+    }
+} g_init;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+milo_compress_params effective(const milo_compress_params *p) {
+    milo_compress_params q = *p;
+    if (q.max_sweeps <= 0) q.max_sweeps = 24;
+    if (!(q.jacobi_tol > 0.f)) q.jacobi_tol = 1e-7f;
+    return q;
+}
+
+bool shape_ok(const milo_cache_shape *s) {
+    return s && s->L > 0 && s->H > 0 && s->T > 0 && s->block_len > 0 &&
+           (s->in_dtype == MILO_F32 || s->in_dtype == MILO_BF16);
+}
+
+int n_blocks(const milo_cache_shape *s) { return (s->T + s->block_len - 1) / s->block_len; }
+
+// sum over one (layer, head) row of the rank caps and of the r_min floors
+void cap_sums(const milo_cache_shape *s, int r_min, int r_max, int64_t &caps, int64_t &floors) {
+    caps = 0;
+    floors = 0;
+    const int nb = n_blocks(s);
+    for (int b = 0; b < nb; ++b) {
+        const int c = block_cap(block_tokens(s->T, s->block_len, b), r_max);
+        caps += c;
+        floors += r_min < c ? r_min : c;
+    }
+}
+
+int64_t budget_of(const milo_cache_shape *s, const milo_compress_params *p) {
+    if (!shape_ok(s) || !p) return -1;
+    if (p->budget_abs > 0) return p->budget_abs;
+    if (!(p->budget_frac >= 0.0 && p->budget_frac <= 1.0)) return -1;
+    int64_t total = 0;
+    const int nb = n_blocks(s);
+    for (int b = 0; b < nb; ++b) {
+        const int tb = block_tokens(s->T, s->block_len, b);
+        total += tb < D ? tb : D;
+    }
+    total *= (int64_t)s->L * s->H;
+    return (int64_t)std::floor(p->budget_frac * (double)total);
+}
+
+// Byte offsets of one kind's arrays inside its arena section.
+struct SectionLayout {
+    size_t ranks, offsets, sigma, eps, scaleA, scaleB, data, bytes;
+};
+
+SectionLayout section_layout(const milo_cache_shape *s, const milo_compress_params *p, int64_t R) {
+    SectionLayout o{};
+    const int64_t nblk = (int64_t)s->L * s->H * n_blocks(s);
+    size_t at = 0;
+    o.ranks = at;   at = align_up(at + sizeof(int32_t) * nblk);
+    o.offsets = at; at = align_up(at + sizeof(int64_t) * (nblk + 1));
+    o.sigma = at;   at = align_up(at + sizeof(float) * nblk * D);
+    o.eps = at;     at = align_up(at + sizeof(double) * (size_t)s->L * s->H);
+    o.scaleA = at;
+    o.scaleB = at;
+    if (p->factor_dtype == MILO_INT8) {
+        at = align_up(at + sizeof(float) * nblk * D);
+        o.scaleB = at;
+        at = align_up(at + sizeof(float) * nblk * D);
+    }
+    o.data = at;
+    at = align_up(at + (size_t)R * (size_t)(round_up(s->block_len, kLdPad) + D) * dtype_bytes(p->factor_dtype));
+    o.bytes = at;
+    return o;
+}
+
+void fill_views(milo_factors *f) {
+    const SectionLayout o = section_layout(&f->shape, &f->params, f->R);
+    for (int k = 0; k < 2; ++k) {
+        char *base = (char *)f->arena + (size_t)k * o.bytes;
+        f->kv[k].ranks = (int32_t *)(base + o.ranks);
+        f->kv[k].offsets = (int64_t *)(base + o.offsets);
+        f->kv[k].sigma = (float *)(base + o.sigma);
+        f->kv[k].eps = (double *)(base + o.eps);
+        f->kv[k].scaleA = f->params.factor_dtype == MILO_INT8 ? (float *)(base + o.scaleA) : nullptr;
+        f->kv[k].scaleB = f->params.factor_dtype == MILO_INT8 ? (float *)(base + o.scaleB) : nullptr;
+        f->kv[k].data = base + o.data;
+    }
+}
+
+milo_status params_ok(const milo_cache_shape *s, const milo_compress_params *p, int64_t *R_out) {
+    if (!shape_ok(s) || !p) return MILO_ERR_INVALID_ARG;
+    if (s->d != D) return MILO_ERR_UNSUPPORTED;
+    if (p->factor_dtype != MILO_F32 && p->factor_dtype != MILO_BF16 && p->factor_dtype != MILO_INT8)
+        return MILO_ERR_INVALID_ARG;
+    if (p->r_min < 0 || p->r_max < 0 || p->eps_scope < 0 || p->eps_scope > 1 || !(p->eps_rel >= 0.0))
+        return MILO_ERR_INVALID_ARG;
+    const int64_t R = budget_of(s, p);
+    if (R < 0) return MILO_ERR_INVALID_ARG;
+    int64_t caps, floors;
+    cap_sums(s, p->r_min, p->r_max, caps, floors);
+    const int64_t lh = (int64_t)s->L * s->H;
+    if (R < floors * lh || R > caps * lh) return MILO_ERR_INVALID_ARG;
+    if (R_out) *R_out = R;
+    return MILO_OK;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+milo_status cuda_check(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return MILO_OK;
+    if (g_log) fprintf(stderr, "[milo] %s: %s\n", what, cudaGetErrorString(e));
+    return MILO_ERR_CUDA;
+}
+
+int g_sm_count = 0;
+int sm_count() {
+    if (g_sm_count == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (g_sm_count <= 0) g_sm_count = 148;
+    }
+    return g_sm_count;
+}
+
+// Allocation scratch layout for two kinds.
+struct AllocScratch {
+    SelState *st;       // [2]
+    int32_t *gt, *eq;   // [2][n_blk] each
+    size_t bytes;
+};
+
+AllocScratch alloc_scratch(void *ws, int64_t n_blk) {
+    AllocScratch a{};
+    size_t at = 0;
+    char *b = (char *)ws;
+    a.st = (SelState *)(b + at); at = align_up(at + 2 * sizeof(SelState));
+    a.gt = (int32_t *)(b + at);  at = align_up(at + 2 * sizeof(int32_t) * n_blk);
+    a.eq = (int32_t *)(b + at);  at = align_up(at + 2 * sizeof(int32_t) * n_blk);
+    a.bytes = at;
+    return a;
+}
+
+// The selection launches for two kinds (kinds == 1 runs the first only).
+milo_status launch_select(SelArgs a0, SelArgs a1, const SelShape &sh, int kinds, cudaStream_t st) {
+    k_sel_init<<<kinds, 256, 0, st>>>(a0, a1);
+    const int64_t elems = sh.n_blk * D;
+    int grid = (int)std::min<int64_t>((elems + 255) / 256, (int64_t)sm_count() * 8);
+    if (grid < 1) grid = 1;
+    for (int pass = 0; pass < 8; ++pass)
+        k_sel_pass<<<dim3(grid, kinds), 256, 0, st>>>(a0, a1, sh, 56 - 8 * pass);
+    const int cgrid = (int)((sh.n_blk * 32 + 255) / 256);
+    k_sel_count<<<dim3(cgrid > 0 ? cgrid : 1, kinds), 256, 0, st>>>(a0, a1, sh);
+    k_sel_ranks<<<kinds, 1024, 0, st>>>(a0, a1, sh);
+    return cuda_check(cudaGetLastError(), "select launch");
+}
+
+bool g_smem_set = false;
+milo_status set_smem_attrs() {
+    if (g_smem_set) return MILO_OK;
+    cudaError_t e = cudaFuncSetAttribute(k_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)jacobi_smem_bytes());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_decode_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(DecodeSimtSmem));
+    if (e == cudaSuccess) e = gram_tc_set_attrs();
+    if (e == cudaSuccess) e = decode_tc_set_attrs();
+    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute");
+    g_smem_set = true;
+    return MILO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *milo_version(void) { return "0.1.0"; }
+
+const char *milo_status_string(milo_status s) {
+    switch (s) {
+    case MILO_OK: return "ok";
+    case MILO_WARN_NOT_CONVERGED: return "a Jacobi eigensolve reached its sweep cap";
+    case MILO_ERR_INVALID_ARG: return "invalid argument";
+    case MILO_ERR_UNSUPPORTED: return "unsupported shape or dtype (d must be 128)";
+    case MILO_ERR_CUDA: return "CUDA runtime error";
+    case MILO_ERR_WORKSPACE: return "workspace or arena too small";
+    case MILO_ERR_NONFINITE: return "non-finite value met on the device";
+    case MILO_ERR_BOUNDS: return "index out of range met on the device";
+    }
+    return "unknown status";
+}
+
+void milo_default_params(milo_compress_params *p) {
+    if (!p) return;
+    memset(p, 0, sizeof(*p));
+    p->budget_frac = 0.5;
+    p->budget_abs = 0;
+    p->eps_rel = 1e-2;
+    p->eps_scope = 0;
+    p->r_min = 0;
+    p->r_max = 0;
+    p->factor_dtype = MILO_BF16;
+    p->max_sweeps = 24;
+    p->jacobi_tol = 1e-7f;
+}
+
+int64_t milo_rank_budget(const milo_cache_shape *shape, const milo_compress_params *params) {
+    int64_t R = -1;
+    if (params_ok(shape, params, &R) != MILO_OK) return -1;
+    return R;
+}
+
+size_t milo_factor_arena_size(const milo_cache_shape *shape, const milo_compress_params *params) {
+    int64_t R;
+    if (params_ok(shape, params, &R) != MILO_OK) return 0;
+    return 2 * section_layout(shape, params, R).bytes;
+}
+
+size_t milo_compress_workspace_size(const milo_cache_shape *shape, const milo_compress_params *params) {
+    if (params_ok(shape, params, nullptr) != MILO_OK) return 0;
+    const int64_t nblk = (int64_t)shape->L * shape->H * n_blocks(shape);
+    const size_t gw = align_up(sizeof(float) * 2 * (size_t)nblk * D * D);
+    return gw + alloc_scratch(nullptr, nblk).bytes;
+}
+
+milo_status milo_compress(const milo_cache_shape *shape, const void *K, const void *V,
+                          const milo_compress_params *params_in, void *workspace, size_t ws_bytes,
+                          void *arena, size_t arena_bytes, milo_factors **out, milo_stream_t stream) {
+    if (!out) return MILO_ERR_INVALID_ARG;
+    *out = nullptr;
+    int64_t R;
+    milo_status st = params_ok(shape, params_in, &R);
+    if (st != MILO_OK) return st;
+    if (!K || !V || !workspace || !arena) return MILO_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(workspace, kAlign) || !aligned(arena, kAlign))
+        return MILO_ERR_INVALID_ARG;
+    if (ws_bytes < milo_compress_workspace_size(shape, params_in) ||
+        arena_bytes < milo_factor_arena_size(shape, params_in))
+        return MILO_ERR_WORKSPACE;
+    if ((st = set_smem_attrs()) != MILO_OK) return st;
+    const milo_compress_params p = effective(params_in);
+    milo_factors *f = new (std::nothrow) milo_factors();
+    if (!f) return MILO_ERR_INVALID_ARG;
+    f->shape = *shape;
+    f->params = p;
+    f->arena = arena;
+    f->arena_bytes = arena_bytes;
+    f->n_b = n_blocks(shape);
+    f->n_blk = (int64_t)shape->L * shape->H * f->n_b;
+    f->R = R;
+    fill_views(f);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t nblk = f->n_blk;
+    float *GW = (float *)workspace;
+    AllocScratch as = alloc_scratch((char *)workspace + align_up(sizeof(float) * 2 * (size_t)nblk * D * D), nblk);
+
+    // 1. Gram matrices of every block of K and V
+    const dim3 grid2((unsigned)nblk, 2);
+    if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->block_len)) {
+        st = launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H, shape->T,
+                            shape->block_len, f->n_b, GW, nblk, s);
+        if (st != MILO_OK) { delete f; return st; }
+    } else if (shape->in_dtype == MILO_BF16) {
+        k_gram_simt<__nv_bfloat16><<<grid2, 256, 0, s>>>((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
+                                                          shape->H, shape->T, shape->block_len, f->n_b, GW, nblk);
+    } else {
+        k_gram_simt<float><<<grid2, 256, 0, s>>>((const float *)K, (const float *)V, shape->H, shape->T,
+                                                  shape->block_len, f->n_b, GW, nblk);
+    }
+    // 2. eigensolve: sigma into the arena, sorted eigenvectors back into GW
+    k_jacobi<<<grid2, JAC_THREADS, jacobi_smem_bytes(), s>>>(GW, f->kv[0].sigma, f->kv[1].sigma, nblk, shape->T,
+                                                             shape->block_len, f->n_b, p.max_sweeps, p.jacobi_tol);
+    // 3. eps per (layer, head, kind)
+    const int ngroups = shape->L * shape->H;
+    k_eps<<<dim3(ngroups, 2), 256, 0, s>>>(f->kv[0].sigma, f->kv[1].sigma, f->kv[0].eps, f->kv[1].eps, f->n_b,
+                                           p.eps_rel);
+    if (p.eps_scope == 1) k_eps_global<<<2, 1024, 0, s>>>(f->kv[0].eps, f->kv[1].eps, ngroups);
+    // 4. global top-R selection, ranks and packed offsets
+    int64_t caps, floors;
+    cap_sums(shape, p.r_min, p.r_max, caps, floors);
+    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk, kLdPad};
+    SelArgs a[2];
+    for (int k = 0; k < 2; ++k) {
+        a[k].sigma = f->kv[k].sigma;
+        a[k].eps = f->kv[k].eps;
+        a[k].ranks = f->kv[k].ranks;
+        a[k].offsets = f->kv[k].offsets;
+        a[k].st = as.st + k;
+        a[k].gt = as.gt + k * nblk;
+        a[k].eq = as.eq + k * nblk;
+        a[k].need0 = R - floors * ngroups;
+    }
+    if ((st = launch_select(a[0], a[1], sh, 2, s)) != MILO_OK) { delete f; return st; }
+    // 5. projection A_b = X_b W_{:,1:r_b}, B_b = W_{:,1:r_b}^T, packing
+    ProjArgs pa{};
+    pa.X[0] = K;
+    pa.X[1] = V;
+    pa.W[0] = GW;
+    pa.W[1] = GW + (size_t)nblk * D * D;
+    pa.kv[0] = f->kv[0];
+    pa.kv[1] = f->kv[1];
+    pa.T = shape->T;
+    pa.block_len = shape->block_len;
+    pa.n_b = f->n_b;
+    pa.in_dtype = shape->in_dtype;
+    pa.out_dtype = p.factor_dtype;
+    pa.n_blk = nblk;
+    if (shape->in_dtype == MILO_BF16)
+        k_project_a<__nv_bfloat16><<<dim3((unsigned)nblk, D / 32, 2), 256, 0, s>>>(pa);
+    else
+        k_project_a<float><<<dim3((unsigned)nblk, D / 32, 2), 256, 0, s>>>(pa);
+    k_project_b<<<grid2, D, 0, s>>>(pa);
+    st = cuda_check(cudaGetLastError(), "compress launch");
+    if (st != MILO_OK) { delete f; return st; }
+    log_msg("compress launched");
+    *out = f;
+    return MILO_OK;
+}
+
+size_t milo_allocate_workspace_size(int32_t n_groups, int32_t n_b, int32_t d) {
+    if (n_groups <= 0 || n_b <= 0 || d != D) return 0;
+    return alloc_scratch(nullptr, (int64_t)n_groups * n_b).bytes;
+}
+
+milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_groups, int32_t n_b, int32_t d,
+                          int32_t T, int32_t block_len, int64_t R, int32_t r_min, int32_t r_max,
+                          int32_t *ranks_out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
+    if (d != D) return MILO_ERR_UNSUPPORTED;
+    if (!sigma || !eps || !ranks_out || !workspace || n_groups <= 0 || n_b <= 0 || block_len <= 0 || T <= 0 ||
+        r_min < 0 || r_max < 0 || R < 0)
+        return MILO_ERR_INVALID_ARG;
+    if ((int64_t)(T + block_len - 1) / block_len != n_b) return MILO_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign) || !aligned(sigma, 4) || !aligned(eps, 8) || !aligned(ranks_out, 4))
+        return MILO_ERR_INVALID_ARG;
+    const int64_t nblk = (int64_t)n_groups * n_b;
+    if (ws_bytes < milo_allocate_workspace_size(n_groups, n_b, d)) return MILO_ERR_WORKSPACE;
+    milo_cache_shape shp{1, 1, T, D, block_len, MILO_F32};
+    int64_t caps, floors;
+    cap_sums(&shp, r_min, r_max, caps, floors);
+    if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
+    AllocScratch as = alloc_scratch(workspace, nblk);
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, kLdPad};
+    SelArgs a{};
+    a.sigma = sigma;
+    a.eps = eps;
+    a.ranks = ranks_out;
+    a.offsets = nullptr;
+    a.st = as.st;
+    a.gt = as.gt;
+    a.eq = as.eq;
+    a.need0 = R - floors * n_groups;
+    return launch_select(a, a, sh, 1, (cudaStream_t)stream);
+}
+
+size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    if (!f || S <= 0 || Hq <= 0 || n_sel <= 0) return 0;
+    const int64_t slots = (int64_t)S * n_sel;
+    const int64_t rows = (int64_t)f->shape.L * S * Hq;
+    size_t at = 0;
+    at = align_up(at + sizeof(int32_t) * (f->n_b + 1) * 2);            // counts / cursor, starts
+    at = align_up(at + sizeof(int32_t) * slots);                       // slot list
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
+    at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
+    at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
+    return at;
+}
+
+milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                             const int32_t *selected, const int32_t *positions, int32_t n_sel, double rope_base,
+                             float *out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
+    if (!f || !q || !selected || !out || !workspace || S <= 0 || Hq <= 0 || n_sel <= 0)
+        return MILO_ERR_INVALID_ARG;
+    if (Hq % f->shape.H != 0 || !(rope_base > 0.0)) return MILO_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, kAlign) || !aligned(selected, 4))
+        return MILO_ERR_INVALID_ARG;
+    if (ws_bytes < milo_decode_workspace_size(f, S, Hq, n_sel)) return MILO_ERR_WORKSPACE;
+    milo_status st = set_smem_attrs();
+    if (st != MILO_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int n_b = f->n_b;
+    const int64_t slots = (int64_t)S * n_sel;
+    const int64_t rows = (int64_t)f->shape.L * S * Hq;
+    char *w = (char *)workspace;
+    size_t at = 0;
+    int32_t *cnt = (int32_t *)(w + at);
+    int32_t *start = cnt + (n_b + 1);
+    at = align_up(at + sizeof(int32_t) * (n_b + 1) * 2);
+    int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
+    float2 *rope_q = (float2 *)(w + at);
+    float2 *rope_t = rope_q + slots * HALF;
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);
+    float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
+    float2 *part_ml = (float2 *)(w + at);
+
+    DecodeArgs a{};
+    a.kv[0] = f->kv[0];
+    a.kv[1] = f->kv[1];
+    a.L = f->shape.L; a.H = f->shape.H; a.G = Hq / f->shape.H; a.T = f->shape.T;
+    a.block_len = f->shape.block_len; a.n_b = n_b; a.factor_dtype = f->params.factor_dtype;
+    a.S = S; a.Hq = Hq; a.n_sel = n_sel;
+    a.q = q; a.sel = selected; a.pos = positions;
+    a.slot_start = start; a.slot_list = list;
+    a.rope_q = rope_q; a.rope_t = rope_t;
+    a.part_o = part_o; a.part_ml = part_ml; a.out = out;
+
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (n_b + 1), s);
+    if (e != cudaSuccess) return cuda_check(e, "memset");
+    const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
+    k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
+    k_slot_scan<<<1, 32, 0, s>>>(cnt, start, n_b);
+    k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
+    const int64_t rt = (slots + f->shape.block_len) * HALF;
+    k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
+        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
+    if (decode_tc_supported(a)) {
+        st = launch_decode_tc(a, s);
+        if (st != MILO_OK) return st;
+    } else {
+        k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
+    }
+    k_combine<<<(unsigned)rows, D, 0, s>>>(a);
+    return cuda_check(cudaGetLastError(), "decode launch");
+}
+
+milo_status milo_factors_get(const milo_factors *f, int32_t kind, int32_t **ranks, int64_t **offsets,
+                             float **sigma, double **eps, void **data, float **scaleA, float **scaleB,
+                             int64_t *R) {
+    if (!f || kind < 0 || kind > 1) return MILO_ERR_INVALID_ARG;
+    const KindView &v = f->kv[kind];
+    if (ranks) *ranks = v.ranks;
+    if (offsets) *offsets = v.offsets;
+    if (sigma) *sigma = v.sigma;
+    if (eps) *eps = v.eps;
+    if (data) *data = v.data;
+    if (scaleA) *scaleA = v.scaleA;
+    if (scaleB) *scaleB = v.scaleB;
+    if (R) *R = f->R;
+    return MILO_OK;
+}
+
+milo_status milo_factors_wrap(const milo_cache_shape *shape, const milo_compress_params *params, void *arena,
+                              size_t arena_bytes, milo_factors **out) {
+    if (!out) return MILO_ERR_INVALID_ARG;
+    *out = nullptr;
+    int64_t R;
+    milo_status st = params_ok(shape, params, &R);
+    if (st != MILO_OK) return st;
+    if (!arena || !aligned(arena, kAlign)) return MILO_ERR_INVALID_ARG;
+    if (arena_bytes < milo_factor_arena_size(shape, params)) return MILO_ERR_WORKSPACE;
+    milo_factors *f = new (std::nothrow) milo_factors();
+    if (!f) return MILO_ERR_INVALID_ARG;
+    f->shape = *shape;
+    f->params = effective(params);
+    f->arena = arena;
+    f->arena_bytes = arena_bytes;
+    f->n_b = n_blocks(shape);
+    f->n_blk = (int64_t)shape->L * shape->H * f->n_b;
+    f->R = R;
+    fill_views(f);
+    *out = f;
+    return MILO_OK;
+}
+
+namespace {
+struct BlobHeader {
+    char magic[8];
+    uint32_t version;
+    uint32_t pad;
+    milo_cache_shape shape;
+    milo_compress_params params;
+    uint64_t arena_bytes;
+};
+}  // namespace
+
+milo_status milo_factors_export(const milo_factors *f, void *host_buf, size_t *bytes, milo_stream_t stream) {
+    if (!f || !bytes) return MILO_ERR_INVALID_ARG;
+    const size_t need = sizeof(BlobHeader) + milo_factor_arena_size(&f->shape, &f->params);
+    if (!host_buf) { *bytes = need; return MILO_OK; }
+    if (*bytes < need) { *bytes = need; return MILO_ERR_WORKSPACE; }
+    BlobHeader h{};
+    memcpy(h.magic, "MILOFAC1", 8);
+    h.version = 1;
+    h.shape = f->shape;
+    h.params = f->params;
+    h.arena_bytes = need - sizeof(BlobHeader);
+    memcpy(host_buf, &h, sizeof(h));
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync((char *)host_buf + sizeof(h), f->arena, h.arena_bytes, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    *bytes = need;
+    return cuda_check(e, "export copy");
+}
+
+milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena, size_t arena_bytes,
+                                milo_factors **out, milo_stream_t stream) {
+    if (!out) return MILO_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!host_buf || bytes < sizeof(BlobHeader) || !arena) return MILO_ERR_INVALID_ARG;
+    BlobHeader h;
+    memcpy(&h, host_buf, sizeof(h));
+    if (memcmp(h.magic, "MILOFAC1", 8) != 0 || h.version != 1) return MILO_ERR_INVALID_ARG;
+    if (bytes < sizeof(h) + h.arena_bytes) return MILO_ERR_INVALID_ARG;
+    if (h.arena_bytes != milo_factor_arena_size(&h.shape, &h.params)) return MILO_ERR_INVALID_ARG;
+    milo_factors *f = nullptr;
+    milo_status st = milo_factors_wrap(&h.shape, &h.params, arena, arena_bytes, &f);
+    if (st != MILO_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(arena, (const char *)host_buf + sizeof(h), h.arena_bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) { delete f; return cuda_check(e, "import copy"); }
+    *out = f;
+    return MILO_OK;
+}
+
+void milo_factors_destroy(milo_factors *f) { delete f; }
+
+milo_status milo_get_status(milo_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_check(e, "stream sync");
+    unsigned bits = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&bits, g_status, sizeof(bits));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_check(e, "status read");
+    if (bits & ST_BOUNDS) return MILO_ERR_BOUNDS;
+    if (bits & ST_NONFINITE) return MILO_ERR_NONFINITE;
+    if (bits & ST_UNSORTED) return MILO_ERR_INVALID_ARG;
+    if (bits & ST_TIMEOUT) return MILO_ERR_CUDA;
+    if (bits & ST_NOT_CONVERGED) return MILO_WARN_NOT_CONVERGED;
+    return MILO_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// project_simt.cuh -- projection and packing of the low-rank factors.
+//
+// Step "keep the top r_b singular triplets of each block and store the
+// cache in compressed low-rank form per block" (evolve.pub review of MILO,
+// Summary and FAQ "What is MILO"): A_b = X_b W_{:,1:r_b} = U_r Sigma_r
+// (T_b x r_b) and B_b = W_{:,1:r_b}^T (r_b x d), written into the packed
+// arena (A_b^T rank rows of ldT_b tokens, then B_b).  INT8 composition
+// (same page, Summary: combined with INT8 quantisation): symmetric per-column
+// absmax codes, scale = absmax / 127, round half to even, clamp to +-127.
+#pragma once
+#include "common.cuh"
+
+namespace milo {
+
+template <typename TO> __device__ __forceinline__ TO from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ int8_t quant_i8(float x, float s) {
+    if (!(s > 0.f)) return 0;
+    float q = rintf(__fdiv_rn(x, s));
+    q = fminf(fmaxf(q, -127.f), 127.f);
+    return (int8_t)q;
+}
+
+struct ProjArgs {
+    const void *X[2];          // K, V caches [L][H][T][D]
+    const float *W[2];         // sorted right singular vectors [n_blk][D][D] (W[j][k])
+    KindView kv[2];
+    int T, block_len, n_b, in_dtype, out_dtype;
+    int64_t n_blk;
+};
+
+// grid (n_blk, D/32 rank chunks, 2 kinds), 256 threads.  Writes the columns
+// k0 .. k0+31 of A_b (as rows of A_b^T) and, for INT8, their scales.
+template <typename TI>
+__global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
+    __shared__ float Wc[D][33];
+    __shared__ float amax[32];
+    const int blk = blockIdx.x, kind = blockIdx.z;
+    const int k0 = blockIdx.y * 32;
+    const KindView &kv = pa.kv[kind];
+    const int r = kv.ranks[blk];
+    if (k0 >= r) return;
+    const int kc = min(32, r - k0);
+    const int b = blk % pa.n_b, lh = blk / pa.n_b;
+    const int Tb = block_tokens(pa.T, pa.block_len, b);
+    const int ldT = (int)round_up(Tb, 16);
+    const TI *Xb = (const TI *)pa.X[kind] + ((int64_t)lh * pa.T + (int64_t)b * pa.block_len) * D;
+    const float *Wb = pa.W[kind] + (int64_t)blk * D * D;
+    for (int e = threadIdx.x; e < D * 32; e += 256) {
+        const int j = e / 32, c = e % 32;
+        Wc[j][c] = c < kc ? Wb[j * D + k0 + c] : 0.f;
+    }
+    if (threadIdx.x < 32) amax[threadIdx.x] = 0.f;
+    __syncthreads();
+    const int64_t base = kv.offsets[blk];
+    const bool is_i8 = pa.out_dtype == MILO_INT8;
+    for (int pass = is_i8 ? 0 : 1; pass < 2; ++pass) {
+        for (int t = threadIdx.x; t < ldT; t += 256) {
+            float acc[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+            if (t < Tb) {
+                const TI *xr = Xb + (int64_t)t * D;
+                for (int j = 0; j < D; ++j) {
+                    const float x = to_f32<TI>(xr[j]);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[c] = fmaf(x, Wc[j][c], acc[c]);
+                }
+            }
+            if (pass == 0) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    if (c < kc) atomicMax((int *)&amax[c], __float_as_int(fabsf(acc[c])));
+            } else {
+                for (int c = 0; c < kc; ++c) {
+                    const int64_t o = base + (int64_t)(k0 + c) * ldT + t;
+                    if (pa.out_dtype == MILO_F32) ((float *)kv.data)[o] = acc[c];
+                    else if (pa.out_dtype == MILO_BF16) ((__nv_bfloat16 *)kv.data)[o] = __float2bfloat16_rn(acc[c]);
+                    else ((int8_t *)kv.data)[o] = quant_i8(acc[c], __fdiv_rn(amax[c], 127.f));
+                }
+            }
+        }
+        __syncthreads();
+        if (pass == 0 && threadIdx.x < kc)
+            kv.scaleA[(int64_t)blk * D + k0 + threadIdx.x] = __fdiv_rn(amax[threadIdx.x], 127.f);
+        __syncthreads();
+    }
+}
+
+// grid (n_blk, 2 kinds), 128 threads: thread j writes column j of B_b
+// (B_b[k][j] = W[j][k], k < r_b) and, for INT8, its scale.
+__global__ void __launch_bounds__(128) k_project_b(ProjArgs pa) {
+    const int blk = blockIdx.x, kind = blockIdx.y, j = threadIdx.x;
+    const KindView &kv = pa.kv[kind];
+    const int r = kv.ranks[blk];
+    const int b = blk % pa.n_b;
+    const int Tb = block_tokens(pa.T, pa.block_len, b);
+    const int64_t base = kv.offsets[blk] + (int64_t)r * round_up(Tb, 16);
+    const float *Wb = pa.W[kind] + (int64_t)blk * D * D + (int64_t)j * D;
+    if (pa.out_dtype == MILO_INT8) {
+        float m = 0.f;
+        for (int k = 0; k < r; ++k) m = fmaxf(m, fabsf(Wb[k]));
+        const float s = __fdiv_rn(m, 127.f);
+        kv.scaleB[(int64_t)blk * D + j] = s;
+        for (int k = 0; k < r; ++k) ((int8_t *)kv.data)[base + (int64_t)k * D + j] = quant_i8(Wb[k], s);
+    } else if (pa.out_dtype == MILO_BF16) {
+        for (int k = 0; k < r; ++k) ((__nv_bfloat16 *)kv.data)[base + (int64_t)k * D + j] = __float2bfloat16_rn(Wb[k]);
+    } else {
+        for (int k = 0; k < r; ++k) ((float *)kv.data)[base + (int64_t)k * D + j] = Wb[k];
+    }
+}
+
+}  // namespace milo

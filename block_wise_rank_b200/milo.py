@@ -1,0 +1,285 @@
+"""Thin ctypes binding of libmilo (include/milo.h), same names as the C ABI.
+
+Argument marshalling only: every step of the path runs in libmilo's CUDA
+kernels.  Tensors are passed as raw device (or host) pointers; PyTorch is
+used for device memory and streams.  There is no fallback: if libmilo.so is
+missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmilo.so")
+
+MILO_OK = 0
+MILO_WARN_NOT_CONVERGED = 1
+MILO_ERR_INVALID_ARG = -1
+MILO_ERR_UNSUPPORTED = -2
+MILO_ERR_CUDA = -3
+MILO_ERR_WORKSPACE = -4
+MILO_ERR_NONFINITE = -5
+MILO_ERR_BOUNDS = -6
+
+MILO_F32, MILO_BF16, MILO_INT8 = 0, 1, 2
+DTYPES = {"f32": MILO_F32, "bf16": MILO_BF16, "int8": MILO_INT8}
+
+
+class milo_cache_shape(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("block_len", ctypes.c_int32), ("in_dtype", ctypes.c_int)]
+
+
+class milo_compress_params(ctypes.Structure):
+    _fields_ = [("budget_frac", ctypes.c_double), ("budget_abs", ctypes.c_int64), ("eps_rel", ctypes.c_double),
+                ("eps_scope", ctypes.c_int32), ("r_min", ctypes.c_int32), ("r_max", ctypes.c_int32),
+                ("factor_dtype", ctypes.c_int), ("max_sweeps", ctypes.c_int32), ("jacobi_tol", ctypes.c_float)]
+
+
+class MiloError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+EXPORTS = [
+    "milo_factor_arena_size", "milo_compress_workspace_size", "milo_rank_budget", "milo_default_params",
+    "milo_compress", "milo_allocate_workspace_size", "milo_allocate", "milo_decode_workspace_size",
+    "milo_decode_attn", "milo_factors_get", "milo_factors_wrap", "milo_factors_export",
+    "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
+]
+
+
+def lib():
+    """Load libmilo.so (raises if it is absent: there is no other path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmilo.so not built at {LIB_PATH}; run block_wise_rank_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        SP, PP = ctypes.POINTER(milo_cache_shape), ctypes.POINTER(milo_compress_params)
+        L.milo_factor_arena_size.argtypes = [SP, PP]; L.milo_factor_arena_size.restype = SZ
+        L.milo_compress_workspace_size.argtypes = [SP, PP]; L.milo_compress_workspace_size.restype = SZ
+        L.milo_rank_budget.argtypes = [SP, PP]; L.milo_rank_budget.restype = I64
+        L.milo_default_params.argtypes = [PP]; L.milo_default_params.restype = None
+        L.milo_compress.argtypes = [SP, P, P, PP, P, SZ, P, SZ, ctypes.POINTER(P), P]
+        L.milo_compress.restype = ctypes.c_int
+        L.milo_allocate_workspace_size.argtypes = [I32, I32, I32]; L.milo_allocate_workspace_size.restype = SZ
+        L.milo_allocate.argtypes = [P, P, I32, I32, I32, I32, I32, I64, I32, I32, P, P, SZ, P]
+        L.milo_allocate.restype = ctypes.c_int
+        L.milo_decode_workspace_size.argtypes = [P, I32, I32, I32]; L.milo_decode_workspace_size.restype = SZ
+        L.milo_decode_attn.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
+        L.milo_decode_attn.restype = ctypes.c_int
+        L.milo_factors_get.argtypes = [P, I32, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
+                                       ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
+                                       ctypes.POINTER(P), ctypes.POINTER(I64)]
+        L.milo_factors_get.restype = ctypes.c_int
+        L.milo_factors_wrap.argtypes = [SP, PP, P, SZ, ctypes.POINTER(P)]; L.milo_factors_wrap.restype = ctypes.c_int
+        L.milo_factors_export.argtypes = [P, P, ctypes.POINTER(SZ), P]; L.milo_factors_export.restype = ctypes.c_int
+        L.milo_factors_import.argtypes = [P, SZ, P, SZ, ctypes.POINTER(P), P]
+        L.milo_factors_import.restype = ctypes.c_int
+        L.milo_factors_destroy.argtypes = [P]; L.milo_factors_destroy.restype = None
+        L.milo_get_status.argtypes = [P]; L.milo_get_status.restype = ctypes.c_int
+        L.milo_status_string.argtypes = [ctypes.c_int]; L.milo_status_string.restype = ctypes.c_char_p
+        L.milo_version.argtypes = []; L.milo_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().milo_status_string(int(s)).decode()
+
+
+def _check(s: int, what: str, allow_warn: bool = False):
+    if s == MILO_OK or (allow_warn and s == MILO_WARN_NOT_CONVERGED):
+        return s
+    raise MiloError(s, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return MILO_F32
+    if t == torch.bfloat16:
+        return MILO_BF16
+    raise ValueError(f"unsupported cache dtype {t}")
+
+
+def default_params(**kw) -> milo_compress_params:
+    p = milo_compress_params()
+    lib().milo_default_params(ctypes.byref(p))
+    for k, v in kw.items():
+        if k == "factor_dtype" and isinstance(v, str):
+            v = DTYPES[v]
+        setattr(p, k, v)
+    return p
+
+
+def cache_shape(L, H, T, d, block_len, in_dtype) -> milo_cache_shape:
+    if isinstance(in_dtype, torch.dtype):
+        in_dtype = _dtype_code(in_dtype)
+    return milo_cache_shape(L, H, T, d, block_len, in_dtype)
+
+
+def milo_factor_arena_size(shape, params) -> int:
+    return lib().milo_factor_arena_size(ctypes.byref(shape), ctypes.byref(params))
+
+
+def milo_compress_workspace_size(shape, params) -> int:
+    return lib().milo_compress_workspace_size(ctypes.byref(shape), ctypes.byref(params))
+
+
+def milo_rank_budget(shape, params) -> int:
+    return lib().milo_rank_budget(ctypes.byref(shape), ctypes.byref(params))
+
+
+def _bytes(n: int, device) -> torch.Tensor:
+    # 256-byte aligned device buffer (the caching allocator aligns to 512 B)
+    return torch.empty(max(int(n), 1), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class Factors:
+    """A libmilo factor handle plus the device arena it views."""
+    handle: ctypes.c_void_p
+    arena: torch.Tensor
+    shape: milo_cache_shape
+    params: milo_compress_params
+
+    def view(self, kind: int):
+        """Device views of one kind as torch tensors (ranks, offsets, sigma, eps, data, scaleA, scaleB, R)."""
+        P = ctypes.c_void_p
+        ptrs = [P() for _ in range(7)]
+        R = ctypes.c_int64()
+        _check(lib().milo_factors_get(self.handle, kind, *[ctypes.byref(p) for p in ptrs], ctypes.byref(R)),
+               "milo_factors_get")
+        return [p.value for p in ptrs], R.value
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            lib().milo_factors_destroy(self.handle)
+            self.handle = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def milo_compress(K: torch.Tensor, V: torch.Tensor, block_len: int, params=None, workspace=None,
+                  arena=None, stream=None) -> Factors:
+    """Compress caches K (pre-RoPE) and V, [L][H][T][d] device tensors."""
+    assert K.shape == V.shape and K.dtype == V.dtype and K.is_cuda and V.is_cuda
+    assert K.is_contiguous() and V.is_contiguous()
+    L, H, T, d = K.shape
+    shape = cache_shape(L, H, T, d, block_len, K.dtype)
+    params = params or default_params()
+    ws_n = milo_compress_workspace_size(shape, params)
+    ar_n = milo_factor_arena_size(shape, params)
+    if ws_n == 0 or ar_n == 0:
+        raise MiloError(MILO_ERR_INVALID_ARG, "milo_compress sizes")
+    if workspace is None:
+        workspace = _bytes(ws_n, K.device)
+    if arena is None:
+        arena = _bytes(ar_n, K.device)
+    h = ctypes.c_void_p()
+    s = lib().milo_compress(ctypes.byref(shape), _ptr(K), _ptr(V), ctypes.byref(params), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _ptr(arena),
+                            arena.numel() * arena.element_size(), ctypes.byref(h), _stream(stream))
+    _check(s, "milo_compress")
+    return Factors(h, arena, shape, params)
+
+
+def milo_allocate_workspace_size(n_groups: int, n_b: int, d: int = 128) -> int:
+    return lib().milo_allocate_workspace_size(n_groups, n_b, d)
+
+
+def milo_allocate(sigma: torch.Tensor, eps: torch.Tensor, n_groups: int, n_b: int, T: int, block_len: int,
+                  R: int, r_min: int = 0, r_max: int = 0, ranks_out=None, workspace=None, stream=None):
+    """Ranks int32 [n_groups * n_b] for sigma float32 [n_groups*n_b][128], eps float64 [n_groups]."""
+    assert sigma.dtype == torch.float32 and eps.dtype == torch.float64 and sigma.is_contiguous()
+    d = sigma.shape[-1]
+    if ranks_out is None:
+        ranks_out = torch.empty(n_groups * n_b, dtype=torch.int32, device=sigma.device)
+    if workspace is None:
+        workspace = _bytes(milo_allocate_workspace_size(n_groups, n_b, d), sigma.device)
+    s = lib().milo_allocate(_ptr(sigma), _ptr(eps), n_groups, n_b, d, T, block_len, int(R), r_min, r_max,
+                            _ptr(ranks_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(s, "milo_allocate")
+    return ranks_out
+
+
+def milo_decode_workspace_size(f: Factors, S: int, Hq: int, n_sel: int) -> int:
+    return lib().milo_decode_workspace_size(f.handle, S, Hq, n_sel)
+
+
+def milo_decode_attn(f: Factors, q: torch.Tensor, selected: torch.Tensor, positions=None, rope_base=1e6,
+                     out=None, workspace=None, stream=None):
+    """GQA decode attention over the selected compressed blocks; q [L][S][Hq][d] fp32."""
+    assert q.dtype == torch.float32 and q.is_contiguous() and q.is_cuda
+    L, S, Hq, d = q.shape
+    n_sel = selected.shape[1]
+    assert selected.dtype == torch.int32 and selected.shape[0] == S and selected.is_contiguous()
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.shape == selected.shape and positions.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = _bytes(milo_decode_workspace_size(f, S, Hq, n_sel), q.device)
+    s = lib().milo_decode_attn(f.handle, _ptr(q), S, Hq, _ptr(selected), _ptr(positions), n_sel, float(rope_base),
+                               _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(s, "milo_decode_attn")
+    return out
+
+
+def milo_factors_wrap(shape, params, arena: torch.Tensor) -> Factors:
+    h = ctypes.c_void_p()
+    _check(lib().milo_factors_wrap(ctypes.byref(shape), ctypes.byref(params), _ptr(arena),
+                                   arena.numel() * arena.element_size(), ctypes.byref(h)), "milo_factors_wrap")
+    return Factors(h, arena, shape, params)
+
+
+def milo_factors_export(f: Factors, stream=None) -> bytes:
+    n = ctypes.c_size_t(0)
+    _check(lib().milo_factors_export(f.handle, None, ctypes.byref(n), _stream(stream)), "milo_factors_export")
+    buf = ctypes.create_string_buffer(n.value)
+    _check(lib().milo_factors_export(f.handle, buf, ctypes.byref(n), _stream(stream)), "milo_factors_export")
+    return buf.raw
+
+
+def milo_factors_import(blob: bytes, arena: torch.Tensor, stream=None) -> Factors:
+    h = ctypes.c_void_p()
+    _check(lib().milo_factors_import(blob, len(blob), _ptr(arena), arena.numel() * arena.element_size(),
+                                     ctypes.byref(h), _stream(stream)), "milo_factors_import")
+    # recover shape/params from the blob header fields
+    shape = milo_cache_shape.from_buffer_copy(blob[16:16 + ctypes.sizeof(milo_cache_shape)])
+    off = 16 + ctypes.sizeof(milo_cache_shape)
+    off = (off + 7) // 8 * 8
+    params = milo_compress_params.from_buffer_copy(blob[off:off + ctypes.sizeof(milo_compress_params)])
+    return Factors(h, arena, shape, params)
+
+
+def milo_get_status(stream=None) -> int:
+    return lib().milo_get_status(_stream(stream))
+
+
+def milo_version() -> str:
+    return lib().milo_version().decode()

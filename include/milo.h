@@ -1,0 +1,235 @@
+/*
+ * milo.h -- C ABI of libmilo: block-wise low-rank compression of a many-shot
+ * KV cache and decode attention over the compressed blocks, on one NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operations follow "MILO: Efficient Many-shot In-Context Learning with
+ * Block-wise Low-rank Compression":
+ *   - evolve.pub review, Summary: the cache is split into blocks of several
+ *     demonstrations; K (taken before RoPE) and V are each decomposed by SVD
+ *     per block; per-block ranks maximise sum log(1 + sigma^2/eps^2) under a
+ *     global rank budget, chosen greedily (Eqs 5-7); at inference a
+ *     retriever picks blocks whose low-rank factors are rebuilt before
+ *     sparse attention.
+ *   - same page, Strengths "Principled, budget-feasible rank allocation":
+ *     greedy marginal gains log(1 + sigma^2/eps^2) under a global budget.
+ *   - same page, FAQ "What is MILO": the cache is stored in compressed
+ *     low-rank form per block and only the blocks a query needs are rebuilt.
+ *   - shd-paper mirror, original abstract: each block holds several
+ *     many-shot examples; rank budgets follow each block's information
+ *     entropy.
+ *
+ * Conventions for every call:
+ *   - Pointers documented as "device" point to memory of the current CUDA
+ *     device; "host" pointers to ordinary host memory.  The caller owns and
+ *     allocates every buffer (sizes come from the *_size queries); libmilo
+ *     allocates no device memory.
+ *   - Calls are asynchronous on the given stream and never synchronise the
+ *     host, except milo_get_status, milo_factors_export and
+ *     milo_factors_import, which say so.  Argument errors are returned
+ *     synchronously and launch nothing.  Errors found on the device (a
+ *     Jacobi sweep cap reached, non-finite input, a bad block id) set bits
+ *     of a per-device status word that milo_get_status reads and clears.
+ *   - No C++ exception crosses this interface.
+ *   - d (head dimension) must be 128.
+ */
+#ifndef MILO_H_
+#define MILO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *milo_stream_t;
+
+typedef enum {
+    MILO_OK = 0,
+    MILO_WARN_NOT_CONVERGED = 1,   /* a Jacobi eigensolve hit its sweep cap  */
+    MILO_ERR_INVALID_ARG = -1,     /* bad pointer, size, shape or budget      */
+    MILO_ERR_UNSUPPORTED = -2,     /* d != 128, dtype not supported here      */
+    MILO_ERR_CUDA = -3,            /* a CUDA runtime call failed              */
+    MILO_ERR_WORKSPACE = -4,       /* workspace or arena smaller than needed  */
+    MILO_ERR_NONFINITE = -5,       /* NaN/Inf met on the device               */
+    MILO_ERR_BOUNDS = -6           /* an index out of range met on the device */
+} milo_status;
+
+typedef enum { MILO_F32 = 0, MILO_BF16 = 1, MILO_INT8 = 2 } milo_dtype;
+
+/* A KV cache of one kind: [L][H][T][d] row-major (d contiguous). */
+typedef struct {
+    int32_t L;          /* layers                                        */
+    int32_t H;          /* KV heads per layer                            */
+    int32_t T;          /* tokens per (layer, head)                      */
+    int32_t d;          /* head dimension; must be 128                   */
+    int32_t block_len;  /* tokens per block (>= 1); the last may be short */
+    milo_dtype in_dtype;/* MILO_F32 or MILO_BF16                         */
+} milo_cache_shape;
+
+typedef struct {
+    /* Global rank budget R per kind (K and V have separate pools, each
+     * global over all (layer, head, block)): budget_abs if > 0, else
+     * floor(budget_frac * sum_b min(T_b, d)), evaluated in double. */
+    double budget_frac;
+    int64_t budget_abs;
+    /* eps = eps_rel * max_b sigma_{b,1}; over the blocks of one
+     * (layer, head, kind) when eps_scope == 0, over all of a kind when 1. */
+    double eps_rel;
+    int32_t eps_scope;
+    /* Rank bounds per block: r_min <= r_b <= min(T_b, d, r_max or d). */
+    int32_t r_min;
+    int32_t r_max;                /* 0 means no cap beyond min(T_b, d) */
+    milo_dtype factor_dtype;      /* MILO_F32, MILO_BF16 or MILO_INT8  */
+    int32_t max_sweeps;           /* Jacobi sweep cap (0 -> 24)        */
+    float jacobi_tol;             /* rotate while |g_pq| > tol*sqrt(g_pp g_qq) (0 -> 1e-7) */
+} milo_compress_params;
+
+/* Opaque host-side handle over a caller-owned factor arena. */
+typedef struct milo_factors milo_factors;
+
+/*
+ * Factor arena layout (device, caller-owned, one section per kind: K then V,
+ * each section start 256-byte aligned; N_blk = L*H*n_b, n_b = ceil(T /
+ * block_len), ldT = round_up(block_len, 16), ldT_b = round_up(T_b, 16)):
+ *   int32  ranks  [N_blk]
+ *   int64  offsets[N_blk + 1]   element offset of block b in data
+ *   float  sigma  [N_blk][d]    singular values, descending
+ *   double eps    [L*H]
+ *   float  scaleA [N_blk][d]    INT8 only: scale of column k of A_b
+ *   float  scaleB [N_blk][d]    INT8 only: scale of column j of B_b
+ *   elem   data   [R*(ldT + d)] elem = factor dtype
+ * Block b at data + offsets[b]: A_b^T as r_b rows of ldT_b elements (token
+ * t of rank row k at k*ldT_b + t; tokens past T_b are zero), followed by
+ * B_b as r_b rows of d elements.  A_b = U_r Sigma_r (T_b x r_b) and
+ * B_b = V_r^T (r_b x d), so X_b ~ A_b B_b.  Blocks are ordered (l, h, b).
+ */
+
+/* ----------------------------------------------------------------- sizes */
+
+/* Bytes of the factor arena for this shape and params (both kinds); 0 on
+ * invalid input. */
+size_t milo_factor_arena_size(const milo_cache_shape *shape, const milo_compress_params *params);
+
+/* Bytes of scratch milo_compress needs; 0 on invalid input. */
+size_t milo_compress_workspace_size(const milo_cache_shape *shape, const milo_compress_params *params);
+
+/* R per kind for this shape and params (the formula above); -1 if invalid. */
+int64_t milo_rank_budget(const milo_cache_shape *shape, const milo_compress_params *params);
+
+/* Fill params with the defaults: budget_frac 0.5, eps_rel 1e-2, scope 0,
+ * r_min 0, r_max 0, factor dtype BF16, 24 sweeps, tol 1e-7. */
+void milo_default_params(milo_compress_params *params);
+
+/* -------------------------------------------------------------- compress */
+
+/*
+ * Compress one cache (both kinds).  K_preRoPE and V: device, [L][H][T][d] in
+ * shape->in_dtype, read only.  workspace: device, >= ws_bytes of
+ * milo_compress_workspace_size.  arena: device, >= milo_factor_arena_size,
+ * 256-byte aligned, filled in the layout above.  On MILO_OK *out receives a
+ * new handle (host memory, free with milo_factors_destroy) whose views point
+ * into arena.  Steps, in order and per kind: per-block Gram X_b^T X_b
+ * (tensor cores for bf16), Jacobi eigensolve (sigma, right singular vectors),
+ * eps, global top-R selection of the gains, ranks and offsets, projection
+ * A_b = X_b W_{:,1:r_b} and packing.  Asynchronous on stream.
+ */
+milo_status milo_compress(const milo_cache_shape *shape, const void *K_preRoPE, const void *V,
+                          const milo_compress_params *params, void *workspace, size_t ws_bytes,
+                          void *arena, size_t arena_bytes, milo_factors **out, milo_stream_t stream);
+
+/* -------------------------------------------------------------- allocate */
+
+/* Bytes of scratch milo_allocate needs for n_blk = n_groups * n_b blocks. */
+size_t milo_allocate_workspace_size(int32_t n_groups, int32_t n_b, int32_t d);
+
+/*
+ * Greedy entropy-gain rank allocation for one kind (the Eqs 5-7 reading):
+ * choose ranks r_b, sum_b r_b = R, r_min_b = min(r_min, cap_b) <= r_b <=
+ * cap_b = min(T_b, d, r_max or d), maximising sum_b sum_{k<r_b}
+ * log(1 + sigma_{b,k}^2/eps_g^2).  Decided exactly by the global top
+ * (R - sum r_min_b) keys (sigma/eps)^2 in double (one division, one
+ * multiply, IEEE), ties to the lower linear index (group, block, k); this
+ * equals the greedy rule when sigma is non-increasing in k.
+ *   sigma:  device, float [n_groups*n_b][d], non-increasing within a block
+ *   eps:    device, double [n_groups] (eps <= 0 makes every key 0)
+ *   T, block_len: block b of a group has T_b = min(block_len, T - b*block_len)
+ *   ranks_out: device, int32 [n_groups*n_b]
+ * MILO_ERR_INVALID_ARG if R is outside [sum r_min_b, sum cap_b].
+ */
+milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_groups, int32_t n_b,
+                          int32_t d, int32_t T, int32_t block_len, int64_t R, int32_t r_min,
+                          int32_t r_max, int32_t *ranks_out, void *workspace, size_t ws_bytes,
+                          milo_stream_t stream);
+
+/* ---------------------------------------------------------------- decode */
+
+/* Bytes of scratch milo_decode_attn needs. */
+size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel);
+
+/*
+ * GQA decode attention over retrieved compressed blocks, all layers in one
+ * call.  For layer l, session s, query head hq (KV head hq / (Hq/H)), the
+ * output is softmax over every token of the selected blocks of
+ *   s_t = q . RoPE(a^K_t B_K, p_j + t) / sqrt(d),
+ * times the rebuilt values a^V_t B_V; keys are rebuilt and rotated per token
+ * (rotate-half pairs (i, i+64), theta_i = rope_base^(-2i/d)) and never
+ * written to memory.
+ *   q:        device, float [L][S][Hq][d], already rotated to its position
+ *   selected: device, int32 [S][n_sel] block ids (0 <= id < n_b), shared by
+ *             all layers and heads
+ *   positions:device, int32 [S][n_sel] start position of each selected
+ *             block, or NULL for id * block_len
+ *   out:      device, float [L][S][Hq][d]
+ * Hq must be a multiple of H.  Block ids out of range set MILO_ERR_BOUNDS in
+ * the status word and contribute nothing.
+ */
+milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                             const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                             double rope_base, float *out, void *workspace, size_t ws_bytes,
+                             milo_stream_t stream);
+
+/* ------------------------------------------------------ factor handles */
+
+/* Views (device pointers into the arena) of one kind (0 = K, 1 = V).  Any
+ * output pointer may be NULL.  R receives the kind's budget. */
+milo_status milo_factors_get(const milo_factors *f, int32_t kind, int32_t **ranks, int64_t **offsets,
+                             float **sigma, double **eps, void **data, float **scaleA,
+                             float **scaleB, int64_t *R);
+
+/* Wrap an arena already filled in the documented layout (for instance by
+ * the caller) in a new handle.  No device access. */
+milo_status milo_factors_wrap(const milo_cache_shape *shape, const milo_compress_params *params,
+                              void *arena, size_t arena_bytes, milo_factors **out);
+
+/* Serialise the handle's shape, params and arena into host_buf.  With
+ * host_buf NULL only *bytes is set to the size needed.  Synchronises stream. */
+milo_status milo_factors_export(const milo_factors *f, void *host_buf, size_t *bytes,
+                                milo_stream_t stream);
+
+/* Copy an exported blob into a caller-owned device arena (>= the arena size
+ * recorded in the blob) and return a handle over it.  Synchronises stream. */
+milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena, size_t arena_bytes,
+                                milo_factors **out, milo_stream_t stream);
+
+/* Free the handle only; the arena stays the caller's. */
+void milo_factors_destroy(milo_factors *f);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronise stream, then read and clear the current device's status word:
+ * MILO_OK, MILO_WARN_NOT_CONVERGED, or the most severe device error. */
+milo_status milo_get_status(milo_stream_t stream);
+
+/* Static description of a status code. */
+const char *milo_status_string(milo_status s);
+
+/* Library version, "major.minor.patch". */
+const char *milo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MILO_H_ */

@@ -1,0 +1,139 @@
+"""The C-ABI library loads, exports every symbol include/milo.h declares, and
+rejects bad arguments on the host (no GPU needed, nothing is launched)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from block_wise_rank_b200 import build as milo_build
+from block_wise_rank_b200 import milo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    milo_build.build()
+    return milo.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "milo.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(milo_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(milo.EXPORTS)
+
+
+def test_version_and_status_strings(L):
+    assert milo.milo_version() == "0.1.0"
+    for s in (0, 1, -1, -2, -3, -4, -5, -6):
+        assert milo.status_string(s) and milo.status_string(s) != "unknown status"
+    assert milo.status_string(42) == "unknown status"
+
+
+def _shape(L=1, H=1, T=2048, d=128, bl=256, dt=milo.MILO_F32):
+    return milo.milo_cache_shape(L, H, T, d, bl, dt)
+
+
+def test_budget_matches_oracle_formula(L, oracle_mod):
+    cases = [(1, 1, 2048, 256, 0.5), (1, 2, 4096, 512, 0.5), (36, 2, 32768, 512, 0.5),
+             (28, 4, 131072, 512, 0.25), (28, 4, 131072, 512, 0.75), (2, 3, 1000, 64, 0.3),
+             (1, 1, 300, 128, 1.0), (1, 1, 300, 128, 0.0)]
+    for Ln, H, T, bl, fr in cases:
+        p = milo.default_params(budget_frac=fr)
+        assert milo.milo_rank_budget(_shape(Ln, H, T, 128, bl), p) == oracle_mod.budget(Ln, H, T, bl, 128, fr)
+    p = milo.default_params(budget_abs=77)
+    assert milo.milo_rank_budget(_shape(), p) == 77
+
+
+def test_arena_size_layout(L):
+    # section = ranks | offsets | sigma | eps | [scaleA | scaleB] | data, each 256-byte aligned
+    def al(x):
+        return (x + 255) // 256 * 256
+    for dt, es in ((milo.MILO_F32, 4), (milo.MILO_BF16, 2), (milo.MILO_INT8, 1)):
+        for (Ln, H, T, bl) in ((1, 1, 2048, 256), (2, 3, 1000, 100), (28, 4, 131072, 512)):
+            p = milo.default_params(factor_dtype=dt)
+            s = _shape(Ln, H, T, 128, bl)
+            nb = math.ceil(T / bl)
+            nblk = Ln * H * nb
+            R = milo.milo_rank_budget(s, p)
+            sec = al(4 * nblk) + al(8 * (nblk + 1)) + al(4 * nblk * 128) + al(8 * Ln * H)
+            if dt == milo.MILO_INT8:
+                sec += 2 * al(4 * nblk * 128)
+            sec += al(R * ((bl + 15) // 16 * 16 + 128) * es)
+            assert milo.milo_factor_arena_size(s, p) == 2 * sec
+
+
+def test_invalid_arguments_rejected_on_host(L):
+    p = milo.default_params()
+    assert milo.milo_factor_arena_size(_shape(d=64), p) == 0                   # d != 128
+    assert milo.milo_factor_arena_size(_shape(bl=0), p) == 0
+    assert milo.milo_factor_arena_size(_shape(T=0), p) == 0
+    assert milo.milo_rank_budget(_shape(), milo.default_params(budget_frac=1.5)) == -1
+    assert milo.milo_rank_budget(_shape(), milo.default_params(budget_abs=10**9)) == -1   # > sum of caps
+    assert milo.milo_rank_budget(_shape(), milo.default_params(r_min=100, budget_frac=0.5)) == -1  # floors > R
+    assert milo.milo_rank_budget(_shape(), milo.default_params(factor_dtype=7)) == -1
+    h = ctypes.c_void_p()
+    s = _shape()
+    # null caches / workspace / arena: invalid argument before any device work
+    rc = L.milo_compress(ctypes.byref(s), None, None, ctypes.byref(p), None, 0, None, 0, ctypes.byref(h), None)
+    assert rc == milo.MILO_ERR_INVALID_ARG and not h.value
+    # d != 128 is unsupported
+    s64 = _shape(d=64)
+    rc = L.milo_compress(ctypes.byref(s64), ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.byref(p),
+                         ctypes.c_void_p(256), 1 << 40, ctypes.c_void_p(256), 1 << 40, ctypes.byref(h), None)
+    assert rc == milo.MILO_ERR_UNSUPPORTED
+    # misaligned pointers
+    rc = L.milo_compress(ctypes.byref(s), ctypes.c_void_p(258), ctypes.c_void_p(256), ctypes.byref(p),
+                         ctypes.c_void_p(256), 1 << 40, ctypes.c_void_p(256), 1 << 40, ctypes.byref(h), None)
+    assert rc == milo.MILO_ERR_INVALID_ARG
+    # too-small workspace / arena
+    rc = L.milo_compress(ctypes.byref(s), ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.byref(p),
+                         ctypes.c_void_p(256), 16, ctypes.c_void_p(256), 1 << 40, ctypes.byref(h), None)
+    assert rc == milo.MILO_ERR_WORKSPACE
+    rc = L.milo_compress(ctypes.byref(s), ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.byref(p),
+                         ctypes.c_void_p(256), 1 << 40, ctypes.c_void_p(256), 16, ctypes.byref(h), None)
+    assert rc == milo.MILO_ERR_WORKSPACE
+    # allocate: wrong d, budget out of range, n_b inconsistent with T
+    P = ctypes.c_void_p(256)
+    assert L.milo_allocate(P, P, 1, 8, 64, 2048, 256, 10, 0, 0, P, P, 1 << 30, None) == milo.MILO_ERR_UNSUPPORTED
+    assert L.milo_allocate(P, P, 1, 8, 128, 2048, 256, 1025, 0, 0, P, P, 1 << 30, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_allocate(P, P, 1, 7, 128, 2048, 256, 10, 0, 0, P, P, 1 << 30, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_allocate(P, P, 1, 8, 128, 2048, 256, 10, 0, 0, P, P, 8, None) == milo.MILO_ERR_WORKSPACE
+    # decode: null handle
+    assert L.milo_decode_attn(None, P, 1, 1, P, None, 1, 1e6, P, P, 1 << 30, None) == milo.MILO_ERR_INVALID_ARG
+
+
+def test_wrap_views_and_export_size(L):
+    p = milo.default_params(factor_dtype=milo.MILO_INT8)
+    s = _shape(2, 3, 1000, 128, 100)
+    n = milo.milo_factor_arena_size(s, p)
+    h = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: wrap does no device access
+    assert L.milo_factors_wrap(ctypes.byref(s), ctypes.byref(p), fake, n, ctypes.byref(h)) == 0
+    P = ctypes.c_void_p
+    ptrs = [P() for _ in range(7)]
+    R = ctypes.c_int64()
+    assert L.milo_factors_get(h, 0, *[ctypes.byref(x) for x in ptrs], ctypes.byref(R)) == 0
+    assert ptrs[0].value == (1 << 20)
+    assert R.value == milo.milo_rank_budget(s, p)
+    k1 = [P() for _ in range(7)]
+    assert L.milo_factors_get(h, 1, *[ctypes.byref(x) for x in k1], ctypes.byref(R)) == 0
+    assert k1[0].value - ptrs[0].value == n // 2
+    assert all(x.value % 256 == 0 for x in ptrs)
+    sz = ctypes.c_size_t(0)
+    assert L.milo_factors_export(h, None, ctypes.byref(sz), None) == 0
+    assert sz.value > n
+    assert L.milo_factors_get(h, 2, *[ctypes.byref(x) for x in k1], ctypes.byref(R)) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_factors_wrap(ctypes.byref(s), ctypes.byref(p), fake, n - 1, ctypes.byref(h)) == \
+        milo.MILO_ERR_WORKSPACE
+    L.milo_factors_destroy(h)

@@ -1,0 +1,279 @@
+"""GPU parity: libmilo (through its C ABI) against the fp64 CPU oracle on the
+same seeded inputs.
+
+Tolerances (written where they are used):
+  sigma:   |s_gpu - s_ref| <= 1e-4 * s_1 per block, and elementwise relative
+           1e-4 where s_ref >= 0.1 * s_1;
+  eps:     bit-exact (eps_rel times the max of the GPU's own sigma_1);
+  ranks:   bit-exact against the oracle allocator fed the GPU's sigma and eps;
+  recon:   | ||X - A B||_F^2 - sum_{k > r_b} s_ref_k^2 | <= 1e-3 * that sum;
+  decode:  ||o_gpu - o_ref||_inf / ||o_ref||_inf per output vector:
+           1e-3 against the oracle on the same factors (fp32, bf16, int8),
+           2e-2 for bf16 factors against the oracle on its own fp64 factors.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_wise_rank_b200 import build as milo_build
+from block_wise_rank_b200 import milo, synth
+from tests import arena as A
+
+pytestmark = pytest.mark.gpu
+
+SIG_TOL = 1e-4
+DEC_TOL = 1e-3
+DEC_TOL_BF16_OWN = 2e-2
+RECON_TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    milo_build.build()
+    milo.lib()
+    assert torch.cuda.is_available()
+
+
+def _oracle_block_svds(oracle_mod, X, block_len, blocks):
+    """Oracle SVD of the listed (l, h, b) blocks of one kind."""
+    out = {}
+    T = X.shape[2]
+    for (l, h, b) in blocks:
+        Xb = X[l, h, b * block_len:min((b + 1) * block_len, T)]
+        out[(l, h, b)] = oracle_mod.svd(Xb)
+    return out
+
+
+def _check_sigma(s_gpu, s_ref):
+    s1 = s_ref[0]
+    assert np.all(np.abs(s_gpu - s_ref) <= SIG_TOL * s1), np.abs(s_gpu - s_ref).max() / s1
+    big = s_ref >= 0.1 * s1
+    assert np.all(np.abs(s_gpu[big] - s_ref[big]) <= SIG_TOL * s_ref[big])
+
+
+def _decode_ref(oracle_mod, U_K, U_V, l, h, nb, q, blocks, positions, base):
+    """Oracle decode of one query vector on unpacked factors (fp64)."""
+    def fa(U):
+        return lambda b: U["A"][(l * U["H"] + h) * nb + b]
+
+    def fb(U):
+        return lambda b: U["B"][(l * U["H"] + h) * nb + b]
+    return oracle_mod.decode_one(fa(U_K), fb(U_K), fa(U_V), fb(U_V), q, blocks, positions, base)
+
+
+def _rel_inf(a, b):
+    return np.abs(a - b).max() / np.abs(b).max()
+
+
+def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None):
+    """Run milo_compress, check sigma/eps/ranks/offsets/reconstruction; return unpacked factors."""
+    Kd, Vd = K.cuda(), V.cuda()
+    f = milo.milo_compress(Kd, Vd, block_len, params)
+    st = milo.milo_get_status()
+    assert st == milo.MILO_OK, milo.status_string(st)
+    L, H, T, d = K.shape
+    nb = math.ceil(T / block_len)
+    Kn = K.double().numpy() if K.dtype != torch.bfloat16 else K.float().double().numpy()
+    Vn = V.double().numpy() if V.dtype != torch.bfloat16 else V.float().double().numpy()
+    R = oracle_mod.budget(L, H, T, block_len, d, params.budget_frac, params.budget_abs)
+    if sample_blocks is None:
+        sample_blocks = [(l, h, b) for l in range(L) for h in range(H) for b in range(nb)]
+    U = []
+    for kind, X in enumerate((Kn, Vn)):
+        u = A.unpack(f, kind)
+        u["H"] = H
+        U.append(u)
+        assert u["R"] == R and int(u["ranks"].sum()) == R
+        # eps: eps_rel * max_b sigma_{b,1} of the GPU's sigma, per (layer, head)
+        s1 = u["sigma"][:, 0].reshape(L * H, nb).astype(np.float64).max(axis=1)
+        if params.eps_scope == 1:
+            s1 = np.full_like(s1, s1.max())
+        assert np.array_equal(u["eps"], params.eps_rel * s1)
+        # ranks: bit-exact against the oracle allocator on the same sigma and eps
+        r_ref = oracle_mod.allocate(u["sigma"].astype(np.float64).reshape(L, H, nb, d), u["eps"].reshape(L, H),
+                                    T, block_len, R, params.r_min, params.r_max)
+        assert np.array_equal(u["ranks"], r_ref.reshape(-1))
+        # offsets: exclusive scan of r_b (ldT_b + d)
+        lens = oracle_mod.block_lengths(T, block_len) * (L * H)
+        sizes = np.array([r * ((tb + 15) // 16 * 16 + d) for r, tb in zip(u["ranks"], lens)], dtype=np.int64)
+        assert np.array_equal(u["offsets"], np.concatenate([[0], np.cumsum(sizes)]))
+        # sigma and reconstruction against the oracle SVD on sampled blocks
+        ref = _oracle_block_svds(oracle_mod, X, block_len, sample_blocks)
+        for (l, h, b), (s_ref, _, _, _) in ref.items():
+            blk = (l * H + h) * nb + b
+            _check_sigma(u["sigma"][blk].astype(np.float64), s_ref)
+            rb = int(u["ranks"][blk])
+            Xb = X[l, h, b * block_len:min((b + 1) * block_len, T)]
+            Xh = u["A"][blk] @ u["B"][blk] if rb else np.zeros_like(Xb)
+            err = np.sum((Xb - Xh) ** 2)
+            tail = np.sum(s_ref[rb:] ** 2)
+            if params.factor_dtype == milo.MILO_F32:
+                # plus fp32 rounding slack of the product A B itself (1e-10 ||X||^2)
+                slack = 1e-10 * np.sum(Xb ** 2)
+                assert abs(err - tail) <= RECON_TOL * tail + slack, (kind, l, h, b, err, tail)
+    return f, U
+
+
+def test_toy_fp32_end_to_end(oracle_mod):
+    w = synth.WORKLOADS["toy"]
+    K, V = synth.workload_cache(w)
+    p = milo.default_params(factor_dtype="f32", budget_frac=0.5)
+    f, U = _compress_and_check(oracle_mod, K, V, w.block_len, p)
+    q, sel, pos = synth.decode_inputs(w)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=w.rope_base)
+    assert milo.milo_get_status() == milo.MILO_OK
+    out = out.cpu().numpy()
+    for l in range(w.L):
+        for s in range(w.sessions):
+            for hq in range(w.Hq):
+                h = hq // w.G
+                ref = _decode_ref(oracle_mod, U[0], U[1], l, h, w.n_b, q[l, s, hq].double().numpy(),
+                                  sel[s].tolist(), pos[s].tolist(), w.rope_base)
+                assert _rel_inf(out[l, s, hq], ref) <= DEC_TOL
+
+
+def test_qwen3b_one_layer_bf16(oracle_mod):
+    w = synth.WORKLOADS["qwen3b-1layer"]
+    K, V = synth.workload_cache(w)
+    p = milo.default_params(factor_dtype="bf16", budget_frac=0.5)
+    f, U = _compress_and_check(oracle_mod, K, V, w.block_len, p,
+                               sample_blocks=[(0, 0, 0), (0, 1, 3), (0, 1, 7), (0, 0, 5)])
+    q, sel, pos = synth.decode_inputs(w)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=w.rope_base).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    # oracle's own fp64 compression of the same bf16 cache
+    own = oracle_mod.compress(K.float().double().numpy(), V.float().double().numpy(), w.block_len, 0.5)
+    for hq in range(w.Hq):
+        h = hq // w.G
+        qv = q[0, 0, hq].double().numpy()
+        same = _decode_ref(oracle_mod, U[0], U[1], 0, h, w.n_b, qv, sel[0].tolist(), pos[0].tolist(), w.rope_base)
+        assert _rel_inf(out[0, 0, hq], same) <= DEC_TOL
+        ref = oracle_mod.decode_one(lambda b: own[0]["A"][0][h][b], lambda b: own[0]["B"][0][h][b],
+                                    lambda b: own[1]["A"][0][h][b], lambda b: own[1]["B"][0][h][b],
+                                    qv, sel[0].tolist(), pos[0].tolist(), w.rope_base)
+        assert _rel_inf(out[0, 0, hq], ref) <= DEC_TOL_BF16_OWN
+
+
+@pytest.mark.parametrize("T,block_len", [(1000, 256), (300, 64), (700, 160)])
+def test_ragged_and_short_blocks(oracle_mod, T, block_len):
+    K = synth.planted_cache(1, 2, T, 128, block_len, (3.0, 20.0), seed=T, out_dtype=torch.float32)
+    V = synth.planted_cache(1, 2, T, 128, block_len, (6.0, 40.0), seed=T + 1, out_dtype=torch.float32)
+    p = milo.default_params(factor_dtype="f32", budget_frac=0.4)
+    f, U = _compress_and_check(oracle_mod, K, V, block_len, p)
+    nb = math.ceil(T / block_len)
+    q = torch.randn(1, 2, 4, 128, generator=torch.Generator().manual_seed(T))
+    sel = torch.tensor([list(range(nb)), list(range(nb - 1, -1, -1))], dtype=torch.int32)
+    pos = torch.tensor([[b * block_len for b in range(nb)], [5000 + 7 * b for b in range(nb)]], dtype=torch.int32)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=1e4).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    for s in range(2):
+        for hq in range(4):
+            ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // 2, nb, q[0, s, hq].double().numpy(),
+                              sel[s].tolist(), pos[s].tolist(), 1e4)
+            assert _rel_inf(out[0, s, hq], ref) <= DEC_TOL
+
+
+@pytest.mark.parametrize("frac,r_min,r_max,scope", [(0.0, 0, 0, 0), (1.0, 0, 0, 0), (0.3, 2, 40, 1),
+                                                    (0.25, 0, 16, 0)])
+def test_budget_edges_and_bounds(oracle_mod, frac, r_min, r_max, scope):
+    K = synth.planted_cache(2, 1, 768, 128, 256, (2.0, 30.0), seed=7, out_dtype=torch.float32)
+    V = synth.planted_cache(2, 1, 768, 128, 256, (8.0, 60.0), seed=8, out_dtype=torch.float32)
+    p = milo.default_params(factor_dtype="f32", budget_frac=frac, r_min=r_min, r_max=r_max, eps_scope=scope)
+    f, U = _compress_and_check(oracle_mod, K, V, 256, p, sample_blocks=[(0, 0, 0), (1, 0, 2)])
+    if frac == 1.0:
+        assert np.all(U[0]["ranks"] == 128)
+    if frac == 0.0:
+        assert np.all(U[0]["ranks"] == 0)
+        q = torch.randn(2, 1, 1, 128)
+        sel = torch.tensor([[0, 2]], dtype=torch.int32)
+        out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), None, rope_base=1e6)
+        assert torch.all(out == 0)
+
+
+def test_int8_codes_and_decode(oracle_mod):
+    K = synth.planted_cache(1, 2, 1024, 128, 256, (4.0, 32.0), seed=31, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(1, 2, 1024, 128, 256, (16.0, 64.0), seed=32, out_dtype=torch.bfloat16)
+    f32 = milo.milo_compress(K.cuda(), V.cuda(), 256, milo.default_params(factor_dtype="f32"))
+    f8 = milo.milo_compress(K.cuda(), V.cuda(), 256, milo.default_params(factor_dtype="int8"))
+    assert milo.milo_get_status() == milo.MILO_OK
+    for kind in range(2):
+        u32, u8 = A.unpack(f32, kind), A.unpack(f8, kind)
+        assert np.array_equal(u32["ranks"], u8["ranks"])
+        for blk in range(u8["nblk"]):
+            r = int(u8["ranks"][blk])
+            if r == 0:
+                continue
+            Qa, sa = oracle_mod.quant_int8_cols(u32["A"][blk].astype(np.float32))
+            assert np.array_equal(Qa.astype(np.float64), u8["Aq"][blk])
+            assert np.array_equal(sa, u8["sA"][blk, :r])
+            Qb, sb = oracle_mod.quant_int8_cols(u32["B"][blk].astype(np.float32))
+            assert np.array_equal(Qb.astype(np.float64), u8["Bq"][blk])
+            assert np.array_equal(sb, u8["sB"][blk])
+    U = [A.unpack(f8, 0), A.unpack(f8, 1)]
+    for u in U:
+        u["H"] = 2
+    q = torch.randn(1, 1, 8, 128, generator=torch.Generator().manual_seed(3))
+    sel = torch.tensor([[0, 1, 3]], dtype=torch.int32)
+    out = milo.milo_decode_attn(f8, q.cuda(), sel.cuda(), None, rope_base=1e6).cpu().numpy()
+    for hq in range(8):
+        ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // 4, 4, q[0, 0, hq].double().numpy(), [0, 1, 3],
+                          [0, 256, 768], 1e6)
+        assert _rel_inf(out[0, 0, hq], ref) <= DEC_TOL
+
+
+@pytest.mark.parametrize("n_groups,n_b,T,bl", [(1, 8, 2048, 256), (3, 5, 1100, 240), (72, 64, 32768, 512)])
+def test_allocate_bit_exact_with_ties(oracle_mod, n_groups, n_b, T, bl):
+    g = torch.Generator().manual_seed(n_groups * 100 + n_b)
+    sig = torch.rand(n_groups * n_b, 128, generator=g) * torch.rand(n_groups * n_b, 1, generator=g)
+    sig[::3] = sig[0]                           # exact ties across blocks
+    sig[:, 60:70] = sig[:, 60:61]               # ties inside blocks
+    sig = torch.sort(sig, dim=1, descending=True).values.contiguous()
+    eps = (torch.rand(n_groups, generator=g, dtype=torch.float64) * 0.05 + 1e-3)
+    caps = [min(min(bl, T - b * bl), 128) for b in range(n_b)] * n_groups
+    for frac in (0.0, 0.13, 0.5, 0.9, 1.0):
+        R = int(math.floor(frac * sum(caps)))
+        for r_min, r_max in ((0, 0), (3, 50)):
+            lo = sum(min(r_min, c) for c in caps)
+            capm = [min(c, r_max) if r_max else c for c in caps]
+            if R < lo or R > sum(capm):
+                continue
+            ranks = milo.milo_allocate(sig.cuda(), eps.cuda(), n_groups, n_b, T, bl, R, r_min, r_max).cpu().numpy()
+            assert milo.milo_get_status() == milo.MILO_OK
+            ref = oracle_mod.allocate(sig.double().numpy().reshape(n_groups, 1, n_b, 128),
+                                      eps.numpy().reshape(n_groups, 1), T, bl, R, r_min, r_max)
+            assert np.array_equal(ranks, ref.reshape(-1)), (frac, r_min, r_max)
+
+
+def test_status_word(oracle_mod):
+    # Jacobi sweep cap of 1: a warning status, results still written
+    K = synth.planted_cache(1, 1, 512, 128, 256, (4.0, 32.0), seed=1, out_dtype=torch.float32)
+    f = milo.milo_compress(K.cuda(), K.cuda(), 256, milo.default_params(max_sweeps=1, factor_dtype="f32"))
+    assert milo.milo_get_status() == milo.MILO_WARN_NOT_CONVERGED
+    assert milo.milo_get_status() == milo.MILO_OK          # cleared by the read
+    # unsorted sigma to milo_allocate: flagged on the device
+    sig = torch.rand(4, 128).cuda()
+    eps = torch.full((1,), 0.1, dtype=torch.float64).cuda()
+    milo.milo_allocate(sig, eps, 1, 4, 1024, 256, 100)
+    assert milo.milo_get_status() == milo.MILO_ERR_INVALID_ARG
+    # out-of-range block id in decode: bounds status, the slot contributes nothing
+    q = torch.randn(1, 1, 1, 128).cuda()
+    sel = torch.tensor([[0, 5]], dtype=torch.int32).cuda()
+    milo.milo_decode_attn(f, q, sel, None)
+    assert milo.milo_get_status() == milo.MILO_ERR_BOUNDS
+    del f
+
+
+def test_export_import_roundtrip(oracle_mod):
+    K = synth.planted_cache(1, 1, 512, 128, 256, (4.0, 32.0), seed=5, out_dtype=torch.bfloat16)
+    f = milo.milo_compress(K.cuda(), K.cuda(), 256, milo.default_params())
+    blob = milo.milo_factors_export(f)
+    arena2 = torch.zeros_like(f.arena)
+    g = milo.milo_factors_import(blob, arena2)
+    assert torch.equal(f.arena, arena2)
+    q = torch.randn(1, 1, 2, 128).cuda()
+    sel = torch.tensor([[1, 0]], dtype=torch.int32).cuda()
+    o1 = milo.milo_decode_attn(f, q, sel)
+    o2 = milo.milo_decode_attn(g, q, sel)
+    assert torch.equal(o1, o2)
