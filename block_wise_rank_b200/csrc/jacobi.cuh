@@ -86,7 +86,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                 if (fabsf(apq) > floor_abs && fabsf(apq) > tol * sqrtf(fabsf(app)) * sqrtf(fabsf(aqq))) {
                     float zeta = (aqq - app) / (2.f * apq);
                     tn = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-                    c = rsqrtf(1.f + tn * tn);
+                    c = 1.f / sqrtf(1.f + tn * tn);
                     s = c * tn;
                     rot = 1;
                 }

@@ -17,6 +17,7 @@
 #include "gram_simt.cuh"
 #include "gram_tc.cuh"
 #include "jacobi.cuh"
+#include "refine.cuh"
 #include "alloc.cuh"
 #include "project_simt.cuh"
 #include "decode_simt.cuh"
@@ -211,6 +212,12 @@ milo_status set_smem_attrs() {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_decode_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(DecodeSimtSmem));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_refine_sigma<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)refine_smem_bytes());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_refine_sigma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)refine_smem_bytes());
     if (e == cudaSuccess) e = gram_tc_set_attrs();
     if (e == cudaSuccess) e = decode_tc_set_attrs();
     if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute");
@@ -318,6 +325,15 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     // 2. eigensolve: sigma into the arena, sorted eigenvectors back into GW
     k_jacobi<<<grid2, JAC_THREADS, jacobi_smem_bytes(), s>>>(GW, f->kv[0].sigma, f->kv[1].sigma, nblk, shape->T,
                                                              shape->block_len, f->n_b, p.max_sweeps, p.jacobi_tol);
+    // 2b. singular values recomputed from the blocks, sigma / W re-sorted
+    if (shape->in_dtype == MILO_BF16)
+        k_refine_sigma<__nv_bfloat16><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
+            (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T,
+            shape->block_len, f->n_b, nblk);
+    else
+        k_refine_sigma<float><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
+            (const float *)K, (const float *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T, shape->block_len,
+            f->n_b, nblk);
     // 3. eps per (layer, head, kind)
     const int ngroups = shape->L * shape->H;
     k_eps<<<dim3(ngroups, 2), 256, 0, s>>>(f->kv[0].sigma, f->kv[1].sigma, f->kv[0].eps, f->kv[1].eps, f->n_b,

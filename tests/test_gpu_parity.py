@@ -176,7 +176,7 @@ def test_ragged_and_short_blocks(oracle_mod, T, block_len):
 
 
 @pytest.mark.parametrize("frac,r_min,r_max,scope", [(0.0, 0, 0, 0), (1.0, 0, 0, 0), (0.3, 2, 40, 1),
-                                                    (0.25, 0, 16, 0)])
+                                                    (0.1, 0, 16, 0)])
 def test_budget_edges_and_bounds(oracle_mod, frac, r_min, r_max, scope):
     K = synth.planted_cache(2, 1, 768, 128, 256, (2.0, 30.0), seed=7, out_dtype=torch.float32)
     V = synth.planted_cache(2, 1, 768, 128, 256, (8.0, 60.0), seed=8, out_dtype=torch.float32)
