@@ -74,7 +74,6 @@ struct SelArgs {
 struct SelShape {
     int n_b, T, block_len, r_min, r_max;
     int64_t n_blk;
-    int ld_pad;              // token stride rounding of the packed A (16)
 };
 
 // key bits of component k of block blk ((sigma/eps)^2 as a double, 0 if eps <= 0)
@@ -189,7 +188,8 @@ __global__ void k_sel_count(SelArgs a0, SelArgs a1, SelShape sh) {
 }
 
 // Single CTA per kind: ties handed out in block order, ranks, and the
-// packed-arena offsets (exclusive scan of r_b (ldT_b + d)).
+// packed-arena offsets (exclusive scan of the padded block sizes
+// round_up(r_b, 8) * (128 * ceil(T_b / 128) + d)).
 __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelShape sh) {
     const SelArgs &a = blockIdx.x == 0 ? a0 : a1;
     const int tid = threadIdx.x, nt = blockDim.x;
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
         const int r = k0 + a.gt[i] + (int)take;
         a.ranks[i] = r;
         const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
-        elems += (long long)r * (round_up(tb, sh.ld_pad) + D);
+        elems += block_elems(r, tb);
     }
     if (a.offsets == nullptr) return;
     sB[tid] = elems;
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
     for (int64_t i = lo; i < hi; ++i) {
         a.offsets[i] = off;
         const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
-        off += (long long)a.ranks[i] * (round_up(tb, sh.ld_pad) + D);
+        off += block_elems(a.ranks[i], tb);
     }
     if (hi == n && lo < hi) a.offsets[n] = off;
     if (n == 0 && tid == 0) a.offsets[0] = 0;

@@ -58,6 +58,30 @@ __host__ __device__ __forceinline__ int dtype_bytes(int dtype) {
     return dtype == MILO_F32 ? 4 : (dtype == MILO_BF16 ? 2 : 1);
 }
 
+// Packed factor layout of one block (element offsets from the block start).
+// Ranks are padded to R8 = round_up(r_b, 8) with zero rows and tokens to
+// whole tiles of FTILE = 128 with zero columns.  Tile tau of A_b^T holds
+// tokens [128 tau, 128 tau + 128) as [k/8][u/8][k%8][u%8]; B_b follows the
+// tiles as [k/8][j/8][k%8][j%8].  This is the tensor cores' canonical
+// no-swizzle operand layout (8 x 8 core matrices, 16 bytes per bf16 row),
+// so one contiguous copy lands a tile ready for the MMA.
+constexpr int FTILE = 128;
+
+__host__ __device__ __forceinline__ int rank_pad(int r) { return (r + 7) & ~7; }
+__host__ __device__ __forceinline__ int token_tiles(int Tb) { return (Tb + FTILE - 1) / FTILE; }
+__host__ __device__ __forceinline__ int64_t block_elems(int r, int Tb) {
+    return (int64_t)rank_pad(r) * (token_tiles(Tb) * FTILE + D);
+}
+// A_b[t][k] (token t, rank k); R8 = rank_pad(r_b)
+__host__ __device__ __forceinline__ int64_t a_index(int R8, int t, int k) {
+    const int tau = t / FTILE, u = t % FTILE;
+    return (int64_t)tau * R8 * FTILE + (k >> 3) * (8 * FTILE) + (u >> 3) * 64 + (k & 7) * 8 + (u & 7);
+}
+// B_b[k][j] (rank k, channel j)
+__host__ __device__ __forceinline__ int64_t b_index(int R8, int n_tiles, int k, int j) {
+    return (int64_t)n_tiles * R8 * FTILE + (k >> 3) * (8 * D) + (j >> 3) * 64 + (k & 7) * 8 + (j & 7);
+}
+
 // One kind's section of the factor arena (device pointers).
 struct KindView {
     int32_t *ranks;

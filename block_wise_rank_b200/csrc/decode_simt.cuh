@@ -95,13 +95,14 @@ struct DecodeSimtSmem {
     int qslot[DS_QC], qhead[DS_QC];
 };
 
-__device__ __forceinline__ float factor_a(const KindView &kv, int dt, int64_t blk, int64_t base, int k, int ldT, int t) {
-    float v = load_elem(kv.data, base + (int64_t)k * ldT + t, dt);
+__device__ __forceinline__ float factor_a(const KindView &kv, int dt, int64_t blk, int64_t base, int R8, int k, int t) {
+    float v = load_elem(kv.data, base + a_index(R8, t, k), dt);
     if (dt == MILO_INT8) v *= kv.scaleA[blk * D + k];
     return v;
 }
-__device__ __forceinline__ float factor_b(const KindView &kv, int dt, int64_t blk, int64_t base, int k, int j) {
-    float v = load_elem(kv.data, base + (int64_t)k * D + j, dt);
+__device__ __forceinline__ float factor_b(const KindView &kv, int dt, int64_t blk, int64_t base, int R8, int nt, int k,
+                                          int j) {
+    float v = load_elem(kv.data, base + b_index(R8, nt, k, j), dt);
     if (dt == MILO_INT8) v *= kv.scaleB[blk * D + j];
     return v;
 }
@@ -119,9 +120,9 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
     const KindView &K = a.kv[0], &V = a.kv[1];
     const int rK = K.ranks[blk], rV = V.ranks[blk];
     const int Tb = block_tokens(a.T, a.block_len, b);
-    const int ldT = (int)round_up(Tb, 16);
+    const int nt = token_tiles(Tb);
+    const int R8K = rank_pad(rK), R8V = rank_pad(rV);
     const int64_t baseK = K.offsets[blk], baseV = V.offsets[blk];
-    const int64_t bK = baseK + (int64_t)rK * ldT, bV = baseV + (int64_t)rV * ldT;
     const float scale = rsqrtf((float)D);
     const int nq_total = ns * a.G;
 
@@ -150,8 +151,8 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
             const int tt = min(DS_TT, Tb - t0);
             for (int e = tid; e < D * DS_TT; e += 256) {
                 const int k = e / DS_TT, t = e % DS_TT;
-                sm.aK[k][t] = (k < rK && t < tt) ? factor_a(K, dt, blk, baseK, k, ldT, t0 + t) : 0.f;
-                sm.aV[k][t] = (k < rV && t < tt) ? factor_a(V, dt, blk, baseV, k, ldT, t0 + t) : 0.f;
+                sm.aK[k][t] = (k < rK && t < tt) ? factor_a(K, dt, blk, baseK, R8K, k, t0 + t) : 0.f;
+                sm.aV[k][t] = (k < rV && t < tt) ? factor_a(V, dt, blk, baseV, R8V, k, t0 + t) : 0.f;
             }
             __syncthreads();
             {   // rebuild pre-RoPE keys: kt[t][j] = sum_k aK[k][t] B_K[k][j]
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
 #pragma unroll
                 for (int u = 0; u < DS_TT / 2; ++u) acc[u] = 0.f;
                 for (int k = 0; k < rK; ++k) {
-                    const float bk = factor_b(K, dt, blk, bK, k, j);
+                    const float bk = factor_b(K, dt, blk, baseK, R8K, nt, k, j);
 #pragma unroll
                     for (int u = 0; u < DS_TT / 2; ++u) acc[u] = fmaf(sm.aK[k][th * (DS_TT / 2) + u], bk, acc[u]);
                 }
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
             const int qi = e / D, j = e % D;
             if (qi >= nq) continue;
             float acc = 0.f;
-            for (int k = 0; k < rV; ++k) acc = fmaf(sm.oA[qi][k], factor_b(V, dt, blk, bV, k, j), acc);
+            for (int k = 0; k < rV; ++k) acc = fmaf(sm.oA[qi][k], factor_b(V, dt, blk, baseV, R8V, nt, k, j), acc);
             const int slot = sm.qslot[qi], hq = sm.qhead[qi];
             const int s = slot / a.n_sel, jj = slot % a.n_sel;
             const int64_t pidx = (((int64_t)l * a.S + s) * a.Hq + hq) * a.n_sel + jj;

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -38,7 +39,6 @@ struct milo_factors {
 
 namespace {
 
-constexpr int kLdPad = 16;     // token stride rounding of packed A^T rows
 constexpr size_t kAlign = 256;
 
 bool g_log = false;
@@ -117,7 +117,9 @@ SectionLayout section_layout(const milo_cache_shape *s, const milo_compress_para
         at = align_up(at + sizeof(float) * nblk * D);
     }
     o.data = at;
-    at = align_up(at + (size_t)R * (size_t)(round_up(s->block_len, kLdPad) + D) * dtype_bytes(p->factor_dtype));
+    // sum_b round_up(r_b, 8) (128 ceil(T_b/128) + d) <= (R + 7 N_blk) (128 ceil(block_len/128) + d)
+    at = align_up(at + (size_t)(R + 7 * nblk) * (size_t)(round_up(s->block_len, FTILE) + D) *
+                           dtype_bytes(p->factor_dtype));
     o.bytes = at;
     return o;
 }
@@ -311,9 +313,9 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
 
     // 1. Gram matrices of every block of K and V
     const dim3 grid2((unsigned)nblk, 2);
-    if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->block_len)) {
+    if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->T, shape->block_len)) {
         st = launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H, shape->T,
-                            shape->block_len, f->n_b, GW, nblk, s);
+                            shape->block_len, f->n_b, GW, nblk, sm_count(), s);
         if (st != MILO_OK) { delete f; return st; }
     } else if (shape->in_dtype == MILO_BF16) {
         k_gram_simt<__nv_bfloat16><<<grid2, 256, 0, s>>>((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
@@ -342,7 +344,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     // 4. global top-R selection, ranks and packed offsets
     int64_t caps, floors;
     cap_sums(shape, p.r_min, p.r_max, caps, floors);
-    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk, kLdPad};
+    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk};
     SelArgs a[2];
     for (int k = 0; k < 2; ++k) {
         a[k].sigma = f->kv[k].sigma;
@@ -403,7 +405,7 @@ milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_group
     cap_sums(&shp, r_min, r_max, caps, floors);
     if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
     AllocScratch as = alloc_scratch(workspace, nblk);
-    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, kLdPad};
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk};
     SelArgs a{};
     a.sigma = sigma;
     a.eps = eps;

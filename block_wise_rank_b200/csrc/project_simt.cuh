@@ -4,7 +4,7 @@
 // cache in compressed low-rank form per block" (evolve.pub review of MILO,
 // Summary and FAQ "What is MILO"): A_b = X_b W_{:,1:r_b} = U_r Sigma_r
 // (T_b x r_b) and B_b = W_{:,1:r_b}^T (r_b x d), written into the packed
-// arena (A_b^T rank rows of ldT_b tokens, then B_b).  INT8 composition
+// arena in the tiled layout of common.cuh (A_b^T tiles, then B_b).  INT8 composition
 // (same page, Summary: combined with INT8 quantisation): symmetric per-column
 // absmax codes, scale = absmax / 127, round half to even, clamp to +-127.
 #pragma once
@@ -31,8 +31,9 @@ struct ProjArgs {
     int64_t n_blk;
 };
 
-// grid (n_blk, D/32 rank chunks, 2 kinds), 256 threads.  Writes the columns
-// k0 .. k0+31 of A_b (as rows of A_b^T) and, for INT8, their scales.
+// grid (n_blk, D/32 rank chunks, 2 kinds), 256 threads.  Writes the rank
+// rows k0 .. k0+31 of A_b^T (rows r_b .. R8-1 and tokens past T_b as zeros,
+// in the tiled layout of common.cuh) and, for INT8, their scales.
 template <typename TI>
 __global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
     __shared__ float Wc[D][33];
@@ -41,11 +42,13 @@ __global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
     const int k0 = blockIdx.y * 32;
     const KindView &kv = pa.kv[kind];
     const int r = kv.ranks[blk];
-    if (k0 >= r) return;
-    const int kc = min(32, r - k0);
+    const int R8 = rank_pad(r);
+    if (k0 >= R8) return;
+    const int kw = min(32, R8 - k0);          // rows written (incl. zero padding)
+    const int kc = max(0, min(32, r - k0));   // rows with data
     const int b = blk % pa.n_b, lh = blk / pa.n_b;
     const int Tb = block_tokens(pa.T, pa.block_len, b);
-    const int ldT = (int)round_up(Tb, 16);
+    const int ldT = token_tiles(Tb) * FTILE;
     const TI *Xb = (const TI *)pa.X[kind] + ((int64_t)lh * pa.T + (int64_t)b * pa.block_len) * D;
     const float *Wb = pa.W[kind] + (int64_t)blk * D * D;
     for (int e = threadIdx.x; e < D * 32; e += 256) {
@@ -74,41 +77,46 @@ __global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
                 for (int c = 0; c < 32; ++c)
                     if (c < kc) atomicMax((int *)&amax[c], __float_as_int(fabsf(acc[c])));
             } else {
-                for (int c = 0; c < kc; ++c) {
-                    const int64_t o = base + (int64_t)(k0 + c) * ldT + t;
+                for (int c = 0; c < kw; ++c) {
+                    const int64_t o = base + a_index(R8, t, k0 + c);
                     if (pa.out_dtype == MILO_F32) ((float *)kv.data)[o] = acc[c];
                     else if (pa.out_dtype == MILO_BF16) ((__nv_bfloat16 *)kv.data)[o] = __float2bfloat16_rn(acc[c]);
-                    else ((int8_t *)kv.data)[o] = quant_i8(acc[c], __fdiv_rn(amax[c], 127.f));
+                    else ((int8_t *)kv.data)[o] = c < kc ? quant_i8(acc[c], __fdiv_rn(amax[c], 127.f)) : (int8_t)0;
                 }
             }
         }
         __syncthreads();
-        if (pass == 0 && threadIdx.x < kc)
-            kv.scaleA[(int64_t)blk * D + k0 + threadIdx.x] = __fdiv_rn(amax[threadIdx.x], 127.f);
+        if (pass == 0 && threadIdx.x < 32 && k0 + threadIdx.x < D)
+            kv.scaleA[(int64_t)blk * D + k0 + threadIdx.x] =
+                threadIdx.x < kc ? __fdiv_rn(amax[threadIdx.x], 127.f) : 0.f;
         __syncthreads();
     }
 }
 
 // grid (n_blk, 2 kinds), 128 threads: thread j writes column j of B_b
-// (B_b[k][j] = W[j][k], k < r_b) and, for INT8, its scale.
+// (B_b[k][j] = W[j][k], k < r_b; zero rows up to R8) and, for INT8, its scale.
 __global__ void __launch_bounds__(128) k_project_b(ProjArgs pa) {
     const int blk = blockIdx.x, kind = blockIdx.y, j = threadIdx.x;
     const KindView &kv = pa.kv[kind];
     const int r = kv.ranks[blk];
+    const int R8 = rank_pad(r);
     const int b = blk % pa.n_b;
-    const int Tb = block_tokens(pa.T, pa.block_len, b);
-    const int64_t base = kv.offsets[blk] + (int64_t)r * round_up(Tb, 16);
+    const int nt = token_tiles(block_tokens(pa.T, pa.block_len, b));
+    const int64_t base = kv.offsets[blk];
     const float *Wb = pa.W[kind] + (int64_t)blk * D * D + (int64_t)j * D;
+    float s = 0.f;
     if (pa.out_dtype == MILO_INT8) {
         float m = 0.f;
         for (int k = 0; k < r; ++k) m = fmaxf(m, fabsf(Wb[k]));
-        const float s = __fdiv_rn(m, 127.f);
+        s = __fdiv_rn(m, 127.f);
         kv.scaleB[(int64_t)blk * D + j] = s;
-        for (int k = 0; k < r; ++k) ((int8_t *)kv.data)[base + (int64_t)k * D + j] = quant_i8(Wb[k], s);
-    } else if (pa.out_dtype == MILO_BF16) {
-        for (int k = 0; k < r; ++k) ((__nv_bfloat16 *)kv.data)[base + (int64_t)k * D + j] = __float2bfloat16_rn(Wb[k]);
-    } else {
-        for (int k = 0; k < r; ++k) ((float *)kv.data)[base + (int64_t)k * D + j] = Wb[k];
+    }
+    for (int k = 0; k < R8; ++k) {
+        const float w = k < r ? Wb[k] : 0.f;
+        const int64_t o = base + b_index(R8, nt, k, j);
+        if (pa.out_dtype == MILO_INT8) ((int8_t *)kv.data)[o] = quant_i8(w, s);
+        else if (pa.out_dtype == MILO_BF16) ((__nv_bfloat16 *)kv.data)[o] = __float2bfloat16_rn(w);
+        else ((float *)kv.data)[o] = w;
     }
 }
 

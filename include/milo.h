@@ -93,18 +93,25 @@ typedef struct milo_factors milo_factors;
 /*
  * Factor arena layout (device, caller-owned, one section per kind: K then V,
  * each section start 256-byte aligned; N_blk = L*H*n_b, n_b = ceil(T /
- * block_len), ldT = round_up(block_len, 16), ldT_b = round_up(T_b, 16)):
+ * block_len)):
  *   int32  ranks  [N_blk]
  *   int64  offsets[N_blk + 1]   element offset of block b in data
  *   float  sigma  [N_blk][d]    singular values, descending
  *   double eps    [L*H]
  *   float  scaleA [N_blk][d]    INT8 only: scale of column k of A_b
  *   float  scaleB [N_blk][d]    INT8 only: scale of column j of B_b
- *   elem   data   [R*(ldT + d)] elem = factor dtype
- * Block b at data + offsets[b]: A_b^T as r_b rows of ldT_b elements (token
- * t of rank row k at k*ldT_b + t; tokens past T_b are zero), followed by
- * B_b as r_b rows of d elements.  A_b = U_r Sigma_r (T_b x r_b) and
- * B_b = V_r^T (r_b x d), so X_b ~ A_b B_b.  Blocks are ordered (l, h, b).
+ *   elem   data   [...]         elem = factor dtype
+ * A_b = U_r Sigma_r (T_b x r_b) and B_b = V_r^T (r_b x d), so X_b ~ A_b B_b.
+ * Block b occupies R8 * (128 * nt + d) elements at data + offsets[b], with
+ * R8 = round_up(r_b, 8) and nt = ceil(T_b / 128) token tiles; blocks are
+ * ordered (l, h, b).  Rank rows r_b .. R8-1 and tokens T_b .. 128*nt-1 are
+ * zero.  Inside a block, with t = 128*tau + u:
+ *   A_b[t][k] at  tau*R8*128 + (k/8)*1024 + (u/8)*64 + (k%8)*8 + (u%8)
+ *   B_b[k][j] at  nt*R8*128  + (k/8)*1024 + (j/8)*64 + (k%8)*8 + (j%8)
+ * i.e. 8 x 8 element tiles, the tensor cores' canonical no-swizzle operand
+ * layout, so that each 128-token tile of A_b and the whole of B_b are single
+ * contiguous copies.  The data section holds at most
+ * (R + 7 N_blk) * (128 * ceil(block_len / 128) + d) elements.
  */
 
 /* ----------------------------------------------------------------- sizes */

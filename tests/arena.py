@@ -22,6 +22,46 @@ def arena_tensor(f: milo.Factors, ptr: int, nbytes: int) -> torch.Tensor:
     return f.arena[off:off + nbytes]
 
 
+def padded_rank(r: int) -> int:
+    return (r + 7) // 8 * 8
+
+
+def tiles(tb: int) -> int:
+    return (tb + 127) // 128
+
+
+def untile(region, r, tb, d):
+    """One block's packed region -> (A^T [R8][128*nt], B [R8][d]).
+
+    Layout (include/milo.h): per 128-token tile [k/8][u/8][k%8][u%8], then B
+    as [k/8][j/8][k%8][j%8].
+    """
+    R8, nt = padded_rank(r), tiles(tb)
+    assert region.size == R8 * (128 * nt + d)
+    At = np.zeros((R8, 128 * nt))
+    if R8:
+        for tau in range(nt):
+            tile = region[tau * R8 * 128:(tau + 1) * R8 * 128].reshape(R8 // 8, 16, 8, 8)
+            # tile[kg][ug][k8][u8] -> A^T[kg*8 + k8][tau*128 + ug*8 + u8]
+            At[:, tau * 128:(tau + 1) * 128] = tile.transpose(0, 2, 1, 3).reshape(R8, 128)
+        bt = region[nt * R8 * 128:].reshape(R8 // 8, d // 8, 8, 8)
+        Bm = bt.transpose(0, 2, 1, 3).reshape(R8, d)
+    else:
+        Bm = np.zeros((0, d))
+    return At, Bm
+
+
+def tile(At, Bm, d):
+    """Inverse of untile: (A^T [R8][128*nt], B [R8][d]) -> flat region."""
+    R8, L = At.shape
+    nt = L // 128
+    parts = []
+    for tau in range(nt):
+        parts.append(At[:, tau * 128:(tau + 1) * 128].reshape(R8 // 8, 8, 16, 8).transpose(0, 2, 1, 3).reshape(-1))
+    parts.append(Bm.reshape(R8 // 8, 8, d // 8, 8).transpose(0, 2, 1, 3).reshape(-1))
+    return np.concatenate(parts) if parts else np.zeros(0)
+
+
 def unpack(f: milo.Factors, kind: int):
     """Per-kind host copy: ranks, offsets, sigma, eps, and factor lists.
 
@@ -56,21 +96,18 @@ def unpack(f: milo.Factors, kind: int):
     for blk in range(nblk):
         b = blk % nb
         tb = min(bl, T - b * bl)
-        ld = (tb + 15) // 16 * 16
         r = int(ranks[blk])
-        o = int(offs[blk])
-        At = data[o:o + r * ld].reshape(r, ld)
-        Bm = data[o + r * ld:o + r * ld + r * d].reshape(r, d)
-        pad = At[:, tb:]
-        Aq.append(At[:, :tb].T.copy())
-        Bq.append(Bm.copy())
+        At, Bm = untile(data[int(offs[blk]):int(offs[blk + 1])], r, tb, d)
+        Aq.append(At[:r, :tb].T.copy())
+        Bq.append(Bm[:r].copy())
         if dt == milo.MILO_INT8:
-            A.append(At[:, :tb].T * sA[blk, :r].astype(np.float64)[None, :])
-            B.append(Bm * sB[blk].astype(np.float64)[None, :])
+            A.append(At[:r, :tb].T * sA[blk, :r].astype(np.float64)[None, :])
+            B.append(Bm[:r] * sB[blk].astype(np.float64)[None, :])
         else:
-            A.append(At[:, :tb].T.copy())
-            B.append(Bm.copy())
-        assert np.all(pad == 0), "padding tokens of A^T must be zero"
+            A.append(At[:r, :tb].T.copy())
+            B.append(Bm[:r].copy())
+        assert np.all(At[r:] == 0) and np.all(At[:, tb:] == 0), "A padding must be zero"
+        assert np.all(Bm[r:] == 0), "B padding rows must be zero"
     return dict(ranks=ranks, offsets=offs, sigma=sigma, eps=eps, A=A, B=B, Aq=Aq, Bq=Bq, sA=sA, sB=sB, R=R,
                 nb=nb, nblk=nblk)
 
@@ -98,12 +135,13 @@ def pack(shape, params, A_lists, B_lists, sigma_lists=None, eps_lists=None, devi
         chunks = []
         for blk in range(nblk):
             tb, r = A[blk].shape
-            ld = (tb + 15) // 16 * 16
-            At = np.zeros((r, ld))
-            At[:, :tb] = A[blk].T
-            chunks.append(At.reshape(-1))
-            chunks.append(np.asarray(B[blk], dtype=np.float64).reshape(-1))
-            offs[blk + 1] = offs[blk] + r * (ld + d)
+            R8, nt = padded_rank(r), tiles(tb)
+            At = np.zeros((R8, 128 * nt))
+            At[:r, :tb] = A[blk].T
+            Bm = np.zeros((R8, d))
+            Bm[:r] = B[blk]
+            chunks.append(tile(At, Bm, d))
+            offs[blk + 1] = offs[blk] + R8 * (128 * nt + d)
         arena_tensor(f, p_r, 4 * nblk).copy_(torch.from_numpy(ranks).view(torch.uint8))
         arena_tensor(f, p_o, 8 * (nblk + 1)).copy_(torch.from_numpy(offs).view(torch.uint8))
         if sigma_lists is not None:

@@ -69,7 +69,7 @@ def test_arena_size_layout(L):
             sec = al(4 * nblk) + al(8 * (nblk + 1)) + al(4 * nblk * 128) + al(8 * Ln * H)
             if dt == milo.MILO_INT8:
                 sec += 2 * al(4 * nblk * 128)
-            sec += al(R * ((bl + 15) // 16 * 16 + 128) * es)
+            sec += al((R + 7 * nblk) * ((bl + 127) // 128 * 128 + 128) * es)
             assert milo.milo_factor_arena_size(s, p) == 2 * sec
 
 

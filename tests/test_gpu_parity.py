@@ -95,9 +95,10 @@ def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None)
         r_ref = oracle_mod.allocate(u["sigma"].astype(np.float64).reshape(L, H, nb, d), u["eps"].reshape(L, H),
                                     T, block_len, R, params.r_min, params.r_max)
         assert np.array_equal(u["ranks"], r_ref.reshape(-1))
-        # offsets: exclusive scan of r_b (ldT_b + d)
+        # offsets: exclusive scan of round_up(r_b, 8) (128 ceil(T_b / 128) + d)
         lens = oracle_mod.block_lengths(T, block_len) * (L * H)
-        sizes = np.array([r * ((tb + 15) // 16 * 16 + d) for r, tb in zip(u["ranks"], lens)], dtype=np.int64)
+        sizes = np.array([(r + 7) // 8 * 8 * ((tb + 127) // 128 * 128 + d) for r, tb in zip(u["ranks"], lens)],
+                         dtype=np.int64)
         assert np.array_equal(u["offsets"], np.concatenate([[0], np.cumsum(sizes)]))
         # sigma and reconstruction against the oracle SVD on sampled blocks
         ref = _oracle_block_svds(oracle_mod, X, block_len, sample_blocks)
@@ -277,3 +278,21 @@ def test_export_import_roundtrip(oracle_mod):
     o1 = milo.milo_decode_attn(f, q, sel)
     o2 = milo.milo_decode_attn(g, q, sel)
     assert torch.equal(o1, o2)
+
+
+def test_gram_tensor_core_path_matches_cuda_core_path(oracle_mod, monkeypatch):
+    """bf16 caches take the tcgen05 Gram; forcing the FP32 FFMA Gram must give
+    the same singular values to fp32 accumulation-order accuracy."""
+    K = synth.planted_cache(2, 2, 2048, 128, 512, (4.0, 32.0), seed=41, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(2, 2, 2048, 128, 512, (16.0, 64.0), seed=42, out_dtype=torch.bfloat16)
+    p = milo.default_params(factor_dtype="f32")
+    f_tc = milo.milo_compress(K.cuda(), V.cuda(), 512, p)
+    assert milo.milo_get_status() == milo.MILO_OK
+    monkeypatch.setenv("MILO_FORCE_SIMT", "1")
+    f_cc = milo.milo_compress(K.cuda(), V.cuda(), 512, p)
+    assert milo.milo_get_status() == milo.MILO_OK
+    for kind in range(2):
+        a, b = A.unpack(f_tc, kind), A.unpack(f_cc, kind)
+        s1 = a["sigma"][:, :1]
+        assert np.all(np.abs(a["sigma"] - b["sigma"]) <= 2e-6 * s1)
+        assert abs(int(a["ranks"].sum()) - int(b["ranks"].sum())) == 0
