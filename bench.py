@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--factor", default=None, choices=["bf16", "int8", "f32"])
     ap.add_argument("--decode-steps", type=int, default=0, help="decode steps per step (0: the workload's)")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="only the warm-up and timed steps (for ncu launch lists): no profiler, e2e or CPU legs")
     return ap.parse_args()
 
 
@@ -198,6 +200,11 @@ def run_ours(args, rank, world):
     st = milo.milo_get_status()
     if st not in (milo.MILO_OK, milo.MILO_WARN_NOT_CONVERGED):
         raise milo.MiloError(st, "warm-up")
+    if args.profile:
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        return dict(profile="done", status=milo.status_string(milo.milo_get_status()))
     launches_per_step = count_launches(step)
     ranks = read_ranks(f)
     dbytes = sum(decode_bytes(ranks, w, sel, factor, S, Hq) for (_, sel, _) in dec_inputs)
@@ -391,7 +398,7 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     res = run_ours(args, rank, world)
-    if world == 1 and rank == 0:
+    if world == 1 and rank == 0 and not args.profile:
         args.cpu_sample_s = min(args.cpu_sample_s, 20.0)
         res["cpu_baseline"] = cpu_baseline(args)
     if rank == 0:

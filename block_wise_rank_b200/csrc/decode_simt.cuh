@@ -64,11 +64,21 @@ __global__ void k_slot_count(const int32_t *__restrict__ sel, int n_slots, int n
     }
 }
 
-__global__ void k_slot_scan(int32_t *__restrict__ cnt, int32_t *__restrict__ start, int n_b) {
+// starts of each block id's slot list, and of its query passes (a pass is up
+// to `pass_q` queries = selecting slots times the GQA group)
+__global__ void k_slot_scan(int32_t *__restrict__ cnt, int32_t *__restrict__ start, int32_t *__restrict__ pstart,
+                            int n_b, int G, int pass_q) {
     if (threadIdx.x == 0 && blockIdx.x == 0) {
-        int acc = 0;
-        for (int b = 0; b < n_b; ++b) { start[b] = acc; acc += cnt[b]; cnt[b] = 0; }
+        int acc = 0, pacc = 0;
+        for (int b = 0; b < n_b; ++b) {
+            start[b] = acc;
+            pstart[b] = pacc;
+            acc += cnt[b];
+            pacc += (cnt[b] * G + pass_q - 1) / pass_q;
+            cnt[b] = 0;
+        }
         start[n_b] = acc;
+        pstart[n_b] = pacc;
     }
 }
 
@@ -221,14 +231,15 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
             const int slot = sm.qslot[qi], hq = sm.qhead[qi];
             const int s = slot / a.n_sel, jj = slot % a.n_sel;
             const int64_t pidx = (((int64_t)l * a.S + s) * a.Hq + hq) * a.n_sel + jj;
-            a.part_o[pidx * D + j] = acc;
+            a.part_o[pidx * D + j] = sm.l[qi] > 0.f ? acc / sm.l[qi] : 0.f;
             if (j == 0) a.part_ml[pidx] = make_float2(sm.m[qi], sm.l[qi]);
         }
         __syncthreads();
     }
 }
 
-// out[l][s][hq] = sum_j w_j o_j / sum_j w_j l_j, w_j = exp(m_j - max m).
+// out[l][s][hq] = sum_j w_j l_j o_j / sum_j w_j l_j, w_j = exp(m_j - max m),
+// with o_j the normalised output of slot j.
 // grid (L * S * Hq), 128 threads.  Slots with an out-of-range block id
 // contribute nothing.
 __global__ void __launch_bounds__(128) k_combine(DecodeArgs a) {
@@ -246,9 +257,9 @@ __global__ void __launch_bounds__(128) k_combine(DecodeArgs a) {
         const int bid = a.sel[(int64_t)s * a.n_sel + u];
         if (bid < 0 || bid >= a.n_b) continue;
         const float2 ml = a.part_ml[row * a.n_sel + u];
-        const float w = __expf(ml.x - M);
+        const float w = __expf(ml.x - M) * ml.y;
         num = fmaf(w, a.part_o[(row * a.n_sel + u) * D + j], num);
-        den = fmaf(w, ml.y, den);
+        den += w;
     }
     a.out[row * D + j] = den > 0.f ? num / den : 0.f;
 }

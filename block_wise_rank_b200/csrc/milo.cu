@@ -423,7 +423,7 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     const int64_t slots = (int64_t)S * n_sel;
     const int64_t rows = (int64_t)f->shape.L * S * Hq;
     size_t at = 0;
-    at = align_up(at + sizeof(int32_t) * (f->n_b + 1) * 2);            // counts / cursor, starts
+    at = align_up(at + sizeof(int32_t) * (f->n_b + 1) * 3);            // counts / cursor, starts, passes
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
     at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
@@ -450,7 +450,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     size_t at = 0;
     int32_t *cnt = (int32_t *)(w + at);
     int32_t *start = cnt + (n_b + 1);
-    at = align_up(at + sizeof(int32_t) * (n_b + 1) * 2);
+    int32_t *pstart = start + (n_b + 1);
+    at = align_up(at + sizeof(int32_t) * (n_b + 1) * 3);
     int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
     float2 *rope_q = (float2 *)(w + at);
     float2 *rope_t = rope_q + slots * HALF;
@@ -473,13 +474,13 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     if (e != cudaSuccess) return cuda_check(e, "memset");
     const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
-    k_slot_scan<<<1, 32, 0, s>>>(cnt, start, n_b);
+    k_slot_scan<<<1, 32, 0, s>>>(cnt, start, pstart, n_b, a.G, DT_NQ);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
     const int64_t rt = (slots + f->shape.block_len) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
         selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
     if (decode_tc_supported(a)) {
-        st = launch_decode_tc(a, s);
+        st = launch_decode_tc(a, pstart, sm_count(), s);
         if (st != MILO_OK) return st;
     } else {
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);

@@ -296,3 +296,36 @@ def test_gram_tensor_core_path_matches_cuda_core_path(oracle_mod, monkeypatch):
         s1 = a["sigma"][:, :1]
         assert np.all(np.abs(a["sigma"] - b["sigma"]) <= 2e-6 * s1)
         assert abs(int(a["ranks"].sum()) - int(b["ranks"].sum())) == 0
+
+
+@pytest.mark.parametrize("frac", [0.5, 1.0, 0.03])
+def test_decode_tensor_core_path(oracle_mod, monkeypatch, frac):
+    """bf16 factors take the tcgen05 decode kernel.  Cases: more queries per
+    block than one pass holds (40 sessions x GQA 4 > 128), a ragged last block
+    (1000 = 512 + 488 tokens), arbitrary start positions, full-rank blocks
+    (no spare rank row for the softmax denominator) and tiny ranks.  Checked
+    against the oracle on the same factors and against the CUDA-core path."""
+    L, H, G, T, bl, S = 2, 2, 4, 1000, 512, 40
+    K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=51, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=52, out_dtype=torch.bfloat16)
+    f = milo.milo_compress(K.cuda(), V.cuda(), bl, milo.default_params(factor_dtype="bf16", budget_frac=frac))
+    g = torch.Generator().manual_seed(int(frac * 100))
+    q = torch.randn(L, S, H * G, 128, generator=g)
+    sel = torch.stack([torch.randperm(2, generator=g) for _ in range(S)]).to(torch.int32)
+    pos = torch.randint(0, 120000, (S, 2), generator=g, dtype=torch.int32)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    monkeypatch.setenv("MILO_FORCE_SIMT", "1")
+    ref_cc = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=1e6).cpu().numpy()
+    monkeypatch.delenv("MILO_FORCE_SIMT")
+    for l in range(L):
+        for s in range(S):
+            for hq in range(H * G):
+                assert _rel_inf(out[l, s, hq], ref_cc[l, s, hq]) <= DEC_TOL, (l, s, hq)
+    U = [A.unpack(f, 0), A.unpack(f, 1)]
+    for u in U:
+        u["H"] = H
+    for (l, s, hq) in [(0, 0, 0), (1, 17, 5), (0, 39, 7), (1, 3, 2)]:
+        ref = _decode_ref(oracle_mod, U[0], U[1], l, hq // G, 2, q[l, s, hq].double().numpy(), sel[s].tolist(),
+                          pos[s].tolist(), 1e6)
+        assert _rel_inf(out[l, s, hq], ref) <= DEC_TOL
