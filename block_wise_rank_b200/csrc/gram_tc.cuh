@@ -189,14 +189,14 @@ inline cudaError_t gram_tc_set_attrs() {
     return cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gram_tc_smem_bytes());
 }
 
-inline milo_status launch_gram_tc(const __nv_bfloat16 *K, const __nv_bfloat16 *V, int LH, int T, int block_len,
+inline cudaError_t launch_gram_tc(const __nv_bfloat16 *K, const __nv_bfloat16 *V, int LH, int T, int block_len,
                                   int n_b, float *G, int64_t n_blk, int sms, cudaStream_t s) {
     CUtensorMap mk, mv;
     const uint64_t rows = (uint64_t)LH * T;
-    if (!make_cache_map(&mk, K, rows) || !make_cache_map(&mv, V, rows)) return MILO_ERR_CUDA;
+    if (!make_cache_map(&mk, K, rows) || !make_cache_map(&mv, V, rows)) return cudaErrorInvalidValue;
     const int grid = (int)std::min<int64_t>(2 * n_blk, (int64_t)sms);
     k_gram_tc<<<grid, GT_THREADS, gram_tc_smem_bytes(), s>>>(mk, mv, G, n_blk, n_b, T, block_len);
-    return cudaGetLastError() == cudaSuccess ? MILO_OK : MILO_ERR_CUDA;
+    return cudaGetLastError();
 }
 
 }  // namespace milo

@@ -314,8 +314,9 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     // 1. Gram matrices of every block of K and V
     const dim3 grid2((unsigned)nblk, 2);
     if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->T, shape->block_len)) {
-        st = launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H, shape->T,
-                            shape->block_len, f->n_b, GW, nblk, sm_count(), s);
+        st = cuda_check(launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H,
+                                       shape->T, shape->block_len, f->n_b, GW, nblk, sm_count(), s),
+                        "Gram (tensor cores) launch");
         if (st != MILO_OK) { delete f; return st; }
     } else if (shape->in_dtype == MILO_BF16) {
         k_gram_simt<__nv_bfloat16><<<grid2, 256, 0, s>>>((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
@@ -428,6 +429,8 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
     at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
+    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
+                                                            Hq / f->shape.H));  // tensor-core work items
     return at;
 }
 
@@ -457,7 +460,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     float2 *rope_t = rope_q + slots * HALF;
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);
     float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
-    float2 *part_ml = (float2 *)(w + at);
+    float2 *part_ml = (float2 *)(w + at); at = align_up(at + sizeof(float2) * rows * n_sel);
+    DtItem *items = (DtItem *)(w + at);
 
     DecodeArgs a{};
     a.kv[0] = f->kv[0];
@@ -480,7 +484,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
         selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
     if (decode_tc_supported(a)) {
-        st = launch_decode_tc(a, pstart, sm_count(), s);
+        st = cuda_check(launch_decode_tc(a, pstart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
     } else {
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
