@@ -155,3 +155,43 @@ def pack(shape, params, A_lists, B_lists, sigma_lists=None, eps_lists=None, devi
             arena_tensor(f, p_d, es * int(offs[-1])).copy_(flat.view(torch.uint8))
     torch.cuda.synchronize()
     return f
+
+
+def unpack_meta(f: milo.Factors, kind: int):
+    """ranks, offsets, sigma, eps of one kind (small arrays only)."""
+    (p_r, p_o, p_s, p_e, p_d, p_sa, p_sb), R = f.view(kind)
+    sh = f.shape
+    nb = math.ceil(sh.T / sh.block_len)
+    nblk = sh.L * sh.H * nb
+    ranks = arena_tensor(f, p_r, 4 * nblk).view(torch.int32).cpu().numpy().copy()
+    offs = arena_tensor(f, p_o, 8 * (nblk + 1)).view(torch.int64).cpu().numpy().copy()
+    sigma = arena_tensor(f, p_s, 4 * nblk * sh.d).view(torch.float32).cpu().numpy().reshape(nblk, sh.d).copy()
+    eps = arena_tensor(f, p_e, 8 * sh.L * sh.H).view(torch.float64).cpu().numpy().copy()
+    return dict(ranks=ranks, offsets=offs, sigma=sigma, eps=eps, R=R, nb=nb, nblk=nblk,
+                ptrs=(p_d, p_sa, p_sb))
+
+
+def unpack_blocks(f: milo.Factors, kind: int, blocks, meta=None):
+    """{blk: (A fp64 T_b x r, B fp64 r x d)} for the listed global block ids."""
+    meta = meta or unpack_meta(f, kind)
+    p_d, p_sa, p_sb = meta["ptrs"]
+    sh, dt = f.shape, f.params.factor_dtype
+    es = {milo.MILO_F32: 4, milo.MILO_BF16: 2, milo.MILO_INT8: 1}[dt]
+    tdt = {milo.MILO_F32: torch.float32, milo.MILO_BF16: torch.bfloat16, milo.MILO_INT8: torch.int8}[dt]
+    out = {}
+    for blk in blocks:
+        b = blk % meta["nb"]
+        tb = min(sh.block_len, sh.T - b * sh.block_len)
+        r = int(meta["ranks"][blk])
+        o0, o1 = int(meta["offsets"][blk]), int(meta["offsets"][blk + 1])
+        raw = arena_tensor(f, p_d + es * o0, es * (o1 - o0)) if o1 > o0 else None
+        region = raw.view(tdt).float().cpu().numpy().astype(np.float64) if raw is not None else np.zeros(0)
+        At, Bm = untile(region, r, tb, sh.d)
+        A, B = At[:r, :tb].T.copy(), Bm[:r].copy()
+        if dt == milo.MILO_INT8:
+            sA = arena_tensor(f, p_sa + 4 * blk * sh.d, 4 * sh.d).view(torch.float32).cpu().numpy().astype(np.float64)
+            sB = arena_tensor(f, p_sb + 4 * blk * sh.d, 4 * sh.d).view(torch.float32).cpu().numpy().astype(np.float64)
+            A = A * sA[None, :r]
+            B = B * sB[None, :]
+        out[blk] = (A, B)
+    return out
