@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
@@ -414,6 +415,88 @@ milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_group
     a.offsets = nullptr;
     a.st = as.st;
     a.gt = as.gt;
+    a.eq = as.eq;
+    a.need0 = R - floors * n_groups;
+    return launch_select(a, a, sh, 1, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Rank allocation without a caller workspace.
+//
+// Some callers may not allocate device memory at all: code running inside a
+// framework that owns every device byte through its own pool, or a plug-in
+// operator that is handed only its inputs and outputs.  They call
+// milo_allocate_noalloc, whose scratch (selection state and per-block counts
+// for up to MILO_NOALLOC_MAX_BLOCKS blocks) is this file-scope device array.
+// Every GPU that loads the library holds it (about 1 MiB) until exit.  In
+// host code the array's name is only a host-side stand-in, so its device
+// address is looked up per device with cudaGetSymbolAddress.
+namespace {
+constexpr int64_t kNoAllocBlocks = MILO_NOALLOC_MAX_BLOCKS;
+constexpr size_t kNoAllocBytes = (2 * sizeof(SelState) + kAlign - 1) / kAlign * kAlign +
+                                 2 * ((2 * sizeof(int32_t) * (size_t)kNoAllocBlocks + kAlign - 1) / kAlign * kAlign);
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up once
+// per device, with that device current); nullptr on failure.
+void *noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            cuda_check(e == cudaSuccess ? cudaErrorInvalidSymbol : e, "cudaGetSymbolAddress(noalloc scratch)");
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" {
+
+milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t n_groups, int32_t n_b, int32_t d,
+                                  int32_t T, int32_t block_len, int64_t R, int32_t r_min, int32_t r_max,
+                                  int32_t *ranks_out, milo_stream_t stream) {
+    if (d != D) return MILO_ERR_UNSUPPORTED;
+    if (!sigma || !eps || !ranks_out || n_groups <= 0 || n_b <= 0 || block_len <= 0 || T <= 0 || r_min < 0 ||
+        r_max < 0 || R < 0)
+        return MILO_ERR_INVALID_ARG;
+    if ((int64_t)(T + block_len - 1) / block_len != n_b) return MILO_ERR_INVALID_ARG;
+    if (!aligned(sigma, 4) || !aligned(eps, 8) || !aligned(ranks_out, 4)) return MILO_ERR_INVALID_ARG;
+    const int64_t nblk = (int64_t)n_groups * n_b;
+    if (nblk > kNoAllocBlocks) {
+        log_msg("milo_allocate_noalloc: n_groups * n_b exceeds MILO_NOALLOC_MAX_BLOCKS");
+        return MILO_ERR_WORKSPACE;
+    }
+    milo_cache_shape shp{1, 1, T, D, block_len, MILO_F32};
+    int64_t caps, floors;
+    cap_sums(&shp, r_min, r_max, caps, floors);
+    if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return MILO_ERR_CUDA;
+    // the scratch layout for kNoAllocBlocks also holds any smaller problem
+    AllocScratch as = alloc_scratch(scratch, kNoAllocBlocks);
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk};
+    SelArgs a{};
+    a.sigma = sigma;
+    a.eps = eps;
+    a.ranks = ranks_out;
+    a.offsets = nullptr;
+    a.st = as.st;      // reset by k_sel_init at the start of every call
+    a.gt = as.gt;      // written in full by k_sel_count before any read
     a.eq = as.eq;
     a.need0 = R - floors * n_groups;
     return launch_select(a, a, sh, 1, (cudaStream_t)stream);

@@ -52,7 +52,10 @@ EXPORTS = [
     "milo_compress", "milo_allocate_workspace_size", "milo_allocate", "milo_decode_workspace_size",
     "milo_decode_attn", "milo_factors_get", "milo_factors_wrap", "milo_factors_export",
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
+    "milo_allocate_noalloc",
 ]
+
+MILO_NOALLOC_MAX_BLOCKS = 65536
 
 
 def lib():
@@ -73,6 +76,8 @@ def lib():
         L.milo_allocate_workspace_size.argtypes = [I32, I32, I32]; L.milo_allocate_workspace_size.restype = SZ
         L.milo_allocate.argtypes = [P, P, I32, I32, I32, I32, I32, I64, I32, I32, P, P, SZ, P]
         L.milo_allocate.restype = ctypes.c_int
+        L.milo_allocate_noalloc.argtypes = [P, P, I32, I32, I32, I32, I32, I64, I32, I32, P, P]
+        L.milo_allocate_noalloc.restype = ctypes.c_int
         L.milo_decode_workspace_size.argtypes = [P, I32, I32, I32]; L.milo_decode_workspace_size.restype = SZ
         L.milo_decode_attn.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
         L.milo_decode_attn.restype = ctypes.c_int
@@ -224,6 +229,20 @@ def milo_allocate(sigma: torch.Tensor, eps: torch.Tensor, n_groups: int, n_b: in
     s = lib().milo_allocate(_ptr(sigma), _ptr(eps), n_groups, n_b, d, T, block_len, int(R), r_min, r_max,
                             _ptr(ranks_out), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(s, "milo_allocate")
+    return ranks_out
+
+
+def milo_allocate_noalloc(sigma: torch.Tensor, eps: torch.Tensor, n_groups: int, n_b: int, T: int, block_len: int,
+                          R: int, r_min: int = 0, r_max: int = 0, ranks_out=None, stream=None):
+    """milo_allocate without a workspace: the library's built-in device scratch
+    (at most MILO_NOALLOC_MAX_BLOCKS blocks) stands in for it."""
+    assert sigma.dtype == torch.float32 and eps.dtype == torch.float64 and sigma.is_contiguous()
+    d = sigma.shape[-1]
+    if ranks_out is None:
+        ranks_out = torch.empty(n_groups * n_b, dtype=torch.int32, device=sigma.device)
+    s = lib().milo_allocate_noalloc(_ptr(sigma), _ptr(eps), n_groups, n_b, d, T, block_len, int(R), r_min, r_max,
+                                    _ptr(ranks_out), _stream(stream))
+    _check(s, "milo_allocate_noalloc")
     return ranks_out
 
 

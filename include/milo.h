@@ -171,6 +171,30 @@ milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_group
                           int32_t r_max, int32_t *ranks_out, void *workspace, size_t ws_bytes,
                           milo_stream_t stream);
 
+/* Largest n_groups * n_b that milo_allocate_noalloc accepts. */
+#define MILO_NOALLOC_MAX_BLOCKS 65536
+
+/*
+ * milo_allocate for callers that cannot allocate device memory: code that
+ * runs under a framework owning every device byte through its own pool, or
+ * a plug-in operator that is handed only its inputs and outputs.  The paper
+ * has no counterpart; it is a deployment convenience.  Same arguments,
+ * result and errors as milo_allocate, minus the workspace: the scratch is a
+ * fixed device array inside the library (about 1 MiB, held on every device
+ * that loads the library until the process exits).
+ *   - n_groups * n_b > MILO_NOALLOC_MAX_BLOCKS: MILO_ERR_WORKSPACE (the
+ *     built-in scratch is too small), nothing is launched.
+ *   - The first call on a device looks up the array's device address (host
+ *     set-up, no allocation); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (on
+ *     different streams, or from different threads) race and give wrong
+ *     ranks.  Calls in one stream are ordered and safe.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ */
+milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t n_groups, int32_t n_b,
+                                  int32_t d, int32_t T, int32_t block_len, int64_t R, int32_t r_min,
+                                  int32_t r_max, int32_t *ranks_out, milo_stream_t stream);
+
 /* ---------------------------------------------------------------- decode */
 
 /* Bytes of scratch milo_decode_attn needs. */
