@@ -18,6 +18,10 @@
 #pragma once
 #include "common.cuh"
 
+#ifndef MILO_TRACE_JACOBI
+#define MILO_TRACE_JACOBI(sweeps)
+#endif
+
 namespace milo {
 
 constexpr int JAC_THREADS = 512;
@@ -72,7 +76,9 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
     const float floor_abs = sm.floor_abs;
 
     bool converged = false;
+    int sweeps_done = 0;
     for (int sweep = 0; sweep < max_sweeps && !converged; ++sweep) {
+        ++sweeps_done;
         int any = 0;
         for (int r = 0; r < D - 1; ++r) {
             int rot = 0;
@@ -112,8 +118,9 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                     }
                     continue;
                 }
-                const int p2 = sm.p[i2], q2 = sm.q[i2];
                 const float c2 = sm.c[i2], s2 = sm.s[i2];
+                if (s1 == 0.f && s2 == 0.f) continue;   // neither pair rotates: block unchanged
+                const int p2 = sm.p[i2], q2 = sm.q[i2];
                 const float a = sm.G[p * JAC_LD + p2], bb = sm.G[p * JAC_LD + q2];
                 const float cc = sm.G[q * JAC_LD + p2], ee = sm.G[q * JAC_LD + q2];
                 // columns (p2, q2) by J2, then rows (p, q) by J1^T
@@ -142,6 +149,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
         if (!any) converged = true;
     }
     if (!converged && tid == 0) raise_status(ST_NOT_CONVERGED);
+    MILO_TRACE_JACOBI(sweeps_done);
 
     // eigenvalues, stable descending order
     if (tid < D) sm.lam[tid] = sm.G[tid * JAC_LD + tid];
