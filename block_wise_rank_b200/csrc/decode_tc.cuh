@@ -6,51 +6,62 @@
 // "What is MILO").  A prep kernel lists the work items (layer, KV head,
 // block, query pass); an item covers up to 128 queries (the sessions that
 // selected the block times the GQA group).  One persistent CTA per SM walks
-// the items:
+// the items with four roles that only meet at mbarriers:
 //
 //   producer warp   bulk-copies the block's factors (already in the tensor
-//                   cores' canonical layout in HBM) through a 4-stage ring:
-//                   A_K tile 0, B_K, A_K tiles 1.., A_V tiles.., B_V.
-//   MMA warp        K-hat tile = A_K(tile) B_K       (M=128 tokens, N=128, K=r_K, bf16)
-//                   S = K-tilde (TMEM) Q-tilde^T      (M=128 tokens, N=nq, K=128, fp16)
-//                   O_A^T += A_V(tile)^T P            (M=128 ranks, N=nq, K=128 tokens, fp16)
-//                   O = B_V^T (O_A / l)              (M=128 channels, N=nq, K=r_V, fp16)
-//   8 epilogue      rotate the queries by -p*theta_i; RoPE of each rebuilt
-//   warps           key row in registers (block-relative angle t*theta_i),
-//                   K-tilde back to TMEM as fp16; softmax in the exp2 domain
-//                   with a per-query reference max that is raised (and the
-//                   running O_A^T and sums rescaled) only when a score exceeds
-//                   it by more than 2^8; P (fp16) to shared memory, each A_V
-//                   tile converted to fp16 in place; a ones row in A_V makes
-//                   the PV product also return the softmax denominator.
-//                   Two warps share each TMEM lane quadrant and split the
-//                   columns between them.
+//                   cores' canonical layout in HBM): B_K into its own buffer;
+//                   the A_K tiles, the A_V tiles (each with a row of ones
+//                   appended) and B_V into a ring of variable-size tiles.
+//   MMA warp        polls three independent queues and issues whichever op
+//                   is ready:
+//                     rebuild  K-hat tile = A_K(tile) B_K     (M=128 tokens, N=128, K=r_K, bf16)
+//                     scores   S = K-tilde (TMEM) Q-tilde^T    (M=128 tokens, N=nq, K=128, fp16)
+//                     PV / O   O_A^T += A_V(tile)^T P          (M=128 ranks, N=nq, K=128 tokens, fp16)
+//                              O = B_V^T (O_A / l)            (M=128 channels, N=nq, K=r_V, fp16)
+//   RoPE group      4 warps, one per TMEM lane quadrant, one token row per
+//                   thread: rotates each rebuilt key row by its in-block angle
+//                   t*theta_i and packs K-tilde to fp16 in place.  Two rebuild
+//                   buffers let it run up to two tiles ahead of the scores.
+//   softmax group   4 warps: rotates the queries by -p*theta_i; softmax in the
+//                   exp2 domain against a per-query reference max that is
+//                   raised (with the running O_A^T and sums rescaled) only
+//                   when a score exceeds it by more than 2^8; P (fp16) to
+//                   shared memory; each A_V tile converted to fp16 in place;
+//                   O_A / l staged for the last product; O to the partials.
 //
-// Keys and values are never written to memory.  Each (query, selected slot)
-// gets a partial (max, sum, normalised output) merged by k_combine.
+// The ones row makes the PV product return the softmax denominators as one
+// more row of O_A^T.  Keys and values are never written to memory.  Each
+// (query, selected slot) gets a partial (max, sum, normalised output) merged
+// by k_combine.
 #pragma once
 #include "decode_simt.cuh"
 #include "tc_common.cuh"
 
 // Timeline hooks: empty unless a tracing build defines them.
 #ifndef MILO_TRACE_EVENT
-#define MILO_TRACE_EVENT(id)
+#define MILO_TRACE_EVENT(grp, id)
 #endif
 #ifndef MILO_TRACE_MMA
-#define MILO_TRACE_MMA(id)
+#define MILO_TRACE_MMA(n, id)
+#endif
+#ifndef MILO_TRACE_WARP
+#define MILO_TRACE_WARP(id)
 #endif
 
 namespace milo {
 
-constexpr int DT_EPI_WARPS = 8;
-constexpr int DT_EPI = 32 * DT_EPI_WARPS;             // epilogue threads
-constexpr int DT_THREADS = 64 + DT_EPI;               // warp 0 producer, 1 MMA, 2.. epilogue
-constexpr int DT_STAGES = 4;
-constexpr int DT_STAGE_BYTES = 128 * 256;             // 128 ranks x 128 tokens (or channels) x 16 bit
-constexpr int DT_NQ = 128;                            // queries per item (pass)
+constexpr int DT_GROUP = 128;                          // threads per epilogue group
+constexpr int DT_THREADS = 64 + 2 * DT_GROUP;          // warp 0 producer, 1 MMA, 2-5 RoPE, 6-9 softmax
+constexpr int DT_RING = 96 * 1024;                     // ring bytes for A_K, A_V and B_V tiles
+constexpr int DT_NBAR = 32;                            // ring tiles in flight at most
+constexpr int DT_TILE_MAX = 128 * 256;                 // 128 rank rows x 128 tokens (or channels) x 16 bit
+constexpr int DT_NQ = 128;                             // queries per item (pass)
 constexpr uint32_t DT_TMEM_COLS = 512;
-constexpr uint32_t DT_COL_D1 = 0, DT_COL_KT = 128, DT_COL_D2 = 256, DT_COL_OA = 384;
-constexpr float DT_RESCALE = 8.f;                     // log2 headroom before the reference max moves
+constexpr uint32_t DT_COL_D1 = 0;                      // two 128-column rebuild buffers
+constexpr uint32_t DT_COL_D2 = 256;                    // scores: one 128-column buffer or two of 64
+constexpr uint32_t DT_COL_OA = 384;                    // O_A^T, then O
+constexpr float DT_RESCALE = 8.f;                      // log2 headroom before the reference max moves
+constexpr int DT_BAR_S = 1, DT_BAR_R = 2;              // named barriers of the two groups
 
 // One work item, written by k_dt_items.
 struct DtItem {
@@ -61,20 +72,27 @@ struct DtItem {
 };
 
 struct DecTcSmem {
-    alignas(128) uint8_t stage[DT_STAGES][DT_STAGE_BYTES];
+    alignas(128) uint8_t ring[DT_RING];
+    // B_K of the current item.  It follows the ring so that the 128-row
+    // operand read of an A_V tile near the ring's end stays in shared memory
+    // (rows past the tile only feed rows of O_A^T that are never used).
+    alignas(128) uint8_t bk[DT_TILE_MAX];
     alignas(128) uint8_t qt[DT_NQ * D * 2];      // rotated queries, fp16, K-major
-    alignas(128) uint8_t pbuf[128 * DT_NQ * 2];  // P or O_A / l (fp16), MN-major
+    alignas(128) uint8_t pbuf[128 * DT_NQ * 2];  // P or O_A / l (fp16), MN-major; two halves when nq <= 64
     float2 t1[HALF][32];                         // (cos, sin)((t % 32) theta_i)
     float2 t2[HALF][16];                         // (cos, sin)(32 (t / 32) theta_i)
     float cref[DT_NQ];                           // reference max per query (log2 domain)
-    float cnew[DT_NQ];
+    float cscale[DT_NQ];                         // rescale factors, then 1 / l
     float lsum[DT_NQ];
-    float wred[4][DT_NQ];
-    int qpidx[DT_NQ];
-    int flag;
-    uint64_t full[DT_STAGES], empty[DT_STAGES];
-    uint64_t d1_full, d1_empty, kt_full[2], kt_empty[2], q_full, q_empty;
-    uint64_t d2_full, d2_empty, p_full, p_empty, oa_full, oa_staged, drain;
+    int cmax[DT_NQ];                             // column maxima, order-preserving int encoding
+    int qpidx[2][DT_NQ];                         // partial index of each query, per item parity
+    uint32_t toff[DT_NBAR], tlen[DT_NBAR];       // ring offset and bytes of each tile in flight
+    uint64_t full[DT_NBAR], empty[DT_NBAR];
+    uint64_t bk_full, bk_empty;
+    uint64_t d1_full[2], d1_empty[2], kt_full[2];
+    uint64_t d2_full[2], d2_empty[2];
+    uint64_t p_full[2], p_empty[2];
+    uint64_t q_full, q_empty, oa_full, oa_free, drain;
     uint32_t tmem_base;
     volatile int abort;
 };
@@ -108,34 +126,137 @@ __global__ void k_dt_items(DecodeArgs a, const int32_t *__restrict__ pstart, DtI
     }
 }
 
-__device__ __forceinline__ int r16_of(int R8) { return R8 <= 16 ? 16 : (R8 + 15) & ~15; }
+__host__ __device__ __forceinline__ int r16_of(int R8) { return R8 <= 16 ? 16 : (R8 + 15) & ~15; }
 
-// zero rank rows [R8, R16) of a chunk stored as [r/8][16 x 128 B] groups
-__device__ __forceinline__ void zero_rows(uint8_t *chunk, int R8, int R16) {
-    for (int off = R8 * 256; off < R16 * 256; off += 16) *reinterpret_cast<uint4 *>(chunk + off) = make_uint4(0, 0, 0, 0);
+// Geometry of one item as every role sees it.
+struct DtGeo {
+    int nt;            // 128-token tiles
+    int R8K, R16K;     // key rank padded to 8 / to the MMA's K step
+    int R8V, R16V;
+    int rowsV;         // rank rows of an A_V tile in the ring (with the ones group)
+    int nq, nq16;
+    bool ones;         // rank row R8V of each A_V tile is all ones (needs R8V <= 120)
+    bool dbl;          // nq16 <= 64: scores and P double-buffered
+};
+__device__ __forceinline__ DtGeo dt_geo(int Tb, int rK, int rV, int nq) {
+    DtGeo g;
+    g.nt = token_tiles(Tb);
+    g.R8K = rank_pad(rK);
+    g.R16K = r16_of(g.R8K);
+    g.R8V = rank_pad(rV);
+    g.R16V = r16_of(g.R8V);
+    g.ones = g.R8V <= 120;
+    g.rowsV = g.ones ? max(g.R8V + 8, g.R16V) : g.R8V;
+    g.nq = nq;
+    g.nq16 = (nq + 15) & ~15;
+    g.dbl = g.nq16 <= 64;
+    return g;
+}
+__device__ __forceinline__ DtGeo dt_geo(const DtItem *__restrict__ items, int64_t i, int64_t n_items) {
+    if (i >= n_items) return dt_geo(1, 0, 0, 0);
+    return dt_geo(__ldg(&items[i].Tb), __ldg(&items[i].rK), __ldg(&items[i].rV), __ldg(&items[i].nq));
+}
+
+// ring tiles of an item: A_K 0..nt-1, A_V 0..nt-1, B_V
+__device__ __forceinline__ int dt_ring_tiles(const DtGeo &g) { return 2 * g.nt + 1; }
+
+// named-barrier helpers for one 128-thread group
+template <int ID>
+__device__ __forceinline__ void grp_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(DT_GROUP) : "memory");
+}
+template <int ID>
+__device__ __forceinline__ bool grp_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(ID), "n"(DT_GROUP)
+        : "memory");
+    return r != 0;
+}
+template <int ID>
+__device__ __forceinline__ bool grp_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(ID), "n"(DT_GROUP)
+        : "memory");
+    return r != 0;
+}
+
+// non-blocking probe of an mbarrier phase
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// 2^x with the hardware approximation (relative error ~2^-22)
+__device__ __forceinline__ float dt_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// order-preserving int encoding of a float (for atomicMax)
+__device__ __forceinline__ int ord_enc(float x) {
+    const int i = __float_as_int(x);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float ord_dec(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+
+// bf16 pairs to fp16 pairs, in place, over n16 16-byte chunks
+__device__ __forceinline__ void bf16_to_f16_inplace(uint8_t *base, int n16, int tid, int nthr) {
+    uint4 *w = reinterpret_cast<uint4 *>(base);
+    for (int e = tid; e < n16; e += nthr) {
+        uint4 v = w[e];
+        uint32_t *u = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[k]));
+            const __half2 h = __floats2half2_rn(f.x, f.y);
+            u[k] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        w[e] = v;
+    }
 }
 
 __global__ void __launch_bounds__(DT_THREADS, 1)
 k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__restrict__ items) {
     extern __shared__ __align__(128) unsigned char dt_raw[];
-    DecTcSmem &sm = *reinterpret_cast<DecTcSmem *>(
-        (reinterpret_cast<uintptr_t>(dt_raw) + 127) & ~static_cast<uintptr_t>(127));
+    // aligned by pointer arithmetic, so that the compiler keeps the shared
+    // address space (an integer round trip would turn every access generic)
+    DecTcSmem &sm = *reinterpret_cast<DecTcSmem *>(dt_raw + ((128u - (tc::smem_u32(dt_raw) & 127u)) & 127u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_items = (int64_t)a.L * a.H * pstart[a.n_b];
+    const int64_t stride = gridDim.x;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DT_STAGES; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
-        tc::mbar_init(&sm.d1_full, 1);
-        tc::mbar_init(&sm.d1_empty, DT_EPI);
-        for (int k = 0; k < 2; ++k) { tc::mbar_init(&sm.kt_full[k], DT_EPI); tc::mbar_init(&sm.kt_empty[k], 1); }
-        tc::mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < DT_NBAR; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
+        tc::mbar_init(&sm.bk_full, 1);
+        tc::mbar_init(&sm.bk_empty, 1);
+        for (int k = 0; k < 2; ++k) {
+            tc::mbar_init(&sm.d1_full[k], 1);
+            tc::mbar_init(&sm.d1_empty[k], 1);
+            tc::mbar_init(&sm.kt_full[k], DT_GROUP);
+            tc::mbar_init(&sm.d2_full[k], 1);
+            tc::mbar_init(&sm.d2_empty[k], DT_GROUP);
+            tc::mbar_init(&sm.p_full[k], DT_GROUP);
+            tc::mbar_init(&sm.p_empty[k], 1);
+        }
+        tc::mbar_init(&sm.q_full, DT_GROUP);
         tc::mbar_init(&sm.q_empty, 1);
-        tc::mbar_init(&sm.d2_full, 1);
-        tc::mbar_init(&sm.d2_empty, DT_EPI);
-        tc::mbar_init(&sm.p_full, 1);
-        tc::mbar_init(&sm.p_empty, 1);
         tc::mbar_init(&sm.oa_full, 1);
-        tc::mbar_init(&sm.oa_staged, 1);
+        tc::mbar_init(&sm.oa_free, DT_GROUP);
         tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
         tc::fence_barrier_init();
@@ -157,288 +278,252 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint8_t *dataK = (const uint8_t *)a.kv[0].data;
-    const uint8_t *dataV = (const uint8_t *)a.kv[1].data;
 
     if (warp == 0) {
         // ================================================================ producer
-        if (lane == 0) {
-            uint32_t alloc = 0;
-            auto chunk = [&](const uint8_t *src, int R8, int R16, bool ones) -> bool {
-                const int s = alloc % DT_STAGES;
-                const uint32_t ph = (alloc / DT_STAGES) & 1u;
-                if (!tc::mbar_wait(&sm.empty[s], ph ^ 1u)) return false;
-                uint8_t *dst = sm.stage[s];
-                zero_rows(dst, R8, R16);
-                if (ones) {   // rank row 127 = 1.0 (fp16: the tile is converted before use)
-                    for (int g = 0; g < 16; ++g)
-                        *reinterpret_cast<uint4 *>(dst + 15 * 2048 + g * 128 + 7 * 16) =
-                            make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+        const uint8_t *dataK = (const uint8_t *)a.kv[0].data;
+        const uint8_t *dataV = (const uint8_t *)a.kv[1].data;
+        uint32_t head = 0, seq = 0, live = 0;   // live: bit s % NBAR set while tile s may be unconsumed
+        bool ok = true;
+        // room for a tile of `bytes` in the ring: lane 0 waits for the
+        // barrier slot's previous tile and for every live tile overlapping
+        // the new one (all older, so all freed without this one); the warp
+        // follows.  Returns the tile's offset.
+        auto place = [&](uint32_t bytes) -> uint32_t {
+            const uint32_t off = head + bytes > (uint32_t)DT_RING ? 0u : head;
+            if (lane == 0) {
+                for (uint32_t k = seq >= DT_NBAR ? seq - DT_NBAR : 0; k < seq && ok; ++k) {
+                    const uint32_t s = k % DT_NBAR;
+                    if (!((live >> s) & 1u)) continue;
+                    const bool slot_reuse = k + DT_NBAR == seq;
+                    const bool overlap = sm.toff[s] < off + bytes && off < sm.toff[s] + sm.tlen[s];
+                    if (!slot_reuse && !overlap) continue;
+                    if (!tc::mbar_wait(&sm.empty[s], (k / DT_NBAR) & 1u)) { ok = false; break; }
+                    live &= ~(1u << s);
                 }
-                tc::fence_async_smem();
-                const uint32_t bytes = (uint32_t)R8 * 256u;
+                const uint32_t s = seq % DT_NBAR;
+                sm.toff[s] = off;
+                sm.tlen[s] = bytes;
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            head = off + bytes;
+            return off;
+        };
+        // rank rows [r0, r1) of a tile: zeros; with `ones`, row r0 is fp16 1.0
+        // (A_V tiles are converted to fp16 before use)
+        auto fill_rows = [&](uint8_t *dst, int r0, int r1, bool ones) {
+            for (int e = lane; e < (r1 - r0) * 16; e += 32) {
+                const uint32_t w = (ones && e < 128 && (e & 7) == 0) ? 0x3C003C00u : 0u;
+                *reinterpret_cast<uint4 *>(dst + r0 * 256 + e * 16) = make_uint4(w, w, w, w);
+            }
+            tc::fence_async_smem();
+            __syncwarp();
+        };
+        // one ring tile of `rows` rank rows, `copy` of them from HBM
+        auto ring_tile = [&](const uint8_t *src, int rows, int copy, bool ones) {
+            const uint32_t off = place((uint32_t)rows * 256u);
+            if (!ok) return;
+            uint8_t *dst = sm.ring + off;
+            if (rows > copy) fill_rows(dst, copy, rows, ones);
+            if (lane == 0) {
+                const uint32_t s = seq % DT_NBAR;
+                const uint32_t bytes = (uint32_t)copy * 256u;
                 tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
                 if (bytes) tc::bulk_g2s(dst, src, bytes, &sm.full[s]);
-                ++alloc;
-                return true;
-            };
-            bool ok = true;
-            for (int64_t i = blockIdx.x; i < n_items && ok && !sm.abort; i += gridDim.x) {
-                const DtItem it = items[i];
-                const int nt = token_tiles(it.Tb);
-                const int R8K = rank_pad(it.rK), R8V = rank_pad(it.rV);
-                const int R16K = r16_of(R8K), R16V = r16_of(R8V);
-                const uint8_t *bK = dataK + 2 * it.offK, *bV = dataV + 2 * it.offV;
-                const int64_t tileK = (int64_t)R8K * 256, tileV = (int64_t)R8V * 256;
-                const bool ones = R8V <= 120;
-                ok = ok && chunk(bK, R8K, R16K, false);                          // A_K tile 0
-                ok = ok && chunk(bK + nt * tileK, R8K, R16K, false);             // B_K
-                for (int t = 1; t < nt && ok; ++t) ok = chunk(bK + t * tileK, R8K, R16K, false);
-                for (int t = 0; t < nt && ok; ++t) ok = chunk(bV + t * tileV, R8V, R16V, ones);
-                ok = ok && chunk(bV + nt * tileV, R8V, R16V, false);             // B_V
             }
-            if (!ok) sm.abort = 1;
-            // drain: every stage's last copy has landed before the CTA exits
-            for (int s = 0; s < DT_STAGES && alloc > 0; ++s) {
-                const uint32_t last = alloc - 1 - s;
-                if ((int)last < 0) break;
-                tc::mbar_wait(&sm.full[last % DT_STAGES], (last / DT_STAGES) & 1u);
+            live |= 1u << (seq % DT_NBAR);
+            ++seq;
+        };
+        uint32_t n = 0;
+        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
+            if (__shfl_sync(0xffffffffu, (int)(sm.abort != 0), 0)) break;
+            const DtItem it = items[i];
+            const DtGeo g = dt_geo(it.Tb, it.rK, it.rV, it.nq);
+            const uint8_t *bK = dataK + 2 * it.offK, *bV = dataV + 2 * it.offV;
+            const int64_t tileK = (int64_t)g.R8K * 256, tileV = (int64_t)g.R8V * 256;
+            ring_tile(bK, g.R16K, g.R8K, false);                               // A_K tile 0
+            if (!ok) break;
+            // B_K into its own buffer once the previous item's rebuilds are done
+            if (lane == 0) ok = tc::mbar_wait(&sm.bk_empty, (n & 1u) ^ 1u);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (g.R16K > g.R8K) fill_rows(sm.bk, g.R8K, g.R16K, false);
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&sm.bk_full, (uint32_t)tileK);
+                if (tileK) tc::bulk_g2s(sm.bk, bK + g.nt * tileK, (uint32_t)tileK, &sm.bk_full);
             }
+            for (int t = 1; t < g.nt && ok; ++t) ring_tile(bK + t * tileK, g.R16K, g.R8K, false);
+            for (int t = 0; t < g.nt && ok; ++t) ring_tile(bV + t * tileV, g.rowsV, g.R8V, g.ones);
+            if (ok) ring_tile(bV + g.nt * tileV, g.R16V, g.R8V, false);          // B_V
+        }
+        if (!ok && lane == 0) sm.abort = 1;
+        // drain: every copy issued has landed before the CTA exits
+        if (lane == 0) {
+            for (uint32_t k = seq >= DT_NBAR ? seq - DT_NBAR : 0; k < seq; ++k)
+                tc::mbar_wait(&sm.full[k % DT_NBAR], (k / DT_NBAR) & 1u);
+            if (n > 0) tc::mbar_wait(&sm.bk_full, (n - 1) & 1u);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            uint32_t alloc = 0, n_d1 = 0, n_d2 = 0, n_kt[2] = {0, 0}, n_q = 0, n_p = 0, n_oa = 0;
+            const uint32_t id_rb = tc::idesc_f16(128, 128, 1, 1, 1);   // bf16, A/B MN-major
+            const int64_t i0 = blockIdx.x;
+            const DtGeo g0 = dt_geo(items, i0, n_items), g1 = dt_geo(items, i0 + stride, n_items);
+            // each queue holds the geometry of its item and of the next one
+            int64_t iR = i0, iS = i0, iP = i0;
+            DtGeo gR = g0, gRn = g1, gS = g0, gSn = g1, gP = g0, gPn = g1;
+            uint32_t nR = 0, tR = 0, seqR = 0, rc = 0;             // rebuild queue
+            uint32_t nS = 0, tS = 0, rcS = 0, u2[2] = {0, 0};      // scores queue
+            uint32_t nP = 0, tP = 0, seqP = 0, pu[2] = {0, 0};     // PV / O queue
+            const uint32_t sq = tc::smem_u32(sm.qt);
+            const uint32_t sbk = tc::smem_u32(sm.bk);
+            const uint32_t spb = tc::smem_u32(sm.pbuf);
+            const uint32_t sring = tc::smem_u32(sm.ring);
+            uint64_t t_last = tc::globaltimer();
             bool ok = true;
-            auto stage_of = [&](uint32_t k) { return k % DT_STAGES; };
-            auto wait_full = [&](uint32_t k) { return tc::mbar_wait(&sm.full[stage_of(k)], (k / DT_STAGES) & 1u); };
-            for (int64_t i = blockIdx.x; i < n_items && ok && !sm.abort; i += gridDim.x) {
-                const DtItem it = items[i];
-                const int nt = token_tiles(it.Tb);
-                const int nq16 = (it.nq + 15) & ~15;
-                const int R16K = r16_of(rank_pad(it.rK)), R16V = r16_of(rank_pad(it.rV));
-                const uint32_t aK0 = alloc, aBK = alloc + 1;
-                auto aK = [&](int t) { return t == 0 ? aK0 : aBK + t; };
-                const uint32_t aV0 = aBK + nt;
-                const uint32_t aBV = aV0 + nt;
-                alloc = aBV + 1;
-                const uint32_t id_rb = tc::idesc_f16(128, 128, 1, 1, 1);     // bf16, A/B MN-major
-                const uint32_t id_sc = tc::idesc_f16(128, nq16, 0, 0, 0);    // fp16, A tmem, B K-major
-                const uint32_t id_pv = tc::idesc_f16(128, nq16, 0, 0, 1);    // fp16, A K-major, B MN-major
-                const uint32_t id_o = tc::idesc_f16(128, nq16, 0, 1, 1);     // fp16, A/B MN-major
-                const uint32_t lbo_p = (uint32_t)(nq16 / 8) * 128u;
-                auto rebuild = [&](int t) -> bool {
-                    if (!wait_full(aK(t))) return false;
-                    if (t == 0 && !wait_full(aBK)) return false;
-                    if (!tc::mbar_wait(&sm.d1_empty, (n_d1 & 1u) ^ 1u)) return false;
-                    MILO_TRACE_MMA(t);
-                    tc::tc_fence_after();
-                    const uint32_t sa = tc::smem_u32(sm.stage[stage_of(aK(t))]);
-                    const uint32_t sb = tc::smem_u32(sm.stage[stage_of(aBK)]);
-                    for (int ks = 0; ks < R16K / 16; ++ks)
-                        tc::mma_ss(tmem + DT_COL_D1, tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
-                                   tc::smem_desc(sb + ks * 4096, 2048, 128, tc::LAYOUT_NONE), id_rb, ks > 0);
-                    tc::mma_commit(&sm.d1_full);
-                    ++n_d1;
-                    tc::mma_commit(&sm.empty[stage_of(aK(t))]);
-                    if (t == nt - 1) tc::mma_commit(&sm.empty[stage_of(aBK)]);
-                    return true;
-                };
-                auto scores = [&](int t) -> bool {
-                    const int slot = t & 1;
-                    if (!tc::mbar_wait(&sm.kt_full[slot], n_kt[slot] & 1u)) return false;
-                    if (t == 0 && !tc::mbar_wait(&sm.q_full, n_q & 1u)) return false;
-                    if (!tc::mbar_wait(&sm.d2_empty, (n_d2 & 1u) ^ 1u)) return false;
-                    MILO_TRACE_MMA(4 + t);
-                    tc::tc_fence_after();
-                    const uint32_t sq = tc::smem_u32(sm.qt);
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        tc::mma_ts(tmem + DT_COL_D2, tmem + DT_COL_KT + slot * 64 + ks * 8,
-                                   tc::smem_desc(sq + ks * 256, 128, 2048, tc::LAYOUT_NONE), id_sc, ks > 0);
-                    tc::mma_commit(&sm.d2_full);
-                    ++n_d2;
-                    tc::mma_commit(&sm.kt_empty[slot]);
-                    ++n_kt[slot];
-                    if (t == nt - 1) { tc::mma_commit(&sm.q_empty); ++n_q; }
-                    return true;
-                };
-                auto pv = [&](int t) -> bool {
-                    if (!tc::mbar_wait(&sm.p_full, n_p & 1u)) return false;
-                    if (!wait_full(aV0 + t)) return false;
-                    MILO_TRACE_MMA(8 + t);
-                    tc::tc_fence_after();
-                    const uint32_t sa = tc::smem_u32(sm.stage[stage_of(aV0 + t)]);
-                    const uint32_t sp = tc::smem_u32(sm.pbuf);
-                    for (int ks = 0; ks < 8; ++ks)
-                        tc::mma_ss(tmem + DT_COL_OA, tc::smem_desc(sa + ks * 256, 128, 2048, tc::LAYOUT_NONE),
-                                   tc::smem_desc(sp + ks * 2 * lbo_p, lbo_p, 128, tc::LAYOUT_NONE), id_pv,
-                                   (t | ks) != 0);
-                    tc::mma_commit(&sm.p_empty);
-                    ++n_p;
-                    tc::mma_commit(&sm.empty[stage_of(aV0 + t)]);
-                    if (t == nt - 1) tc::mma_commit(&sm.oa_full);
-                    return true;
-                };
-                ok = rebuild(0);
-                if (ok && nt > 1) ok = rebuild(1);
-                for (int t = 0; t < nt && ok; ++t) {
-                    ok = scores(t);
-                    if (ok && t + 2 < nt) ok = rebuild(t + 2);
-                    if (ok && t >= 1) ok = pv(t - 1);
-                }
-                if (ok) ok = pv(nt - 1);
-                if (ok) {   // O = B_V^T (O_A / l), into the D1 columns
-                    ok = tc::mbar_wait(&sm.oa_staged, n_oa & 1u) && tc::mbar_wait(&sm.d1_empty, (n_d1 & 1u) ^ 1u);
-                    ++n_oa;
-                    MILO_TRACE_MMA(12);
-                    if (ok) {
+            while (ok) {
+                const bool doneR = iR >= n_items, doneS = iS >= n_items, doneP = iP >= n_items;
+                if (doneR && doneS && doneP) break;
+                bool prog = false;
+                // ---------------------------------------------------- rebuild
+                if (!doneR) {
+                    const uint32_t k = seqR + tR, s = k % DT_NBAR, b = rc & 1u;
+                    if (mbar_test(&sm.full[s], (k / DT_NBAR) & 1u) && (tR > 0 || mbar_test(&sm.bk_full, nR & 1u)) &&
+                        mbar_test(&sm.d1_empty[b], ((rc >> 1) & 1u) ^ 1u)) {
+                        MILO_TRACE_MMA(nR, tR);
                         tc::tc_fence_after();
-                        const uint32_t sa = tc::smem_u32(sm.stage[stage_of(aBV)]);
-                        const uint32_t sp = tc::smem_u32(sm.pbuf);
-                        for (int ks = 0; ks < R16V / 16; ++ks)
-                            tc::mma_ss(tmem + DT_COL_D1, tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
-                                       tc::smem_desc(sp + ks * 2 * lbo_p, lbo_p, 128, tc::LAYOUT_NONE), id_o,
-                                       ks > 0);
-                        tc::mma_commit(&sm.d1_full);
-                        ++n_d1;
-                        tc::mma_commit(&sm.p_empty);   // staging buffer free again
-                        tc::mma_commit(&sm.empty[stage_of(aBV)]);
+                        const uint32_t sa = sring + sm.toff[s];
+                        for (int ks = 0; ks < gR.R16K / 16; ++ks)
+                            tc::mma_ss(tmem + DT_COL_D1 + 128 * b,
+                                       tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
+                                       tc::smem_desc(sbk + ks * 4096, 2048, 128, tc::LAYOUT_NONE), id_rb, ks > 0);
+                        tc::mma_commit(&sm.d1_full[b]);
+                        tc::mma_commit(&sm.empty[s]);
+                        if ((int)tR == gR.nt - 1) tc::mma_commit(&sm.bk_empty);
+                        ++rc;
+                        if ((int)++tR == gR.nt) {
+                            seqR += dt_ring_tiles(gR);
+                            tR = 0;
+                            ++nR;
+                            iR += stride;
+                            gR = gRn;
+                            gRn = dt_geo(items, iR + stride, n_items);
+                        }
+                        prog = true;
                     }
+                }
+                // ---------------------------------------------------- scores
+                if (!doneS) {
+                    const uint32_t b = rcS & 1u;
+                    const uint32_t d2b = gS.dbl ? (tS & 1u) : 0u;
+                    // a full-width scores buffer also covers the second half-buffer
+                    if (mbar_test(&sm.kt_full[b], (rcS >> 1) & 1u) && (tS > 0 || mbar_test(&sm.q_full, nS & 1u)) &&
+                        mbar_test(&sm.d2_empty[d2b], (u2[d2b] & 1u) ^ 1u) &&
+                        (gS.dbl || mbar_test(&sm.d2_empty[1], (u2[1] & 1u) ^ 1u))) {
+                        MILO_TRACE_MMA(nS, 4 + tS);
+                        tc::tc_fence_after();
+                        const uint32_t id_sc = tc::idesc_f16(128, gS.nq16, 0, 0, 0);   // fp16, A tmem, B K-major
+                        const uint32_t kt = tmem + DT_COL_D1 + 128 * b;
+                        // K-tilde: x halves packed at columns 0..31, y halves at 64..95
+                        for (int ks = 0; ks < D / 16; ++ks)
+                            tc::mma_ts(tmem + DT_COL_D2 + 64 * d2b, kt + (ks < 4 ? 8 * ks : 32 + 8 * ks),
+                                       tc::smem_desc(sq + ks * 256, 128, 2048, tc::LAYOUT_NONE), id_sc, ks > 0);
+                        tc::mma_commit(&sm.d2_full[d2b]);
+                        tc::mma_commit(&sm.d1_empty[b]);
+                        if ((int)tS == gS.nt - 1) tc::mma_commit(&sm.q_empty);
+                        ++u2[d2b];
+                        ++rcS;
+                        if ((int)++tS == gS.nt) {
+                            tS = 0;
+                            ++nS;
+                            iS += stride;
+                            gS = gSn;
+                            gSn = dt_geo(items, iS + stride, n_items);
+                        }
+                        prog = true;
+                    }
+                }
+                // ---------------------------------------------------- PV and O
+                if (!doneP) {
+                    const uint32_t pb = gP.dbl ? (tP & 1u) : 0u;
+                    const uint32_t lbo_p = (uint32_t)(gP.nq16 / 8) * 128u;
+                    const uint32_t sp = spb + pb * 16384u;
+                    if (mbar_test(&sm.p_full[pb], pu[pb] & 1u) && (tP > 0 || mbar_test(&sm.oa_free, (nP & 1u) ^ 1u))) {
+                        tc::tc_fence_after();
+                        if ((int)tP < gP.nt) {   // O_A^T += A_V(tile)^T P
+                            MILO_TRACE_MMA(nP, 8 + tP);
+                            const uint32_t k = seqP + gP.nt + tP, s = k % DT_NBAR;
+                            const uint32_t sa = sring + sm.toff[s];
+                            const uint32_t id_pv = tc::idesc_f16(128, gP.nq16, 0, 0, 1);   // fp16, A K-major, B MN-major
+                            for (int ks = 0; ks < 8; ++ks)
+                                tc::mma_ss(tmem + DT_COL_OA, tc::smem_desc(sa + ks * 256, 128, 2048, tc::LAYOUT_NONE),
+                                           tc::smem_desc(sp + ks * 2 * lbo_p, lbo_p, 128, tc::LAYOUT_NONE), id_pv,
+                                           (tP | ks) != 0);
+                            tc::mma_commit(&sm.p_empty[pb]);
+                            tc::mma_commit(&sm.empty[s]);
+                            if ((int)tP == gP.nt - 1) tc::mma_commit(&sm.oa_full);
+                            ++pu[pb];
+                            ++tP;
+                        } else {                 // O = B_V^T (O_A / l), over O_A's columns
+                            MILO_TRACE_MMA(nP, 12);
+                            const uint32_t k = seqP + 2 * gP.nt, s = k % DT_NBAR;
+                            const uint32_t sa = sring + sm.toff[s];
+                            const uint32_t id_o = tc::idesc_f16(128, gP.nq16, 0, 1, 1);    // fp16, A/B MN-major
+                            for (int ks = 0; ks < gP.R16V / 16; ++ks)
+                                tc::mma_ss(tmem + DT_COL_OA, tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
+                                           tc::smem_desc(sp + ks * 2 * lbo_p, lbo_p, 128, tc::LAYOUT_NONE), id_o,
+                                           ks > 0);
+                            tc::mma_commit(&sm.p_empty[pb]);
+                            tc::mma_commit(&sm.empty[s]);
+                            tc::mma_commit(&sm.oa_full);
+                            ++pu[pb];
+                            seqP += dt_ring_tiles(gP);
+                            tP = 0;
+                            ++nP;
+                            iP += stride;
+                            gP = gPn;
+                            gPn = dt_geo(items, iP + stride, n_items);
+                        }
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    t_last = tc::globaltimer();
+                } else if (sm.abort || tc::globaltimer() - t_last > 2000000000ull) {
+                    if (!sm.abort) raise_status(ST_TIMEOUT);
+                    ok = false;
+                } else {
+                    __nanosleep(32);   // leave the issue slots to the group warps
                 }
             }
             if (!ok) sm.abort = 1;
             tc::mma_commit(&sm.drain);
             tc::mbar_wait(&sm.drain, 0);
         }
-    } else {
-        // ================================================================ epilogue (8 warps)
-        const int quad = warp & 3;                   // TMEM lane quadrant of this warp
-        const int eh = (warp - 2) >> 2;              // which of the two warps of the quadrant
-        const int row = quad * 32 + lane;            // TMEM lane of this thread
+    } else if (warp < 6) {
+        // ================================================================ RoPE group
+        const int et = threadIdx.x - 64;
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int et = threadIdx.x - 64;             // 0 .. DT_EPI-1
-        const float kscale = 1.4426950408889634f * rsqrtf((float)D);   // log2(e) / sqrt(d)
-        uint32_t alloc = 0, n_d1 = 0, n_d2 = 0, n_kt[2] = {0, 0}, n_q = 0, n_p = 0, n_oa = 0;
+        uint32_t rc = 0, n = 0;
         bool ok = true;
-        auto ebar = [&]() { asm volatile("bar.sync 1, %0;" ::"n"(DT_EPI) : "memory"); };
-        // named-barrier AND of every epilogue thread's flag: a wait that gave up
-        // in one thread ends the loop in all of them, never a lone straggler
-        // named-barrier OR of a flag over the epilogue threads
-        auto any_all = [&](int v) -> bool {
-            uint32_t r;
-            asm volatile(
-                "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
-                "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                : "=r"(r)
-                : "r"((uint32_t)v), "n"(DT_EPI)
-                : "memory");
-            return r != 0;
-        };
-        // 2^x with the hardware approximation (relative error ~2^-22)
-        auto ex2 = [](float x) -> float {
-            float y;
-            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-            return y;
-        };
-        auto all_ok = [&](bool v) -> bool {
-            uint32_t r;
-            asm volatile(
-                "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
-                "bar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                : "=r"(r)
-                : "r"((uint32_t)v), "n"(DT_EPI)
-                : "memory");
-            return r != 0;
-        };
-        for (int64_t i = blockIdx.x; i < n_items && ok && !sm.abort; i += gridDim.x) {
-            const DtItem it = items[i];
-            MILO_TRACE_EVENT(0);
-            const int nt = token_tiles(it.Tb);
-            const int nq = it.nq, nq16 = (nq + 15) & ~15;
-            const int R8V = rank_pad(it.rV), R16V = r16_of(R8V);
-            const uint32_t aV0 = alloc + 1 + nt;
-            const uint32_t aBV = alloc + 1 + 2 * nt;
-            alloc = aBV + 1;
-            const uint32_t lbo_p = (uint32_t)(nq16 / 8) * 128u;
-            const bool ones = R8V <= 120;   // rank row 127 of A_V carries ones
-            const int c_first = 16 * eh;    // this warp's 16-column chunks: c_first, +32, ...
-
-            // ---- rotated queries R(-p) q, fp16, K-major [q/8][j/8][q%8][j%8];
-            // four threads per query, 16 pairs each, every load issued up front
-            ok = all_ok(tc::mbar_wait(&sm.q_empty, (n_q & 1u) ^ 1u));
-            if (!ok) break;
-            MILO_TRACE_EVENT(1);
-            for (int u = et; u < 4 * nq16; u += DT_EPI) {
-                const int qi = u >> 2, part = u & 3;          // pairs 16*part .. 16*part+15
-                uint8_t *qrow = sm.qt + (qi >> 3) * 2048 + (qi & 7) * 16;
-                if (qi < nq) {
-                    const int gq = it.q0 + qi;
-                    const int slot = a.slot_list[it.slot0 + gq / a.G];
-                    const int g = gq % a.G;
-                    const int s = slot / a.n_sel, jj = slot % a.n_sel;
-                    const int hq = it.h * a.G + g;
-                    const float4 *qv = reinterpret_cast<const float4 *>(a.q + (((int64_t)it.l * a.S + s) * a.Hq + hq) * D);
-                    const float4 *cs = reinterpret_cast<const float4 *>(a.rope_q + (int64_t)slot * HALF);
-                    if (part == 0) sm.qpidx[qi] = (int)((((int64_t)it.l * a.S + s) * a.Hq + hq) * a.n_sel + jj);
-                    float4 xa[4], xb[4], cv[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) { xa[k] = qv[4 * part + k]; xb[k] = qv[16 + 4 * part + k]; }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) cv[k] = cs[8 * part + k];
-#pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {          // pairs 16*part + 8*h8 .. +7
-                        const float x0[8] = {xa[2 * h8].x, xa[2 * h8].y, xa[2 * h8].z, xa[2 * h8].w,
-                                             xa[2 * h8 + 1].x, xa[2 * h8 + 1].y, xa[2 * h8 + 1].z, xa[2 * h8 + 1].w};
-                        const float x1[8] = {xb[2 * h8].x, xb[2 * h8].y, xb[2 * h8].z, xb[2 * h8].w,
-                                             xb[2 * h8 + 1].x, xb[2 * h8 + 1].y, xb[2 * h8 + 1].z, xb[2 * h8 + 1].w};
-                        uint32_t lo[4], hi[4];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const float4 c2 = cv[4 * h8 + v];   // (cos, sin) of pairs 2v, 2v+1
-                            const __half2 h0 = __floats2half2_rn(x0[2 * v] * c2.x + x1[2 * v] * c2.y,
-                                                                 x0[2 * v + 1] * c2.z + x1[2 * v + 1] * c2.w);
-                            const __half2 h1 = __floats2half2_rn(x1[2 * v] * c2.x - x0[2 * v] * c2.y,
-                                                                 x1[2 * v + 1] * c2.z - x0[2 * v + 1] * c2.w);
-                            lo[v] = *reinterpret_cast<const uint32_t *>(&h0);
-                            hi[v] = *reinterpret_cast<const uint32_t *>(&h1);
-                        }
-                        const int g8 = 2 * part + h8;
-                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        *reinterpret_cast<uint4 *>(qrow + (8 + g8) * 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    }
-                } else {
-                    for (int g8 = 4 * part; g8 < 4 * part + 4; ++g8)
-                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            tc::fence_async_smem();
-            ebar();
-            if (et == 0) tc::mbar_arrive(&sm.q_full);
-            ++n_q;
-            MILO_TRACE_EVENT(2);
-
-            // ---- RoPE of a rebuilt tile, K-tilde to TMEM (fp16 pairs); this warp: 2 of the 4 pair chunks
-            auto rope = [&](int t) -> bool {
-                const int slot = t & 1;
-                const bool w1 = tc::mbar_wait(&sm.d1_full, n_d1 & 1u);
-                const bool w2 = w1 && tc::mbar_wait(&sm.kt_empty[slot], (n_kt[slot] & 1u) ^ 1u);
-                if (!all_ok(w2)) return false;
-                MILO_TRACE_EVENT(4 + 4 * t);
+        (void)et;
+        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
+            const int nt = token_tiles(__ldg(&items[i].Tb));
+            for (int t = 0; t < nt; ++t) {
+                const uint32_t b = rc & 1u;
+                ok = grp_and<DT_BAR_R>(tc::mbar_wait(&sm.d1_full[b], (rc >> 1) & 1u) && !sm.abort);
+                if (!ok) break;
+                MILO_TRACE_EVENT(0, 2 * t);
                 tc::tc_fence_after();
-                const int tok = t * FTILE + row;             // token of this lane
+                const uint32_t base = tmem + DT_COL_D1 + 128 * b + lane_off;
+                const int tok = t * FTILE + row;   // in-block token of this lane
                 const int tl = tok & 31, th = tok >> 5;
-                uint32_t xr2[2][16], yr2[2][16];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    tc::tmem_ld16(tmem + DT_COL_D1 + lane_off + (2 * eh + c) * 16, xr2[c]);
-                    tc::tmem_ld16(tmem + DT_COL_D1 + lane_off + HALF + (2 * eh + c) * 16, yr2[c]);
-                }
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int pc = 2 * eh + c;
-                    const uint32_t(&xr)[16] = xr2[c];
-                    const uint32_t(&yr)[16] = yr2[c];
+                // pair chunk pc (16 pairs): x at columns 16pc.., y at 64 + 16pc..;
+                // packed fp16 results go to 8pc.. (x) and 64 + 8pc.. (y), columns
+                // this thread has already read
+                auto rot_chunk = [&](const uint32_t (&xr)[16], const uint32_t (&yr)[16], int pc) {
                     uint32_t px[8], py[8];
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
@@ -458,265 +543,392 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         px[v] = *reinterpret_cast<const uint32_t *>(&hx);
                         py[v] = *reinterpret_cast<const uint32_t *>(&hy);
                     }
-                    tc::tmem_st8(tmem + DT_COL_KT + slot * 64 + lane_off + pc * 8, px);
-                    tc::tmem_st8(tmem + DT_COL_KT + slot * 64 + lane_off + 32 + pc * 8, py);
+                    tc::tmem_st8(base + 8 * pc, px);
+                    tc::tmem_st8(base + 64 + 8 * pc, py);
+                };
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {   // pair chunks 2h, 2h+1
+                    uint32_t xa[16], ya[16], xb[16], yb[16];
+                    tc::tmem_ld16(base + 32 * h, xa);
+                    tc::tmem_ld16(base + 64 + 32 * h, ya);
+                    tc::tmem_ld16(base + 32 * h + 16, xb);
+                    tc::tmem_ld16(base + 64 + 32 * h + 16, yb);
+                    tc::tmem_wait_ld();
+                    rot_chunk(xa, ya, 2 * h);
+                    rot_chunk(xb, yb, 2 * h + 1);
                 }
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
-                tc::mbar_arrive(&sm.d1_empty);
-                ++n_d1;
-                tc::mbar_arrive(&sm.kt_full[slot]);
-                ++n_kt[slot];
-                MILO_TRACE_EVENT(5 + 4 * t);
+                tc::mbar_arrive(&sm.kt_full[b]);
+                ++rc;
+                MILO_TRACE_EVENT(0, 2 * t + 1);
+            }
+        }
+        if (!ok) sm.abort = 1;
+    } else {
+        // ================================================================ softmax group
+        const int et = threadIdx.x - 192;
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;             // TMEM lane of this thread
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const float kscale = 1.4426950408889634f * rsqrtf((float)D);   // log2(e) / sqrt(d)
+        uint32_t u2[2] = {0, 0};                      // uses of each scores buffer
+        uint32_t pf[2] = {0, 0}, pe[2] = {0, 0};      // P buffer hand-overs / completions seen
+        uint32_t seqA0 = 0, n = 0;
+        bool ok = true;
+
+        // wait until P buffer b's last product (PV or O) has completed
+        auto p_drain = [&](int b) -> bool {
+            if (pe[b] == pf[b]) return true;
+            const bool w = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.p_empty[b], pe[b] & 1u));
+            ++pe[b];
+            return w;
+        };
+
+        // ---- rotated queries R(-p) q of item j, fp16, K-major [q/8][j/8][q%8][j%8];
+        // four threads per query, 16 pairs each
+        auto qprep = [&](int64_t j, uint32_t nj) -> bool {
+            if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.q_empty, (nj & 1u) ^ 1u))) return false;
+            const int nq = __ldg(&items[j].nq), nq16 = (nq + 15) & ~15;
+            const int jl = __ldg(&items[j].l), jh = __ldg(&items[j].h), jq0 = __ldg(&items[j].q0);
+            const int jslot0 = __ldg(&items[j].slot0);
+            for (int u = et; u < 4 * nq16; u += DT_GROUP) {
+                const int qi = u >> 2, part = u & 3;          // pairs 16*part .. 16*part+15
+                uint8_t *qrow = sm.qt + (qi >> 3) * 2048 + (qi & 7) * 16;
+                if (qi < nq) {
+                    const int gq = jq0 + qi;
+                    const int slot = a.slot_list[jslot0 + gq / a.G];
+                    const int g = gq % a.G;
+                    const int s = slot / a.n_sel, jj = slot % a.n_sel;
+                    const int hq = jh * a.G + g;
+                    const int64_t qbase = ((int64_t)jl * a.S + s) * a.Hq + hq;
+                    const float4 *qv = reinterpret_cast<const float4 *>(a.q + qbase * D);
+                    const float4 *cs = reinterpret_cast<const float4 *>(a.rope_q + (int64_t)slot * HALF);
+                    if (part == 0) sm.qpidx[nj & 1u][qi] = (int)(qbase * a.n_sel + jj);
+#pragma unroll 1
+                    for (int h8 = 0; h8 < 2; ++h8) {          // pairs 16*part + 8*h8 .. +7
+                        const int p0 = 16 * part + 8 * h8;
+                        const float4 xa0 = qv[p0 / 4], xa1 = qv[p0 / 4 + 1];
+                        const float4 xb0 = qv[16 + p0 / 4], xb1 = qv[16 + p0 / 4 + 1];
+                        float4 cv[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) cv[k] = cs[p0 / 2 + k];
+                        const float x0[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+                        const float x1[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+                        uint32_t lo[4], hi[4];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const float4 c2 = cv[v];   // (cos, sin) of pairs p0 + 2v, p0 + 2v + 1
+                            const __half2 h0 = __floats2half2_rn(x0[2 * v] * c2.x + x1[2 * v] * c2.y,
+                                                                 x0[2 * v + 1] * c2.z + x1[2 * v + 1] * c2.w);
+                            const __half2 h1 = __floats2half2_rn(x1[2 * v] * c2.x - x0[2 * v] * c2.y,
+                                                                 x1[2 * v + 1] * c2.z - x0[2 * v + 1] * c2.w);
+                            lo[v] = *reinterpret_cast<const uint32_t *>(&h0);
+                            hi[v] = *reinterpret_cast<const uint32_t *>(&h1);
+                        }
+                        const int g8 = 2 * part + h8;
+                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        *reinterpret_cast<uint4 *>(qrow + (8 + g8) * 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    }
+                } else {
+                    for (int g8 = 4 * part; g8 < 4 * part + 4; ++g8)
+                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            tc::fence_async_smem();
+            tc::mbar_arrive(&sm.q_full);
+            return true;
+        };
+
+        if (blockIdx.x < n_items) ok = qprep(blockIdx.x, 0);
+        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
+            const DtGeo g = dt_geo(items, i, n_items);
+            const int Tb = __ldg(&items[i].Tb);
+            const int nq = g.nq, nq16 = g.nq16;
+            const uint32_t lbo_p = (uint32_t)(nq16 / 8) * 128u;
+            int cv_next = 0, pv_issued = 0;
+            MILO_TRACE_EVENT(1, 0);
+
+            // ---- A_V tile tt (B_V when tt == nt) to fp16 in place; an A_V tile
+            // hands its P buffer to the PV product
+            auto convert = [&](int tt) -> bool {
+                const uint32_t k = seqA0 + g.nt + tt, s = k % DT_NBAR;
+                if (tt < 4) MILO_TRACE_EVENT(1, 48 + tt);
+                if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.full[s], (k / DT_NBAR) & 1u))) return false;
+                if (tt < 4) MILO_TRACE_EVENT(1, 52 + tt);
+                bf16_to_f16_inplace(sm.ring + sm.toff[s], g.R8V * 16, et, DT_GROUP);
+                tc::fence_async_smem();
+                if (tt < 4) MILO_TRACE_EVENT(1, 56 + tt);
+                if (tt < g.nt) {
+                    const int pb = g.dbl ? (tt & 1) : 0;
+                    tc::mbar_arrive(&sm.p_full[pb]);
+                    ++pf[pb];
+                    ++pv_issued;
+                }
                 return true;
             };
 
-            // ---- softmax of one score tile, P (fp16) to shared memory.  One pass
-            // over the scores: p = 2^(x - cref); a CTA-wide vote decides whether
-            // any score exceeded its reference by more than 2^8, in which case
-            // (rare) the reference moves to the exact maximum and the running
-            // O_A^T and sums are rescaled before P is written.
-            auto softmax = [&](int t) -> bool {
-                {
-                    const bool w1 = tc::mbar_wait(&sm.d2_full, n_d2 & 1u);
-                    const bool w2 = w1 && tc::mbar_wait(&sm.p_empty, (n_p & 1u) ^ 1u);   // P buffer free
-                    if (!all_ok(w2)) return false;
-                }
-                MILO_TRACE_EVENT(6 + 4 * t);
-                tc::tc_fence_after();
-                const int tok = t * FTILE + row;
-                const bool valid = tok < it.Tb;
-                const int nch = (nq16 - c_first + 31) / 32;   // this warp's 16-column chunks (<= 4)
-                // two chunks per TMEM round trip: at most 32 score registers live
-                auto load2 = [&](int k, uint32_t (&r0)[16], uint32_t (&r1)[16]) {
-                    tc::tmem_ld16(tmem + DT_COL_D2 + lane_off + c_first + 32 * k, r0);
-                    if (k + 1 < nch) tc::tmem_ld16(tmem + DT_COL_D2 + lane_off + c_first + 32 * (k + 1), r1);
-                    tc::tmem_wait_ld();
-                };
-                if (t == 0) {   // reference max: the scores of the item's first token (lane 0 of quadrant 0)
-                    if (quad == 0) {
-                        for (int k = 0; k < nch; k += 2) {
-                            uint32_t r0[16], r1[16];
-                            load2(k, r0, r1);
-                            if (lane == 0) {
+            // ---- rare path: some p of columns [c0, c0 + w) exceeded 2^8 (or
+            // overflowed).  Raise those columns' reference max to this tile's
+            // maxima (raw scores reloaded from TMEM), rescale the running O_A^T
+            // and sums, and recompute p.
+            auto rescale = [&](int t, int c0, int w, uint32_t dcol, int lim) -> bool {
+                while (cv_next < t)   // P tiles written against the old reference go first
+                    if (!convert(cv_next++)) return false;
+                if (!p_drain(0) || !p_drain(1)) return false;
+                if (et < w) sm.cmax[c0 + et] = ord_enc(-INFINITY);
+                uint32_t r[32];
+                tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                tc::tmem_wait_ld();
+                grp_sync<DT_BAR_S>();
 #pragma unroll
-                                for (int v = 0; v < 16; ++v) sm.cref[c_first + 32 * k + v] = __uint_as_float(r0[v]) * kscale;
-                                if (k + 1 < nch)
-#pragma unroll
-                                    for (int v = 0; v < 16; ++v)
-                                        sm.cref[c_first + 32 * (k + 1) + v] = __uint_as_float(r1[v]) * kscale;
-                            }
-                        }
-                    }
-                    ebar();
+                for (int v = 0; v < 32; ++v) {
+                    if (v >= w) break;
+                    float x = v < lim ? __uint_as_float(r[v]) * kscale : -INFINITY;
+                    for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+                    if (lane == 0) atomicMax(&sm.cmax[c0 + v], ord_enc(x));
                 }
-                int over = 0;
-                for (int k = 0; k < nch; k += 2) {
-                    uint32_t r0[16], r1[16];
-                    load2(k, r0, r1);
-#pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        const int q0 = c_first + 32 * k + v, q1 = q0 + 32;
-                        if (valid && q0 < nq && __uint_as_float(r0[v]) * kscale > sm.cref[q0] + DT_RESCALE) over = 1;
-                        if (valid && k + 1 < nch && q1 < nq && __uint_as_float(r1[v]) * kscale > sm.cref[q1] + DT_RESCALE)
-                            over = 1;
-                    }
+                grp_sync<DT_BAR_S>();
+                if (et < w) {
+                    const int c = c0 + et;
+                    const float cn = fmaxf(sm.cref[c], ord_dec(sm.cmax[c]));
+                    const float f = dt_ex2(sm.cref[c] - cn);
+                    sm.cscale[c] = f;
+                    sm.cref[c] = cn;
+                    sm.lsum[c] *= f;
                 }
-                if (any_all(over)) {
-                    // rare path: exact column maxima of this tile, rescale running state
-                    for (int k = 0; k < nch; ++k) {
-                        uint32_t r0[16];
-                        tc::tmem_ld16(tmem + DT_COL_D2 + lane_off + c_first + 32 * k, r0);
+                grp_sync<DT_BAR_S>();
+                if (pv_issued > 0) {   // O_A^T columns (every rank lane) times 2^(cref_old - cref_new)
+                    tc::tc_fence_after();
+                    for (int h = 0; h < w; h += 16) {
+                        uint32_t o[16];
+                        tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + h, o);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) {
-                            float x = valid ? __uint_as_float(r0[v]) * kscale : -INFINITY;
-                            for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-                            if (lane == 0) sm.wred[quad][c_first + 32 * k + v] = x;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t wv[8];
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                wv[v] = __float_as_uint(__uint_as_float(o[8 * hh + v]) * sm.cscale[c0 + h + 8 * hh + v]);
+                            tc::tmem_st8(tmem + DT_COL_OA + lane_off + c0 + h + 8 * hh, wv);
                         }
                     }
-                    ebar();
-                    if (et < nq16) {
-                        const float m = fmaxf(fmaxf(sm.wred[0][et], sm.wred[1][et]), fmaxf(sm.wred[2][et], sm.wred[3][et]));
-                        sm.cnew[et] = fmaxf(sm.cref[et], m);
-                    }
-                    ebar();
-                    if (t > 0) {   // O_A^T columns (all rank lanes) scaled by 2^(cref - cnew)
-                        for (int k = 0; k < nch; ++k) {
-                            const int c0 = c_first + 32 * k;
-                            uint32_t o[16];
-                            tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, o);
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
+                }
+                return true;
+            };
+
+            // ---- softmax of score tile t: p = 2^(x - cref), fp16, MN-major [t/8][q/8][t%8][q%8]
+            auto softmax = [&](int t) -> bool {
+                const int d2b = g.dbl ? (t & 1) : 0;
+                const uint32_t dcol = tmem + DT_COL_D2 + 64 * d2b + lane_off;
+                if (t == 1) MILO_TRACE_WARP(3);
+                if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.d2_full[d2b], u2[d2b] & 1u))) return false;
+                if (t == 1) MILO_TRACE_WARP(4);
+                ++u2[d2b];
+                MILO_TRACE_EVENT(1, 2 + 2 * t);
+                tc::tc_fence_after();
+                const int tok = t * FTILE + row;
+                const bool valid = tok < Tb;
+                if (t == 0) {   // reference max: the scores of the item's first token
+                    sm.lsum[et] = 0.f;
+                    if (quad == 0) {
+                        for (int c0 = 0; c0 < nq16; c0 += 16) {
+                            uint32_t r[16];
+                            tc::tmem_ld16(dcol + c0, r);
                             tc::tmem_wait_ld();
-                            uint32_t w[8];
-                            #pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                #pragma unroll
-                                for (int v = 0; v < 8; ++v) {
-                                    const int q = c0 + hh * 8 + v;
-                                    w[v] = __float_as_uint(__uint_as_float(o[hh * 8 + v]) * ex2(sm.cref[q] - sm.cnew[q]));
+                            if (lane == 0)
+#pragma unroll
+                                for (int v = 0; v < 16; ++v) sm.cref[c0 + v] = __uint_as_float(r[v]) * kscale;
+                        }
+                    }
+                    grp_sync<DT_BAR_S>();
+                }
+                MILO_TRACE_EVENT(1, 16 + 8 * t);
+                const int pb = g.dbl ? (t & 1) : 0;
+                uint8_t *pbase = sm.pbuf + pb * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
+                bool p_ready = false;
+                for (int c0 = 0; c0 < nq16; c0 += 32) {
+                    const int w = min(32, nq16 - c0);
+                    const int lim = valid ? min(w, nq - c0) : 0;   // this token's live columns
+                    // raw scores, turned into p in place
+                    float pv[32];
+                    tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pv[0]));
+                    if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pv[16]));
+                    tc::tmem_wait_ld();
+                    if (c0 == 0) MILO_TRACE_EVENT(1, 17 + 8 * t);
+                    if (c0 == 32) MILO_TRACE_EVENT(1, 21 + 8 * t);
+                    {
+                        // p = 2^(x - cref); more than 2^8 (or an overflow) sends the
+                        // group down the rare path
+                        const float4 *c4 = reinterpret_cast<const float4 *>(sm.cref + c0);
+                        float pmax = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (4 * k >= w) break;
+                            const float4 f = c4[k];
+                            const float cr[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int v = 4 * k + j;
+                                const float e = dt_ex2(pv[v] * kscale - cr[j]);
+                                pv[v] = v < lim ? e : 0.f;
+                                pmax = fmaxf(pmax, pv[v]);
+                            }
+                        }
+                        const bool any_over = grp_or<DT_BAR_S>(!(pmax <= 256.f));
+                        if (c0 == 0) MILO_TRACE_EVENT(1, 18 + 8 * t);
+                        if (any_over) {
+                            MILO_TRACE_EVENT(1, 23 + 8 * t);
+                            if (!rescale(t, c0, w, dcol, lim)) return false;
+                            tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pv[0]));
+                            if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pv[16]));
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int v = 0; v < 32; ++v)
+                                if (v < w) pv[v] = v < lim ? dt_ex2(pv[v] * kscale - sm.cref[c0 + v]) : 0.f;
+                        }
+                    }
+                    if (c0 + 32 >= nq16) {   // every score of the tile has been used
+                        tc::tc_fence_before();
+                        tc::mbar_arrive(&sm.d2_empty[d2b]);
+                    }
+                    if (!p_ready) {   // the P buffer's previous product has completed
+                        // (at an item's start both halves: the previous item may have
+                        // used the buffer at the other width)
+                        if (t == 0) {
+                            if (!p_drain(0) || !p_drain(1)) return false;
+                        } else if (!p_drain(pb)) {
+                            return false;
+                        }
+                        p_ready = true;
+                        MILO_TRACE_EVENT(1, 19 + 8 * t);
+                    }
+                    // fp16 P, MN-major [t/8][q/8][t%8][q%8]
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (16 * hh >= w) break;
+                        const int ch = c0 + 16 * hh;
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const __half2 hb = __floats2half2_rn(pv[16 * hh + 2 * v], pv[16 * hh + 2 * v + 1]);
+                            pk[v] = *reinterpret_cast<const uint32_t *>(&hb);
+                        }
+                        uint8_t *dst = pbase + (ch >> 3) * 128;
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        if (!g.ones) {
+                            // no spare rank row: column sums of the rounded P by a
+                            // transposing butterfly; lanes 2c and 2c+1 end with column c
+                            float sv[16];
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                const float2 pr = __half22float2(*reinterpret_cast<const __half2 *>(&pk[v]));
+                                sv[2 * v] = pr.x;
+                                sv[2 * v + 1] = pr.y;
+                            }
+#pragma unroll
+                            for (int sz = 8, bit = 16; sz >= 1; sz >>= 1, bit >>= 1) {
+                                const bool hi = lane & bit;
+#pragma unroll
+                                for (int j = 0; j < sz; ++j) {
+                                    const float send = hi ? sv[j] : sv[j + sz];
+                                    const float keep = hi ? sv[j + sz] : sv[j];
+                                    sv[j] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
                                 }
-                                tc::tmem_st8(tmem + DT_COL_OA + lane_off + c0 + hh * 8, w);
                             }
-                        }
-                        tc::tmem_wait_st();
-                        if (et < nq16) sm.lsum[et] *= ex2(sm.cref[et] - sm.cnew[et]);
-                    }
-                    ebar();
-                    if (et < nq16) sm.cref[et] = sm.cnew[et];
-                    ebar();
-                }
-                // p = 2^(x - cref), fp16, MN-major [t/8][q/8][t%8][q%8]
-                for (int k2 = 0; k2 < nch; k2 += 2) {
-                  uint32_t rr[2][16];
-                  load2(k2, rr[0], rr[1]);
-#pragma unroll
-                  for (int kk = 0; kk < 2; ++kk) {
-                    const int k = k2 + kk;
-                    if (k >= nch) break;
-                    const uint32_t(&rk)[16] = rr[kk];
-                    const int c0 = c_first + 32 * k;
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        float p2[2];
-#pragma unroll
-                        for (int w2 = 0; w2 < 2; ++w2) {
-                            const int q = c0 + 2 * v + w2;
-                            p2[w2] = (valid && q < nq) ? ex2(__uint_as_float(rk[2 * v + w2]) * kscale - sm.cref[q]) : 0.f;
-                        }
-                        const __half2 hb = __floats2half2_rn(p2[0], p2[1]);
-                        pk[v] = *reinterpret_cast<const uint32_t *>(&hb);
-                        if (!ones) {   // no spare rank row: column sums of the rounded P
-                            const float2 pr = __half22float2(hb);
-                            float s0 = pr.x, s1 = pr.y;
-                            for (int o = 16; o; o >>= 1) {
-                                s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-                                s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-                            }
-                            if (lane == 0) {
-                                atomicAdd(&sm.lsum[c0 + 2 * v], s0);
-                                atomicAdd(&sm.lsum[c0 + 2 * v + 1], s1);
-                            }
+                            sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
+                            if (!(lane & 1)) atomicAdd(&sm.lsum[ch + ((lane >> 1) & 15)], sv[0]);
                         }
                     }
-                    uint8_t *dst = sm.pbuf + (row >> 3) * lbo_p + (c0 >> 3) * 128 + (row & 7) * 16;
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                  }
+                    if (c0 == 0) MILO_TRACE_EVENT(1, 20 + 8 * t);
                 }
-                tc::tc_fence_before();
-                tc::mbar_arrive(&sm.d2_empty);
-                ++n_d2;
+                MILO_TRACE_EVENT(1, 3 + 2 * t);
                 return true;
             };
 
-            // ---- A_V tile to fp16 in place, then hand P and the tile to the PV
-            // product.  Runs after the next RoPE: the tile's ring slot may only
-            // be refilled once the last rebuild of this block has been issued.
-            auto release_p = [&](int t) -> bool {
-                const uint32_t av = aV0 + t;
-                if (!all_ok(tc::mbar_wait(&sm.full[av % DT_STAGES], (av / DT_STAGES) & 1u))) return false;
-                uint32_t *w = reinterpret_cast<uint32_t *>(sm.stage[av % DT_STAGES]);
-                for (int e = et; e < R8V * 64; e += DT_EPI) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                    const __half2 h2 = __floats2half2_rn(f.x, f.y);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                tc::fence_async_smem();
-                ebar();
-                if (et == 0) tc::mbar_arrive(&sm.p_full);
-                ++n_p;
-                MILO_TRACE_EVENT(7 + 4 * t);
-                return true;
-            };
-
-            if (et < nq16) sm.lsum[et] = 0.f;
-            ebar();
-            ok = rope(0);
-            if (ok && nt > 1) ok = rope(1);
-            for (int t = 0; t < nt && ok; ++t) {
+            for (int t = 0; t < g.nt && ok; ++t) {
                 ok = softmax(t);
-                if (ok && t + 2 < nt) ok = rope(t + 2);
-                if (ok) ok = release_p(t);
+                // the item's last scores are done: the query tile is free for the
+                // next item's queries
+                if (ok && t == g.nt - 1 && i + stride < n_items) ok = qprep(i + stride, n + 1);
+                // A_V tiles hand P over; with two P buffers the first waits one
+                // tile so that its A_V tile has time to land
+                const int target = (g.dbl && t == 0 && g.nt > 1) ? 0 : t + 1;
+                while (ok && cv_next < target) ok = convert(cv_next++);
             }
+            if (ok) ok = convert(g.nt);   // B_V
             if (!ok) break;
-            {   // B_V (bf16, landed in its stage) to fp16 in place, while the last PV runs
-                const uint32_t s = aBV % DT_STAGES;
-                if (!(ok = all_ok(tc::mbar_wait(&sm.full[s], (aBV / DT_STAGES) & 1u)))) break;
-                uint32_t *w = reinterpret_cast<uint32_t *>(sm.stage[s]);
-                for (int e = et; e < R8V * 64; e += DT_EPI) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                    const __half2 h2 = __floats2half2_rn(f.x, f.y);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-            }
+
             // ---- O_A^T finished: denominators, O_A / l to fp16 staging
-            {
-                const bool w1 = tc::mbar_wait(&sm.oa_full, n_oa & 1u);
-                const bool w2 = w1 && tc::mbar_wait(&sm.p_empty, (n_p & 1u) ^ 1u);   // last PV done
-                if (!(ok = all_ok(w2))) break;
-            }
-            MILO_TRACE_EVENT(20);
+            ok = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.oa_full, 0));
+            if (!ok) break;
+            MILO_TRACE_EVENT(1, 12);
             tc::tc_fence_after();
-            if (ones && quad == 3) {   // the ones row (rank lane 127) holds sum_t p
-                for (int c0 = c_first; c0 < nq16; c0 += 32) {
+            if (g.ones && quad == (g.R8V >> 5)) {   // the ones row holds sum_t p
+                for (int c0 = 0; c0 < nq16; c0 += 16) {
                     uint32_t r[16];
                     tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
                     tc::tmem_wait_ld();
-                    if (lane == 31)
-                        #pragma unroll
-                        for (int v = 0; v < 16; ++v) sm.lsum[c0 + v] += __uint_as_float(r[v]);
+                    if (row == g.R8V)
+#pragma unroll
+                        for (int v = 0; v < 16; ++v) sm.lsum[c0 + v] = __uint_as_float(r[v]);
                 }
             }
-            ebar();
-            if (et < nq16) sm.cnew[et] = (et < nq && sm.lsum[et] > 0.f) ? __frcp_rn(sm.lsum[et]) : 0.f;
-            ebar();
-            for (int c0 = c_first; c0 < nq16; c0 += 32) {
-                uint32_t r[16];
-                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
-                tc::tmem_wait_ld();
-                if (row < R16V) {
-                    uint32_t pk[8];
-                    #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        float o2[2];
-                        #pragma unroll
-                        for (int w2 = 0; w2 < 2; ++w2) o2[w2] = __uint_as_float(r[2 * v + w2]) * sm.cnew[c0 + 2 * v + w2];
-                        const __half2 hh = __floats2half2_rn(o2[0], o2[1]);
-                        pk[v] = *reinterpret_cast<const uint32_t *>(&hh);
+            grp_sync<DT_BAR_S>();
+            if (et < nq16) sm.cscale[et] = (et < nq && sm.lsum[et] > 0.f) ? __frcp_rn(sm.lsum[et]) : 0.f;
+            const int pst = g.dbl ? (g.nt & 1) : 0;
+            if (!p_drain(pst)) { ok = false; break; }
+            grp_sync<DT_BAR_S>();
+            if (quad * 32 < g.R16V) {
+                uint8_t *sbase = sm.pbuf + pst * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
+                for (int c0 = 0; c0 < nq16; c0 += 16) {
+                    uint32_t r[16];
+                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
+                    tc::tmem_wait_ld();
+                    if (row < g.R16V) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const __half2 hh = __floats2half2_rn(__uint_as_float(r[2 * v]) * sm.cscale[c0 + 2 * v],
+                                                                 __uint_as_float(r[2 * v + 1]) * sm.cscale[c0 + 2 * v + 1]);
+                            pk[v] = *reinterpret_cast<const uint32_t *>(&hh);
+                        }
+                        uint8_t *dst = sbase + (c0 >> 3) * 128;
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
-                    uint8_t *dst = sm.pbuf + (row >> 3) * lbo_p + (c0 >> 3) * 128 + (row & 7) * 16;
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            ebar();
-            if (et == 0) tc::mbar_arrive(&sm.oa_staged);
-            MILO_TRACE_EVENT(21);
-            ++n_oa;
-            ++n_p;   // the O product's commit frees the staging buffer
+            tc::mbar_arrive(&sm.p_full[pst]);
+            ++pf[pst];
             // ---- O (lanes = channels, columns = queries) to the partials
-            if (!(ok = all_ok(tc::mbar_wait(&sm.d1_full, n_d1 & 1u)))) break;
-            MILO_TRACE_EVENT(22);
+            ok = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.oa_full, 1));
+            if (!ok) break;
+            MILO_TRACE_EVENT(1, 13);
             tc::tc_fence_after();
-            for (int c0 = c_first; c0 < nq16; c0 += 32) {
+            const int *qp = sm.qpidx[n & 1u];
+            for (int c0 = 0; c0 < nq16; c0 += 16) {
                 uint32_t r[16];
-                tc::tmem_ld16(tmem + DT_COL_D1 + lane_off + c0, r);
+                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
                 tc::tmem_wait_ld();
-                #pragma unroll
-                for (int v = 0; v < 16; ++v) {
-                    const int q = c0 + v;
-                    if (q < nq) a.part_o[(int64_t)sm.qpidx[q] * D + row] = __uint_as_float(r[v]);
-                }
+#pragma unroll
+                for (int v = 0; v < 16; ++v)
+                    if (c0 + v < nq) a.part_o[(int64_t)qp[c0 + v] * D + row] = __uint_as_float(r[v]);
             }
-            if (et < nq) a.part_ml[sm.qpidx[et]] = make_float2(sm.cref[et] * 0.69314718055994531f, sm.lsum[et]);
+            if (et < nq) a.part_ml[qp[et]] = make_float2(sm.cref[et] * 0.69314718055994531f, sm.lsum[et]);
             tc::tc_fence_before();
-            tc::mbar_arrive(&sm.d1_empty);
-            ++n_d1;
-            ebar();
-            MILO_TRACE_EVENT(23);
+            tc::mbar_arrive(&sm.oa_free);
+            seqA0 += dt_ring_tiles(g);
+            // one group-wide decision per item (also orders this item's reads of
+            // cref / lsum before the next item's writes)
+            ok = grp_and<DT_BAR_S>(!sm.abort);
+            MILO_TRACE_EVENT(1, 14);
         }
         if (!ok) sm.abort = 1;
     }

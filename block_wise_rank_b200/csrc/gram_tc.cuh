@@ -34,8 +34,8 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 k_gram_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, float *__restrict__ G_out,
           int64_t n_blk, int n_b, int Tn, int block_len) {
     extern __shared__ __align__(1024) unsigned char gt_raw[];
-    GramTcSmem &sm = *reinterpret_cast<GramTcSmem *>(
-        (reinterpret_cast<uintptr_t>(gt_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // aligned by pointer arithmetic: the compiler keeps the shared address space
+    GramTcSmem &sm = *reinterpret_cast<GramTcSmem *>(gt_raw + ((1024u - (tc::smem_u32(gt_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_items = 2 * n_blk;
     const int chunks = block_len / GT_CHUNK;
