@@ -22,12 +22,14 @@
 //                   thread: rotates each rebuilt key row by its in-block angle
 //                   t*theta_i and packs K-tilde to fp16 in place.  Two rebuild
 //                   buffers let it run up to two tiles ahead of the scores.
-//   softmax group   4 warps: rotates the queries by -p*theta_i; softmax in the
-//                   exp2 domain against a per-query reference max that is
-//                   raised (with the running O_A^T and sums rescaled) only
-//                   when a score exceeds it by more than 2^8; P (fp16) to
-//                   shared memory; each A_V tile converted to fp16 in place;
-//                   O_A / l staged for the last product; O to the partials.
+//   softmax group   4 warps: softmax in the exp2 domain against a per-query
+//                   reference max that is raised (with the running O_A^T and
+//                   sums rescaled) only when a score exceeds it by more than
+//                   2^8; P (fp16) to shared memory; O_A / l staged for the
+//                   last product; O to the partials.
+//   helper warps    2 warps: convert each A_V tile and B_V to fp16 in place as
+//                   they land; rotate the next item's queries by -p*theta_i
+//                   once the current item's scores are done.
 //
 // The ones row makes the PV product return the softmax denominators as one
 // more row of O_A^T.  Keys and values are never written to memory.  Each
@@ -47,11 +49,19 @@
 #ifndef MILO_TRACE_WARP
 #define MILO_TRACE_WARP(id)
 #endif
+#ifndef MILO_TRACE_WAIT
+#define MILO_TRACE_WAIT(dist, reuse, overlap)
+#endif
+#ifndef MILO_TRACE_TILE
+#define MILO_TRACE_TILE(role, n, k)
+#endif
+
 
 namespace milo {
 
 constexpr int DT_GROUP = 128;                          // threads per epilogue group
-constexpr int DT_THREADS = 64 + 2 * DT_GROUP;          // warp 0 producer, 1 MMA, 2-5 RoPE, 6-9 softmax
+constexpr int DT_HELP = 64;                            // helper threads
+constexpr int DT_THREADS = 64 + 2 * DT_GROUP + DT_HELP; // warp 0 producer, 1 MMA, 2-5 RoPE, 6-9 softmax, 10-11 helpers
 constexpr int DT_RING = 96 * 1024;                     // ring bytes for A_K, A_V and B_V tiles
 constexpr int DT_NBAR = 32;                            // ring tiles in flight at most
 constexpr int DT_TILE_MAX = 128 * 256;                 // 128 rank rows x 128 tokens (or channels) x 16 bit
@@ -61,7 +71,7 @@ constexpr uint32_t DT_COL_D1 = 0;                      // two 128-column rebuild
 constexpr uint32_t DT_COL_D2 = 256;                    // scores: one 128-column buffer or two of 64
 constexpr uint32_t DT_COL_OA = 384;                    // O_A^T, then O
 constexpr float DT_RESCALE = 8.f;                      // log2 headroom before the reference max moves
-constexpr int DT_BAR_S = 1, DT_BAR_R = 2;              // named barriers of the two groups
+constexpr int DT_BAR_S = 1, DT_BAR_R = 2, DT_BAR_H = 3; // named barriers of the groups
 
 // One work item, written by k_dt_items.
 struct DtItem {
@@ -85,9 +95,12 @@ struct DecTcSmem {
     float cscale[DT_NQ];                         // rescale factors, then 1 / l
     float lsum[DT_NQ];
     int cmax[DT_NQ];                             // column maxima, order-preserving int encoding
-    int qpidx[2][DT_NQ];                         // partial index of each query, per item parity
+    int qpidx[4][DT_NQ];                         // partial index of each query, per item (mod 4)
     uint32_t toff[DT_NBAR], tlen[DT_NBAR];       // ring offset and bytes of each tile in flight
-    uint64_t full[DT_NBAR], empty[DT_NBAR];
+    // conv: one arrival per ring tile, in ring order, once an A_V / B_V tile
+    // is fp16 (A_K tiles pass straight through), so that slot k % NBAR is in
+    // phase k / NBAR exactly like full and empty
+    uint64_t full[DT_NBAR], empty[DT_NBAR], conv[DT_NBAR];
     uint64_t bk_full, bk_empty;
     uint64_t d1_full[2], d1_empty[2], kt_full[2];
     uint64_t d2_full[2], d2_empty[2];
@@ -157,33 +170,47 @@ __device__ __forceinline__ DtGeo dt_geo(const DtItem *__restrict__ items, int64_
     return dt_geo(__ldg(&items[i].Tb), __ldg(&items[i].rK), __ldg(&items[i].rV), __ldg(&items[i].nq));
 }
 
-// ring tiles of an item: A_K 0..nt-1, A_V 0..nt-1, B_V
+// Ring tiles of an item, 2 nt + 1 of them, in the order they are consumed:
+// A_V(t) follows A_K(t + 2) (the rebuilds run two tiles ahead of the PV
+// products), B_V comes last:  A_K0 A_K1 A_K2 A_V0 A_K3 A_V1 A_V2 A_V3 B_V.
 __device__ __forceinline__ int dt_ring_tiles(const DtGeo &g) { return 2 * g.nt + 1; }
+__host__ __device__ __forceinline__ int dt_pos_k(int t) { return t + (t > 2 ? t - 2 : 0); }
+__host__ __device__ __forceinline__ int dt_pos_v(int nt, int t) { return (t + 3 < nt ? t + 3 : nt) + t; }
+// kind of ring position k: 0 = A_K, 1 = A_V, 2 = B_V; *t = its tile
+__host__ __device__ __forceinline__ int dt_tile_at(int nt, int k, int *t) {
+    if (k == 2 * nt) { *t = nt; return 2; }
+    for (int u = 0; u < nt; ++u) {
+        if (dt_pos_k(u) == k) { *t = u; return 0; }
+        if (dt_pos_v(nt, u) == k) { *t = u; return 1; }
+    }
+    *t = 0;
+    return 0;
+}
 
 // named-barrier helpers for one 128-thread group
-template <int ID>
+template <int ID, int N = DT_GROUP>
 __device__ __forceinline__ void grp_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(DT_GROUP) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
 }
-template <int ID>
+template <int ID, int N = DT_GROUP>
 __device__ __forceinline__ bool grp_and(bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
         "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v), "n"(ID), "n"(DT_GROUP)
+        : "r"((uint32_t)v), "n"(ID), "n"(N)
         : "memory");
     return r != 0;
 }
-template <int ID>
+template <int ID, int N = DT_GROUP>
 __device__ __forceinline__ bool grp_or(bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
         "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v), "n"(ID), "n"(DT_GROUP)
+        : "r"((uint32_t)v), "n"(ID), "n"(N)
         : "memory");
     return r != 0;
 }
@@ -241,7 +268,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
     const int64_t stride = gridDim.x;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DT_NBAR; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
+        for (int s = 0; s < DT_NBAR; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.empty[s], 1);
+            tc::mbar_init(&sm.conv[s], 1);
+        }
         tc::mbar_init(&sm.bk_full, 1);
         tc::mbar_init(&sm.bk_empty, 1);
         for (int k = 0; k < 2; ++k) {
@@ -253,7 +284,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             tc::mbar_init(&sm.p_full[k], DT_GROUP);
             tc::mbar_init(&sm.p_empty[k], 1);
         }
-        tc::mbar_init(&sm.q_full, DT_GROUP);
+        tc::mbar_init(&sm.q_full, DT_HELP);
         tc::mbar_init(&sm.q_empty, 1);
         tc::mbar_init(&sm.oa_full, 1);
         tc::mbar_init(&sm.oa_free, DT_GROUP);
@@ -283,23 +314,31 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // ================================================================ producer
         const uint8_t *dataK = (const uint8_t *)a.kv[0].data;
         const uint8_t *dataV = (const uint8_t *)a.kv[1].data;
-        uint32_t head = 0, seq = 0, live = 0;   // live: bit s % NBAR set while tile s may be unconsumed
+        // The ring is a FIFO byte buffer: tiles are placed at `head` (or at 0
+        // when they would cross the end) and released oldest first; `tail`
+        // is the oldest tile not yet seen released.
+        uint32_t head = 0, seq = 0, tail = 0;
+        uint32_t trace_n = 0;
+        int trace_k = 0;
+        (void)trace_n;
+        (void)trace_k;
         bool ok = true;
-        // room for a tile of `bytes` in the ring: lane 0 waits for the
-        // barrier slot's previous tile and for every live tile overlapping
-        // the new one (all older, so all freed without this one); the warp
-        // follows.  Returns the tile's offset.
+        // room for a tile of `bytes`: lane 0 releases tiles from the tail
+        // (all older than the new tile, so all released without it) until the
+        // bytes are free and a barrier slot is; the warp follows.  Returns
+        // the tile's offset.
         auto place = [&](uint32_t bytes) -> uint32_t {
             const uint32_t off = head + bytes > (uint32_t)DT_RING ? 0u : head;
             if (lane == 0) {
-                for (uint32_t k = seq >= DT_NBAR ? seq - DT_NBAR : 0; k < seq && ok; ++k) {
-                    const uint32_t s = k % DT_NBAR;
-                    if (!((live >> s) & 1u)) continue;
-                    const bool slot_reuse = k + DT_NBAR == seq;
-                    const bool overlap = sm.toff[s] < off + bytes && off < sm.toff[s] + sm.tlen[s];
-                    if (!slot_reuse && !overlap) continue;
-                    if (!tc::mbar_wait(&sm.empty[s], (k / DT_NBAR) & 1u)) { ok = false; break; }
-                    live &= ~(1u << s);
+                while (ok && tail < seq) {
+                    const uint32_t t0 = sm.toff[tail % DT_NBAR];   // oldest live byte
+                    // live bytes run from t0 up to head, circularly
+                    const bool room = t0 < head ? (off == head || off + bytes <= t0)
+                                                : (off >= head && off + bytes <= t0);
+                    if (room && seq - tail < DT_NBAR) break;
+                    MILO_TRACE_WAIT(seq - tail, 0, 1);
+                    if (!tc::mbar_wait(&sm.empty[tail % DT_NBAR], (tail / DT_NBAR) & 1u)) { ok = false; break; }
+                    ++tail;
                 }
                 const uint32_t s = seq % DT_NBAR;
                 sm.toff[s] = off;
@@ -323,6 +362,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         auto ring_tile = [&](const uint8_t *src, int rows, int copy, bool ones) {
             const uint32_t off = place((uint32_t)rows * 256u);
             if (!ok) return;
+            if (lane == 0) MILO_TRACE_TILE(3, trace_n, trace_k);
             uint8_t *dst = sm.ring + off;
             if (rows > copy) fill_rows(dst, copy, rows, ones);
             if (lane == 0) {
@@ -331,7 +371,6 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
                 if (bytes) tc::bulk_g2s(dst, src, bytes, &sm.full[s]);
             }
-            live |= 1u << (seq % DT_NBAR);
             ++seq;
         };
         uint32_t n = 0;
@@ -341,7 +380,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             const DtGeo g = dt_geo(it.Tb, it.rK, it.rV, it.nq);
             const uint8_t *bK = dataK + 2 * it.offK, *bV = dataV + 2 * it.offV;
             const int64_t tileK = (int64_t)g.R8K * 256, tileV = (int64_t)g.R8V * 256;
-            ring_tile(bK, g.R16K, g.R8K, false);                               // A_K tile 0
+            ring_tile(bK, g.R16K, g.R8K, false);                               // A_K tile 0 (position 0)
             if (!ok) break;
             // B_K into its own buffer once the previous item's rebuilds are done
             if (lane == 0) ok = tc::mbar_wait(&sm.bk_empty, (n & 1u) ^ 1u);
@@ -351,10 +390,20 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             if (lane == 0) {
                 tc::mbar_arrive_expect_tx(&sm.bk_full, (uint32_t)tileK);
                 if (tileK) tc::bulk_g2s(sm.bk, bK + g.nt * tileK, (uint32_t)tileK, &sm.bk_full);
+                MILO_TRACE_TILE(0, n, 15);
             }
-            for (int t = 1; t < g.nt && ok; ++t) ring_tile(bK + t * tileK, g.R16K, g.R8K, false);
-            for (int t = 0; t < g.nt && ok; ++t) ring_tile(bV + t * tileV, g.rowsV, g.R8V, g.ones);
-            if (ok) ring_tile(bV + g.nt * tileV, g.R16V, g.R8V, false);          // B_V
+            MILO_TRACE_TILE(0, n, 0);
+            for (int k = 1; k <= 2 * g.nt && ok; ++k) {
+                int t;
+                const int kind = dt_tile_at(g.nt, k, &t);
+                if (lane == 0) MILO_TRACE_TILE(2, n, k);
+                trace_n = n;
+                trace_k = k;
+                if (kind == 0) ring_tile(bK + t * tileK, g.R16K, g.R8K, false);          // A_K(t)
+                else if (kind == 1) ring_tile(bV + t * tileV, g.rowsV, g.R8V, g.ones);   // A_V(t)
+                else ring_tile(bV + g.nt * tileV, g.R16V, g.R8V, false);                // B_V
+                if (lane == 0) MILO_TRACE_TILE(0, n, k);
+            }
         }
         if (!ok && lane == 0) sm.abort = 1;
         // drain: every copy issued has landed before the CTA exits
@@ -387,7 +436,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 bool prog = false;
                 // ---------------------------------------------------- rebuild
                 if (!doneR) {
-                    const uint32_t k = seqR + tR, s = k % DT_NBAR, b = rc & 1u;
+                    const uint32_t k = seqR + dt_pos_k(tR), s = k % DT_NBAR, b = rc & 1u;
                     if (mbar_test(&sm.full[s], (k / DT_NBAR) & 1u) && (tR > 0 || mbar_test(&sm.bk_full, nR & 1u)) &&
                         mbar_test(&sm.d1_empty[b], ((rc >> 1) & 1u) ^ 1u)) {
                         MILO_TRACE_MMA(nR, tR);
@@ -448,11 +497,14 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     const uint32_t pb = gP.dbl ? (tP & 1u) : 0u;
                     const uint32_t lbo_p = (uint32_t)(gP.nq16 / 8) * 128u;
                     const uint32_t sp = spb + pb * 16384u;
-                    if (mbar_test(&sm.p_full[pb], pu[pb] & 1u) && (tP > 0 || mbar_test(&sm.oa_free, (nP & 1u) ^ 1u))) {
+                    // A_V tile tP, or B_V when tP == nt
+                    const uint32_t kv = seqP + ((int)tP < gP.nt ? dt_pos_v(gP.nt, tP) : 2 * gP.nt);
+                    if (mbar_test(&sm.p_full[pb], pu[pb] & 1u) && mbar_test(&sm.conv[kv % DT_NBAR], (kv / DT_NBAR) & 1u) &&
+                        (tP > 0 || mbar_test(&sm.oa_free, (nP & 1u) ^ 1u))) {
                         tc::tc_fence_after();
                         if ((int)tP < gP.nt) {   // O_A^T += A_V(tile)^T P
                             MILO_TRACE_MMA(nP, 8 + tP);
-                            const uint32_t k = seqP + gP.nt + tP, s = k % DT_NBAR;
+                            const uint32_t k = kv, s = k % DT_NBAR;
                             const uint32_t sa = sring + sm.toff[s];
                             const uint32_t id_pv = tc::idesc_f16(128, gP.nq16, 0, 0, 1);   // fp16, A K-major, B MN-major
                             for (int ks = 0; ks < 8; ++ks)
@@ -466,7 +518,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             ++tP;
                         } else {                 // O = B_V^T (O_A / l), over O_A's columns
                             MILO_TRACE_MMA(nP, 12);
-                            const uint32_t k = seqP + 2 * gP.nt, s = k % DT_NBAR;
+                            const uint32_t k = kv, s = k % DT_NBAR;
                             const uint32_t sa = sring + sm.toff[s];
                             const uint32_t id_o = tc::idesc_f16(128, gP.nq16, 0, 1, 1);    // fp16, A/B MN-major
                             for (int ks = 0; ks < gP.R16V / 16; ++ks)
@@ -493,7 +545,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     if (!sm.abort) raise_status(ST_TIMEOUT);
                     ok = false;
                 } else {
-                    __nanosleep(32);   // leave the issue slots to the group warps
+                    __nanosleep(64);   // leave the issue slots to the group warps
                 }
             }
             if (!ok) sm.abort = 1;
@@ -565,7 +617,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
         }
         if (!ok) sm.abort = 1;
-    } else {
+    } else if (warp < 10) {
         // ================================================================ softmax group
         const int et = threadIdx.x - 192;
         const int quad = warp & 3;
@@ -585,87 +637,21 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             return w;
         };
 
-        // ---- rotated queries R(-p) q of item j, fp16, K-major [q/8][j/8][q%8][j%8];
-        // four threads per query, 16 pairs each
-        auto qprep = [&](int64_t j, uint32_t nj) -> bool {
-            if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.q_empty, (nj & 1u) ^ 1u))) return false;
-            const int nq = __ldg(&items[j].nq), nq16 = (nq + 15) & ~15;
-            const int jl = __ldg(&items[j].l), jh = __ldg(&items[j].h), jq0 = __ldg(&items[j].q0);
-            const int jslot0 = __ldg(&items[j].slot0);
-            for (int u = et; u < 4 * nq16; u += DT_GROUP) {
-                const int qi = u >> 2, part = u & 3;          // pairs 16*part .. 16*part+15
-                uint8_t *qrow = sm.qt + (qi >> 3) * 2048 + (qi & 7) * 16;
-                if (qi < nq) {
-                    const int gq = jq0 + qi;
-                    const int slot = a.slot_list[jslot0 + gq / a.G];
-                    const int g = gq % a.G;
-                    const int s = slot / a.n_sel, jj = slot % a.n_sel;
-                    const int hq = jh * a.G + g;
-                    const int64_t qbase = ((int64_t)jl * a.S + s) * a.Hq + hq;
-                    const float4 *qv = reinterpret_cast<const float4 *>(a.q + qbase * D);
-                    const float4 *cs = reinterpret_cast<const float4 *>(a.rope_q + (int64_t)slot * HALF);
-                    if (part == 0) sm.qpidx[nj & 1u][qi] = (int)(qbase * a.n_sel + jj);
-#pragma unroll 1
-                    for (int h8 = 0; h8 < 2; ++h8) {          // pairs 16*part + 8*h8 .. +7
-                        const int p0 = 16 * part + 8 * h8;
-                        const float4 xa0 = qv[p0 / 4], xa1 = qv[p0 / 4 + 1];
-                        const float4 xb0 = qv[16 + p0 / 4], xb1 = qv[16 + p0 / 4 + 1];
-                        float4 cv[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) cv[k] = cs[p0 / 2 + k];
-                        const float x0[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-                        const float x1[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
-                        uint32_t lo[4], hi[4];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const float4 c2 = cv[v];   // (cos, sin) of pairs p0 + 2v, p0 + 2v + 1
-                            const __half2 h0 = __floats2half2_rn(x0[2 * v] * c2.x + x1[2 * v] * c2.y,
-                                                                 x0[2 * v + 1] * c2.z + x1[2 * v + 1] * c2.w);
-                            const __half2 h1 = __floats2half2_rn(x1[2 * v] * c2.x - x0[2 * v] * c2.y,
-                                                                 x1[2 * v + 1] * c2.z - x0[2 * v + 1] * c2.w);
-                            lo[v] = *reinterpret_cast<const uint32_t *>(&h0);
-                            hi[v] = *reinterpret_cast<const uint32_t *>(&h1);
-                        }
-                        const int g8 = 2 * part + h8;
-                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        *reinterpret_cast<uint4 *>(qrow + (8 + g8) * 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    }
-                } else {
-                    for (int g8 = 4 * part; g8 < 4 * part + 4; ++g8)
-                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            tc::fence_async_smem();
-            tc::mbar_arrive(&sm.q_full);
-            return true;
-        };
-
-        if (blockIdx.x < n_items) ok = qprep(blockIdx.x, 0);
         for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
             const DtGeo g = dt_geo(items, i, n_items);
             const int Tb = __ldg(&items[i].Tb);
             const int nq = g.nq, nq16 = g.nq16;
             const uint32_t lbo_p = (uint32_t)(nq16 / 8) * 128u;
-            int cv_next = 0, pv_issued = 0;
+            int pv_issued = 0;
             MILO_TRACE_EVENT(1, 0);
 
-            // ---- A_V tile tt (B_V when tt == nt) to fp16 in place; an A_V tile
-            // hands its P buffer to the PV product
-            auto convert = [&](int tt) -> bool {
-                const uint32_t k = seqA0 + g.nt + tt, s = k % DT_NBAR;
-                if (tt < 4) MILO_TRACE_EVENT(1, 48 + tt);
-                if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.full[s], (k / DT_NBAR) & 1u))) return false;
-                if (tt < 4) MILO_TRACE_EVENT(1, 52 + tt);
-                bf16_to_f16_inplace(sm.ring + sm.toff[s], g.R8V * 16, et, DT_GROUP);
+            // ---- P tile tt to the PV product (its A_V tile is converted by the helpers)
+            auto handoff = [&](int tt) {
                 tc::fence_async_smem();
-                if (tt < 4) MILO_TRACE_EVENT(1, 56 + tt);
-                if (tt < g.nt) {
-                    const int pb = g.dbl ? (tt & 1) : 0;
-                    tc::mbar_arrive(&sm.p_full[pb]);
-                    ++pf[pb];
-                    ++pv_issued;
-                }
-                return true;
+                const int pb = g.dbl ? (tt & 1) : 0;
+                tc::mbar_arrive(&sm.p_full[pb]);
+                ++pf[pb];
+                ++pv_issued;
             };
 
             // ---- rare path: some p of columns [c0, c0 + w) exceeded 2^8 (or
@@ -673,9 +659,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             // maxima (raw scores reloaded from TMEM), rescale the running O_A^T
             // and sums, and recompute p.
             auto rescale = [&](int t, int c0, int w, uint32_t dcol, int lim) -> bool {
-                while (cv_next < t)   // P tiles written against the old reference go first
-                    if (!convert(cv_next++)) return false;
-                if (!p_drain(0) || !p_drain(1)) return false;
+                (void)t;
+                if (!p_drain(0) || !p_drain(1)) return false;   // every P handed over has been used
                 if (et < w) sm.cmax[c0 + et] = ord_enc(-INFINITY);
                 uint32_t r[32];
                 tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
@@ -852,15 +837,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
 
             for (int t = 0; t < g.nt && ok; ++t) {
                 ok = softmax(t);
-                // the item's last scores are done: the query tile is free for the
-                // next item's queries
-                if (ok && t == g.nt - 1 && i + stride < n_items) ok = qprep(i + stride, n + 1);
-                // A_V tiles hand P over; with two P buffers the first waits one
-                // tile so that its A_V tile has time to land
-                const int target = (g.dbl && t == 0 && g.nt > 1) ? 0 : t + 1;
-                while (ok && cv_next < target) ok = convert(cv_next++);
+                if (ok) handoff(t);
             }
-            if (ok) ok = convert(g.nt);   // B_V
             if (!ok) break;
 
             // ---- O_A^T finished: denominators, O_A / l to fp16 staging
@@ -885,21 +863,29 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             grp_sync<DT_BAR_S>();
             if (quad * 32 < g.R16V) {
                 uint8_t *sbase = sm.pbuf + pst * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
-                for (int c0 = 0; c0 < nq16; c0 += 16) {
-                    uint32_t r[16];
-                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
+                for (int c0 = 0; c0 < nq16; c0 += 32) {
+                    uint32_t r[32];
+                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                    if (c0 + 16 < nq16)
+                        tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
                     tc::tmem_wait_ld();
                     if (row < g.R16V) {
-                        uint32_t pk[8];
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            const __half2 hh = __floats2half2_rn(__uint_as_float(r[2 * v]) * sm.cscale[c0 + 2 * v],
-                                                                 __uint_as_float(r[2 * v + 1]) * sm.cscale[c0 + 2 * v + 1]);
-                            pk[v] = *reinterpret_cast<const uint32_t *>(&hh);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int ch = c0 + 16 * hh;
+                            if (ch >= nq16) break;
+                            uint32_t pk[8];
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                const __half2 h2 = __floats2half2_rn(
+                                    __uint_as_float(r[16 * hh + 2 * v]) * sm.cscale[ch + 2 * v],
+                                    __uint_as_float(r[16 * hh + 2 * v + 1]) * sm.cscale[ch + 2 * v + 1]);
+                                pk[v] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            uint8_t *dst = sbase + (ch >> 3) * 128;
+                            *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                         }
-                        uint8_t *dst = sbase + (c0 >> 3) * 128;
-                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
                 }
             }
@@ -912,13 +898,15 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             if (!ok) break;
             MILO_TRACE_EVENT(1, 13);
             tc::tc_fence_after();
-            const int *qp = sm.qpidx[n & 1u];
-            for (int c0 = 0; c0 < nq16; c0 += 16) {
-                uint32_t r[16];
-                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
+            const int *qp = sm.qpidx[n & 3u];
+            for (int c0 = 0; c0 < nq16; c0 += 32) {
+                uint32_t r[32];
+                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                if (c0 + 16 < nq16)
+                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int v = 0; v < 16; ++v)
+                for (int v = 0; v < 32; ++v)
                     if (c0 + v < nq) a.part_o[(int64_t)qp[c0 + v] * D + row] = __uint_as_float(r[v]);
             }
             if (et < nq) a.part_ml[qp[et]] = make_float2(sm.cref[et] * 0.69314718055994531f, sm.lsum[et]);
@@ -929,6 +917,117 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             // cref / lsum before the next item's writes)
             ok = grp_and<DT_BAR_S>(!sm.abort);
             MILO_TRACE_EVENT(1, 14);
+        }
+        if (!ok) sm.abort = 1;
+    } else {
+        // ================================================================ helper warps
+        const int et = threadIdx.x - (64 + 2 * DT_GROUP);
+        bool ok = true;
+        // ---- rotated queries R(-p) q of item j, fp16, K-major [q/8][j/8][q%8][j%8];
+        // four threads per query, 16 pairs each
+        auto qprep = [&](int64_t j, uint32_t nj) -> bool {
+            if (!grp_and<DT_BAR_H, DT_HELP>(tc::mbar_wait(&sm.q_empty, (nj & 1u) ^ 1u))) return false;
+            const int nq = __ldg(&items[j].nq), nq16 = (nq + 15) & ~15;
+            const int jl = __ldg(&items[j].l), jh = __ldg(&items[j].h), jq0 = __ldg(&items[j].q0);
+            const int jslot0 = __ldg(&items[j].slot0);
+            for (int u = et; u < 4 * nq16; u += DT_HELP) {
+                const int qi = u >> 2, part = u & 3;          // pairs 16*part .. 16*part+15
+                uint8_t *qrow = sm.qt + (qi >> 3) * 2048 + (qi & 7) * 16;
+                if (qi < nq) {
+                    const int gq = jq0 + qi;
+                    const int slot = a.slot_list[jslot0 + gq / a.G];
+                    const int g = gq % a.G;
+                    const int s = slot / a.n_sel, jj = slot % a.n_sel;
+                    const int hq = jh * a.G + g;
+                    const int64_t qbase = ((int64_t)jl * a.S + s) * a.Hq + hq;
+                    const float4 *qv = reinterpret_cast<const float4 *>(a.q + qbase * D);
+                    const float4 *cs = reinterpret_cast<const float4 *>(a.rope_q + (int64_t)slot * HALF);
+                    if (part == 0) sm.qpidx[nj & 3u][qi] = (int)(qbase * a.n_sel + jj);
+#pragma unroll 1
+                    for (int h8 = 0; h8 < 2; ++h8) {          // pairs 16*part + 8*h8 .. +7
+                        const int p0 = 16 * part + 8 * h8;
+                        const float4 xa0 = qv[p0 / 4], xa1 = qv[p0 / 4 + 1];
+                        const float4 xb0 = qv[16 + p0 / 4], xb1 = qv[16 + p0 / 4 + 1];
+                        float4 cv[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) cv[k] = cs[p0 / 2 + k];
+                        const float x0[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+                        const float x1[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+                        uint32_t lo[4], hi[4];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const float4 c2 = cv[v];   // (cos, sin) of pairs p0 + 2v, p0 + 2v + 1
+                            const __half2 h0 = __floats2half2_rn(x0[2 * v] * c2.x + x1[2 * v] * c2.y,
+                                                                 x0[2 * v + 1] * c2.z + x1[2 * v + 1] * c2.w);
+                            const __half2 h1 = __floats2half2_rn(x1[2 * v] * c2.x - x0[2 * v] * c2.y,
+                                                                 x1[2 * v + 1] * c2.z - x0[2 * v + 1] * c2.w);
+                            lo[v] = *reinterpret_cast<const uint32_t *>(&h0);
+                            hi[v] = *reinterpret_cast<const uint32_t *>(&h1);
+                        }
+                        const int g8 = 2 * part + h8;
+                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        *reinterpret_cast<uint4 *>(qrow + (8 + g8) * 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    }
+                } else {
+                    for (int g8 = 4 * part; g8 < 4 * part + 4; ++g8)
+                        *reinterpret_cast<uint4 *>(qrow + g8 * 128) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            tc::fence_async_smem();
+            tc::mbar_arrive(&sm.q_full);
+            return true;
+        };
+
+        // Two independent streams, served whichever is ready: the ring tiles
+        // in order (A_K tiles pass, A_V tiles and B_V to fp16 in place), and
+        // each next item's queries once the current item's scores are done.
+        int64_t ic = blockIdx.x, iq = blockIdx.x;
+        uint32_t seqC = 0, nqp = 0;
+        int kc = 0;
+        DtGeo gc = dt_geo(items, ic, n_items);
+        uint64_t t_last = tc::globaltimer();
+        while (ok && (ic < n_items || iq < n_items)) {
+            bool did = false;
+            if (ic < n_items) {
+                int tt;
+                const int kind = dt_tile_at(gc.nt, kc, &tt);
+                const uint32_t k = seqC + kc, s = k % DT_NBAR;
+                bool go = kind == 0;
+                if (!go) go = grp_and<DT_BAR_H, DT_HELP>(mbar_test(&sm.full[s], (k / DT_NBAR) & 1u));
+                if (go) {
+                    if (kind != 0) {
+                        bf16_to_f16_inplace(sm.ring + sm.toff[s], gc.R8V * 16, et, DT_HELP);
+                        tc::fence_async_smem();
+                        grp_sync<DT_BAR_H, DT_HELP>();
+                    }
+                    if (et == 0) tc::mbar_arrive(&sm.conv[s]);
+                    if (et == 0) MILO_TRACE_TILE(1, (uint32_t)((ic - blockIdx.x) / stride), kc);
+                    if (++kc == dt_ring_tiles(gc)) {
+                        seqC += dt_ring_tiles(gc);
+                        kc = 0;
+                        ic += stride;
+                        gc = dt_geo(items, ic, n_items);
+                    }
+                    did = true;
+                }
+            }
+            if (iq < n_items && grp_and<DT_BAR_H, DT_HELP>(mbar_test(&sm.q_empty, (nqp & 1u) ^ 1u))) {
+                ok = qprep(iq, nqp);
+                if (et == 0) MILO_TRACE_TILE(1, nqp, 14);
+                iq += stride;
+                ++nqp;
+                did = true;
+            }
+            if (did) {
+                t_last = tc::globaltimer();
+            } else {
+                const bool stop = grp_or<DT_BAR_H, DT_HELP>(sm.abort || tc::globaltimer() - t_last > 2000000000ull);
+                if (stop) {
+                    if (!sm.abort) raise_status(ST_TIMEOUT);
+                    ok = false;
+                }
+                __nanosleep(256);
+            }
         }
         if (!ok) sm.abort = 1;
     }

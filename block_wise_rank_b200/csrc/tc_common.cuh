@@ -29,17 +29,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  "r"(bytes)
                  : "memory");
 }
-// try_wait with a suspend-time hint: the thread sleeps (up to the hint, in
-// ns) until the phase completes instead of spinning, so waiting warps leave
-// their scheduler's issue slots to the warps doing work.
+// try_wait without a suspend-time hint: the thread may be parked for the
+// hardware's own short limit.  (With a long hint, a thread waiting for an
+// arrival made by tcgen05.commit was measured to resume microseconds late.)
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -51,8 +51,19 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // Wait for the phase with this parity to complete.  Gives up after ~2 s of
 // wall time, raises ST_TIMEOUT and returns false, so that a broken pipeline
 // ends the kernel instead of hanging the GPU.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;   // already complete: no suspend round trip
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
