@@ -66,19 +66,53 @@ __global__ void k_slot_count(const int32_t *__restrict__ sel, int n_slots, int n
 
 // starts of each block id's slot list, and of its query passes (a pass is up
 // to `pass_q` queries = selecting slots times the GQA group)
-__global__ void k_slot_scan(int32_t *__restrict__ cnt, int32_t *__restrict__ start, int32_t *__restrict__ pstart,
-                            int n_b, int G, int pass_q) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) {
-        int acc = 0, pacc = 0;
-        for (int b = 0; b < n_b; ++b) {
-            start[b] = acc;
-            pstart[b] = pacc;
-            acc += cnt[b];
-            pacc += (cnt[b] * G + pass_q - 1) / pass_q;
-            cnt[b] = 0;
+// Exclusive prefix sums of the per-block slot counts (start) and of the
+// per-block query passes (pstart), one CTA of 1024 threads; counts are reset
+// for k_slot_fill's cursors.
+constexpr int SCAN_THREADS = 1024;
+__global__ void __launch_bounds__(SCAN_THREADS) k_slot_scan(int32_t *__restrict__ cnt, int32_t *__restrict__ start,
+                                                            int32_t *__restrict__ pstart, int n_b, int G, int pass_q) {
+    __shared__ int2 wsum[SCAN_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int chunk = (n_b + SCAN_THREADS - 1) / SCAN_THREADS;
+    const int b0 = min(n_b, tid * chunk), b1 = min(n_b, b0 + chunk);
+    int2 mine = make_int2(0, 0);
+    for (int b = b0; b < b1; ++b) {
+        const int c = cnt[b];
+        mine.x += c;
+        mine.y += (c * G + pass_q - 1) / pass_q;
+    }
+    // inclusive scan of (slots, passes) over the CTA
+    int2 inc = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc.x, o), y = __shfl_up_sync(0xffffffffu, inc.y, o);
+        if (lane >= o) { inc.x += x; inc.y += y; }
+    }
+    if (lane == 31) wsum[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        int2 v = wsum[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, v.x, o), y = __shfl_up_sync(0xffffffffu, v.y, o);
+            if (lane >= o) { v.x += x; v.y += y; }
         }
-        start[n_b] = acc;
-        pstart[n_b] = pacc;
+        wsum[lane] = v;
+    }
+    __syncthreads();
+    int acc = inc.x - mine.x + (wid > 0 ? wsum[wid - 1].x : 0);
+    int pacc = inc.y - mine.y + (wid > 0 ? wsum[wid - 1].y : 0);
+    for (int b = b0; b < b1; ++b) {
+        const int c = cnt[b];
+        start[b] = acc;
+        pstart[b] = pacc;
+        acc += c;
+        pacc += (c * G + pass_q - 1) / pass_q;
+    }
+    __syncthreads();   // every count read before any is reset
+    for (int b = b0; b < b1; ++b) cnt[b] = 0;
+    if (tid == SCAN_THREADS - 1) {
+        start[n_b] = wsum[31].x;
+        pstart[n_b] = wsum[31].y;
     }
 }
 

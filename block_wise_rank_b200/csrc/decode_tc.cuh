@@ -61,7 +61,7 @@ namespace milo {
 
 constexpr int DT_GROUP = 128;                          // threads per epilogue group
 constexpr int DT_HELP = 64;                            // helper threads
-constexpr int DT_THREADS = 64 + 2 * DT_GROUP + DT_HELP; // warp 0 producer, 1 MMA, 2-5 RoPE, 6-9 softmax, 10-11 helpers
+constexpr int DT_THREADS = 64 + 3 * DT_GROUP + DT_HELP; // warp 0 producer, 1 MMA, 2-5 RoPE, 6-13 softmax, 14-15 helpers
 constexpr int DT_RING = 96 * 1024;                     // ring bytes for A_K, A_V and B_V tiles
 constexpr int DT_NBAR = 32;                            // ring tiles in flight at most
 constexpr int DT_TILE_MAX = 128 * 256;                 // 128 rank rows x 128 tokens (or channels) x 16 bit
@@ -71,7 +71,7 @@ constexpr uint32_t DT_COL_D1 = 0;                      // two 128-column rebuild
 constexpr uint32_t DT_COL_D2 = 256;                    // scores: one 128-column buffer or two of 64
 constexpr uint32_t DT_COL_OA = 384;                    // O_A^T, then O
 constexpr float DT_RESCALE = 8.f;                      // log2 headroom before the reference max moves
-constexpr int DT_BAR_S = 1, DT_BAR_R = 2, DT_BAR_H = 3; // named barriers of the groups
+constexpr int DT_BAR_S = 1, DT_BAR_R = 2, DT_BAR_H = 3, DT_BAR_S2 = 4; // named barriers of the groups
 
 // One work item, written by k_dt_items.
 struct DtItem {
@@ -105,7 +105,7 @@ struct DecTcSmem {
     uint64_t d1_full[2], d1_empty[2], kt_full[2];
     uint64_t d2_full[2], d2_empty[2];
     uint64_t p_full[2], p_empty[2];
-    uint64_t q_full, q_empty, oa_full, oa_free, drain;
+    uint64_t q_full, q_empty, oa_full, o_full, oa_free, drain;
     uint32_t tmem_base;
     volatile int abort;
 };
@@ -187,6 +187,16 @@ __host__ __device__ __forceinline__ int dt_tile_at(int nt, int k, int *t) {
     return 0;
 }
 
+// Two counters selected by a runtime index without a local-memory array.
+struct DtPair {
+    uint32_t c0 = 0, c1 = 0;
+    __device__ __forceinline__ uint32_t operator[](uint32_t b) const { return b ? c1 : c0; }
+    __device__ __forceinline__ void inc(uint32_t b) {
+        if (b) ++c1;
+        else ++c0;
+    }
+};
+
 // named-barrier helpers for one 128-thread group
 template <int ID, int N = DT_GROUP>
 __device__ __forceinline__ void grp_sync() {
@@ -211,6 +221,31 @@ __device__ __forceinline__ bool grp_or(bool v) {
         "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)v), "n"(ID), "n"(N)
+        : "memory");
+    return r != 0;
+}
+
+// the same with the barrier id in a register
+__device__ __forceinline__ void grp_sync_rt(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(DT_GROUP) : "memory");
+}
+__device__ __forceinline__ bool grp_and_rt(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "n"(DT_GROUP)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool grp_or_rt(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "n"(DT_GROUP)
         : "memory");
     return r != 0;
 }
@@ -280,13 +315,14 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             tc::mbar_init(&sm.d1_empty[k], 1);
             tc::mbar_init(&sm.kt_full[k], DT_GROUP);
             tc::mbar_init(&sm.d2_full[k], 1);
-            tc::mbar_init(&sm.d2_empty[k], DT_GROUP);
-            tc::mbar_init(&sm.p_full[k], DT_GROUP);
+            tc::mbar_init(&sm.d2_empty[k], 2 * DT_GROUP);
+            tc::mbar_init(&sm.p_full[k], 2 * DT_GROUP);
             tc::mbar_init(&sm.p_empty[k], 1);
         }
         tc::mbar_init(&sm.q_full, DT_HELP);
         tc::mbar_init(&sm.q_empty, 1);
         tc::mbar_init(&sm.oa_full, 1);
+        tc::mbar_init(&sm.o_full, 1);
         tc::mbar_init(&sm.oa_free, DT_GROUP);
         tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
@@ -422,13 +458,15 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             int64_t iR = i0, iS = i0, iP = i0;
             DtGeo gR = g0, gRn = g1, gS = g0, gSn = g1, gP = g0, gPn = g1;
             uint32_t nR = 0, tR = 0, seqR = 0, rc = 0;             // rebuild queue
-            uint32_t nS = 0, tS = 0, rcS = 0, u2[2] = {0, 0};      // scores queue
-            uint32_t nP = 0, tP = 0, seqP = 0, pu[2] = {0, 0};     // PV / O queue
+            uint32_t nS = 0, tS = 0, rcS = 0;                      // scores queue
+            uint32_t nP = 0, tP = 0, seqP = 0;                     // PV / O queue
+            DtPair u2, pu;                                         // uses of each scores / P buffer
             const uint32_t sq = tc::smem_u32(sm.qt);
             const uint32_t sbk = tc::smem_u32(sm.bk);
             const uint32_t spb = tc::smem_u32(sm.pbuf);
             const uint32_t sring = tc::smem_u32(sm.ring);
             uint64_t t_last = tc::globaltimer();
+            uint32_t backoff = 32;
             bool ok = true;
             while (ok) {
                 const bool doneR = iR >= n_items, doneS = iS >= n_items, doneP = iP >= n_items;
@@ -480,7 +518,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         tc::mma_commit(&sm.d2_full[d2b]);
                         tc::mma_commit(&sm.d1_empty[b]);
                         if ((int)tS == gS.nt - 1) tc::mma_commit(&sm.q_empty);
-                        ++u2[d2b];
+                        u2.inc(d2b);
                         ++rcS;
                         if ((int)++tS == gS.nt) {
                             tS = 0;
@@ -514,7 +552,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             tc::mma_commit(&sm.p_empty[pb]);
                             tc::mma_commit(&sm.empty[s]);
                             if ((int)tP == gP.nt - 1) tc::mma_commit(&sm.oa_full);
-                            ++pu[pb];
+                            pu.inc(pb);
                             ++tP;
                         } else {                 // O = B_V^T (O_A / l), over O_A's columns
                             MILO_TRACE_MMA(nP, 12);
@@ -527,8 +565,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                                            ks > 0);
                             tc::mma_commit(&sm.p_empty[pb]);
                             tc::mma_commit(&sm.empty[s]);
-                            tc::mma_commit(&sm.oa_full);
-                            ++pu[pb];
+                            tc::mma_commit(&sm.o_full);
+                            pu.inc(pb);
                             seqP += dt_ring_tiles(gP);
                             tP = 0;
                             ++nP;
@@ -541,11 +579,15 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 }
                 if (prog) {
                     t_last = tc::globaltimer();
+                    backoff = 32;
                 } else if (sm.abort || tc::globaltimer() - t_last > 2000000000ull) {
                     if (!sm.abort) raise_status(ST_TIMEOUT);
                     ok = false;
                 } else {
-                    __nanosleep(64);   // leave the issue slots to the group warps
+                    // idle: sleep, longer while nothing happens, so that the
+                    // polling leaves issue slots and i-cache to the group warps
+                    __nanosleep(backoff);
+                    backoff = min(backoff * 2, 64u);
                 }
             }
             if (!ok) sm.abort = 1;
@@ -561,6 +603,30 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         uint32_t rc = 0, n = 0;
         bool ok = true;
         (void)et;
+        // O = B_V^T (O_A / l) of item m (lanes = channels, columns = queries)
+        // to the partials; frees O_A^T for the next item's PV products
+        int pend_nq = -1;   // queries of the item whose O is still to be read, or -1
+        uint32_t pend_n = 0;
+        auto readout = [&]() -> bool {
+            if (!grp_and<DT_BAR_R>(tc::mbar_wait(&sm.o_full, pend_n & 1u) && !sm.abort)) return false;
+            tc::tc_fence_after();
+            const int *qp = sm.qpidx[pend_n & 3u];
+            const int nq = pend_nq, nq16 = (nq + 15) & ~15;
+            for (int c0 = 0; c0 < nq16; c0 += 32) {
+                uint32_t r[32];
+                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                if (c0 + 16 < nq16)
+                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int v = 0; v < 32; ++v)
+                    if (c0 + v < nq) a.part_o[(int64_t)qp[c0 + v] * D + row] = __uint_as_float(r[v]);
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&sm.oa_free);
+            pend_nq = -1;
+            return true;
+        };
         for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
             const int nt = token_tiles(__ldg(&items[i].Tb));
             for (int t = 0; t < nt; ++t) {
@@ -573,8 +639,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 const int tok = t * FTILE + row;   // in-block token of this lane
                 const int tl = tok & 31, th = tok >> 5;
                 // pair chunk pc (16 pairs): x at columns 16pc.., y at 64 + 16pc..;
-                // packed fp16 results go to 8pc.. (x) and 64 + 8pc.. (y), columns
-                // this thread has already read
+                // packed fp16 results go to 8pc.. (x) and 64 + 8pc.. (y), columns of
+                // chunks this thread has already read
                 auto rot_chunk = [&](const uint32_t (&xr)[16], const uint32_t (&yr)[16], int pc) {
                     uint32_t px[8], py[8];
 #pragma unroll
@@ -599,41 +665,52 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     tc::tmem_st8(base + 64 + 8 * pc, py);
                 };
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {   // pair chunks 2h, 2h+1
-                    uint32_t xa[16], ya[16], xb[16], yb[16];
-                    tc::tmem_ld16(base + 32 * h, xa);
-                    tc::tmem_ld16(base + 64 + 32 * h, ya);
-                    tc::tmem_ld16(base + 32 * h + 16, xb);
-                    tc::tmem_ld16(base + 64 + 32 * h + 16, yb);
+                for (int pc = 0; pc < 4; ++pc) {   // pair chunk pc: writes land in columns of chunks <= pc
+                    uint32_t xa[16], ya[16];
+                    tc::tmem_ld16(base + 16 * pc, xa);
+                    tc::tmem_ld16(base + 64 + 16 * pc, ya);
                     tc::tmem_wait_ld();
-                    rot_chunk(xa, ya, 2 * h);
-                    rot_chunk(xb, yb, 2 * h + 1);
+                    rot_chunk(xa, ya, pc);
                 }
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 tc::mbar_arrive(&sm.kt_full[b]);
                 ++rc;
                 MILO_TRACE_EVENT(0, 2 * t + 1);
+                // the previous item's output, once this item's first two tiles
+                // are rotated (the softmax group has work queued meanwhile)
+                if (t == min(1, nt - 1) && pend_nq >= 0 && !(ok = readout())) break;
             }
+            if (!ok) break;
+            pend_nq = __ldg(&items[i].nq);
+            pend_n = n;
         }
+        if (ok && pend_nq >= 0) ok = readout();
         if (!ok) sm.abort = 1;
-    } else if (warp < 10) {
-        // ================================================================ softmax group
-        const int et = threadIdx.x - 192;
+    } else if (warp < 14) {
+        // ================================================================ softmax groups
+        // Two groups of 4 warps (one per TMEM lane quadrant, one token row per
+        // thread); group sg owns the 32-column query slabs sg, sg + 2, ...  The
+        // reference max, sums and P of a column belong to one group, so the
+        // groups only meet at the counted arrivals.
+        const int sg = (warp - 6) >> 2;
+        const int gt = threadIdx.x - 192 - DT_GROUP * sg;   // thread within the group
+        const int et = gt + DT_GROUP * sg;                 // trace hooks: thread 0 of group 0
+        const int bar_id = sg == 0 ? DT_BAR_S : DT_BAR_S2;
         const int quad = warp & 3;
-        const int row = quad * 32 + lane;             // TMEM lane of this thread
+        const int row = quad * 32 + lane;                  // TMEM lane of this thread
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const float kscale = 1.4426950408889634f * rsqrtf((float)D);   // log2(e) / sqrt(d)
-        uint32_t u2[2] = {0, 0};                      // uses of each scores buffer
-        uint32_t pf[2] = {0, 0}, pe[2] = {0, 0};      // P buffer hand-overs / completions seen
-        uint32_t seqA0 = 0, n = 0;
+        DtPair u2;                                         // uses of each scores buffer
+        DtPair pf, pe;                                     // P buffer hand-overs / completions seen
+        uint32_t n = 0;
         bool ok = true;
 
         // wait until P buffer b's last product (PV or O) has completed
         auto p_drain = [&](int b) -> bool {
             if (pe[b] == pf[b]) return true;
-            const bool w = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.p_empty[b], pe[b] & 1u));
-            ++pe[b];
+            const bool w = grp_and_rt(bar_id, tc::mbar_wait(&sm.p_empty[b], pe[b] & 1u));
+            pe.inc(b);
             return w;
         };
 
@@ -650,40 +727,63 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 tc::fence_async_smem();
                 const int pb = g.dbl ? (tt & 1) : 0;
                 tc::mbar_arrive(&sm.p_full[pb]);
-                ++pf[pb];
+                pf.inc(pb);
                 ++pv_issued;
+            };
+
+            // ---- no spare rank row: column sums of the rounded P by a transposing
+            // butterfly; lanes 2c and 2c+1 end with column c of the 16
+            auto colsum = [&](const uint32_t (&pk)[8], int ch) {
+                float sv[16];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float2 pr = __half22float2(*reinterpret_cast<const __half2 *>(&pk[v]));
+                    sv[2 * v] = pr.x;
+                    sv[2 * v + 1] = pr.y;
+                }
+#pragma unroll
+                for (int sz = 8, bit = 16; sz >= 1; sz >>= 1, bit >>= 1) {
+                    const bool hi = lane & bit;
+#pragma unroll
+                    for (int j = 0; j < sz; ++j) {
+                        const float send = hi ? sv[j] : sv[j + sz];
+                        const float keep = hi ? sv[j + sz] : sv[j];
+                        sv[j] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+                    }
+                }
+                sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
+                if (!(lane & 1)) atomicAdd(&sm.lsum[ch + ((lane >> 1) & 15)], sv[0]);
             };
 
             // ---- rare path: some p of columns [c0, c0 + w) exceeded 2^8 (or
             // overflowed).  Raise those columns' reference max to this tile's
-            // maxima (raw scores reloaded from TMEM), rescale the running O_A^T
-            // and sums, and recompute p.
-            auto rescale = [&](int t, int c0, int w, uint32_t dcol, int lim) -> bool {
-                (void)t;
+            // maxima (raw scores reloaded from TMEM) and rescale the running
+            // O_A^T and sums; the caller recomputes p.
+            auto rescale = [&](int c0, int w, uint32_t dcol, int lim) -> bool {
                 if (!p_drain(0) || !p_drain(1)) return false;   // every P handed over has been used
-                if (et < w) sm.cmax[c0 + et] = ord_enc(-INFINITY);
-                uint32_t r[32];
-                tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-                tc::tmem_wait_ld();
-                grp_sync<DT_BAR_S>();
+                if (gt < w) sm.cmax[c0 + gt] = ord_enc(-INFINITY);
+                grp_sync_rt(bar_id);
+                for (int h = 0; h < w; h += 16) {   // column maxima over the tile's live rows
+                    uint32_t r[16];
+                    tc::tmem_ld16(dcol + c0 + h, r);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int v = 0; v < 32; ++v) {
-                    if (v >= w) break;
-                    float x = v < lim ? __uint_as_float(r[v]) * kscale : -INFINITY;
-                    for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-                    if (lane == 0) atomicMax(&sm.cmax[c0 + v], ord_enc(x));
+                    for (int v = 0; v < 16; ++v) {
+                        float x = h + v < lim ? __uint_as_float(r[v]) * kscale : -INFINITY;
+                        for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+                        if (lane == 0) atomicMax(&sm.cmax[c0 + h + v], ord_enc(x));
+                    }
                 }
-                grp_sync<DT_BAR_S>();
-                if (et < w) {
-                    const int c = c0 + et;
+                grp_sync_rt(bar_id);
+                if (gt < w) {
+                    const int c = c0 + gt;
                     const float cn = fmaxf(sm.cref[c], ord_dec(sm.cmax[c]));
                     const float f = dt_ex2(sm.cref[c] - cn);
                     sm.cscale[c] = f;
                     sm.cref[c] = cn;
                     sm.lsum[c] *= f;
                 }
-                grp_sync<DT_BAR_S>();
+                grp_sync_rt(bar_id);
                 if (pv_issued > 0) {   // O_A^T columns (every rank lane) times 2^(cref_old - cref_new)
                     tc::tc_fence_after();
                     for (int h = 0; h < w; h += 16) {
@@ -705,132 +805,103 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 return true;
             };
 
-            // ---- softmax of score tile t: p = 2^(x - cref), fp16, MN-major [t/8][q/8][t%8][q%8]
+            // ---- softmax of score tile t over this group's slabs:
+            // p = 2^(x - cref), fp16, MN-major [t/8][q/8][t%8][q%8]
             auto softmax = [&](int t) -> bool {
                 const int d2b = g.dbl ? (t & 1) : 0;
                 const uint32_t dcol = tmem + DT_COL_D2 + 64 * d2b + lane_off;
-                if (t == 1) MILO_TRACE_WARP(3);
-                if (!grp_and<DT_BAR_S>(tc::mbar_wait(&sm.d2_full[d2b], u2[d2b] & 1u))) return false;
-                if (t == 1) MILO_TRACE_WARP(4);
-                ++u2[d2b];
+                if (!grp_and_rt(bar_id, tc::mbar_wait(&sm.d2_full[d2b], u2[d2b] & 1u))) return false;
+                u2.inc(d2b);
                 MILO_TRACE_EVENT(1, 2 + 2 * t);
                 tc::tc_fence_after();
                 const int tok = t * FTILE + row;
                 const bool valid = tok < Tb;
                 if (t == 0) {   // reference max: the scores of the item's first token
-                    sm.lsum[et] = 0.f;
-                    if (quad == 0) {
-                        for (int c0 = 0; c0 < nq16; c0 += 16) {
-                            uint32_t r[16];
-                            tc::tmem_ld16(dcol + c0, r);
-                            tc::tmem_wait_ld();
-                            if (lane == 0)
+                    for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
+                        const int w = min(32, nq16 - c0);
+                        if (gt < w) sm.lsum[c0 + gt] = 0.f;
+                        if (quad == 0)
+                            for (int h = 0; h < w; h += 16) {
+                                uint32_t r[16];
+                                tc::tmem_ld16(dcol + c0 + h, r);
+                                tc::tmem_wait_ld();
+                                if (lane == 0)
 #pragma unroll
-                                for (int v = 0; v < 16; ++v) sm.cref[c0 + v] = __uint_as_float(r[v]) * kscale;
-                        }
+                                    for (int v = 0; v < 16; ++v) sm.cref[c0 + h + v] = __uint_as_float(r[v]) * kscale;
+                            }
                     }
-                    grp_sync<DT_BAR_S>();
+                    grp_sync_rt(bar_id);
                 }
-                MILO_TRACE_EVENT(1, 16 + 8 * t);
                 const int pb = g.dbl ? (t & 1) : 0;
                 uint8_t *pbase = sm.pbuf + pb * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
+                // the P buffer's previous product has completed (at an item's start
+                // both halves: the previous item may have used it at another width)
+                auto drain = [&]() -> bool {
+                    if (t == 0) return p_drain(0) && p_drain(1);
+                    return p_drain(pb);
+                };
                 bool p_ready = false;
-                for (int c0 = 0; c0 < nq16; c0 += 32) {
+                for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
                     const int w = min(32, nq16 - c0);
                     const int lim = valid ? min(w, nq - c0) : 0;   // this token's live columns
-                    // raw scores, turned into p in place
-                    float pv[32];
-                    tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pv[0]));
-                    if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pv[16]));
+                    // raw scores; p = 2^(x - cref) packed to fp16 pairs in place (pk[v] <-
+                    // columns 2v, 2v+1).  More than 2^8 (or an overflow) sends the slab
+                    // down the rare path, which recomputes it.
+                    uint32_t pk[32];
+                    tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                    if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
                     tc::tmem_wait_ld();
                     if (c0 == 0) MILO_TRACE_EVENT(1, 17 + 8 * t);
-                    if (c0 == 32) MILO_TRACE_EVENT(1, 21 + 8 * t);
-                    {
-                        // p = 2^(x - cref); more than 2^8 (or an overflow) sends the
-                        // group down the rare path
-                        const float4 *c4 = reinterpret_cast<const float4 *>(sm.cref + c0);
-                        float pmax = 0.f;
+                    auto make_p = [&](float &pmax) {
+                        const float2 *c2 = reinterpret_cast<const float2 *>(sm.cref + c0);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            if (4 * k >= w) break;
-                            const float4 f = c4[k];
-                            const float cr[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int v = 4 * k + j;
-                                const float e = dt_ex2(pv[v] * kscale - cr[j]);
-                                pv[v] = v < lim ? e : 0.f;
-                                pmax = fmaxf(pmax, pv[v]);
-                            }
+                        for (int v = 0; v < 16; ++v) {
+                            if (2 * v >= w) break;
+                            const float2 cr = c2[v];
+                            float e0 = dt_ex2(__uint_as_float(pk[2 * v]) * kscale - cr.x);
+                            float e1 = dt_ex2(__uint_as_float(pk[2 * v + 1]) * kscale - cr.y);
+                            e0 = 2 * v < lim ? e0 : 0.f;
+                            e1 = 2 * v + 1 < lim ? e1 : 0.f;
+                            pmax = fmaxf(pmax, fmaxf(e0, e1));
+                            const __half2 hb = __floats2half2_rn(e0, e1);
+                            pk[v] = *reinterpret_cast<const uint32_t *>(&hb);
                         }
-                        const bool any_over = grp_or<DT_BAR_S>(!(pmax <= 256.f));
-                        if (c0 == 0) MILO_TRACE_EVENT(1, 18 + 8 * t);
-                        if (any_over) {
-                            MILO_TRACE_EVENT(1, 23 + 8 * t);
-                            if (!rescale(t, c0, w, dcol, lim)) return false;
-                            tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pv[0]));
-                            if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pv[16]));
-                            tc::tmem_wait_ld();
-#pragma unroll
-                            for (int v = 0; v < 32; ++v)
-                                if (v < w) pv[v] = v < lim ? dt_ex2(pv[v] * kscale - sm.cref[c0 + v]) : 0.f;
-                        }
+                    };
+                    float pmax = 0.f;
+                    make_p(pmax);
+                    const bool any_over = grp_or_rt(bar_id, !(pmax <= 256.f));
+                    if (c0 == 0) MILO_TRACE_EVENT(1, 18 + 8 * t);
+                    if (any_over) {
+                        MILO_TRACE_EVENT(1, 23 + 8 * t);
+                        if (!rescale(c0, w, dcol, lim)) return false;
+                        tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                        if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+                        tc::tmem_wait_ld();
+                        float pm2 = 0.f;
+                        make_p(pm2);
                     }
-                    if (c0 + 32 >= nq16) {   // every score of the tile has been used
-                        tc::tc_fence_before();
-                        tc::mbar_arrive(&sm.d2_empty[d2b]);
-                    }
-                    if (!p_ready) {   // the P buffer's previous product has completed
-                        // (at an item's start both halves: the previous item may have
-                        // used the buffer at the other width)
-                        if (t == 0) {
-                            if (!p_drain(0) || !p_drain(1)) return false;
-                        } else if (!p_drain(pb)) {
-                            return false;
-                        }
+                    if (!p_ready) {
+                        if (!drain()) return false;
                         p_ready = true;
                         MILO_TRACE_EVENT(1, 19 + 8 * t);
                     }
-                    // fp16 P, MN-major [t/8][q/8][t%8][q%8]
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         if (16 * hh >= w) break;
                         const int ch = c0 + 16 * hh;
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            const __half2 hb = __floats2half2_rn(pv[16 * hh + 2 * v], pv[16 * hh + 2 * v + 1]);
-                            pk[v] = *reinterpret_cast<const uint32_t *>(&hb);
-                        }
+                        const uint32_t(&q8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[8 * hh]);
                         uint8_t *dst = pbase + (ch >> 3) * 128;
-                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        if (!g.ones) {
-                            // no spare rank row: column sums of the rounded P by a
-                            // transposing butterfly; lanes 2c and 2c+1 end with column c
-                            float sv[16];
-#pragma unroll
-                            for (int v = 0; v < 8; ++v) {
-                                const float2 pr = __half22float2(*reinterpret_cast<const __half2 *>(&pk[v]));
-                                sv[2 * v] = pr.x;
-                                sv[2 * v + 1] = pr.y;
-                            }
-#pragma unroll
-                            for (int sz = 8, bit = 16; sz >= 1; sz >>= 1, bit >>= 1) {
-                                const bool hi = lane & bit;
-#pragma unroll
-                                for (int j = 0; j < sz; ++j) {
-                                    const float send = hi ? sv[j] : sv[j + sz];
-                                    const float keep = hi ? sv[j + sz] : sv[j];
-                                    sv[j] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-                                }
-                            }
-                            sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
-                            if (!(lane & 1)) atomicAdd(&sm.lsum[ch + ((lane >> 1) & 15)], sv[0]);
-                        }
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(q8[0], q8[1], q8[2], q8[3]);
+                        *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(q8[4], q8[5], q8[6], q8[7]);
+                        if (!g.ones) colsum(q8, ch);
                     }
                     if (c0 == 0) MILO_TRACE_EVENT(1, 20 + 8 * t);
                 }
+                // every score of the tile this thread needed has been read
+                tc::tc_fence_before();
+                tc::mbar_arrive(&sm.d2_empty[d2b]);
+                // a group without slabs keeps the same drain sequence
+                if (!p_ready && !drain()) return false;
                 MILO_TRACE_EVENT(1, 3 + 2 * t);
                 return true;
             };
@@ -841,50 +912,56 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
             if (!ok) break;
 
-            // ---- O_A^T finished: denominators, O_A / l to fp16 staging
-            ok = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.oa_full, 0));
+            // ---- O_A^T finished: denominators, O_A / l to fp16 staging (this
+            // group's columns); the last product and its read-out are the RoPE group's
+            ok = grp_and_rt(bar_id, tc::mbar_wait(&sm.oa_full, n & 1u));
             if (!ok) break;
             MILO_TRACE_EVENT(1, 12);
             tc::tc_fence_after();
             if (g.ones && quad == (g.R8V >> 5)) {   // the ones row holds sum_t p
-                for (int c0 = 0; c0 < nq16; c0 += 16) {
-                    uint32_t r[16];
-                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, r);
-                    tc::tmem_wait_ld();
-                    if (row == g.R8V)
+                for (int c0 = 32 * sg; c0 < nq16; c0 += 64)
+                    for (int h = 0; h < min(32, nq16 - c0); h += 16) {
+                        uint32_t r[16];
+                        tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + h, r);
+                        tc::tmem_wait_ld();
+                        if (row == g.R8V)
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) sm.lsum[c0 + v] = __uint_as_float(r[v]);
-                }
+                            for (int v = 0; v < 16; ++v) sm.lsum[c0 + h + v] = __uint_as_float(r[v]);
+                    }
             }
-            grp_sync<DT_BAR_S>();
-            if (et < nq16) sm.cscale[et] = (et < nq && sm.lsum[et] > 0.f) ? __frcp_rn(sm.lsum[et]) : 0.f;
+            grp_sync_rt(bar_id);
+            for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
+                const int c = c0 + gt;
+                if (gt < min(32, nq16 - c0)) sm.cscale[c] = (c < nq && sm.lsum[c] > 0.f) ? __frcp_rn(sm.lsum[c]) : 0.f;
+            }
             const int pst = g.dbl ? (g.nt & 1) : 0;
             if (!p_drain(pst)) { ok = false; break; }
-            grp_sync<DT_BAR_S>();
+            grp_sync_rt(bar_id);
             if (quad * 32 < g.R16V) {
                 uint8_t *sbase = sm.pbuf + pst * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
-                for (int c0 = 0; c0 < nq16; c0 += 32) {
+                for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
+                    const int w = min(32, nq16 - c0);
                     uint32_t r[32];
                     tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                    if (c0 + 16 < nq16)
+                    if (w == 32)
                         tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
                     tc::tmem_wait_ld();
                     if (row < g.R16V) {
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int ch = c0 + 16 * hh;
-                            if (ch >= nq16) break;
-                            uint32_t pk[8];
+                            if (16 * hh >= w) break;
+                            uint32_t q8[8];
 #pragma unroll
                             for (int v = 0; v < 8; ++v) {
                                 const __half2 h2 = __floats2half2_rn(
                                     __uint_as_float(r[16 * hh + 2 * v]) * sm.cscale[ch + 2 * v],
                                     __uint_as_float(r[16 * hh + 2 * v + 1]) * sm.cscale[ch + 2 * v + 1]);
-                                pk[v] = *reinterpret_cast<const uint32_t *>(&h2);
+                                q8[v] = *reinterpret_cast<const uint32_t *>(&h2);
                             }
                             uint8_t *dst = sbase + (ch >> 3) * 128;
-                            *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                            *reinterpret_cast<uint4 *>(dst) = make_uint4(q8[0], q8[1], q8[2], q8[3]);
+                            *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(q8[4], q8[5], q8[6], q8[7]);
                         }
                     }
                 }
@@ -892,36 +969,22 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             tc::fence_async_smem();
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.p_full[pst]);
-            ++pf[pst];
-            // ---- O (lanes = channels, columns = queries) to the partials
-            ok = grp_and<DT_BAR_S>(tc::mbar_wait(&sm.oa_full, 1));
-            if (!ok) break;
-            MILO_TRACE_EVENT(1, 13);
-            tc::tc_fence_after();
-            const int *qp = sm.qpidx[n & 3u];
-            for (int c0 = 0; c0 < nq16; c0 += 32) {
-                uint32_t r[32];
-                tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                if (c0 + 16 < nq16)
-                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int v = 0; v < 32; ++v)
-                    if (c0 + v < nq) a.part_o[(int64_t)qp[c0 + v] * D + row] = __uint_as_float(r[v]);
+            pf.inc(pst);
+            // the reference max and the sum of this group's queries
+            for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
+                const int c = c0 + gt;
+                if (gt < min(32, nq16 - c0) && c < nq)
+                    a.part_ml[sm.qpidx[n & 3u][c]] = make_float2(sm.cref[c] * 0.69314718055994531f, sm.lsum[c]);
             }
-            if (et < nq) a.part_ml[qp[et]] = make_float2(sm.cref[et] * 0.69314718055994531f, sm.lsum[et]);
-            tc::tc_fence_before();
-            tc::mbar_arrive(&sm.oa_free);
-            seqA0 += dt_ring_tiles(g);
             // one group-wide decision per item (also orders this item's reads of
             // cref / lsum before the next item's writes)
-            ok = grp_and<DT_BAR_S>(!sm.abort);
+            ok = grp_and_rt(bar_id, !sm.abort);
             MILO_TRACE_EVENT(1, 14);
         }
         if (!ok) sm.abort = 1;
     } else {
         // ================================================================ helper warps
-        const int et = threadIdx.x - (64 + 2 * DT_GROUP);
+        const int et = threadIdx.x - (64 + 3 * DT_GROUP);
         bool ok = true;
         // ---- rotated queries R(-p) q of item j, fp16, K-major [q/8][j/8][q%8][j%8];
         // four threads per query, 16 pairs each
@@ -986,6 +1049,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         int kc = 0;
         DtGeo gc = dt_geo(items, ic, n_items);
         uint64_t t_last = tc::globaltimer();
+        uint32_t backoff = 64;
         while (ok && (ic < n_items || iq < n_items)) {
             bool did = false;
             if (ic < n_items) {
@@ -1020,13 +1084,15 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
             if (did) {
                 t_last = tc::globaltimer();
+                backoff = 64;
             } else {
                 const bool stop = grp_or<DT_BAR_H, DT_HELP>(sm.abort || tc::globaltimer() - t_last > 2000000000ull);
                 if (stop) {
                     if (!sm.abort) raise_status(ST_TIMEOUT);
                     ok = false;
                 }
-                __nanosleep(256);
+                __nanosleep(backoff);
+                backoff = min(backoff * 2, 256u);
             }
         }
         if (!ok) sm.abort = 1;

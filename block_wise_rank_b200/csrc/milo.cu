@@ -561,7 +561,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     if (e != cudaSuccess) return cuda_check(e, "memset");
     const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
-    k_slot_scan<<<1, 32, 0, s>>>(cnt, start, pstart, n_b, a.G, DT_NQ);
+    k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, pstart, n_b, a.G, DT_NQ);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
     const int64_t rt = (slots + f->shape.block_len) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
