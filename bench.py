@@ -19,6 +19,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -48,6 +49,8 @@ def parse():
     ap.add_argument("--factor", default=None, choices=["bf16", "int8", "f32"])
     ap.add_argument("--decode-steps", type=int, default=0, help="decode steps per step (0: the workload's)")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (0: the workload's); for small profiling slices")
     ap.add_argument("--profile", action="store_true",
                     help="only the warm-up and timed steps (for ncu launch lists): no profiler, e2e or CPU legs")
     return ap.parse_args()
@@ -161,10 +164,18 @@ def count_launches(fn):
 
 
 # ------------------------------------------------------------------ arms
+def workload_of(args):
+    import dataclasses
+    w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = dataclasses.replace(w, name=f"{w.name} ({args.layers}-layer slice)", L=args.layers)
+    return w
+
+
 def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     factor = args.factor or ("f32" if w.dtype == "f32" else "bf16")
     params = milo.default_params(factor_dtype=factor, budget_frac=args.budget)
     gen_dtype = torch.float64 if w.T * w.L * w.H <= 1 << 16 else torch.float32
@@ -257,12 +268,46 @@ def run_ours(args, rank, world):
         compress=dict(blocks_per_s=round(comp_bps, 1), ms=round(comp_sum / args.steps, 3),
                       blocks=n_blocks),
         roofline=dict(bound="hbm", achieved=round(kernel["gbs"], 1), peak=pk["hbm"], unit="GB/s",
-                      frac=round(kernel["gbs"] / pk["hbm"], 4), traffic=None, kernel=kernel["name"],
-                      peak_src=f"{pk['src']} hbm_gbs"),
+                      frac=round(kernel["gbs"] / pk["hbm"], 4), traffic=decode_traffic(w, factor),
+                      kernel=kernel["name"], peak_src=f"{pk['src']} hbm_gbs"),
         e2e=e2e, clocks=clk, gpu_launches=launches_per_step * args.steps,
         status=milo.status_string(st),
     )
     return res
+
+
+DECODE_SOURCES = ("block_wise_rank_b200/csrc/decode_tc.cuh", "block_wise_rank_b200/csrc/tc_common.cuh",
+                  "block_wise_rank_b200/csrc/common.cuh")
+DECODE_PROFILE = "profiles/decode_tc_qwen7b-128k_4layer.md"
+
+
+def decode_traffic(w, factor):
+    """DRAM bytes (read + write) of one k_decode_tc launch, from the committed
+    ncu summary of the qwen7b-128k-shaped slice scaled by the layer count;
+    None for another shape or factor type, or once the kernel's sources differ
+    from the ones the counters were taken on."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    if not w.name.startswith("qwen7b-128k") or factor != "bf16":
+        return None
+    try:
+        h = hashlib.sha256()
+        for f in DECODE_SOURCES:   # code only: comments and blank space do not count
+            with open(os.path.join(here, f)) as fh:
+                text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+            text = re.sub(r"//[^\n]*", "", text)
+            h.update(re.sub(r"\s+", " ", text).strip().encode())
+        fields = {}
+        with open(os.path.join(here, DECODE_PROFILE)) as fh:
+            for line in fh:
+                k, _, v = line.strip().partition(":")
+                if k in ("traffic_bytes_per_layer", "source_sha256_16"):
+                    fields[k] = v.strip()
+        if fields.get("source_sha256_16") != h.hexdigest()[:16]:
+            return None
+        return int(fields["traffic_bytes_per_layer"]) * w.L
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def decode_kernel_timing(f, w, dec_inputs, out, dws, stream):
@@ -321,7 +366,7 @@ def run_reference(args):
     import numpy as np
 
     import oracle
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     factor = args.factor or ("f32" if w.dtype == "f32" else "bf16")
     cores = 1   # the oracle is single-threaded C
     # bounded sample: the cache of 1 (layer, head) for compression; queries of

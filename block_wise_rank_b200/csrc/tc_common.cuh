@@ -30,8 +30,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 // try_wait without a suspend-time hint: the thread may be parked for the
-// hardware's own short limit.  (With a long hint, a thread waiting for an
-// arrival made by tcgen05.commit was measured to resume microseconds late.)
+// hardware's own short limit before the caller checks its time budget again.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

@@ -122,8 +122,12 @@ def planted_cache(L: int, H: int, T: int, d: int, block_len: int, tau_range, see
         sig = torch.exp(-k[None, :] / taus[:, None])
         X = (U * sig[:, None, :]) @ Vm.transpose(1, 2)
         X = X + noise * torch.randn(n, block_len, d, generator=g, device=device, dtype=gen_dtype)
-        for j, (lh, b) in enumerate(part):
-            flat[lh, b * block_len:(b + 1) * block_len] = X[j].to(out_dtype)
+        if not ragged:   # every block full: one indexed copy for the chunk
+            rows = torch.tensor([lh * nb + b for lh, b in part], device=device)
+            flat.view(L * H * nb, block_len, d)[rows] = X.to(out_dtype)
+        else:
+            for j, (lh, b) in enumerate(part):
+                flat[lh, b * block_len:(b + 1) * block_len] = X[j].to(out_dtype)
     for lh in range(L * H):
         for b in ragged:
             tb = lengths[b]
