@@ -18,15 +18,17 @@
 //                     scores   S = K-tilde (TMEM) Q-tilde^T    (M=128 tokens, N=nq, K=128, fp16)
 //                     PV / O   O_A^T += A_V(tile)^T P          (M=128 ranks, N=nq, K=128 tokens, fp16)
 //                              O = B_V^T (O_A / l)            (M=128 channels, N=nq, K=r_V, fp16)
-//   RoPE group      4 warps, one per TMEM lane quadrant, one token row per
-//                   thread: rotates each rebuilt key row by its in-block angle
-//                   t*theta_i and packs K-tilde to fp16 in place.  Two rebuild
-//                   buffers let it run up to two tiles ahead of the scores.
-//   softmax group   4 warps: softmax in the exp2 domain against a per-query
-//                   reference max that is raised (with the running O_A^T and
-//                   sums rescaled) only when a score exceeds it by more than
-//                   2^8; P (fp16) to shared memory; O_A / l staged for the
-//                   last product; O to the partials.
+//   RoPE group      8 warps, two per TMEM lane quadrant (one token row per
+//                   thread, half the pairs each): rotates each rebuilt key row
+//                   by its in-block angle t*theta_i and packs K-tilde to fp16 in
+//                   place; two rebuild buffers let it run up to two tiles ahead
+//                   of the scores.  It also reads each item's O out to the
+//                   partials.
+//   softmax groups  2 x 4 warps, alternate 32-query slabs: softmax in the exp2
+//                   domain against a per-query reference max that is raised
+//                   (with the running O_A^T and sums rescaled) only when a p
+//                   exceeds 2^8; P (fp16) to shared memory; O_A / l staged for
+//                   the last product.
 //   helper warps    2 warps: convert each A_V tile and B_V to fp16 in place as
 //                   they land; rotate the next item's queries by -p*theta_i
 //                   once the current item's scores are done.
@@ -61,7 +63,11 @@ namespace milo {
 
 constexpr int DT_GROUP = 128;                          // threads per epilogue group
 constexpr int DT_HELP = 64;                            // helper threads
-constexpr int DT_THREADS = 64 + 3 * DT_GROUP + DT_HELP; // warp 0 producer, 1 MMA, 2-5 RoPE, 6-13 softmax, 14-15 helpers
+constexpr int DT_RGROUP = 2 * DT_GROUP;                // RoPE threads: two warps per TMEM lane quadrant
+constexpr int DT_THREADS = 64 + DT_RGROUP + 2 * DT_GROUP + DT_HELP; // warp 0 producer, 1 MMA, 2-9 RoPE,
+                                                                    // 10-17 softmax, 18-19 helpers
+constexpr int DT_W_S = 2 + DT_RGROUP / 32;             // first softmax warp
+constexpr int DT_W_H = DT_W_S + 2 * DT_GROUP / 32;     // first helper warp
 constexpr int DT_RING = 96 * 1024;                     // ring bytes for A_K, A_V and B_V tiles
 constexpr int DT_NBAR = 32;                            // ring tiles in flight at most
 constexpr int DT_TILE_MAX = 128 * 256;                 // 128 rank rows x 128 tokens (or channels) x 16 bit
@@ -313,7 +319,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         for (int k = 0; k < 2; ++k) {
             tc::mbar_init(&sm.d1_full[k], 1);
             tc::mbar_init(&sm.d1_empty[k], 1);
-            tc::mbar_init(&sm.kt_full[k], DT_GROUP);
+            tc::mbar_init(&sm.kt_full[k], DT_RGROUP);
             tc::mbar_init(&sm.d2_full[k], 1);
             tc::mbar_init(&sm.d2_empty[k], 2 * DT_GROUP);
             tc::mbar_init(&sm.p_full[k], 2 * DT_GROUP);
@@ -323,7 +329,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         tc::mbar_init(&sm.q_empty, 1);
         tc::mbar_init(&sm.oa_full, 1);
         tc::mbar_init(&sm.o_full, 1);
-        tc::mbar_init(&sm.oa_free, DT_GROUP);
+        tc::mbar_init(&sm.oa_free, DT_RGROUP);
         tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
         tc::fence_barrier_init();
@@ -511,9 +517,12 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         tc::tc_fence_after();
                         const uint32_t id_sc = tc::idesc_f16(128, gS.nq16, 0, 0, 0);   // fp16, A tmem, B K-major
                         const uint32_t kt = tmem + DT_COL_D1 + 128 * b;
-                        // K-tilde: x halves packed at columns 0..31, y halves at 64..95
+                        // K-tilde packed in place: the 16 dims of k-step ks (pairs
+                        // 16(ks % 4).. of the x or y half) at columns (ks >= 4 ? 64 : 0)
+                        // + {0, 8, 32, 40}[ks % 4]
                         for (int ks = 0; ks < D / 16; ++ks)
-                            tc::mma_ts(tmem + DT_COL_D2 + 64 * d2b, kt + (ks < 4 ? 8 * ks : 32 + 8 * ks),
+                            tc::mma_ts(tmem + DT_COL_D2 + 64 * d2b,
+                                       kt + (ks >= 4 ? 64 : 0) + ((ks & 3) < 2 ? 8 * (ks & 3) : 16 + 8 * (ks & 3)),
                                        tc::smem_desc(sq + ks * 256, 128, 2048, tc::LAYOUT_NONE), id_sc, ks > 0);
                         tc::mma_commit(&sm.d2_full[d2b]);
                         tc::mma_commit(&sm.d1_empty[b]);
@@ -594,9 +603,12 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             tc::mma_commit(&sm.drain);
             tc::mbar_wait(&sm.drain, 0);
         }
-    } else if (warp < 6) {
+    } else if (warp < DT_W_S) {
         // ================================================================ RoPE group
+        // Two warps per TMEM lane quadrant; half rh rotates pair chunks 2rh and
+        // 2rh + 1 (pairs 32rh .. 32rh + 31) of every token row of its quadrant.
         const int et = threadIdx.x - 64;
+        const int rh = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -608,11 +620,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         int pend_nq = -1;   // queries of the item whose O is still to be read, or -1
         uint32_t pend_n = 0;
         auto readout = [&]() -> bool {
-            if (!grp_and<DT_BAR_R>(tc::mbar_wait(&sm.o_full, pend_n & 1u) && !sm.abort)) return false;
+            if (!grp_and<DT_BAR_R, DT_RGROUP>(tc::mbar_wait(&sm.o_full, pend_n & 1u) && !sm.abort)) return false;
             tc::tc_fence_after();
             const int *qp = sm.qpidx[pend_n & 3u];
             const int nq = pend_nq, nq16 = (nq + 15) & ~15;
-            for (int c0 = 0; c0 < nq16; c0 += 32) {
+            for (int c0 = 32 * rh; c0 < nq16; c0 += 64) {   // this half's 32-query slabs
                 uint32_t r[32];
                 tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
                 if (c0 + 16 < nq16)
@@ -631,7 +643,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             const int nt = token_tiles(__ldg(&items[i].Tb));
             for (int t = 0; t < nt; ++t) {
                 const uint32_t b = rc & 1u;
-                ok = grp_and<DT_BAR_R>(tc::mbar_wait(&sm.d1_full[b], (rc >> 1) & 1u) && !sm.abort);
+                ok = grp_and<DT_BAR_R, DT_RGROUP>(tc::mbar_wait(&sm.d1_full[b], (rc >> 1) & 1u) && !sm.abort);
                 if (!ok) break;
                 MILO_TRACE_EVENT(0, 2 * t);
                 tc::tc_fence_after();
@@ -639,9 +651,10 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 const int tok = t * FTILE + row;   // in-block token of this lane
                 const int tl = tok & 31, th = tok >> 5;
                 // pair chunk pc (16 pairs): x at columns 16pc.., y at 64 + 16pc..;
-                // packed fp16 results go to 8pc.. (x) and 64 + 8pc.. (y), columns of
-                // chunks this thread has already read
-                auto rot_chunk = [&](const uint32_t (&xr)[16], const uint32_t (&yr)[16], int pc) {
+                // packed fp16 results go to 32rh + 8j (x) and 64 + 32rh + 8j (y) for
+                // the half's j-th chunk: columns of the half's first chunk, which
+                // this thread has already read
+                auto rot_chunk = [&](const uint32_t (&xr)[16], const uint32_t (&yr)[16], int pc, int j) {
                     uint32_t px[8], py[8];
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
@@ -661,16 +674,17 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         px[v] = *reinterpret_cast<const uint32_t *>(&hx);
                         py[v] = *reinterpret_cast<const uint32_t *>(&hy);
                     }
-                    tc::tmem_st8(base + 8 * pc, px);
-                    tc::tmem_st8(base + 64 + 8 * pc, py);
+                    tc::tmem_st8(base + 32 * rh + 8 * j, px);
+                    tc::tmem_st8(base + 64 + 32 * rh + 8 * j, py);
                 };
 #pragma unroll 1
-                for (int pc = 0; pc < 4; ++pc) {   // pair chunk pc: writes land in columns of chunks <= pc
+                for (int j = 0; j < 2; ++j) {
+                    const int pc = 2 * rh + j;
                     uint32_t xa[16], ya[16];
                     tc::tmem_ld16(base + 16 * pc, xa);
                     tc::tmem_ld16(base + 64 + 16 * pc, ya);
                     tc::tmem_wait_ld();
-                    rot_chunk(xa, ya, pc);
+                    rot_chunk(xa, ya, pc, j);
                 }
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
@@ -687,14 +701,14 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         }
         if (ok && pend_nq >= 0) ok = readout();
         if (!ok) sm.abort = 1;
-    } else if (warp < 14) {
+    } else if (warp < DT_W_H) {
         // ================================================================ softmax groups
         // Two groups of 4 warps (one per TMEM lane quadrant, one token row per
         // thread); group sg owns the 32-column query slabs sg, sg + 2, ...  The
         // reference max, sums and P of a column belong to one group, so the
         // groups only meet at the counted arrivals.
-        const int sg = (warp - 6) >> 2;
-        const int gt = threadIdx.x - 192 - DT_GROUP * sg;   // thread within the group
+        const int sg = (warp - DT_W_S) >> 2;
+        const int gt = threadIdx.x - 32 * DT_W_S - DT_GROUP * sg;   // thread within the group
         const int et = gt + DT_GROUP * sg;                 // trace hooks: thread 0 of group 0
         const int bar_id = sg == 0 ? DT_BAR_S : DT_BAR_S2;
         const int quad = warp & 3;
@@ -939,24 +953,17 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             grp_sync_rt(bar_id);
             if (quad * 32 < g.R16V) {
                 uint8_t *sbase = sm.pbuf + pst * 16384 + (row >> 3) * lbo_p + (row & 7) * 16;
-                for (int c0 = 32 * sg; c0 < nq16; c0 += 64) {
-                    const int w = min(32, nq16 - c0);
-                    uint32_t r[32];
-                    tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                    if (w == 32)
-                        tc::tmem_ld16(tmem + DT_COL_OA + lane_off + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-                    tc::tmem_wait_ld();
-                    if (row < g.R16V) {
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int ch = c0 + 16 * hh;
-                            if (16 * hh >= w) break;
+                for (int c0 = 32 * sg; c0 < nq16; c0 += 64)
+                    for (int ch = c0; ch < min(c0 + 32, nq16); ch += 16) {
+                        uint32_t r[16];
+                        tc::tmem_ld16(tmem + DT_COL_OA + lane_off + ch, r);
+                        tc::tmem_wait_ld();
+                        if (row < g.R16V) {
                             uint32_t q8[8];
 #pragma unroll
                             for (int v = 0; v < 8; ++v) {
-                                const __half2 h2 = __floats2half2_rn(
-                                    __uint_as_float(r[16 * hh + 2 * v]) * sm.cscale[ch + 2 * v],
-                                    __uint_as_float(r[16 * hh + 2 * v + 1]) * sm.cscale[ch + 2 * v + 1]);
+                                const __half2 h2 = __floats2half2_rn(__uint_as_float(r[2 * v]) * sm.cscale[ch + 2 * v],
+                                                                     __uint_as_float(r[2 * v + 1]) * sm.cscale[ch + 2 * v + 1]);
                                 q8[v] = *reinterpret_cast<const uint32_t *>(&h2);
                             }
                             uint8_t *dst = sbase + (ch >> 3) * 128;
@@ -964,7 +971,6 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(q8[4], q8[5], q8[6], q8[7]);
                         }
                     }
-                }
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
@@ -984,7 +990,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         if (!ok) sm.abort = 1;
     } else {
         // ================================================================ helper warps
-        const int et = threadIdx.x - (64 + 3 * DT_GROUP);
+        const int et = threadIdx.x - 32 * DT_W_H;
         bool ok = true;
         // ---- rotated queries R(-p) q of item j, fp16, K-major [q/8][j/8][q%8][j%8];
         // four threads per query, 16 pairs each
