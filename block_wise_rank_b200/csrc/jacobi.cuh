@@ -29,6 +29,10 @@ constexpr int JAC_NPAIR = D / 2;                       // 64 pairs per round
 constexpr int JAC_NTRI = JAC_NPAIR * (JAC_NPAIR + 1) / 2;  // 2080 pair blocks (i <= i2)
 constexpr int JAC_LD = D + 1;                          // padded row stride of G and W
 
+// G is symmetric: only its upper triangle is kept up to date, entry (x, y)
+// lives at row min(x, y), column max(x, y)
+__device__ __forceinline__ int jac_g(int x, int y) { return min(x, y) * JAC_LD + max(x, y); }
+
 struct JacobiSmem {
     float G[D * JAC_LD];
     float W[D * JAC_LD];
@@ -102,7 +106,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
             rot = __syncthreads_or(rot);
             any |= rot;
             if (!rot) continue;   // uniform across the CTA
-            // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2, mirrored
+            // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2 (upper triangle)
             for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
                 const int i = sm.tri[e][0], i2 = sm.tri[e][1];
                 const int p = sm.p[i], q = sm.q[i];
@@ -114,24 +118,24 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                         sm.G[p * JAC_LD + p] -= tn * apq;
                         sm.G[q * JAC_LD + q] += tn * apq;
                         sm.G[p * JAC_LD + q] = 0.f;
-                        sm.G[q * JAC_LD + p] = 0.f;
                     }
                     continue;
                 }
                 const float c2 = sm.c[i2], s2 = sm.s[i2];
                 if (s1 == 0.f && s2 == 0.f) continue;   // neither pair rotates: block unchanged
                 const int p2 = sm.p[i2], q2 = sm.q[i2];
-                const float a = sm.G[p * JAC_LD + p2], bb = sm.G[p * JAC_LD + q2];
-                const float cc = sm.G[q * JAC_LD + p2], ee = sm.G[q * JAC_LD + q2];
+                const int ia = jac_g(p, p2), ib = jac_g(p, q2), ic = jac_g(q, p2), ie = jac_g(q, q2);
+                const float a = sm.G[ia], bb = sm.G[ib];
+                const float cc = sm.G[ic], ee = sm.G[ie];
                 // columns (p2, q2) by J2, then rows (p, q) by J1^T
                 const float a1 = c2 * a - s2 * bb, b1 = s2 * a + c2 * bb;
                 const float c1_ = c2 * cc - s2 * ee, e1 = s2 * cc + c2 * ee;
                 const float na = c1 * a1 - s1 * c1_, nc = s1 * a1 + c1 * c1_;
                 const float nb = c1 * b1 - s1 * e1, ne = s1 * b1 + c1 * e1;
-                sm.G[p * JAC_LD + p2] = na; sm.G[p2 * JAC_LD + p] = na;
-                sm.G[p * JAC_LD + q2] = nb; sm.G[q2 * JAC_LD + p] = nb;
-                sm.G[q * JAC_LD + p2] = nc; sm.G[p2 * JAC_LD + q] = nc;
-                sm.G[q * JAC_LD + q2] = ne; sm.G[q2 * JAC_LD + q] = ne;
+                sm.G[ia] = na;
+                sm.G[ib] = nb;
+                sm.G[ic] = nc;
+                sm.G[ie] = ne;
             }
             // W <- W J: columns (p_i, q_i) of every row
             for (int e = tid; e < D * JAC_NPAIR; e += JAC_THREADS) {
