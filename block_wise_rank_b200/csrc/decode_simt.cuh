@@ -33,6 +33,7 @@ struct DecodeArgs {
     float *part_o;             // [L][S][Hq][n_sel][D]
     float2 *part_ml;           // [L][S][Hq][n_sel] (max, sum)
     float *out;                // [L][S][Hq][D]
+    int32_t *claim;            // tensor-core path: next unclaimed work item (zeroed before the launch)
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every

@@ -72,6 +72,7 @@ constexpr int DT_RING = 96 * 1024;                     // ring bytes for A_K, A_
 constexpr int DT_NBAR = 32;                            // ring tiles in flight at most
 constexpr int DT_TILE_MAX = 128 * 256;                 // 128 rank rows x 128 tokens (or channels) x 16 bit
 constexpr int DT_NQ = 128;                             // queries per item (pass)
+constexpr int DT_NITAB = 32;                           // claimed items in flight at most
 constexpr uint32_t DT_TMEM_COLS = 512;
 constexpr uint32_t DT_COL_D1 = 0;                      // two 128-column rebuild buffers
 constexpr uint32_t DT_COL_D2 = 256;                    // scores: one 128-column buffer or two of 64
@@ -103,6 +104,8 @@ struct DecTcSmem {
     int cmax[DT_NQ];                             // column maxima, order-preserving int encoding
     int qpidx[4][DT_NQ];                         // partial index of each query, per item (mod 4)
     uint32_t toff[DT_NBAR], tlen[DT_NBAR];       // ring offset and bytes of each tile in flight
+    int itab[DT_NITAB];                          // n-th item claimed by this CTA (slot n % NITAB), -1: none left
+    uint64_t item_full[DT_NITAB];                // slot n % NITAB holds item n
     // conv: one arrival per ring tile, in ring order, once an A_V / B_V tile
     // is fp16 (A_K tiles pass straight through), so that slot k % NBAR is in
     // phase k / NBAR exactly like full and empty
@@ -306,7 +309,14 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
     DecTcSmem &sm = *reinterpret_cast<DecTcSmem *>(dt_raw + ((128u - (tc::smem_u32(dt_raw) & 127u)) & 127u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_items = (int64_t)a.L * a.H * pstart[a.n_b];
-    const int64_t stride = gridDim.x;
+    // Items are claimed dynamically: the producer takes the next unclaimed one
+    // from a global counter and publishes it in the item table; every role
+    // walks the same sequence n = 0, 1, ... of this CTA's items.  (The factor
+    // ring keeps the producer fewer than NITAB items ahead of the slowest role,
+    // so a slot is never rewritten before every role has read it.)
+    auto item_ready = [&](uint32_t n) { return mbar_test(&sm.item_full[n % DT_NITAB], (n / DT_NITAB) & 1u); };
+    auto item_wait = [&](uint32_t n) { return tc::mbar_wait(&sm.item_full[n % DT_NITAB], (n / DT_NITAB) & 1u); };
+    auto item_at = [&](uint32_t n) -> int64_t { return sm.itab[n % DT_NITAB]; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < DT_NBAR; ++s) {
@@ -314,6 +324,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             tc::mbar_init(&sm.empty[s], 1);
             tc::mbar_init(&sm.conv[s], 1);
         }
+        for (int s = 0; s < DT_NITAB; ++s) tc::mbar_init(&sm.item_full[s], 1);
         tc::mbar_init(&sm.bk_full, 1);
         tc::mbar_init(&sm.bk_empty, 1);
         for (int k = 0; k < 2; ++k) {
@@ -416,8 +427,18 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             ++seq;
         };
         uint32_t n = 0;
-        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
-            if (__shfl_sync(0xffffffffu, (int)(sm.abort != 0), 0)) break;
+        for (; ok; ++n) {
+            int claimed = -1;
+            if (lane == 0) {
+                if (!sm.abort) {
+                    const int c = atomicAdd(a.claim, 1);
+                    if (c < n_items) claimed = c;
+                }
+                sm.itab[n % DT_NITAB] = claimed;
+                tc::mbar_arrive(&sm.item_full[n % DT_NITAB]);   // releases the table entry
+            }
+            const int64_t i = __shfl_sync(0xffffffffu, claimed, 0);
+            if (i < 0) break;
             const DtItem it = items[i];
             const DtGeo g = dt_geo(it.Tb, it.rK, it.rV, it.nq);
             const uint8_t *bK = dataK + 2 * it.offK, *bV = dataV + 2 * it.offV;
@@ -458,11 +479,25 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // ================================================================ MMA issuer
         if (lane == 0) {
             const uint32_t id_rb = tc::idesc_f16(128, 128, 1, 1, 1);   // bf16, A/B MN-major
-            const int64_t i0 = blockIdx.x;
-            const DtGeo g0 = dt_geo(items, i0, n_items), g1 = dt_geo(items, i0 + stride, n_items);
-            // each queue holds the geometry of its item and of the next one
-            int64_t iR = i0, iS = i0, iP = i0;
-            DtGeo gR = g0, gRn = g1, gS = g0, gSn = g1, gP = g0, gPn = g1;
+            // each queue holds its item (kPend until the producer has claimed it,
+            // -1 once none is left) and the next one when already known
+            constexpr int64_t kPend = -2;
+            int64_t iR = kPend, iS = kPend, iP = kPend, iRn = kPend, iSn = kPend, iPn = kPend;
+            DtGeo gR = dt_geo(1, 0, 0, 0), gS = gR, gP = gR, gRn = gR, gSn = gR, gPn = gR;
+            // resolve a queue's current / next item from the item table
+            auto resolve = [&](int64_t &i, DtGeo &g, int64_t &in, DtGeo &gn, uint32_t n) {
+                if (i == kPend && in != kPend) {
+                    i = in; g = gn; in = kPend;
+                }
+                if (i == kPend && item_ready(n)) {
+                    i = item_at(n);
+                    if (i >= 0) g = dt_geo(items, i, n_items);
+                }
+                if (i >= 0 && in == kPend && item_ready(n + 1)) {
+                    in = item_at(n + 1);
+                    if (in >= 0) gn = dt_geo(items, in, n_items);
+                }
+            };
             uint32_t nR = 0, tR = 0, seqR = 0, rc = 0;             // rebuild queue
             uint32_t nS = 0, tS = 0, rcS = 0;                      // scores queue
             uint32_t nP = 0, tP = 0, seqP = 0;                     // PV / O queue
@@ -475,11 +510,13 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             uint32_t backoff = 32;
             bool ok = true;
             while (ok) {
-                const bool doneR = iR >= n_items, doneS = iS >= n_items, doneP = iP >= n_items;
-                if (doneR && doneS && doneP) break;
+                resolve(iR, gR, iRn, gRn, nR);
+                resolve(iS, gS, iSn, gSn, nS);
+                resolve(iP, gP, iPn, gPn, nP);
+                if (iR == -1 && iS == -1 && iP == -1) break;
                 bool prog = false;
                 // ---------------------------------------------------- rebuild
-                if (!doneR) {
+                if (iR >= 0) {
                     const uint32_t k = seqR + dt_pos_k(tR), s = k % DT_NBAR, b = rc & 1u;
                     if (mbar_test(&sm.full[s], (k / DT_NBAR) & 1u) && (tR > 0 || mbar_test(&sm.bk_full, nR & 1u)) &&
                         mbar_test(&sm.d1_empty[b], ((rc >> 1) & 1u) ^ 1u)) {
@@ -498,15 +535,13 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             seqR += dt_ring_tiles(gR);
                             tR = 0;
                             ++nR;
-                            iR += stride;
-                            gR = gRn;
-                            gRn = dt_geo(items, iR + stride, n_items);
+                            iR = kPend;
                         }
                         prog = true;
                     }
                 }
                 // ---------------------------------------------------- scores
-                if (!doneS) {
+                if (iS >= 0) {
                     const uint32_t b = rcS & 1u;
                     const uint32_t d2b = gS.dbl ? (tS & 1u) : 0u;
                     // a full-width scores buffer also covers the second half-buffer
@@ -532,15 +567,13 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         if ((int)++tS == gS.nt) {
                             tS = 0;
                             ++nS;
-                            iS += stride;
-                            gS = gSn;
-                            gSn = dt_geo(items, iS + stride, n_items);
+                            iS = kPend;
                         }
                         prog = true;
                     }
                 }
                 // ---------------------------------------------------- PV and O
-                if (!doneP) {
+                if (iP >= 0) {
                     const uint32_t pb = gP.dbl ? (tP & 1u) : 0u;
                     const uint32_t lbo_p = (uint32_t)(gP.nq16 / 8) * 128u;
                     const uint32_t sp = spb + pb * 16384u;
@@ -579,9 +612,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             seqP += dt_ring_tiles(gP);
                             tP = 0;
                             ++nP;
-                            iP += stride;
-                            gP = gPn;
-                            gPn = dt_geo(items, iP + stride, n_items);
+                            iP = kPend;
                         }
                         prog = true;
                     }
@@ -639,7 +670,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             pend_nq = -1;
             return true;
         };
-        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
+        for (; ok; ++n) {
+            ok = grp_and<DT_BAR_R, DT_RGROUP>(item_wait(n) && !sm.abort);
+            if (!ok) break;
+            const int64_t i = item_at(n);
+            if (i < 0) break;
             const int nt = token_tiles(__ldg(&items[i].Tb));
             for (int t = 0; t < nt; ++t) {
                 const uint32_t b = rc & 1u;
@@ -728,7 +763,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             return w;
         };
 
-        for (int64_t i = blockIdx.x; i < n_items && ok; i += stride, ++n) {
+        for (; ok; ++n) {
+            ok = grp_and_rt(bar_id, item_wait(n) && !sm.abort);
+            if (!ok) break;
+            const int64_t i = item_at(n);
+            if (i < 0) break;
             const DtGeo g = dt_geo(items, i, n_items);
             const int Tb = __ldg(&items[i].Tb);
             const int nq = g.nq, nq16 = g.nq16;
@@ -1050,15 +1089,24 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // Two independent streams, served whichever is ready: the ring tiles
         // in order (A_K tiles pass, A_V tiles and B_V to fp16 in place), and
         // each next item's queries once the current item's scores are done.
-        int64_t ic = blockIdx.x, iq = blockIdx.x;
-        uint32_t seqC = 0, nqp = 0;
+        // Each stream's item is kPend until the producer has claimed it, -1 once
+        // none is left.
+        constexpr int64_t kPend = -2;
+        int64_t ic = kPend, iq = kPend;
+        uint32_t seqC = 0, nc = 0, nqp = 0;
         int kc = 0;
-        DtGeo gc = dt_geo(items, ic, n_items);
+        DtGeo gc = dt_geo(1, 0, 0, 0);
         uint64_t t_last = tc::globaltimer();
         uint32_t backoff = 64;
-        while (ok && (ic < n_items || iq < n_items)) {
+        while (ok) {
+            if (ic == kPend && grp_and<DT_BAR_H, DT_HELP>(item_ready(nc))) {
+                ic = item_at(nc);
+                if (ic >= 0) gc = dt_geo(items, ic, n_items);
+            }
+            if (iq == kPend && grp_and<DT_BAR_H, DT_HELP>(item_ready(nqp))) iq = item_at(nqp);
+            if (ic == -1 && iq == -1) break;
             bool did = false;
-            if (ic < n_items) {
+            if (ic >= 0) {
                 int tt;
                 const int kind = dt_tile_at(gc.nt, kc, &tt);
                 const uint32_t k = seqC + kc, s = k % DT_NBAR;
@@ -1071,21 +1119,21 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         grp_sync<DT_BAR_H, DT_HELP>();
                     }
                     if (et == 0) tc::mbar_arrive(&sm.conv[s]);
-                    if (et == 0) MILO_TRACE_TILE(1, (uint32_t)((ic - blockIdx.x) / stride), kc);
+                    if (et == 0) MILO_TRACE_TILE(1, nc, kc);
                     if (++kc == dt_ring_tiles(gc)) {
                         seqC += dt_ring_tiles(gc);
                         kc = 0;
-                        ic += stride;
-                        gc = dt_geo(items, ic, n_items);
+                        ++nc;
+                        ic = kPend;
                     }
                     did = true;
                 }
             }
-            if (iq < n_items && grp_and<DT_BAR_H, DT_HELP>(mbar_test(&sm.q_empty, (nqp & 1u) ^ 1u))) {
+            if (iq >= 0 && grp_and<DT_BAR_H, DT_HELP>(mbar_test(&sm.q_empty, (nqp & 1u) ^ 1u))) {
                 ok = qprep(iq, nqp);
                 if (et == 0) MILO_TRACE_TILE(1, nqp, 14);
-                iq += stride;
                 ++nqp;
+                iq = kPend;
                 did = true;
             }
             if (did) {

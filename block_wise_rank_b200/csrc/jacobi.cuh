@@ -137,9 +137,10 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                 sm.G[ic] = nc;
                 sm.G[ie] = ne;
             }
-            // W <- W J: columns (p_i, q_i) of every row
+            // W <- W J: columns (p_i, q_i) of every row; consecutive threads take
+            // consecutive rows of one pair (row stride 129: no bank conflicts)
             for (int e = tid; e < D * JAC_NPAIR; e += JAC_THREADS) {
-                const int i = e % JAC_NPAIR, j = e / JAC_NPAIR;
+                const int j = e % D, i = e / D;
                 const float s1 = sm.s[i];
                 if (s1 == 0.f) continue;
                 const float c1 = sm.c[i];

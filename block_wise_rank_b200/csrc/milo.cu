@@ -507,7 +507,7 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     const int64_t slots = (int64_t)S * n_sel;
     const int64_t rows = (int64_t)f->shape.L * S * Hq;
     size_t at = 0;
-    at = align_up(at + sizeof(int32_t) * (f->n_b + 1) * 3);            // counts / cursor, starts, passes
+    at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursor, starts, passes, claim
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
     at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
@@ -537,7 +537,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     int32_t *cnt = (int32_t *)(w + at);
     int32_t *start = cnt + (n_b + 1);
     int32_t *pstart = start + (n_b + 1);
-    at = align_up(at + sizeof(int32_t) * (n_b + 1) * 3);
+    int32_t *claim = pstart + (n_b + 1);   // next unclaimed tensor-core work item
+    at = align_up(at + sizeof(int32_t) * ((n_b + 1) * 3 + 1));
     int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
     float2 *rope_q = (float2 *)(w + at);
     float2 *rope_t = rope_q + slots * HALF;
@@ -556,8 +557,10 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.slot_start = start; a.slot_list = list;
     a.rope_q = rope_q; a.rope_t = rope_t;
     a.part_o = part_o; a.part_ml = part_ml; a.out = out;
+    a.claim = claim;
 
-    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (n_b + 1), s);
+    // counts and the claim counter to 0 (starts and passes are written by the scan)
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ((n_b + 1) * 3 + 1), s);
     if (e != cudaSuccess) return cuda_check(e, "memset");
     const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
