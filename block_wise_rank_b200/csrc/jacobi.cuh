@@ -27,14 +27,20 @@ namespace milo {
 constexpr int JAC_THREADS = 512;
 constexpr int JAC_NPAIR = D / 2;                       // 64 pairs per round
 constexpr int JAC_NTRI = JAC_NPAIR * (JAC_NPAIR + 1) / 2;  // 2080 pair blocks (i <= i2)
-constexpr int JAC_LD = D + 1;                          // padded row stride of G and W
+constexpr int JAC_LD = D + 1;                          // padded row stride of W
+constexpr int JAC_GT = D * (D + 1) / 2;                // packed upper triangle of G
 
-// G is symmetric: only its upper triangle is kept up to date, entry (x, y)
-// lives at row min(x, y), column max(x, y)
-__device__ __forceinline__ int jac_g(int x, int y) { return min(x, y) * JAC_LD + max(x, y); }
+// G is symmetric and only its upper triangle is stored, packed by rows:
+// entry (x, y) lives at row u = min(x, y), offset max(x, y) - u into a row
+// that starts at u (2d - u + 1) / 2.  (Half of the full tile, so that two
+// CTAs fit on an SM.)
+__device__ __forceinline__ int jac_g(int x, int y) {
+    const int u = min(x, y), v = max(x, y);
+    return ((u * (2 * D + 1 - u)) >> 1) + (v - u);
+}
 
 struct JacobiSmem {
-    float G[D * JAC_LD];
+    float G[JAC_GT];
     float W[D * JAC_LD];
     float c[JAC_NPAIR], s[JAC_NPAIR], t[JAC_NPAIR];
     int p[JAC_NPAIR], q[JAC_NPAIR];
@@ -48,7 +54,7 @@ struct JacobiSmem {
 // eigenvectors, columns sorted by descending eigenvalue (W[j][k] = v_k[j]).
 // sigma_K/sigma_V: [n_blk][128] singular values, descending; entries past
 // min(T_b, d) are set to 0 (the rank of a T_b x d block).
-__global__ void __launch_bounds__(JAC_THREADS, 1)
+__global__ void __launch_bounds__(JAC_THREADS, 2)
 k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restrict__ sigma_V,
          int64_t n_blk, int Tn, int block_len, int n_b, int max_sweeps, float tol) {
     extern __shared__ __align__(16) unsigned char jac_raw[];
@@ -59,7 +65,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
 
     for (int e = tid; e < D * D; e += JAC_THREADS) {
         int i = e / D, j = e % D;
-        sm.G[i * JAC_LD + j] = Gg[e];
+        if (i <= j) sm.G[jac_g(i, j)] = Gg[e];
         sm.W[i * JAC_LD + j] = (i == j) ? 1.f : 0.f;
     }
     for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
@@ -72,7 +78,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
     __syncthreads();
     if (tid < 32) {
         float tr = 0.f;
-        for (int k = tid; k < D; k += 32) tr += fabsf(sm.G[k * JAC_LD + k]);
+        for (int k = tid; k < D; k += 32) tr += fabsf(sm.G[jac_g(k, k)]);
         for (int o = 16; o; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
         if (tid == 0) sm.floor_abs = 1e-10f * tr;
     }
@@ -91,7 +97,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                 if (tid == 0) { a = r; b = D - 1; }
                 else { a = (r + tid) % (D - 1); b = (r - tid + (D - 1)) % (D - 1); }
                 int p = min(a, b), q = max(a, b);
-                float app = sm.G[p * JAC_LD + p], aqq = sm.G[q * JAC_LD + q], apq = sm.G[p * JAC_LD + q];
+                float app = sm.G[jac_g(p, p)], aqq = sm.G[jac_g(q, q)], apq = sm.G[jac_g(p, q)];
                 float c = 1.f, s = 0.f, tn = 0.f;
                 if (fabsf(apq) > floor_abs && fabsf(apq) > tol * sqrtf(fabsf(app)) * sqrtf(fabsf(aqq))) {
                     float zeta = (aqq - app) / (2.f * apq);
@@ -114,10 +120,11 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                 if (i == i2) {
                     if (s1 != 0.f) {
                         const float tn = sm.t[i];
-                        const float apq = sm.G[p * JAC_LD + q];
-                        sm.G[p * JAC_LD + p] -= tn * apq;
-                        sm.G[q * JAC_LD + q] += tn * apq;
-                        sm.G[p * JAC_LD + q] = 0.f;
+                        const int ipq = jac_g(p, q);
+                        const float apq = sm.G[ipq];
+                        sm.G[jac_g(p, p)] -= tn * apq;
+                        sm.G[jac_g(q, q)] += tn * apq;
+                        sm.G[ipq] = 0.f;
                     }
                     continue;
                 }
@@ -157,7 +164,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
     MILO_TRACE_JACOBI(sweeps_done);
 
     // eigenvalues, stable descending order
-    if (tid < D) sm.lam[tid] = sm.G[tid * JAC_LD + tid];
+    if (tid < D) sm.lam[tid] = sm.G[jac_g(tid, tid)];
     __syncthreads();
     if (tid < D) {
         const float lk = sm.lam[tid];
