@@ -329,3 +329,39 @@ def test_decode_tensor_core_path(oracle_mod, monkeypatch, frac):
         ref = _decode_ref(oracle_mod, U[0], U[1], l, hq // G, 2, q[l, s, hq].double().numpy(), sel[s].tolist(),
                           pos[s].tolist(), 1e6)
         assert _rel_inf(out[l, s, hq], ref) <= DEC_TOL
+
+
+@pytest.mark.parametrize("qscale", [60.0, 150.0])
+def test_decode_tensor_core_large_scores(oracle_mod, monkeypatch, qscale):
+    """Scores spanning far more than 2^8 in the exp2 domain (queries scaled up):
+    the tensor-core kernel must raise its per-query reference max and rescale
+    the running O_A^T and sums, tile after tile (at 150x the scores span ~30
+    units of log2, so P would overflow fp16 without it), giving the softmax of
+    the oracle.  The fp16 rounding of the rotated keys
+    and queries grows with the score magnitude, so the bound is the one for
+    bf16 factors (2e-2), against the oracle and the fp32 CUDA-core path on the
+    same factors."""
+    L, H, G, T, bl, S = 1, 2, 4, 1536, 512, 6
+    K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=61, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=62, out_dtype=torch.bfloat16)
+    f = milo.milo_compress(K.cuda(), V.cuda(), bl, milo.default_params(factor_dtype="bf16", budget_frac=0.5))
+    g = torch.Generator().manual_seed(int(qscale))
+    q = torch.randn(L, S, H * G, 128, generator=g) * qscale
+    sel = torch.stack([torch.randperm(3, generator=g) for _ in range(S)]).to(torch.int32)
+    pos = (sel * bl).to(torch.int32)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    assert np.all(np.isfinite(out))
+    monkeypatch.setenv("MILO_FORCE_SIMT", "1")
+    ref_cc = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), pos.cuda(), rope_base=1e6).cpu().numpy()
+    monkeypatch.delenv("MILO_FORCE_SIMT")
+    U = [A.unpack(f, 0), A.unpack(f, 1)]
+    for u in U:
+        u["H"] = H
+    nb = math.ceil(T / bl)
+    for s in range(S):
+        for hq in range(H * G):
+            assert _rel_inf(out[0, s, hq], ref_cc[0, s, hq]) <= DEC_TOL_BF16_OWN, (s, hq)
+            ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // G, nb, q[0, s, hq].double().numpy(),
+                              sel[s].tolist(), pos[s].tolist(), 1e6)
+            assert _rel_inf(out[0, s, hq], ref) <= DEC_TOL_BF16_OWN, (s, hq)
