@@ -19,8 +19,9 @@ together in the order the pages give them:
   abstract: each block holds several many-shot examples; rank budgets follow
   the information entropy of each block.
 
-Readings of what the pages leave open (eps, budget rounding, tie order, RoPE
-convention, rank-0 blocks, INT8 rounding) are the ones listed in the design doc.
+Where the pages leave a point open (eps, budget rounding, tie order, RoPE
+convention, rank-0 blocks, INT8 rounding), the routine concerned states the
+reading it takes.
 """
 from __future__ import annotations
 

@@ -19,8 +19,8 @@
  *    greedy marginal gains log(1 + sigma^2/eps^2) under a global budget.
  *
  * Every routine is the plain definition written out, in fp64, with the
- * steps in the order the pages give them.  Readings of points the pages
- * leave open are listed in the design doc and repeated at each routine.
+ * steps in the order the pages give them.  Where the pages leave a point
+ * open, the routine concerned states the reading it takes.
  */
 #include <float.h>
 #include <math.h>
