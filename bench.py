@@ -163,6 +163,25 @@ def count_launches(fn):
     return n
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(values_ms, world, device):
+    """Element-wise maximum of per-rank device timings over all ranks: the
+    slowest rank sets the job's time."""
+    t = torch.tensor(values_ms, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(dec_bytes_per_rank, blocks_per_rank, steps, dec_ms, comp_ms, world):
+    """Whole-job decode GB/s and compression blocks/s: every rank is a replica
+    doing the same work, so the job moves world x one rank's work in the
+    slowest rank's time."""
+    dec_gbs = dec_bytes_per_rank * steps / (dec_ms / 1e3) / 1e9 * world
+    comp_bps = blocks_per_rank * steps / (comp_ms / 1e3) * world
+    return dec_gbs, comp_bps
+
+
 # ------------------------------------------------------------------ arms
 def workload_of(args):
     import dataclasses
@@ -241,17 +260,13 @@ def run_ours(args, rank, world):
     comp_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
     st = milo.milo_get_status()
-    times = torch.tensor([total_ms, sum(comp_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, comp_sum, dec_sum = times.tolist()
+    total_ms, comp_sum, dec_sum = max_over_ranks([total_ms, sum(comp_ms), sum(dec_ms)], world, dev)
 
     # end-to-end decode through the public call with host buffers
     e2e = run_e2e(f, w, dec_inputs, out, dws, stream, args.steps)
     kernel = decode_kernel_timing(f, w, dec_inputs, out, dws, stream)
     pk = peaks()
-    dec_gbs = dbytes * args.steps / (dec_sum / 1e3) / 1e9 * world
-    comp_bps = n_blocks * args.steps / (comp_sum / 1e3) * world
+    dec_gbs, comp_bps = job_throughput(dbytes, n_blocks, args.steps, dec_sum, comp_sum, world)
     res = dict(
         metric=METRIC, value=round(dec_gbs, 2), unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=round(total_ms / args.steps, 3), higher_is_better=True, scaling="weak", vs_baseline=None,
