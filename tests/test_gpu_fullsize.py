@@ -2,7 +2,7 @@
 64K-token 28-layer and 131K-token 28-layer Qwen2.5-shaped caches), through
 the C ABI, on sampled outputs the oracle can compute one by one:
 
-  * sum of ranks == R and eps == eps_rel * max sigma_1, exactly;
+  * sum of ranks == R and eps == the oracle's eps of the GPU's sigma, exactly;
   * every rank bit-exact against the oracle allocator fed the GPU's sigma/eps
     (all N_blk * 128 keys of a kind);
   * packed offsets == exclusive scan of the padded block sizes;
@@ -41,8 +41,9 @@ def _check_kind(oracle_mod, f, kind, w, X, params, rng, n_sigma_blocks=3):
     nb = w.n_b
     R = oracle_mod.budget(L, H, T, bl, d, params.budget_frac, params.budget_abs)
     assert meta["R"] == R and int(meta["ranks"].sum()) == R
-    s1 = meta["sigma"][:, 0].reshape(L * H, nb).astype(np.float64).max(axis=1)
-    assert np.array_equal(meta["eps"], params.eps_rel * s1)
+    eps_ref = oracle_mod.eps_of(meta["sigma"].astype(np.float64).reshape(L, H, nb, d), params.eps_rel,
+                                params.eps_scope)
+    assert np.array_equal(meta["eps"], eps_ref.reshape(-1))
     ref = oracle_mod.allocate(meta["sigma"].astype(np.float64).reshape(L, H, nb, d), meta["eps"].reshape(L, H),
                               T, bl, R, params.r_min, params.r_max)
     assert np.array_equal(meta["ranks"], ref.reshape(-1))

@@ -4,7 +4,7 @@ same seeded inputs.
 Tolerances (written where they are used):
   sigma:   |s_gpu - s_ref| <= 1e-4 * s_1 per block, and elementwise relative
            1e-4 where s_ref >= 0.1 * s_1;
-  eps:     bit-exact (eps_rel times the max of the GPU's own sigma_1);
+  eps:     bit-exact against the oracle's eps of the GPU's own sigma;
   ranks:   bit-exact against the oracle allocator fed the GPU's sigma and eps;
   recon:   | ||X - A B||_F^2 - sum_{k > r_b} s_ref_k^2 | <= 1e-3 * that sum;
   decode:  ||o_gpu - o_ref||_inf / ||o_ref||_inf per output vector:
@@ -86,11 +86,10 @@ def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None)
         u["H"] = H
         U.append(u)
         assert u["R"] == R and int(u["ranks"].sum()) == R
-        # eps: eps_rel * max_b sigma_{b,1} of the GPU's sigma, per (layer, head)
-        s1 = u["sigma"][:, 0].reshape(L * H, nb).astype(np.float64).max(axis=1)
-        if params.eps_scope == 1:
-            s1 = np.full_like(s1, s1.max())
-        assert np.array_equal(u["eps"], params.eps_rel * s1)
+        # eps: the oracle's eps of the GPU's own sigma, bit for bit
+        eps_ref = oracle_mod.eps_of(u["sigma"].astype(np.float64).reshape(L, H, nb, d), params.eps_rel,
+                                    params.eps_scope)
+        assert np.array_equal(u["eps"], eps_ref.reshape(-1))
         # ranks: bit-exact against the oracle allocator on the same sigma and eps
         r_ref = oracle_mod.allocate(u["sigma"].astype(np.float64).reshape(L, H, nb, d), u["eps"].reshape(L, H),
                                     T, block_len, R, params.r_min, params.r_max)

@@ -179,6 +179,44 @@ def test_keys_groups_and_zero_eps(oracle_mod):
     assert key.tolist() == [[4.0, 1.0], [1.0, 0.25], [0.0, 0.0]]
 
 
+def _eps_fixture_ok(eps_fn, c):
+    """True when eps_fn reproduces the hand-worked values of both scopes."""
+    sig = np.array(c["sigma"], dtype=np.float64)
+    for scope, key in ((0, "eps_scope0"), (1, "eps_scope1")):
+        got = np.asarray(eps_fn(sig, c["eps_rel"], scope), dtype=np.float64)
+        want = np.array(c[key], dtype=np.float64)
+        if got.shape != want.shape or not np.allclose(got, want, rtol=1e-15, atol=0):
+            return False
+    return True
+
+
+def test_eps_golden_both_scopes(oracle_mod):
+    """eps = eps_rel * max_b sigma_{b,1}: hand-worked values for scope 0 (per
+    layer and head) and scope 1 (one per kind).  Plausible slips in the
+    reduction (wrong axis, wrong component, no global max for scope 1) are
+    run against the same fixture and must be rejected by it."""
+    c = json.load(open(os.path.join(GOLDEN, "eps_tiny.json")))
+    assert _eps_fixture_ok(oracle_mod.eps_of, c)
+
+    def wrong_axis(s, rel, scope):            # max over heads instead of blocks
+        top = s[..., 0].max(axis=1)
+        return rel * (np.full_like(top, top.max()) if scope == 1 else top)
+
+    def wrong_component(s, rel, scope):       # sigma_2 instead of sigma_1
+        top = s[..., 1].max(axis=-1)
+        return rel * (np.full_like(top, top.max()) if scope == 1 else top)
+
+    def last_block(s, rel, scope):            # first-to-last instead of the max
+        top = s[:, :, -1, 0]
+        return rel * (np.full_like(top, top.max()) if scope == 1 else top)
+
+    def scope_ignored(s, rel, scope):         # scope 1 treated like scope 0
+        return rel * s[..., 0].max(axis=-1)
+
+    for bad in (wrong_axis, wrong_component, last_block, scope_ignored):
+        assert not _eps_fixture_ok(bad, c), bad.__name__
+
+
 def test_budget_and_blocking(oracle_mod):
     assert oracle_mod.block_lengths(2048, 256) == [256] * 8
     assert oracle_mod.block_lengths(1000, 256) == [256, 256, 256, 232]
