@@ -12,8 +12,8 @@
 // K-hat nor V-hat is written to memory.  Each (query, selected slot) gets a
 // partial (max, sum, unnormalised output) merged by k_combine.
 //
-// This kernel serves every factor dtype and is the FP32 path; the tensor
-// core kernel in decode_tc.cuh serves bf16 / int8 factors.
+// This kernel is the FP32 path: it serves f32 and int8 factors; the tensor
+// core kernel in decode_tc.cuh serves bf16 factors.
 #pragma once
 #include "common.cuh"
 
@@ -30,29 +30,45 @@ struct DecodeArgs {
     const int32_t *slot_list;  // [S * n_sel] slot = s * n_sel + j
     const float2 *rope_q;      // [S * n_sel][64] (cos, sin)(p theta_i)
     const float2 *rope_t;      // [block_len][64] (cos, sin)(t theta_i)
-    float *part_o;             // [L][S][Hq][n_sel][D]
+    const float2 *rope_lo;     // [32][64] (cos, sin)(u theta_i), u < 32: in-block angle, low five bits
+    const float4 *rope_hi;     // [16][32] (cos, sin)(32 v theta_i) of pairs (2k, 2k+1): (c0, c1, s0, s1)
+    float *part_o;             // [L][S][Hq][n_sel][D] (CUDA-core path)
+    __half *part_o16;          // [L][S][Hq][n_sel][D] (tensor-core path)
     float2 *part_ml;           // [L][S][Hq][n_sel] (max, sum)
     float *out;                // [L][S][Hq][D]
     int32_t *claim;            // tensor-core path: next unclaimed work item (zeroed before the launch)
+    uint64_t wait_ns;          // tensor-core path: limit of every wait on the device
+    int inject;                // tensor-core path: 1 = withhold one copy (tests of the bounded waits)
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
-// in-block token, angles in double, theta_i = base^(-2i/d).
+// in-block token, angles in double, theta_i = base^(-2i/d).  The same
+// in-block angles split as t = 32 v + u (u < 32, v < 16) for the tensor-core
+// path: (u theta_i) per pair and (32 v theta_i) per pair of pairs.
 __global__ void k_rope_tables(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int n_slots,
-                              int block_len, double base, float2 *__restrict__ rope_q, float2 *__restrict__ rope_t) {
-    const int64_t total = (int64_t)(n_slots + block_len) * HALF;
+                              int block_len, double base, float2 *__restrict__ rope_q, float2 *__restrict__ rope_t,
+                              float2 *__restrict__ rope_lo, float4 *__restrict__ rope_hi) {
+    const int64_t total = (int64_t)(n_slots + block_len + 32 + 16) * HALF;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int i = (int)(e % HALF);
         const int64_t row = e / HALF;
         const double theta = pow(base, -2.0 * (double)i / (double)D);
         double p;
         if (row < n_slots) p = pos ? (double)pos[row] : (double)sel[row] * (double)block_len;
-        else p = (double)(row - n_slots);
+        else if (row < n_slots + block_len) p = (double)(row - n_slots);
+        else if (row < n_slots + block_len + 32) p = (double)(row - n_slots - block_len);
+        else p = 32.0 * (double)(row - n_slots - block_len - 32);
         double sn, cs;
         sincos(p * theta, &sn, &cs);
         const float2 v = make_float2((float)cs, (float)sn);
         if (row < n_slots) rope_q[row * HALF + i] = v;
-        else rope_t[(row - n_slots) * HALF + i] = v;
+        else if (row < n_slots + block_len) rope_t[(row - n_slots) * HALF + i] = v;
+        else if (row < n_slots + block_len + 32) rope_lo[(row - n_slots - block_len) * HALF + i] = v;
+        else {
+            float *h = reinterpret_cast<float *>(rope_hi + (row - n_slots - block_len - 32) * (HALF / 2) + i / 2);
+            h[i & 1] = v.x;
+            h[2 + (i & 1)] = v.y;
+        }
     }
 }
 
@@ -274,10 +290,18 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
 }
 
 // out[l][s][hq] = sum_j w_j l_j o_j / sum_j w_j l_j, w_j = exp(m_j - max m),
-// with o_j the normalised output of slot j.
+// with o_j the normalised output of slot j (fp32 from the CUDA-core path,
+// fp16 from the tensor-core path).
 // grid (L * S * Hq), 128 threads.  Slots with an out-of-range block id
 // contribute nothing.
-__global__ void __launch_bounds__(128) k_combine(DecodeArgs a) {
+template <typename PT> __device__ __forceinline__ float part_elem(const PT *p, int64_t i);
+template <> __device__ __forceinline__ float part_elem<float>(const float *p, int64_t i) { return p[i]; }
+template <> __device__ __forceinline__ float part_elem<__half>(const __half *p, int64_t i) {
+    return __half2float(p[i]);
+}
+
+template <typename PT>
+__global__ void __launch_bounds__(128) k_combine(DecodeArgs a, const PT *__restrict__ part_o) {
     const int64_t row = blockIdx.x;
     const int s = (int)((row / a.Hq) % a.S);
     const int j = threadIdx.x;
@@ -293,7 +317,7 @@ __global__ void __launch_bounds__(128) k_combine(DecodeArgs a) {
         if (bid < 0 || bid >= a.n_b) continue;
         const float2 ml = a.part_ml[row * a.n_sel + u];
         const float w = __expf(ml.x - M) * ml.y;
-        num = fmaf(w, a.part_o[(row * a.n_sel + u) * D + j], num);
+        num = fmaf(w, part_elem(part_o, (row * a.n_sel + u) * D + j), num);
         den += w;
     }
     a.out[row * D + j] = den > 0.f ? num / den : 0.f;

@@ -164,6 +164,14 @@ milo_status cuda_check(cudaError_t e, const char *what) {
     return MILO_ERR_CUDA;
 }
 
+// Limit of every wait inside the tensor-core decode kernel (ns of the GPU's
+// global timer), and a fault injected into the next decode call by the test
+// hook milo_test_decode_inject.
+constexpr uint64_t kWaitNs = 2000000000ull;
+std::mutex g_inject_mu;
+int g_inject_mode = 0;
+uint64_t g_inject_wait_ns = 0;
+
 int g_sm_count = 0;
 int sm_count() {
     if (g_sm_count == 0) {
@@ -244,6 +252,7 @@ const char *milo_status_string(milo_status s) {
     case MILO_ERR_WORKSPACE: return "workspace or arena too small";
     case MILO_ERR_NONFINITE: return "non-finite value met on the device";
     case MILO_ERR_BOUNDS: return "index out of range met on the device";
+    case MILO_ERR_TIMEOUT: return "a bounded wait on the device ran out (pipeline stalled)";
     }
     return "unknown status";
 }
@@ -509,8 +518,8 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     size_t at = 0;
     at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursor, starts, passes, claim
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
-    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
-    at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);  // rope tables
+    at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o (fp32, or fp16 in its first half)
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
                                                             Hq / f->shape.H));  // tensor-core work items
@@ -542,7 +551,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
     float2 *rope_q = (float2 *)(w + at);
     float2 *rope_t = rope_q + slots * HALF;
-    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);
+    float2 *rope_lo = rope_t + (int64_t)f->shape.block_len * HALF;
+    float4 *rope_hi = (float4 *)(rope_lo + 32 * HALF);
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);
     float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
     float2 *part_ml = (float2 *)(w + at); at = align_up(at + sizeof(float2) * rows * n_sel);
     DtItem *items = (DtItem *)(w + at);
@@ -555,9 +566,16 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.S = S; a.Hq = Hq; a.n_sel = n_sel;
     a.q = q; a.sel = selected; a.pos = positions;
     a.slot_start = start; a.slot_list = list;
-    a.rope_q = rope_q; a.rope_t = rope_t;
-    a.part_o = part_o; a.part_ml = part_ml; a.out = out;
+    a.rope_q = rope_q; a.rope_t = rope_t; a.rope_lo = rope_lo; a.rope_hi = rope_hi;
+    a.part_o = part_o; a.part_o16 = (__half *)part_o; a.part_ml = part_ml; a.out = out;
     a.claim = claim;
+    {   // a test-injected fault applies to this call only
+        std::lock_guard<std::mutex> lk(g_inject_mu);
+        a.wait_ns = g_inject_wait_ns ? g_inject_wait_ns : kWaitNs;
+        a.inject = g_inject_mode;
+        g_inject_mode = 0;
+        g_inject_wait_ns = 0;
+    }
 
     // counts and the claim counter to 0 (starts and passes are written by the scan)
     cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ((n_b + 1) * 3 + 1), s);
@@ -566,16 +584,17 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
     k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, pstart, n_b, a.G, DT_NQ);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
-    const int64_t rt = (slots + f->shape.block_len) * HALF;
+    const int64_t rt = (slots + f->shape.block_len + 32 + 16) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
-        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
+        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t, rope_lo, rope_hi);
     if (decode_tc_supported(a)) {
         st = cuda_check(launch_decode_tc(a, pstart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
+        k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
     } else {
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
+        k_combine<float><<<(unsigned)rows, D, 0, s>>>(a, a.part_o);
     }
-    k_combine<<<(unsigned)rows, D, 0, s>>>(a);
     return cuda_check(cudaGetLastError(), "decode launch");
 }
 
@@ -671,6 +690,14 @@ milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena,
 
 void milo_factors_destroy(milo_factors *f) { delete f; }
 
+milo_status milo_test_decode_inject(int32_t mode, uint64_t wait_ns) {
+    if (mode < 0 || mode > 1 || (mode == 1 && (wait_ns == 0 || wait_ns > kWaitNs))) return MILO_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_inject_mu);
+    g_inject_mode = mode;
+    g_inject_wait_ns = wait_ns;
+    return MILO_OK;
+}
+
 milo_status milo_get_status(milo_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_check(e, "stream sync");
@@ -681,7 +708,7 @@ milo_status milo_get_status(milo_stream_t stream) {
     if (bits & ST_BOUNDS) return MILO_ERR_BOUNDS;
     if (bits & ST_NONFINITE) return MILO_ERR_NONFINITE;
     if (bits & ST_UNSORTED) return MILO_ERR_INVALID_ARG;
-    if (bits & ST_TIMEOUT) return MILO_ERR_CUDA;
+    if (bits & ST_TIMEOUT) return MILO_ERR_TIMEOUT;
     if (bits & ST_NOT_CONVERGED) return MILO_WARN_NOT_CONVERGED;
     return MILO_OK;
 }

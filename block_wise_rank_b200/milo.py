@@ -24,6 +24,7 @@ MILO_ERR_CUDA = -3
 MILO_ERR_WORKSPACE = -4
 MILO_ERR_NONFINITE = -5
 MILO_ERR_BOUNDS = -6
+MILO_ERR_TIMEOUT = -7
 
 MILO_F32, MILO_BF16, MILO_INT8 = 0, 1, 2
 DTYPES = {"f32": MILO_F32, "bf16": MILO_BF16, "int8": MILO_INT8}
@@ -52,7 +53,7 @@ EXPORTS = [
     "milo_compress", "milo_allocate_workspace_size", "milo_allocate", "milo_decode_workspace_size",
     "milo_decode_attn", "milo_factors_get", "milo_factors_wrap", "milo_factors_export",
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
-    "milo_allocate_noalloc",
+    "milo_allocate_noalloc", "milo_test_decode_inject",
 ]
 
 MILO_NOALLOC_MAX_BLOCKS = 65536
@@ -93,6 +94,8 @@ def lib():
         L.milo_get_status.argtypes = [P]; L.milo_get_status.restype = ctypes.c_int
         L.milo_status_string.argtypes = [ctypes.c_int]; L.milo_status_string.restype = ctypes.c_char_p
         L.milo_version.argtypes = []; L.milo_version.restype = ctypes.c_char_p
+        L.milo_test_decode_inject.argtypes = [I32, ctypes.c_uint64]
+        L.milo_test_decode_inject.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -298,6 +301,12 @@ def milo_factors_import(blob: bytes, arena: torch.Tensor, stream=None) -> Factor
 
 def milo_get_status(stream=None) -> int:
     return lib().milo_get_status(_stream(stream))
+
+
+def milo_test_decode_inject(mode: int, wait_ns: int = 0) -> int:
+    """Test hook: arm (mode 1) a withheld copy and a wait limit of wait_ns for
+    the next tensor-core decode call, or disarm (mode 0).  Returns the status."""
+    return lib().milo_test_decode_inject(int(mode), int(wait_ns))
 
 
 def milo_version() -> str:

@@ -28,7 +28,8 @@
  *     host, except milo_get_status, milo_factors_export and
  *     milo_factors_import, which say so.  Argument errors are returned
  *     synchronously and launch nothing.  Errors found on the device (a
- *     Jacobi sweep cap reached, non-finite input, a bad block id) set bits
+ *     Jacobi sweep cap reached, non-finite input, a bad block id, a wait on
+ *     the device that ran out) set bits
  *     of a per-device status word that milo_get_status reads and clears.
  *   - No C++ exception crosses this interface.
  *   - d (head dimension) must be 128.
@@ -54,7 +55,8 @@ typedef enum {
     MILO_ERR_CUDA = -3,            /* a CUDA runtime call failed              */
     MILO_ERR_WORKSPACE = -4,       /* workspace or arena smaller than needed  */
     MILO_ERR_NONFINITE = -5,       /* NaN/Inf met on the device               */
-    MILO_ERR_BOUNDS = -6           /* an index out of range met on the device */
+    MILO_ERR_BOUNDS = -6,          /* an index out of range met on the device */
+    MILO_ERR_TIMEOUT = -7          /* a bounded wait on the device ran out    */
 } milo_status;
 
 typedef enum { MILO_F32 = 0, MILO_BF16 = 1, MILO_INT8 = 2 } milo_dtype;
@@ -247,6 +249,20 @@ milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena,
 
 /* Free the handle only; the arena stays the caller's. */
 void milo_factors_destroy(milo_factors *f);
+
+/*
+ * Test hook (no counterpart on the pages): arms a fault for the next
+ * milo_decode_attn call that takes the tensor-core path, then disarms.
+ *   mode 1: the kernel withholds the copy of the first work item's B_K (no
+ *           copy is issued, so none is in flight), every wait on the device
+ *           gives up after wait_ns nanoseconds (1 .. 2e9) instead of 2 s, and
+ *           the call's status word reports MILO_ERR_TIMEOUT; the kernel
+ *           still waits for its issued copies and products and frees its
+ *           tensor memory before it returns, so later calls run normally.
+ *   mode 0: disarm.
+ * MILO_ERR_INVALID_ARG for another mode or an out-of-range wait_ns.
+ */
+milo_status milo_test_decode_inject(int32_t mode, uint64_t wait_ns);
 
 /* ---------------------------------------------------------------- status */
 

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_status_strings(L):
     assert milo.milo_version() == "0.1.0"
-    for s in (0, 1, -1, -2, -3, -4, -5, -6):
+    for s in (0, 1, -1, -2, -3, -4, -5, -6, -7):
         assert milo.status_string(s) and milo.status_string(s) != "unknown status"
     assert milo.status_string(42) == "unknown status"
 
@@ -111,6 +111,11 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.milo_allocate(P, P, 1, 8, 128, 2048, 256, 10, 0, 0, P, P, 8, None) == milo.MILO_ERR_WORKSPACE
     # decode: null handle
     assert L.milo_decode_attn(None, P, 1, 1, P, None, 1, 1e6, P, P, 1 << 30, None) == milo.MILO_ERR_INVALID_ARG
+    # test hook: unknown mode, or a wait limit of 0 or above the 2 s default
+    assert milo.milo_test_decode_inject(2, 1000) == milo.MILO_ERR_INVALID_ARG
+    assert milo.milo_test_decode_inject(1, 0) == milo.MILO_ERR_INVALID_ARG
+    assert milo.milo_test_decode_inject(1, 3 * 10**9) == milo.MILO_ERR_INVALID_ARG
+    assert milo.milo_test_decode_inject(0, 0) == milo.MILO_OK
 
 
 def test_wrap_views_and_export_size(L):
