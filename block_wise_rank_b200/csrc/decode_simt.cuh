@@ -39,6 +39,9 @@ struct DecodeArgs {
     int32_t *claim;            // tensor-core path: next unclaimed work item (zeroed before the launch)
     uint64_t wait_ns;          // tensor-core path: limit of every wait on the device
     int inject;                // tensor-core path: 1 = withhold one copy (tests of the bounded waits)
+    int G8;                    // tensor-core path: GQA group padded to a multiple of 8
+    int spi;                   // tensor-core path: sessions per work item (64 / G8 queries, at most 8)
+    const __half *qpack;       // tensor-core path: [L][S][H][G8 x 128] packed fp16 queries (k_q_pack)
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
@@ -81,56 +84,43 @@ __global__ void k_slot_count(const int32_t *__restrict__ sel, int n_slots, int n
     }
 }
 
-// starts of each block id's slot list, and of its query passes (a pass is up
-// to `pass_q` queries = selecting slots times the GQA group)
-// Exclusive prefix sums of the per-block slot counts (start) and of the
-// per-block query passes (pstart), one CTA of 1024 threads; counts are reset
-// for k_slot_fill's cursors.
+// Exclusive prefix sum of the per-block slot counts (start, start[n_b] = the
+// total), one CTA of 1024 threads; the counts are reset for k_slot_fill's
+// cursors.
 constexpr int SCAN_THREADS = 1024;
 __global__ void __launch_bounds__(SCAN_THREADS) k_slot_scan(int32_t *__restrict__ cnt, int32_t *__restrict__ start,
-                                                            int32_t *__restrict__ pstart, int n_b, int G, int pass_q) {
-    __shared__ int2 wsum[SCAN_THREADS / 32];
+                                                            int n_b) {
+    __shared__ int wsum[SCAN_THREADS / 32];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int chunk = (n_b + SCAN_THREADS - 1) / SCAN_THREADS;
     const int b0 = min(n_b, tid * chunk), b1 = min(n_b, b0 + chunk);
-    int2 mine = make_int2(0, 0);
-    for (int b = b0; b < b1; ++b) {
-        const int c = cnt[b];
-        mine.x += c;
-        mine.y += (c * G + pass_q - 1) / pass_q;
-    }
-    // inclusive scan of (slots, passes) over the CTA
-    int2 inc = mine;
+    int mine = 0;
+    for (int b = b0; b < b1; ++b) mine += cnt[b];
+    int inc = mine;
     for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, inc.x, o), y = __shfl_up_sync(0xffffffffu, inc.y, o);
-        if (lane >= o) { inc.x += x; inc.y += y; }
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
     }
     if (lane == 31) wsum[wid] = inc;
     __syncthreads();
     if (wid == 0) {
-        int2 v = wsum[lane];
+        int v = wsum[lane];
         for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, v.x, o), y = __shfl_up_sync(0xffffffffu, v.y, o);
-            if (lane >= o) { v.x += x; v.y += y; }
+            const int x = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += x;
         }
         wsum[lane] = v;
     }
     __syncthreads();
-    int acc = inc.x - mine.x + (wid > 0 ? wsum[wid - 1].x : 0);
-    int pacc = inc.y - mine.y + (wid > 0 ? wsum[wid - 1].y : 0);
+    int acc = inc - mine + (wid > 0 ? wsum[wid - 1] : 0);
     for (int b = b0; b < b1; ++b) {
         const int c = cnt[b];
         start[b] = acc;
-        pstart[b] = pacc;
         acc += c;
-        pacc += (c * G + pass_q - 1) / pass_q;
     }
     __syncthreads();   // every count read before any is reset
     for (int b = b0; b < b1; ++b) cnt[b] = 0;
-    if (tid == SCAN_THREADS - 1) {
-        start[n_b] = wsum[31].x;
-        pstart[n_b] = wsum[31].y;
-    }
+    if (tid == SCAN_THREADS - 1) start[n_b] = wsum[31];
 }
 
 __global__ void k_slot_fill(const int32_t *__restrict__ sel, int n_slots, int n_b, const int32_t *__restrict__ start,
@@ -139,6 +129,110 @@ __global__ void k_slot_fill(const int32_t *__restrict__ sel, int n_slots, int n_
         const int b = sel[e];
         if (b < 0 || b >= n_b) continue;
         list[start[b] + atomicAdd(&cursor[b], 1)] = e;
+    }
+}
+
+// Position of a selected slot: the caller's start position, or block id *
+// block_len.
+__device__ __forceinline__ int slot_pos(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int slot,
+                                        int block_len) {
+    return pos ? pos[slot] : sel[slot] * block_len;
+}
+
+// Tensor-core path: per block id, sort its slot list by (position, slot) in
+// place and count its work items: runs of equal position, up to `spi`
+// sessions each.  One thread per block id.
+__global__ void k_blk_items(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int n_b, int block_len,
+                            const int32_t *__restrict__ start, int32_t *__restrict__ list, int spi,
+                            int32_t *__restrict__ nitems) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= n_b) return;
+    const int s0 = start[b], s1 = start[b + 1];
+    for (int i = s0 + 1; i < s1; ++i) {   // insertion sort by (position, slot)
+        const int x = list[i];
+        const int px = slot_pos(sel, pos, x, block_len);
+        int k = i - 1;
+        while (k >= s0) {
+            const int y = list[k];
+            const int py = slot_pos(sel, pos, y, block_len);
+            if (py < px || (py == px && y < x)) break;
+            list[k + 1] = y;
+            --k;
+        }
+        list[k + 1] = x;
+    }
+    int cnt = 0;
+    for (int i = s0; i < s1;) {
+        const int p = slot_pos(sel, pos, list[i], block_len);
+        int k = i;
+        while (k < s1 && slot_pos(sel, pos, list[k], block_len) == p) ++k;
+        cnt += (k - i + spi - 1) / spi;
+        i = k;
+    }
+    nitems[b] = cnt;
+}
+
+// Exclusive prefix sum of n values (one CTA of 1024 threads): out[i] for i <=
+// n, out[n] = the total.
+__global__ void __launch_bounds__(SCAN_THREADS) k_scan_counts(const int32_t *__restrict__ in, int32_t *__restrict__ out,
+                                                              int n) {
+    __shared__ int wsum[SCAN_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int chunk = (n + SCAN_THREADS - 1) / SCAN_THREADS;
+    const int b0 = min(n, tid * chunk), b1 = min(n, b0 + chunk);
+    int mine = 0;
+    for (int b = b0; b < b1; ++b) mine += in[b];
+    int inc = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+    }
+    if (lane == 31) wsum[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        int v = wsum[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += x;
+        }
+        wsum[lane] = v;
+    }
+    __syncthreads();
+    int acc = inc - mine + (wid > 0 ? wsum[wid - 1] : 0);
+    for (int b = b0; b < b1; ++b) {
+        out[b] = acc;
+        acc += in[b];
+    }
+    if (tid == SCAN_THREADS - 1) out[n] = wsum[31];
+}
+
+// Tensor-core path: the queries of every (layer, session, KV head) in fp16,
+// GQA heads padded to G8 = round_up(G, 8) with zeros, already in the tensor
+// cores' K-major operand layout [g/8][cg][g%8][8]: core-matrix column 2c holds
+// channels 8c .. 8c+7, column 2c+1 channels 64+8c .. 64+8c+7 (the order the
+// rotated keys are packed in).  One 16-byte chunk per thread.
+__global__ void k_q_pack(const float *__restrict__ q, int L, int S, int H, int G, int G8, __half *__restrict__ qp) {
+    const int64_t total = (int64_t)L * S * H * G8 * 16;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int r = (int)(e & 7);
+        const int cg = (int)((e >> 3) & 15);
+        const int64_t rest = e >> 7;                  // (lsh, g / 8)
+        const int rg = (int)(rest % (G8 / 8));
+        const int64_t lsh = rest / (G8 / 8);
+        const int h = (int)(lsh % H);
+        const int64_t ls = lsh / H;                   // l * S + s
+        const int g = rg * 8 + r;
+        const int ch = (cg & 1) ? HALF + 8 * (cg >> 1) : 8 * (cg >> 1);
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (g < G) {
+            const float4 *src = reinterpret_cast<const float4 *>(q + (ls * (H * G) + h * G + g) * D + ch);
+            const float4 a = src[0], b = src[1];
+            const __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
+            const __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
+            out = make_uint4(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1),
+                             *reinterpret_cast<const uint32_t *>(&h2), *reinterpret_cast<const uint32_t *>(&h3));
+        }
+        *reinterpret_cast<uint4 *>(qp + lsh * (int64_t)G8 * D + rg * 1024 + cg * 64 + r * 8) = out;
     }
 }
 

@@ -516,13 +516,14 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     const int64_t slots = (int64_t)S * n_sel;
     const int64_t rows = (int64_t)f->shape.L * S * Hq;
     size_t at = 0;
-    at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursor, starts, passes, claim
+    at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursors / item counts, slot starts, item starts, claim
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);  // rope tables
     at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o (fp32, or fp16 in its first half)
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
-    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
-                                                            Hq / f->shape.H));  // tensor-core work items
+    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));  // tensor-core work items
+    at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H *
+                           decode_tc_g8(Hq / f->shape.H) * D);              // packed fp16 queries
     return at;
 }
 
@@ -545,8 +546,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     size_t at = 0;
     int32_t *cnt = (int32_t *)(w + at);
     int32_t *start = cnt + (n_b + 1);
-    int32_t *pstart = start + (n_b + 1);
-    int32_t *claim = pstart + (n_b + 1);   // next unclaimed tensor-core work item
+    int32_t *istart = start + (n_b + 1);   // tensor-core work items of each block id, scanned
+    int32_t *claim = istart + (n_b + 1);   // next unclaimed tensor-core work item
     at = align_up(at + sizeof(int32_t) * ((n_b + 1) * 3 + 1));
     int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
     float2 *rope_q = (float2 *)(w + at);
@@ -557,6 +558,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
     float2 *part_ml = (float2 *)(w + at); at = align_up(at + sizeof(float2) * rows * n_sel);
     DtItem *items = (DtItem *)(w + at);
+    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));
+    __half *qpack = (__half *)(w + at);
 
     DecodeArgs a{};
     a.kv[0] = f->kv[0];
@@ -569,6 +572,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.rope_q = rope_q; a.rope_t = rope_t; a.rope_lo = rope_lo; a.rope_hi = rope_hi;
     a.part_o = part_o; a.part_o16 = (__half *)part_o; a.part_ml = part_ml; a.out = out;
     a.claim = claim;
+    a.G8 = decode_tc_g8(a.G);
+    a.spi = decode_tc_spi(a.G);
+    a.qpack = qpack;
     {   // a test-injected fault applies to this call only
         std::lock_guard<std::mutex> lk(g_inject_mu);
         a.wait_ns = g_inject_wait_ns ? g_inject_wait_ns : kWaitNs;
@@ -577,18 +583,26 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
         g_inject_wait_ns = 0;
     }
 
-    // counts and the claim counter to 0 (starts and passes are written by the scan)
+    // counts and the claim counter to 0 (the starts are written by the scans)
     cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ((n_b + 1) * 3 + 1), s);
     if (e != cudaSuccess) return cuda_check(e, "memset");
     const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
-    k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, pstart, n_b, a.G, DT_NQ);
+    k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, n_b);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
     const int64_t rt = (slots + f->shape.block_len + 32 + 16) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
         selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t, rope_lo, rope_hi);
     if (decode_tc_supported(a)) {
-        st = cuda_check(launch_decode_tc(a, pstart, items, sm_count(), s), "decode (tensor cores) launch");
+        // items: each block's slots sorted by position (the fill order is not
+        // deterministic), cut into runs of equal position; item starts per block
+        k_blk_items<<<(n_b + 127) / 128, 128, 0, s>>>(selected, positions, n_b, f->shape.block_len, start, list,
+                                                     a.spi, cnt);
+        k_scan_counts<<<1, SCAN_THREADS, 0, s>>>(cnt, istart, n_b);
+        const int64_t qchunks = (int64_t)a.L * S * a.H * a.G8 * 16;
+        k_q_pack<<<(int)std::min<int64_t>((qchunks + 255) / 256, 8192), 256, 0, s>>>(q, a.L, S, a.H, a.G, a.G8,
+                                                                                     qpack);
+        st = cuda_check(launch_decode_tc(a, istart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
         k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
     } else {
