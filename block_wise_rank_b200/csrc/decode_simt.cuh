@@ -42,6 +42,7 @@ struct DecodeArgs {
     int G8;                    // tensor-core path: GQA group padded to a multiple of 8
     int spi;                   // tensor-core path: sessions per work item (64 / G8 queries, at most 8)
     const __half *qpack;       // tensor-core path: [L][S][H][G8 x 128] packed fp16 queries (k_q_pack)
+    const float4 *rot_slot;    // tensor-core path: [S * n_sel][16][32] (cos, sin)((p + 32 v) theta_i) (k_rot_slots)
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every

@@ -13,26 +13,28 @@
 // streams them through warp roles that meet only at mbarriers, every wait
 // bounded:
 //
-//   K producer (warp 0)   claims items into a shared-memory table;
-//                         bulk-copies each item's B_K into its own ring, its
-//                         sessions' packed queries into one of two query
-//                         buffers, and the 128-token A_K tiles into a ring
-//                         (factors already in the canonical operand layout).
+//   K producer (warp 0)   claims items into a shared-memory table; per item
+//                         one entry of a resident ring holds its sessions'
+//                         packed queries (16-byte asynchronous copies by the
+//                         warp's lanes) and B_K (one bulk copy); the 128-token
+//                         A_K tiles are bulk-copied into a tile ring (factors
+//                         already in the canonical operand layout).
 //   V producer (warp 1)   bulk-copies the A_V tiles and B_V into a third ring.
 //   K MMA (warp 2)        rebuild  K-hat tile = A_K(tile) B_K        (M=128 tokens, N=128, K=r_K, bf16)
 //                         scores   S = K-tilde (TMEM) Q^T             (M=128 tokens, N=nq, K=128, fp16)
 //                         in the order R0 R1 S0 R2 S1 ...
-//   V warp (warp 3)       converts each A_V tile and B_V to fp16 in place
-//                         (appending a row of ones to A_V when a rank row is
-//                         free) and issues O_A^T += A_V(tile)^T P, then
+//   V warp (warp 3)       issues O_A^T += A_V(tile)^T P, then
 //                         O = B_V^T (O_A / l)                        (M=128, N=nq, fp16)
 //   RoPE group (8 warps)  two per TMEM lane quadrant, a token row per thread,
 //                         32 pairs each: rotates the rebuilt keys by
 //                         (p + 32 v + u) theta_i, u = the thread's lane, with
 //                         (cos, sin)(u theta_i) in registers and (p + 32 v)
-//                         theta_i from a per-item table in shared memory,
-//                         f32x2 arithmetic; packs K-tilde to fp16 in place.
-//                         Also reads each item's O out to the fp16 partials.
+//                         theta_i from a per-slot table (L2-resident), f32x2
+//                         arithmetic; packs K-tilde to fp16 in place.
+//                         Then converts the same tile of A_V (and, last, B_V)
+//                         to fp16 in place, appending a row of ones to A_V
+//                         when a rank row is free.  Also reads each item's O
+//                         out to the fp16 partials.
 //   softmax group (8 w.)  two column halves of four warps, a token row per
 //                         thread: exp2 against a per-query reference max
 //                         raised only when some p exceeds 2^8, P (fp16) to
@@ -55,6 +57,20 @@
 #ifndef MILO_DT_TRACE
 #define MILO_DT_TRACE(code, n, t)
 #endif
+#ifndef MILO_DT_TRACE_STATE
+#define MILO_DT_TRACE_STATE
+#endif
+// Copy-latency hooks (tracing builds): issue time of a ring slot's copy, and
+// its landing as the consumer sees it.
+#ifndef MILO_DT_STAMP
+#define MILO_DT_STAMP(kind, slot)
+#define MILO_DT_LAT(kind, slot)
+#endif
+// Debug hooks (tracing builds): the shared-memory base, and a wait that ran out.
+#ifndef MILO_DT_ON_TIMEOUT
+#define MILO_DT_BASE(p)
+#define MILO_DT_ON_TIMEOUT(bar, parity)
+#endif
 
 namespace milo {
 
@@ -66,17 +82,16 @@ constexpr int DT_W_SM = 12;                       // softmax warps 12 .. 19
 constexpr int DT_NROPE = 256, DT_NSM = 256;
 // registers per thread: at launch (65536 / 640, in steps of 8) and per
 // warpgroup after setmaxnreg; the shares add up to the launch total
-constexpr int DT_REG_LAUNCH = 96, DT_REG_CTRL = 48, DT_REG_ROPE = 136, DT_REG_SM = 80;
+constexpr int DT_REG_LAUNCH = 96, DT_REG_CTRL = 48, DT_REG_ROPE = 128, DT_REG_SM = 88;
 static_assert(DT_REG_CTRL + 2 * DT_REG_ROPE + 2 * DT_REG_SM <= 5 * DT_REG_LAUNCH, "register split over the launch");
 constexpr int DT_VRING = 64 * 1024;               // A_V tiles (+ ones group) and B_V
 constexpr int DT_AKRING = 48 * 1024;              // A_K tiles
-constexpr int DT_BKRING = 32 * 1024;              // B_K per item (one of rank 128 fills it)
+constexpr int DT_RRING = 72 * 1024;               // per item: packed queries, then B_K
 constexpr int DT_NSLOT = 16;                      // tiles in flight per tile ring
-constexpr int DT_NBK = 4;                         // B_K in flight
+constexpr int DT_NRES = 4;                        // items in flight in the resident ring
 constexpr int DT_NITAB = 16;                      // item table entries
 constexpr int DT_AHEAD = 4;                       // items claimed ahead of the copies
 constexpr int DT_PBUF = 128 * DT_NQ * 2;          // one P buffer: 128 tokens x 64 queries, fp16
-constexpr int DT_QBUF = DT_NQ * D * 2;            // one query buffer: 64 queries x 128, fp16
 constexpr uint32_t DT_TMEM_COLS = 512;
 constexpr uint32_t DT_COL_KH = 0;                 // two 128-column rebuild buffers
 constexpr uint32_t DT_COL_S = 256;                // two 64-column score buffers
@@ -100,10 +115,12 @@ struct DecTcSmem {
     // CTA's shared memory (the rows they feed are never used).
     alignas(1024) uint8_t vring[DT_VRING];
     alignas(1024) uint8_t akring[DT_AKRING];
-    alignas(1024) uint8_t bkring[DT_BKRING];
-    alignas(1024) uint8_t qt[2][DT_QBUF];         // packed queries, fp16, K-major, per item parity
+    alignas(1024) uint8_t rring[DT_RRING];
     alignas(1024) uint8_t pbuf[2][DT_PBUF];       // P, or O_A / l for an item's last product (fp16, MN-major)
-    float4 rot[16][HALF / 2];                     // (cos, sin)((p + 32 v) theta_i), pairs (2k, 2k+1): (c0, c1, s0, s1)
+    // 8 rank rows of zeros in the B_K operand layout: the second half of the
+    // last K step when the padded rank is an odd multiple of 8, or both
+    // halves (leading offset 0) for a block of rank 0
+    alignas(1024) uint8_t zero[2048];
     DtItem itab[DT_NITAB];                        // claimed items, entry n % NITAB = this CTA's n-th
     float cref[2][DT_NQ];                         // reference max per query (log2 domain), per item parity
     float cscale[2][DT_NQ];                       // rescale factors, then 1 / l
@@ -111,12 +128,11 @@ struct DecTcSmem {
     int cmax[DT_NQ];                              // column maxima, order-preserving int encoding
     int qp_sm[4][DT_NQ];                          // partial index of each query column (-1: none), per item
     int qp_rope[4][DT_NQ];                        // the same, the RoPE group's copy
-    uint32_t ak_off[DT_NSLOT], v_off[DT_NSLOT], bk_off[DT_NBK];
+    uint32_t ak_off[DT_NSLOT], v_off[DT_NSLOT], res_off[DT_NRES];
     uint64_t item_full[DT_NITAB], item_free[DT_NITAB];
     uint64_t akfull[DT_NSLOT], akempty[DT_NSLOT];
-    uint64_t vfull[DT_NSLOT], vempty[DT_NSLOT];
-    uint64_t bkfull[DT_NBK], bkempty[DT_NBK];
-    uint64_t qt_full[2], qt_free[2];
+    uint64_t vfull[DT_NSLOT], vconv[DT_NSLOT], vempty[DT_NSLOT];
+    uint64_t res_full[DT_NRES], res_empty[DT_NRES];
     uint64_t kh_full[2], kh_free[2], kt_full[2];
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], p_free[2];
@@ -158,6 +174,25 @@ __global__ void k_dt_items(DecodeArgs a, const int32_t *__restrict__ istart, DtI
             it.slots[it.ns++] = a.slot_list[i++];
         for (int k = it.ns; k < DT_MAXS; ++k) it.slots[k] = -1;
         items[out++] = it;
+    }
+}
+
+// Per selected slot, (cos, sin)((p + 32 v) theta_i) for v < 16, the angle of
+// the first token of each 32-token group of the block at start position p,
+// by angle addition from (p theta_i) and (32 v theta_i); pairs (2k, 2k+1) as
+// (c0, c1, s0, s1).  16 x 32 float4 (8 KB) per slot.
+__global__ void k_rot_slots(const float2 *__restrict__ rope_q, const float4 *__restrict__ rope_hi, int n_slots,
+                            float4 *__restrict__ rot) {
+    const int64_t total = (int64_t)n_slots * 16 * (HALF / 2);
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int k = (int)(e % (HALF / 2));
+        const int v = (int)((e / (HALF / 2)) % 16);
+        const int64_t slot = e / (16 * (HALF / 2));
+        const float4 p = reinterpret_cast<const float4 *>(rope_q + slot * HALF)[k];   // (c0, s0, c1, s1) of p theta
+        const float4 h = rope_hi[v * (HALF / 2) + k];                                   // (c0, c1, s0, s1) of 32 v theta
+        const float c0 = fmaf(p.x, h.x, -p.y * h.z), s0 = fmaf(p.y, h.x, p.x * h.z);
+        const float c1 = fmaf(p.z, h.y, -p.w * h.w), s1 = fmaf(p.w, h.y, p.z * h.w);
+        rot[e] = make_float4(c0, c1, s0, s1);
     }
 }
 
@@ -234,6 +269,7 @@ __device__ __forceinline__ bool dt_wait(uint64_t *bar, uint32_t parity, uint64_t
     for (;;) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if (tc::globaltimer() - t0 > limit) {
+            MILO_DT_ON_TIMEOUT(bar, parity);
             raise_status(ST_TIMEOUT);
             return false;
         }
@@ -306,32 +342,34 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t lim = a.wait_ns;
     const int G8 = a.G8;
+    if (threadIdx.x == 0) MILO_DT_BASE(&sm);
 
     // ---------------------------------------------------------------- set-up
-    {   // zero the tile rings: pad rows of a tile hold older ring contents,
-        // which must be finite (they meet zero rows of the other operand)
+    {   // zero the rings (pad rows of a tile hold older ring contents, which
+        // must be finite: they meet zero rows of the other operand) and the
+        // zero rows
         uint4 *z = reinterpret_cast<uint4 *>(sm.vring);
-        const int n16 = (DT_VRING + DT_AKRING + DT_BKRING) / 16;
+        const int n16 = (DT_VRING + DT_AKRING + DT_RRING) / 16;
         for (int e = threadIdx.x; e < n16; e += DT_THREADS) z[e] = make_uint4(0, 0, 0, 0);
+        for (int e = threadIdx.x; e < 2048 / 16; e += DT_THREADS) reinterpret_cast<uint4 *>(sm.zero)[e] = make_uint4(0, 0, 0, 0);
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < DT_NSLOT; ++s) {
             tc::mbar_init(&sm.akfull[s], 1);
             tc::mbar_init(&sm.akempty[s], 1);
             tc::mbar_init(&sm.vfull[s], 1);
+            tc::mbar_init(&sm.vconv[s], DT_NROPE);
             tc::mbar_init(&sm.vempty[s], 1);
         }
-        for (int s = 0; s < DT_NBK; ++s) {
-            tc::mbar_init(&sm.bkfull[s], 1);
-            tc::mbar_init(&sm.bkempty[s], 1);
+        for (int s = 0; s < DT_NRES; ++s) {
+            tc::mbar_init(&sm.res_full[s], 32 + 1);   // the K producer's lanes' query copies, B_K's bulk copy
+            tc::mbar_init(&sm.res_empty[s], 1);
         }
         for (int s = 0; s < DT_NITAB; ++s) {
             tc::mbar_init(&sm.item_full[s], 1);
             tc::mbar_init(&sm.item_free[s], DT_ITEM_READERS);
         }
         for (int k = 0; k < 2; ++k) {
-            tc::mbar_init(&sm.qt_full[k], 1);
-            tc::mbar_init(&sm.qt_free[k], 1);
             tc::mbar_init(&sm.kh_full[k], 1);
             tc::mbar_init(&sm.kh_free[k], 1);
             tc::mbar_init(&sm.kt_full[k], DT_NROPE);
@@ -362,9 +400,10 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         reg_dealloc<DT_REG_CTRL>();
         if (warp == 0) {
             // ======================================================== K producer
+            MILO_DT_TRACE_STATE;
             const int64_t n_items = (int64_t)a.L * a.H * istart[a.n_b];
-            DtRing ak, bk;
-            uint32_t claimed = 0, qissued = 0;
+            DtRing ak, rr;
+            uint32_t claimed = 0;
             bool ok = true, done = false;
             bool withheld = false;               // first B_K copy never issued (tests only)
             // publish the item with global index c (or the end) as this CTA's item `claimed`
@@ -395,80 +434,74 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 // the claim for a later item is in flight while this one's copies go out
                 int c = -2;
                 if (lane == 0 && !done) c = claim();
-                const int R8K = rank_pad(it.rK), R16K = r16_of(R8K);
+                if (lane == 0) MILO_DT_TRACE(28, n, 0);
+                const int R8K = rank_pad(it.rK);
                 const uint32_t tile = (uint32_t)R8K * 256u;
-                // B_K: R16K rows, the pad rows R8K .. R16K-1 zero
-                uint32_t off = 0;
-                if (lane == 0)
-                    ok = bk.place((uint32_t)R16K * 256u, DT_BKRING, sm.bk_off, sm.bkempty, DT_NBK, lim, off);
+                // resident entry: the queries (nq16 rows; rows past ns * G8 are
+                // not copied: their score columns are masked), then B_K
+                const uint32_t qbytes = (uint32_t)((it.ns * G8 + 15) & ~15) * 256u;
+                uint32_t off = 0, rs = 0;
+                if (lane == 0) {
+                    ok = rr.place(qbytes + tile, DT_RRING, sm.res_off, sm.res_empty, DT_NRES, lim, off);
+                    rs = (rr.seq - 1) % DT_NRES;
+                }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 off = __shfl_sync(0xffffffffu, off, 0);
+                rs = __shfl_sync(0xffffffffu, rs, 0);
                 if (!ok) break;
-                if (R16K > R8K) {
-                    uint4 *z = reinterpret_cast<uint4 *>(sm.bkring + off + tile);
-                    for (int e = lane; e < (R16K - R8K) * 16; e += 32) z[e] = make_uint4(0, 0, 0, 0);
+                if (lane == 0) MILO_DT_TRACE(29, n, 0);
+                // each session's G8 packed query rows (G8 x 256 bytes, contiguous in
+                // the packed queries and in the entry), 16 bytes per lane and copy
+                for (int k = 0; k < it.ns; ++k) {
+                    const int slot = it.slots[k];
+                    const int64_t lsh = ((int64_t)it.l * a.S + slot / a.n_sel) * a.H + it.h;
+                    const __half *src = a.qpack + lsh * G8 * D;
+                    uint8_t *dst = sm.rring + off + k * G8 * 256;
+                    for (int w = lane; w < G8 * 16; w += 32) tc::cp_async16(dst + w * 16, src + w * 8);
                 }
-                // the query buffer of this item's parity is free once the scores of
-                // item n-2 have run; query rows past ns * G8 (up to 16) zero
-                const uint32_t qb = n & 1u;
-                if (lane == 0 && n >= 2) ok = dt_wait(&sm.qt_free[qb], ((n - 2) >> 1) & 1u, lim);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                const int nq = it.ns * G8, nq16 = (nq + 15) & ~15;
-                if (nq16 > nq) {
-                    uint4 *z = reinterpret_cast<uint4 *>(sm.qt[qb] + nq * 256);
-                    for (int e = lane; e < (nq16 - nq) * 16; e += 32) z[e] = make_uint4(0, 0, 0, 0);
-                }
-                tc::fence_async_smem();
+                tc::cp_async_arrive_noinc(&sm.res_full[rs]);
                 __syncwarp();
                 if (lane == 0) {
                     const uint8_t *src = (const uint8_t *)a.kv[0].data + 2 * it.offK;
                     const int nt = token_tiles(it.Tb);
-                    const uint32_t s = (bk.seq - 1) % DT_NBK;
                     if (a.inject == 1 && n == 0) {
                         withheld = true;         // no copy, no arrival: the K MMA's wait runs out
                     } else {
-                        tc::mbar_arrive_expect_tx(&sm.bkfull[s], tile);
-                        if (tile) tc::bulk_g2s(sm.bkring + off, src + (size_t)nt * tile, tile, &sm.bkfull[s]);
+                        tc::mbar_arrive_expect_tx(&sm.res_full[rs], tile);
+                        if (tile) tc::bulk_g2s(sm.rring + off + qbytes, src + (size_t)nt * tile, tile, &sm.res_full[rs]);
                     }
-                    // each session's G8 packed query rows, 256 bytes a row
-                    const uint32_t qbytes = (uint32_t)G8 * 256u;
-                    tc::mbar_arrive_expect_tx(&sm.qt_full[qb], (uint32_t)it.ns * qbytes);
-                    for (int k = 0; k < it.ns; ++k) {
-                        const int slot = it.slots[k];
-                        const int64_t lsh = ((int64_t)it.l * a.S + slot / a.n_sel) * a.H + it.h;
-                        tc::bulk_g2s(sm.qt[qb] + k * qbytes, a.qpack + lsh * G8 * D, qbytes, &sm.qt_full[qb]);
-                    }
-                    ++qissued;
                     // A_K tiles (R16K rows reserved; rows past R8K meet B_K's zero rows)
+                    const uint32_t rows16 = (uint32_t)r16_of(R8K);
                     for (int t = 0; t < nt && ok; ++t) {
-                        ok = ak.place((uint32_t)R16K * 256u, DT_AKRING, sm.ak_off, sm.akempty, DT_NSLOT, lim, off);
+                        ok = ak.place(rows16 * 256u, DT_AKRING, sm.ak_off, sm.akempty, DT_NSLOT, lim, off);
                         if (!ok) break;
                         MILO_DT_TRACE(1, n, t);
                         const uint32_t sl = (ak.seq - 1) % DT_NSLOT;
                         tc::mbar_arrive_expect_tx(&sm.akfull[sl], tile);
                         if (tile) tc::bulk_g2s(sm.akring + off, src + (size_t)t * tile, tile, &sm.akfull[sl]);
+                        MILO_DT_STAMP(0, sl);
                     }
                     if (ok && c != -2) ok = publish(c);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 __syncwarp();
             }
+            // every query copy of this warp has landed before the CTA exits
+            tc::cp_async_wait_all();
             if (lane == 0) {
                 if (!ok) sm.abort = 1;
                 // an end marker after the last entry published, for the roles
                 // still walking the table
                 if (!done) publish(-1);
-                // every copy issued has landed before the CTA exits
+                // every bulk copy issued has landed before the CTA exits
                 for (uint32_t k = ak.seq > DT_NSLOT ? ak.seq - DT_NSLOT : 0; k < ak.seq; ++k)
                     dt_wait(&sm.akfull[k % DT_NSLOT], (k / DT_NSLOT) & 1u, lim);
-                for (uint32_t k = bk.seq > DT_NBK ? bk.seq - DT_NBK : 0; k < bk.seq; ++k)
-                    if (!(withheld && k == 0)) dt_wait(&sm.bkfull[k % DT_NBK], (k / DT_NBK) & 1u, lim);
-                for (uint32_t k = qissued > 2 ? qissued - 2 : 0; k < qissued; ++k)
-                    dt_wait(&sm.qt_full[k & 1u], (k >> 1) & 1u, lim);
+                for (uint32_t k = rr.seq > DT_NRES ? rr.seq - DT_NRES : 0; k < rr.seq; ++k)
+                    if (!(withheld && k == 0)) dt_wait(&sm.res_full[k % DT_NRES], (k / DT_NRES) & 1u, lim);
             }
         } else if (warp == 1) {
             // ======================================================== V producer
+            MILO_DT_TRACE_STATE;
             DtRing vr;
             bool ok = true;
             if (lane == 0) {
@@ -490,6 +523,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                         const uint32_t s = (vr.seq - 1) % DT_NSLOT;
                         tc::mbar_arrive_expect_tx(&sm.vfull[s], tile);
                         if (tile) tc::bulk_g2s(sm.vring + off, src + (size_t)t * tile, tile, &sm.vfull[s]);
+                        MILO_DT_STAMP(1, s);
                     }
                 }
                 if (!ok) sm.abort = 1;
@@ -498,33 +532,33 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
             }
         } else if (warp == 2) {
             // ======================================================== K MMA
+            MILO_DT_TRACE_STATE;
             if (lane == 0) {
                 const uint32_t id_rb = tc::idesc_f16(128, 128, 1, 1, 1);   // bf16, A/B MN-major
-                const uint32_t s_ak = tc::smem_u32(sm.akring), s_bk = tc::smem_u32(sm.bkring);
-                const uint32_t s_q = tc::smem_u32(sm.qt[0]);
-                uint32_t g = 0, ka = 0, kb = 0;
+                const uint32_t s_ak = tc::smem_u32(sm.akring), s_rr = tc::smem_u32(sm.rring);
+                const uint32_t s_zero = tc::smem_u32(sm.zero);
+                uint32_t g = 0, ka = 0, kr = 0;
                 bool ok = true;
-                // the tile whose scores are still to be issued
+                // the tile whose scores are still to be issued: its buffer, the
+                // queries of its item and the item's resident entry
                 bool have_prev = false;
-                uint32_t pg = 0, pn = 0;
-                int ptau = 0, pnt = 0, pnq16 = 16;
+                uint32_t pg = 0, pq = 0, prs = 0;
+                int plast = 0, pnq16 = 16;
                 auto scores = [&]() -> bool {
-                    const uint32_t b = pg & 1u, qb = pn & 1u;
+                    const uint32_t b = pg & 1u;
                     if (!dt_wait(&sm.kt_full[b], (pg >> 1) & 1u, lim)) return false;
-                    if (ptau == 0 && !dt_wait(&sm.qt_full[qb], (pn >> 1) & 1u, lim)) return false;
                     if (pg >= 2 && !dt_wait(&sm.s_free[b], ((pg - 2) >> 1) & 1u, lim)) return false;
                     tc::tc_fence_after();
-                    MILO_DT_TRACE(4, pn, ptau);
+                    MILO_DT_TRACE(4, 0, 0);
                     const uint32_t id_sc = tc::idesc_f16(128, pnq16, 0, 0, 0);   // fp16, A tmem, B K-major
                     // K step ks: columns 8 ks .. 8 ks + 7 of K-tilde, core-matrix
                     // columns 2 ks, 2 ks + 1 of the packed queries
                     for (int ks = 0; ks < D / 16; ++ks)
                         tc::mma_ts(tmem + DT_COL_S + 64 * b, tmem + DT_COL_KH + 128 * b + 8 * ks,
-                                   tc::smem_desc(s_q + qb * DT_QBUF + ks * 256, 128, 2048, tc::LAYOUT_NONE), id_sc,
-                                   ks > 0);
+                                   tc::smem_desc(pq + ks * 256, 128, 2048, tc::LAYOUT_NONE), id_sc, ks > 0);
                     tc::mma_commit(&sm.s_full[b]);
                     tc::mma_commit(&sm.kh_free[b]);
-                    if (ptau == pnt - 1) tc::mma_commit(&sm.qt_free[qb]);
+                    if (plast) tc::mma_commit(&sm.res_empty[prs]);   // the item's queries and B_K are done
                     return true;
                 };
                 for (uint32_t n = 0; ok; ++n) {
@@ -534,34 +568,50 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                     const DtGeo geo = dt_geo(e, G8);
                     tc::mbar_arrive(&sm.item_free[n % DT_NITAB]);
                     if (!live || sm.abort) break;
+                    // the item's queries and B_K.  The previous item's entry is freed by
+                    // its last scores: they go first unless this entry has landed, so
+                    // that no wait for an entry holds back the release of another
+                    // (two large entries need not fit in the ring together)
+                    const uint32_t rs = kr % DT_NRES;
+                    if (have_prev && !tc::mbar_test_wait(&sm.res_full[rs], (kr / DT_NRES) & 1u)) {
+                        if (!(ok = scores())) break;
+                        have_prev = false;
+                    }
+                    if (!(ok = dt_wait(&sm.res_full[rs], (kr / DT_NRES) & 1u, lim))) break;
+                    tc::fence_async_smem();   // the queries came through the generic proxy
+                    const uint32_t q_addr = s_rr + sm.res_off[rs];
+                    const uint32_t sb = q_addr + (uint32_t)geo.nq16 * 256u;
+                    const int nks = geo.R16K / 16;
+                    const bool odd = geo.R16K != geo.R8K;   // the last K step's upper 8 ranks read zeros
                     for (int t = 0; t < geo.nt && ok; ++t) {
                         const uint32_t b = g & 1u;
                         ok = dt_wait(&sm.akfull[ka % DT_NSLOT], (ka / DT_NSLOT) & 1u, lim);
-                        if (ok && t == 0) ok = dt_wait(&sm.bkfull[kb % DT_NBK], (kb / DT_NBK) & 1u, lim);
+                        MILO_DT_LAT(0, ka % DT_NSLOT);
+                        MILO_DT_TRACE(31, n, t);
                         if (ok && g >= 2) ok = dt_wait(&sm.kh_free[b], ((g - 2) >> 1) & 1u, lim);
                         if (!ok) break;
                         tc::tc_fence_after();
                         MILO_DT_TRACE(3, n, t);
                         const uint32_t sa = s_ak + sm.ak_off[ka % DT_NSLOT];
-                        const uint32_t sb = s_bk + sm.bk_off[kb % DT_NBK];
-                        for (int ks = 0; ks < geo.R16K / 16; ++ks)
-                            tc::mma_ss(tmem + DT_COL_KH + 128 * b,
-                                       tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
-                                       tc::smem_desc(sb + ks * 4096, 2048, 128, tc::LAYOUT_NONE), id_rb, ks > 0);
+                        for (int ks = 0; ks < nks; ++ks) {
+                            const uint32_t bk = geo.R8K ? sb + ks * 4096 : s_zero;
+                            const uint32_t lbo = geo.R8K == 0 ? 0u : (odd && ks == nks - 1) ? s_zero - bk : 2048u;
+                            tc::mma_ss(tmem + DT_COL_KH + 128 * b, tc::smem_desc(sa + ks * 4096, 2048, 128, tc::LAYOUT_NONE),
+                                       tc::smem_desc(bk, lbo, 128, tc::LAYOUT_NONE), id_rb, ks > 0);
+                        }
                         tc::mma_commit(&sm.kh_full[b]);
                         tc::mma_commit(&sm.akempty[ka % DT_NSLOT]);
-                        if (t == geo.nt - 1) tc::mma_commit(&sm.bkempty[kb % DT_NBK]);
                         ++ka;
-                        if (t == geo.nt - 1) ++kb;
                         if (have_prev && !(ok = scores())) break;
                         have_prev = true;
                         pg = g;
-                        pn = n;
-                        ptau = t;
-                        pnt = geo.nt;
+                        pq = q_addr;
+                        prs = rs;
+                        plast = t == geo.nt - 1;
                         pnq16 = geo.nq16;
                         ++g;
                     }
+                    ++kr;
                 }
                 if (ok && have_prev) ok = scores();
                 if (!ok) sm.abort = 1;
@@ -569,7 +619,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 dt_wait(&sm.drain_k, 0, lim);
             }
         } else {
-            // ======================================================== V warp: conversion + PV / O
+            // ======================================================== V warp: PV / O
+            MILO_DT_TRACE_STATE;
             const uint32_t s_v = tc::smem_u32(sm.vring);
             const uint32_t s_p = tc::smem_u32(sm.pbuf[0]);
             uint32_t g = 0, va = 0;
@@ -593,22 +644,9 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 for (int t = 0; t <= geo.nt && ok; ++t) {
                     const bool last = t == geo.nt;      // B_V
                     const uint32_t slot = va % DT_NSLOT;
-                    if (!(ok = wait_all(&sm.vfull[slot], (va / DT_NSLOT) & 1u))) break;
+                    // the tile in fp16 (the RoPE group converts it)
+                    if (!(ok = wait_all(&sm.vconv[slot], (va / DT_NSLOT) & 1u))) break;
                     if (lane == 0) MILO_DT_TRACE(5, n, t);
-                    uint8_t *tp = sm.vring + sm.v_off[slot];
-                    bf16_to_f16_inplace(tp, geo.R8V * 16, lane, 32);
-                    if (!last && geo.ones) {            // rank row R8V: fp16 ones, rows R8V+1 .. +7: zero
-                        uint4 *z = reinterpret_cast<uint4 *>(tp + geo.R8V * 256);
-                        for (int e2 = lane; e2 < 128; e2 += 32) {
-                            const uint32_t w = (e2 & 7) == 0 ? 0x3C003C00u : 0u;
-                            z[e2] = make_uint4(w, w, w, w);
-                        }
-                    } else if (last && geo.R16V > geo.R8V) {   // B_V pad rows: zero
-                        uint4 *z = reinterpret_cast<uint4 *>(tp + geo.R8V * 256);
-                        for (int e2 = lane; e2 < (geo.R16V - geo.R8V) * 16; e2 += 32) z[e2] = make_uint4(0, 0, 0, 0);
-                    }
-                    tc::fence_async_smem();
-                    __syncwarp();
                     if (!last && t == 0 && n >= 2 && !(ok = wait_all(&sm.oa_free[n & 1u], ((n - 2) >> 1) & 1u)))
                         break;
                     // PV: this tile's P buffer; O: the item's O_A / l, handed over in
@@ -653,6 +691,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         }
     } else if (warp < DT_W_SM) {
         // ============================================================ RoPE group
+        MILO_DT_TRACE_STATE;
         reg_alloc<DT_REG_ROPE>();
         const int quad = warp & 3;
         const int half = (warp - DT_W_ROPE) >> 2;         // RoPE pairs 32 half .. +31, O columns 32 half .. +31
@@ -675,27 +714,9 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
             const bool w = gt == 0 ? (dt_wait(b, par, lim) && !sm.abort) : true;
             return grp_and(DT_BAR_ROPE, DT_NROPE, w);
         };
-        // (cos, sin)(p theta) of pairs 2k, 2k+1 (k = gt % 32) of a slot: (c0, s0, c1, s1)
-        auto load_pcs = [&](int slot) -> float4 {
-            return reinterpret_cast<const float4 *>(a.rope_q + (int64_t)slot * HALF)[gt & 31];
-        };
-        // the table for position p from (cos, sin)(p theta) and (cos, sin)(32 v theta):
-        // this thread's entries (v, k) = (gt / 32 + 8 i, gt % 32)
-        auto build_rot = [&](float4 pcs) {
-            const float2 pc = make_float2(pcs.x, pcs.z), ps = make_float2(pcs.y, pcs.w);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int v = (gt >> 5) + 8 * i;
-                const float4 h = a.rope_hi[v * (HALF / 2) + (gt & 31)];
-                const float2 hc = make_float2(h.x, h.y), hs = make_float2(h.z, h.w);
-                const float2 c = __ffma2_rn(pc, hc, __fmul2_rn(make_float2(-ps.x, -ps.y), hs));
-                const float2 s = __ffma2_rn(ps, hc, __fmul2_rn(pc, hs));
-                sm.rot[v][gt & 31] = make_float4(c.x, c.y, s.x, s.y);
-            }
-        };
         // an item's geometry and, for the read-out, its partial indices (entry
-        // n of the table; read before the entry is freed)
-        int nxt_live = 0, nxt_nt = 0, nxt_nq = 0, nxt_slot0 = 0;
+        // m of the table; read before the entry is freed)
+        int nxt_live = 0, nxt_nt = 0, nxt_nq = 0, nxt_slot0 = 0, nxt_rV = 0;
         auto take = [&](uint32_t m) {
             const DtItem &e = sm.itab[m % DT_NITAB];
             nxt_live = e.l >= 0;
@@ -703,10 +724,40 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 nxt_nt = token_tiles(e.Tb);
                 nxt_nq = e.ns * G8;
                 nxt_slot0 = e.slots[0];
+                nxt_rV = e.rV;
                 if (gt < DT_NQ) sm.qp_rope[m & 3u][gt] = dt_pidx(a, e, gt);
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.item_free[m % DT_NITAB]);
+        };
+
+        // ---- the next tile of the V ring (an A_V tile, or B_V when last) to
+        // fp16 in place; A_V's rank row R8V to ones and rows R8V+1 .. +7 to zero
+        // when R8V <= 120, B_V's pad rows to zero
+        uint32_t va = 0;
+        auto vconvert = [&](int R8V, bool last, uint32_t n, int t) -> bool {
+            const uint32_t slot = va % DT_NSLOT;
+            if (!gwait(&sm.vfull[slot], (va / DT_NSLOT) & 1u)) return false;
+            if (gt == 0) {
+                MILO_DT_TRACE(27, n, t);
+                MILO_DT_LAT(1, slot);
+            }
+            uint8_t *tp = sm.vring + sm.v_off[slot];
+            bf16_to_f16_inplace(tp, R8V * 16, gt, DT_NROPE);
+            const int R16V = r16_of(R8V);
+            if (!last && R8V <= 120) {
+                if (gt < 128) {
+                    const uint32_t w = (gt & 7) == 0 ? 0x3C003C00u : 0u;
+                    reinterpret_cast<uint4 *>(tp + R8V * 256)[gt] = make_uint4(w, w, w, w);
+                }
+            } else if (last) {
+                for (int e2 = gt; e2 < (R16V - R8V) * 16; e2 += DT_NROPE)
+                    reinterpret_cast<uint4 *>(tp + R8V * 256)[e2] = make_uint4(0, 0, 0, 0);
+            }
+            tc::fence_async_smem();
+            tc::mbar_arrive(&sm.vconv[slot]);
+            ++va;
+            return true;
         };
 
         // ---- item m's O = B_V^T (O_A / l) (lanes = channels, columns = queries)
@@ -733,23 +784,21 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         };
 
         // ---------------------------------------------------- the item loop
-        // per item: RoPE of every tile against the item's rotation table, the
-        // next item's table (its (cos, sin)(p theta) loaded one item ahead),
+        // per item: RoPE and the V conversion of every tile, B_V's conversion,
         // then the previous item's read-out
         uint32_t g = 0, n = 0;
-        int cur_nt = 0, cur_nq = 0, prev_nq = 0;
+        int cur_nt = 0, cur_nq = 0, cur_R8V = 0, cur_slot0 = 0, prev_nq = 0;
         if (!(ok = gwait(&sm.item_full[0], 0))) {
             sm.abort = 1;
         } else {
             take(0);
-            if (nxt_live) build_rot(load_pcs(nxt_slot0));
-            grp_sync(DT_BAR_ROPE, DT_NROPE);
             for (; ok && nxt_live; ++n) {
                 cur_nt = nxt_nt;
                 cur_nq = nxt_nq;
+                cur_R8V = rank_pad(nxt_rV);
+                cur_slot0 = nxt_slot0;
                 if (!(ok = gwait(&sm.item_full[(n + 1) % DT_NITAB], ((n + 1) / DT_NITAB) & 1u))) break;
                 take(n + 1);
-                const float4 pcs_next = nxt_live ? load_pcs(nxt_slot0) : make_float4(1.f, 0.f, 1.f, 0.f);
                 for (int t = 0; t < cur_nt; ++t, ++g) {
                     const uint32_t b = g & 1u;
                     if (!(ok = gwait(&sm.kh_full[b], (g >> 1) & 1u))) break;
@@ -757,7 +806,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                     if (gt == 0) MILO_DT_TRACE(7, n, t);
                     const uint32_t base = tmem + DT_COL_KH + 128 * b + lane_off;
                     // (p + 32 v) theta for the rows of this warp: v = (128 t + 32 quad) / 32
-                    const float4 *hi = sm.rot[4 * t + quad] + c0 / 2;
+                    const float4 *hi = a.rot_slot + ((int64_t)cur_slot0 * 16 + 4 * t + quad) * (HALF / 2) + c0 / 2;
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {       // 16 pairs: x at columns i0 .., y at 64 + i0 ..
                         const int i0 = c0 + 16 * j;
@@ -765,11 +814,12 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                         tc::tmem_ld16(base + i0, xr);
                         tc::tmem_ld16(base + HALF + i0, yr);
                         tc::tmem_wait_ld();
+                        if (gt == 0 && j == 0) MILO_DT_TRACE(26, n, t);
                         uint32_t px[8], py[8];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {   // pairs i0 + 2v, i0 + 2v + 1
                             const int k = 8 * j + v;
-                            const float4 h4 = hi[k];
+                            const float4 h4 = __ldg(hi + k);
                             const float2 ch = make_float2(h4.x, h4.y), shh = make_float2(h4.z, h4.w);
                             // (cos, sin)((p + 32 v' + u) theta): rotation by (p + 32 v') theta after u theta
                             const float2 c = __ffma2_rn(ch, cl[k], __fmul2_rn(make_float2(-shh.x, -shh.y), sl[k]));
@@ -796,12 +846,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                     tc::tc_fence_before();
                     tc::mbar_arrive(&sm.kt_full[b]);
                     if (gt == 0) MILO_DT_TRACE(8, n, t);
+                    // the same tile of A_V
+                    if (!(ok = vconvert(cur_R8V, false, n, t))) break;
                 }
                 if (!ok) break;
-                // every read of this item's table done; the next item's in its place
-                grp_sync(DT_BAR_ROPE, DT_NROPE);
-                if (nxt_live) build_rot(pcs_next);
-                grp_sync(DT_BAR_ROPE, DT_NROPE);
+                if (!(ok = vconvert(cur_R8V, true, n, cur_nt))) break;   // B_V
                 if (n >= 1 && !(ok = readout(prev_nq, n - 1))) break;
                 prev_nq = cur_nq;
             }
@@ -810,6 +859,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         }
     } else {
         // ============================================================ softmax group
+        MILO_DT_TRACE_STATE;
         reg_dealloc<DT_REG_SM>();
         const int quad = warp & 3;
         const int half = (warp - DT_W_SM) >> 2;           // query columns 32 half .. +31
@@ -914,6 +964,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                     uint32_t r[16];
                     tc::tmem_ld16(dcol + c0 + 16 * hh, r);
                     tc::tmem_wait_ld();
+                    if (gt == 0 && hh == 0) MILO_DT_TRACE(22 + 2 * half, n, t);
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         const int k = 8 * hh + v;
@@ -928,6 +979,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 }
             };
             if (wc > 0 && w) make_p();
+            if (gt == 0) MILO_DT_TRACE(23 + 2 * half, n, t);
             // one barrier: the P buffer's previous product done (thread 0's wait),
             // no p above 2^8 (or not finite) in the half, no failed wait
             const bool pw = p_wait0(b);

@@ -524,6 +524,7 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));  // tensor-core work items
     at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H *
                            decode_tc_g8(Hq / f->shape.H) * D);              // packed fp16 queries
+    at = align_up(at + sizeof(float4) * slots * 16 * (HALF / 2));      // per-slot rotation tables
     return at;
 }
 
@@ -560,6 +561,8 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     DtItem *items = (DtItem *)(w + at);
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));
     __half *qpack = (__half *)(w + at);
+    at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H * decode_tc_g8(Hq / f->shape.H) * D);
+    float4 *rot_slot = (float4 *)(w + at);
 
     DecodeArgs a{};
     a.kv[0] = f->kv[0];
@@ -575,6 +578,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.G8 = decode_tc_g8(a.G);
     a.spi = decode_tc_spi(a.G);
     a.qpack = qpack;
+    a.rot_slot = rot_slot;
     {   // a test-injected fault applies to this call only
         std::lock_guard<std::mutex> lk(g_inject_mu);
         a.wait_ns = g_inject_wait_ns ? g_inject_wait_ns : kWaitNs;
@@ -602,6 +606,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
         const int64_t qchunks = (int64_t)a.L * S * a.H * a.G8 * 16;
         k_q_pack<<<(int)std::min<int64_t>((qchunks + 255) / 256, 8192), 256, 0, s>>>(q, a.L, S, a.H, a.G, a.G8,
                                                                                      qpack);
+        const int64_t nrot = slots * 16 * (HALF / 2);
+        k_rot_slots<<<(int)std::min<int64_t>((nrot + 255) / 256, 8192), 256, 0, s>>>(rope_q, rope_hi, (int)slots,
+                                                                                    rot_slot);
         st = cuda_check(launch_decode_tc(a, istart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
         k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
