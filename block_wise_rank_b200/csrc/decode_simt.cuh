@@ -33,7 +33,7 @@ struct DecodeArgs {
     const float2 *rope_lo;     // [32][64] (cos, sin)(u theta_i), u < 32: in-block angle, low five bits
     const float4 *rope_hi;     // [16][32] (cos, sin)(32 v theta_i) of pairs (2k, 2k+1): (c0, c1, s0, s1)
     float *part_o;             // [L][S][Hq][n_sel][D] (CUDA-core path)
-    __half *part_o16;          // [L][S][Hq][n_sel][D] (tensor-core path)
+    __half *part_o16;          // tensor-core path: rows of D, one per (item, query column) (see pmap)
     float2 *part_ml;           // [L][S][Hq][n_sel] (max, sum)
     float *out;                // [L][S][Hq][D]
     int32_t *claim;            // tensor-core path: next unclaimed work item (zeroed before the launch)
@@ -43,6 +43,7 @@ struct DecodeArgs {
     int spi;                   // tensor-core path: sessions per work item (64 / G8 queries, at most 8)
     const __half *qpack;       // tensor-core path: [L][S][H][G8 x 128] packed fp16 queries (k_q_pack)
     const float4 *rot_slot;    // tensor-core path: [S * n_sel][16][32] (cos, sin)((p + 32 v) theta_i) (k_rot_slots)
+    int32_t *pmap;             // tensor-core path: row of part_o16 holding each partial (written by k_dt_items)
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
@@ -412,7 +413,8 @@ __global__ void __launch_bounds__(128) k_combine(DecodeArgs a, const PT *__restr
         if (bid < 0 || bid >= a.n_b) continue;
         const float2 ml = a.part_ml[row * a.n_sel + u];
         const float w = __expf(ml.x - M) * ml.y;
-        num = fmaf(w, part_elem(part_o, (row * a.n_sel + u) * D + j), num);
+        const int64_t prow = a.pmap ? (int64_t)a.pmap[row * a.n_sel + u] : row * a.n_sel + u;
+        num = fmaf(w, part_elem(part_o, prow * D + j), num);
         den += w;
     }
     a.out[row * D + j] = den > 0.f ? num / den : 0.f;

@@ -34,7 +34,8 @@
 //                         Then converts the same tile of A_V (and, last, B_V)
 //                         to fp16 in place, appending a row of ones to A_V
 //                         when a rank row is free.  Also reads each item's O
-//                         out to the fp16 partials.
+//                         out (fp16, query-major in shared memory, then one
+//                         bulk store of the item's rows of partials).
 //   softmax group (8 w.)  two column halves of four warps, a token row per
 //                         thread: exp2 against a per-query reference max
 //                         raised only when some p exceeds 2^8, P (fp16) to
@@ -86,7 +87,7 @@ constexpr int DT_REG_LAUNCH = 96, DT_REG_CTRL = 48, DT_REG_ROPE = 128, DT_REG_SM
 static_assert(DT_REG_CTRL + 2 * DT_REG_ROPE + 2 * DT_REG_SM <= 5 * DT_REG_LAUNCH, "register split over the launch");
 constexpr int DT_VRING = 64 * 1024;               // A_V tiles (+ ones group) and B_V
 constexpr int DT_AKRING = 48 * 1024;              // A_K tiles
-constexpr int DT_RRING = 72 * 1024;               // per item: packed queries, then B_K
+constexpr int DT_RRING = 56 * 1024;               // per item: packed queries, then B_K (48 KB at most)
 constexpr int DT_NSLOT = 16;                      // tiles in flight per tile ring
 constexpr int DT_NRES = 4;                        // items in flight in the resident ring
 constexpr int DT_NITAB = 16;                      // item table entries
@@ -107,6 +108,7 @@ struct DtItem {
     int32_t ns, Tb, rK, rV; // sessions, tokens, ranks
     int64_t offK, offV;     // element offsets of the block in the data sections
     int32_t slots[DT_MAXS]; // the sessions' slots (s * n_sel + j); -1 past ns
+    int32_t row0, pad;      // first row of the item's partial outputs (ns x G8 rows of D)
 };
 
 struct DecTcSmem {
@@ -117,6 +119,7 @@ struct DecTcSmem {
     alignas(1024) uint8_t akring[DT_AKRING];
     alignas(1024) uint8_t rring[DT_RRING];
     alignas(1024) uint8_t pbuf[2][DT_PBUF];       // P, or O_A / l for an item's last product (fp16, MN-major)
+    alignas(1024) uint8_t ostage[DT_NQ * D * 2];  // an item's O, fp16, query-major, for its bulk store
     // 8 rank rows of zeros in the B_K operand layout: the second half of the
     // last K step when the padded rank is an odd multiple of 8, or both
     // halves (leading offset 0) for a block of rank 0
@@ -127,7 +130,6 @@ struct DecTcSmem {
     float lsum[2][DT_NQ];
     int cmax[DT_NQ];                              // column maxima, order-preserving int encoding
     int qp_sm[4][DT_NQ];                          // partial index of each query column (-1: none), per item
-    int qp_rope[4][DT_NQ];                        // the same, the RoPE group's copy
     uint32_t ak_off[DT_NSLOT], v_off[DT_NSLOT], res_off[DT_NRES];
     uint64_t item_full[DT_NITAB], item_free[DT_NITAB];
     uint64_t akfull[DT_NSLOT], akempty[DT_NSLOT];
@@ -144,6 +146,14 @@ struct DecTcSmem {
 
 // readers that free an item table entry: V producer, K MMA, V warp, 8 RoPE and 8 softmax warps
 constexpr int DT_ITEM_READERS = 1 + 1 + 1 + 8 + 8;
+
+// Partial index of query column c of an item (-1: a padding column).
+__device__ __forceinline__ int dt_pidx(const DecodeArgs &a, const DtItem &it, int c) {
+    const int k = c / a.G8, g = c % a.G8;
+    if (k >= it.ns || g >= a.G) return -1;
+    const int slot = it.slots[k];
+    return (int)((((int64_t)it.l * a.S + slot / a.n_sel) * a.Hq + it.h * a.G + g) * a.n_sel + slot % a.n_sel);
+}
 
 // Items of every (layer, head, block): the block's slot list (sorted by
 // (position, slot) by k_blk_items) cut into runs of equal position of at
@@ -166,13 +176,19 @@ __global__ void k_dt_items(DecodeArgs a, const int32_t *__restrict__ istart, DtI
     it.offV = a.kv[1].offsets[blk];
     int64_t out = lh * istart[a.n_b] + istart[b];
     const int s1 = a.slot_start[b + 1];
+    const int64_t nslots = (int64_t)a.S * a.n_sel;
+    it.pad = 0;
     for (int i = a.slot_start[b]; i < s1;) {
         const int p = slot_pos(a.sel, a.pos, a.slot_list[i], a.block_len);
         it.pos = p;
         it.ns = 0;
+        // the item's rows of partials: G8 per session, in the block's slot-list order
+        it.row0 = (int32_t)((lh * nslots + i) * a.G8);
         while (i < s1 && it.ns < a.spi && slot_pos(a.sel, a.pos, a.slot_list[i], a.block_len) == p)
             it.slots[it.ns++] = a.slot_list[i++];
         for (int k = it.ns; k < DT_MAXS; ++k) it.slots[k] = -1;
+        for (int k = 0; k < it.ns; ++k)
+            for (int g = 0; g < a.G; ++g) a.pmap[dt_pidx(a, it, k * a.G8 + g)] = it.row0 + k * a.G8 + g;
         items[out++] = it;
     }
 }
@@ -223,13 +239,6 @@ __device__ __forceinline__ DtGeo dt_geo(const DtItem &it, int G8) {
     return g;
 }
 
-// Partial index of query column c of an item (-1: a padding column).
-__device__ __forceinline__ int dt_pidx(const DecodeArgs &a, const DtItem &it, int c) {
-    const int k = c / a.G8, g = c % a.G8;
-    if (k >= it.ns || g >= a.G) return -1;
-    const int slot = it.slots[k];
-    return (int)((((int64_t)it.l * a.S + slot / a.n_sel) * a.Hq + it.h * a.G + g) * a.n_sel + slot % a.n_sel);
-}
 
 // named barriers, id and thread count in registers
 __device__ __forceinline__ void grp_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -714,9 +723,9 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
             const bool w = gt == 0 ? (dt_wait(b, par, lim) && !sm.abort) : true;
             return grp_and(DT_BAR_ROPE, DT_NROPE, w);
         };
-        // an item's geometry and, for the read-out, its partial indices (entry
-        // m of the table; read before the entry is freed)
-        int nxt_live = 0, nxt_nt = 0, nxt_nq = 0, nxt_slot0 = 0, nxt_rV = 0;
+        // an item's geometry and the first row of its partials (entry m of the
+        // table; read before the entry is freed)
+        int nxt_live = 0, nxt_nt = 0, nxt_nq = 0, nxt_slot0 = 0, nxt_rV = 0, nxt_row0 = 0;
         auto take = [&](uint32_t m) {
             const DtItem &e = sm.itab[m % DT_NITAB];
             nxt_live = e.l >= 0;
@@ -725,7 +734,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 nxt_nq = e.ns * G8;
                 nxt_slot0 = e.slots[0];
                 nxt_rV = e.rV;
-                if (gt < DT_NQ) sm.qp_rope[m & 3u][gt] = dt_pidx(a, e, gt);
+                nxt_row0 = e.row0;
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.item_free[m % DT_NITAB]);
@@ -761,25 +770,32 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         };
 
         // ---- item m's O = B_V^T (O_A / l) (lanes = channels, columns = queries)
-        // to the fp16 partials; frees the item's O_A^T buffer
-        auto readout = [&](int nq, uint32_t m) -> bool {
+        // to its nq rows of fp16 partials: query-major in shared memory, then one
+        // bulk store; frees the item's O_A^T buffer
+        auto readout = [&](int nq, int row0, uint32_t m) -> bool {
+            if (gt == 0) tc::bulk_wait_read_all();   // the previous item's store has read the buffer
             if (!gwait(&sm.o_full[m & 1u], (m >> 1) & 1u)) return false;
             tc::tc_fence_after();
             if (gt == 0) MILO_DT_TRACE(14, m, 0);
-            const int *qp = sm.qp_rope[m & 3u];
             if (c0 < nq) {
                 uint32_t r[32];
                 tc::tmem_ld32(tmem + DT_COL_OA + 64 * (m & 1u) + lane_off + c0, r);
                 tc::tmem_wait_ld();
+                if (gt == 0) MILO_DT_TRACE(32, m, 0);
+                __half *st = reinterpret_cast<__half *>(sm.ostage) + row;
 #pragma unroll
-                for (int v = 0; v < 32; ++v) {
-                    const int pi = qp[c0 + v];
-                    if (pi >= 0) a.part_o16[(int64_t)pi * D + row] = __float2half_rn(__uint_as_float(r[v]));
-                }
+                for (int v = 0; v < 32; ++v) st[(c0 + v) * D] = __float2half_rn(__uint_as_float(r[v]));
             }
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.oa_free[m & 1u]);
-            if (gt == 0) MILO_DT_TRACE(15, m, 0);
+            tc::fence_async_smem();
+            grp_sync(DT_BAR_ROPE, DT_NROPE);
+            if (gt == 0) {
+                MILO_DT_TRACE(33, m, 0);
+                tc::bulk_s2g(a.part_o16 + (int64_t)row0 * D, sm.ostage, (uint32_t)nq * D * 2u);
+                tc::bulk_commit();
+                MILO_DT_TRACE(15, m, 0);
+            }
             return true;
         };
 
@@ -787,7 +803,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
         // per item: RoPE and the V conversion of every tile, B_V's conversion,
         // then the previous item's read-out
         uint32_t g = 0, n = 0;
-        int cur_nt = 0, cur_nq = 0, cur_R8V = 0, cur_slot0 = 0, prev_nq = 0;
+        int cur_nt = 0, cur_nq = 0, cur_R8V = 0, cur_slot0 = 0, cur_row0 = 0, prev_nq = 0, prev_row0 = 0;
         if (!(ok = gwait(&sm.item_full[0], 0))) {
             sm.abort = 1;
         } else {
@@ -797,6 +813,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 cur_nq = nxt_nq;
                 cur_R8V = rank_pad(nxt_rV);
                 cur_slot0 = nxt_slot0;
+                cur_row0 = nxt_row0;
                 if (!(ok = gwait(&sm.item_full[(n + 1) % DT_NITAB], ((n + 1) / DT_NITAB) & 1u))) break;
                 take(n + 1);
                 for (int t = 0; t < cur_nt; ++t, ++g) {
@@ -851,12 +868,14 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 }
                 if (!ok) break;
                 if (!(ok = vconvert(cur_R8V, true, n, cur_nt))) break;   // B_V
-                if (n >= 1 && !(ok = readout(prev_nq, n - 1))) break;
+                if (n >= 1 && !(ok = readout(prev_nq, prev_row0, n - 1))) break;
                 prev_nq = cur_nq;
+                prev_row0 = cur_row0;
             }
-            if (ok && n >= 1) ok = readout(prev_nq, n - 1);
+            if (ok && n >= 1) ok = readout(prev_nq, prev_row0, n - 1);
             if (!ok) sm.abort = 1;
         }
+        if (gt == 0) tc::bulk_wait_all();   // the partials stored before the CTA exits
     } else {
         // ============================================================ softmax group
         MILO_DT_TRACE_STATE;

@@ -511,6 +511,16 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
     return launch_select(a, a, sh, 1, (cudaStream_t)stream);
 }
 
+// Partial outputs: fp32 rows (L, S, Hq, n_sel) of D for the CUDA-core path;
+// fp16 rows of D, G8 per selected slot and (layer, KV head), for the tensor
+// cores.  The region holds either.
+static size_t part_o_bytes(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    const int64_t slots = (int64_t)S * n_sel;
+    const size_t simt = sizeof(float) * (size_t)f->shape.L * S * Hq * n_sel * D;
+    const size_t tc = sizeof(__half) * (size_t)f->shape.L * f->shape.H * slots * decode_tc_g8(Hq / f->shape.H) * D;
+    return std::max(simt, tc);
+}
+
 size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
     if (!f || S <= 0 || Hq <= 0 || n_sel <= 0) return 0;
     const int64_t slots = (int64_t)S * n_sel;
@@ -519,8 +529,9 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursors / item counts, slot starts, item starts, claim
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);  // rope tables
-    at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o (fp32, or fp16 in its first half)
+    at = align_up(at + part_o_bytes(f, S, Hq, n_sel));                 // partial o
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
+    at = align_up(at + sizeof(int32_t) * rows * n_sel);                // partial -> row of partial o (tensor cores)
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));  // tensor-core work items
     at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H *
                            decode_tc_g8(Hq / f->shape.H) * D);              // packed fp16 queries
@@ -556,8 +567,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     float2 *rope_lo = rope_t + (int64_t)f->shape.block_len * HALF;
     float4 *rope_hi = (float4 *)(rope_lo + 32 * HALF);
     at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);
-    float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
+    float *part_o = (float *)(w + at); at = align_up(at + part_o_bytes(f, S, Hq, n_sel));
     float2 *part_ml = (float2 *)(w + at); at = align_up(at + sizeof(float2) * rows * n_sel);
+    int32_t *pmap = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * rows * n_sel);
     DtItem *items = (DtItem *)(w + at);
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));
     __half *qpack = (__half *)(w + at);
@@ -579,6 +591,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.spi = decode_tc_spi(a.G);
     a.qpack = qpack;
     a.rot_slot = rot_slot;
+    a.pmap = nullptr;   // the CUDA-core path's partials are indexed directly
     {   // a test-injected fault applies to this call only
         std::lock_guard<std::mutex> lk(g_inject_mu);
         a.wait_ns = g_inject_wait_ns ? g_inject_wait_ns : kWaitNs;
@@ -609,6 +622,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
         const int64_t nrot = slots * 16 * (HALF / 2);
         k_rot_slots<<<(int)std::min<int64_t>((nrot + 255) / 256, 8192), 256, 0, s>>>(rope_q, rope_hi, (int)slots,
                                                                                     rot_slot);
+        a.pmap = pmap;
         st = cuda_check(launch_decode_tc(a, istart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
         k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
