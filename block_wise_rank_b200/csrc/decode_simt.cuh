@@ -44,6 +44,7 @@ struct DecodeArgs {
     const __half *qpack;       // tensor-core path: [L][S][H][G8 x 128] packed fp16 queries (k_q_pack)
     const float4 *rot_slot;    // tensor-core path: [S * n_sel][16][32] (cos, sin)((p + 32 v) theta_i) (k_rot_slots)
     int32_t *pmap;             // tensor-core path: row of part_o16 holding each partial (written by k_dt_items)
+    int f16;                   // tensor-core path: kv[].data holds fp16 factors (INT8 dequantised), else bf16
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every

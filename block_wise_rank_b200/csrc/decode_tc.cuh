@@ -1,5 +1,6 @@
 // decode_tc.cuh -- decode attention over retrieved compressed blocks on
-// tcgen05 tensor cores (bf16 factors).
+// tcgen05 tensor cores (bf16 factors, or INT8 factors dequantised to fp16 by
+// k_dequant_selected).
 //
 // Step "at inference a retriever selects blocks, whose low-rank factors are
 // rebuilt before sparse attention" (evolve.pub review of MILO, Summary; FAQ
@@ -543,7 +544,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
             // ======================================================== K MMA
             MILO_DT_TRACE_STATE;
             if (lane == 0) {
-                const uint32_t id_rb = tc::idesc_f16(128, 128, 1, 1, 1);   // bf16, A/B MN-major
+                const uint32_t id_rb = tc::idesc_f16(128, 128, a.f16 ? 0 : 1, 1, 1);   // bf16 (or fp16), A/B MN-major
                 const uint32_t s_ak = tc::smem_u32(sm.akring), s_rr = tc::smem_u32(sm.rring);
                 const uint32_t s_zero = tc::smem_u32(sm.zero);
                 uint32_t g = 0, ka = 0, kr = 0;
@@ -752,7 +753,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ istart, const DtItem *__re
                 MILO_DT_LAT(1, slot);
             }
             uint8_t *tp = sm.vring + sm.v_off[slot];
-            bf16_to_f16_inplace(tp, R8V * 16, gt, DT_NROPE);
+            if (!a.f16) bf16_to_f16_inplace(tp, R8V * 16, gt, DT_NROPE);
             const int R16V = r16_of(R8V);
             if (!last && R8V <= 120) {
                 if (gt < 128) {
@@ -1198,7 +1199,54 @@ inline int decode_tc_spi(int G) { return std::min(DT_MAXS, DT_NQ / decode_tc_g8(
 
 inline bool decode_tc_supported(const DecodeArgs &a) {
     if (getenv("MILO_FORCE_SIMT")) return false;
-    return a.factor_dtype == MILO_BF16 && a.block_len <= 512 && decode_tc_g8(a.G) <= DT_NQ;
+    return (a.factor_dtype == MILO_BF16 || a.factor_dtype == MILO_INT8) && a.block_len <= 512 &&
+           decode_tc_g8(a.G) <= DT_NQ;
+}
+
+// INT8 factors for the tensor cores: the selected blocks' factors of both
+// kinds, code x per-column scale (A: per rank, B: per channel) rounded to
+// fp16, written at the same element offsets into `out` (one section per
+// kind, laid out like the INT8 data).  Grid (L*H*n_b, 2); blocks no slot
+// selected are skipped.  8 elements (one core-matrix row) per thread step.
+__global__ void __launch_bounds__(256) k_dequant_selected(DecodeArgs a, __half *out0, __half *out1) {
+    const int64_t blk = blockIdx.x;
+    const int kind = blockIdx.y;
+    const int b = (int)(blk % a.n_b);
+    if (a.slot_start[b + 1] == a.slot_start[b]) return;
+    const KindView &kv = a.kv[kind];
+    const int R8 = rank_pad(kv.ranks[blk]);
+    if (R8 == 0) return;
+    const int Tb = block_tokens(a.T, a.block_len, b);
+    const int nt = token_tiles(Tb);
+    const int64_t base = kv.offsets[blk];
+    const int64_t nA = (int64_t)nt * R8 * FTILE, nAll = nA + (int64_t)R8 * D;
+    const int8_t *src = (const int8_t *)kv.data + base;
+    __half *dst = (kind ? out1 : out0) + base;
+    const float *sA = kv.scaleA + blk * D, *sB = kv.scaleB + blk * D;
+    for (int64_t e = (int64_t)threadIdx.x * 8; e < nAll; e += 256 * 8) {
+        const uint2 codes = *reinterpret_cast<const uint2 *>(src + e);   // 8 codes, one row of a core matrix
+        const int8_t *c = reinterpret_cast<const int8_t *>(&codes);
+        float sc[8];
+        if (e < nA) {   // A tile: [k/8][u/8][k%8][u%8], one rank k per 8 elements
+            const int r = (int)(e % (R8 * FTILE));
+            const float s = sA[(r >> 10) * 8 + ((r & 63) >> 3)];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] = s;
+        } else {        // B: [k/8][j/8][k%8][j%8], eight channels j per 8 elements
+            const int r = (int)(e - nA);
+            const int j0 = ((r & 1023) >> 6) * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] = sB[j0 + i];
+        }
+        uint4 o;
+        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = __floats2half2_rn((float)c[2 * i] * sc[2 * i], (float)c[2 * i + 1] * sc[2 * i + 1]);
+            ow[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(dst + e) = o;
+    }
 }
 
 // The warpgroups' register split assumes the launch value; a build that

@@ -87,6 +87,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
 
     bool converged = false;
     int sweeps_done = 0;
+    unsigned rounds_applied = 0;
     for (int sweep = 0; sweep < max_sweeps && !converged; ++sweep) {
         ++sweeps_done;
         int any = 0;
@@ -112,6 +113,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
             rot = __syncthreads_or(rot);
             any |= rot;
             if (!rot) continue;   // uniform across the CTA
+            ++rounds_applied;
             // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2 (upper triangle)
             for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
                 const int i = sm.tri[e][0], i2 = sm.tri[e][1];
@@ -162,6 +164,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
     }
     if (!converged && tid == 0) raise_status(ST_NOT_CONVERGED);
     MILO_TRACE_JACOBI(sweeps_done);
+    if (tid == 0) atomicAdd(&g_jacobi_rounds, (unsigned long long)rounds_applied);
 
     // eigenvalues, stable descending order
     if (tid < D) sm.lam[tid] = sm.G[jac_g(tid, tid)];

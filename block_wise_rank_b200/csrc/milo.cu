@@ -13,6 +13,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 #include <new>
 
 #include "common.cuh"
@@ -169,6 +171,42 @@ milo_status cuda_check(cudaError_t e, const char *what) {
 // hook milo_test_decode_inject.
 constexpr uint64_t kWaitNs = 2000000000ull;
 std::mutex g_inject_mu;
+
+// Kernel timing: event pairs per stage, recorded while enabled.
+struct StageTiming {
+    std::mutex mu;
+    bool on = false;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[MILO_TK_COUNT];
+} g_timing;
+
+cudaEvent_t tmark(cudaStream_t s) {
+    if (!g_timing.on) return nullptr;
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    if (cudaEventRecord(e, s) != cudaSuccess) {
+        cudaEventDestroy(e);
+        return nullptr;
+    }
+    return e;
+}
+void tpush(int stage, cudaEvent_t a, cudaEvent_t b) {
+    if (!a || !b) {
+        if (a) cudaEventDestroy(a);
+        if (b) cudaEventDestroy(b);
+        return;
+    }
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    g_timing.ev[stage].emplace_back(a, b);
+}
+void timing_drop_locked() {
+    for (auto &v : g_timing.ev) {
+        for (auto &p : v) {
+            cudaEventDestroy(p.first);
+            cudaEventDestroy(p.second);
+        }
+        v.clear();
+    }
+}
 int g_inject_mode = 0;
 uint64_t g_inject_wait_ns = 0;
 
@@ -323,6 +361,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
 
     // 1. Gram matrices of every block of K and V
     const dim3 grid2((unsigned)nblk, 2);
+    cudaEvent_t t0 = tmark(s);
     if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->T, shape->block_len)) {
         st = cuda_check(launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H,
                                        shape->T, shape->block_len, f->n_b, GW, nblk, sm_count(), s),
@@ -335,10 +374,15 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
         k_gram_simt<float><<<grid2, 256, 0, s>>>((const float *)K, (const float *)V, shape->H, shape->T,
                                                   shape->block_len, f->n_b, GW, nblk);
     }
+    cudaEvent_t t1 = tmark(s);
+    tpush(MILO_TK_GRAM, t0, t1);
     // 2. eigensolve: sigma into the arena, sorted eigenvectors back into GW
+    t0 = tmark(s);
     k_jacobi<<<grid2, JAC_THREADS, jacobi_smem_bytes(), s>>>(GW, f->kv[0].sigma, f->kv[1].sigma, nblk, shape->T,
                                                              shape->block_len, f->n_b, p.max_sweeps, p.jacobi_tol);
+    tpush(MILO_TK_JACOBI, t0, tmark(s));
     // 2b. singular values recomputed from the blocks, sigma / W re-sorted
+    t0 = tmark(s);
     if (shape->in_dtype == MILO_BF16)
         k_refine_sigma<__nv_bfloat16><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
             (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T,
@@ -347,8 +391,10 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
         k_refine_sigma<float><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
             (const float *)K, (const float *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T, shape->block_len,
             f->n_b, nblk);
+    tpush(MILO_TK_REFINE, t0, tmark(s));
     // 3. eps per (layer, head, kind)
     const int ngroups = shape->L * shape->H;
+    t0 = tmark(s);
     k_eps<<<dim3(ngroups, 2), 256, 0, s>>>(f->kv[0].sigma, f->kv[1].sigma, f->kv[0].eps, f->kv[1].eps, f->n_b,
                                            p.eps_rel);
     if (p.eps_scope == 1) k_eps_global<<<2, 1024, 0, s>>>(f->kv[0].eps, f->kv[1].eps, ngroups);
@@ -368,6 +414,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
         a[k].need0 = R - floors * ngroups;
     }
     if ((st = launch_select(a[0], a[1], sh, 2, s)) != MILO_OK) { delete f; return st; }
+    tpush(MILO_TK_SELECT, t0, tmark(s));
     // 5. projection A_b = X_b W_{:,1:r_b}, B_b = W_{:,1:r_b}^T, packing
     ProjArgs pa{};
     pa.X[0] = K;
@@ -382,11 +429,13 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     pa.in_dtype = shape->in_dtype;
     pa.out_dtype = p.factor_dtype;
     pa.n_blk = nblk;
+    t0 = tmark(s);
     if (shape->in_dtype == MILO_BF16)
         k_project_a<__nv_bfloat16><<<dim3((unsigned)nblk, D / 32, 2), 256, 0, s>>>(pa);
     else
         k_project_a<float><<<dim3((unsigned)nblk, D / 32, 2), 256, 0, s>>>(pa);
     k_project_b<<<grid2, D, 0, s>>>(pa);
+    tpush(MILO_TK_PROJECT, t0, tmark(s));
     st = cuda_check(cudaGetLastError(), "compress launch");
     if (st != MILO_OK) { delete f; return st; }
     log_msg("compress launched");
@@ -511,6 +560,14 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
     return launch_select(a, a, sh, 1, (cudaStream_t)stream);
 }
 
+// INT8 factors on the tensor cores: an fp16 copy of each kind's data section
+// (the selected blocks' elements are written, at the INT8 element offsets).
+static size_t shadow_bytes_per_kind(const milo_factors *f) {
+    if (f->params.factor_dtype != MILO_INT8) return 0;
+    return align_up(sizeof(__half) * (size_t)(f->R + 7 * f->n_blk) *
+                    (size_t)(round_up(f->shape.block_len, FTILE) + D));
+}
+
 // Partial outputs: fp32 rows (L, S, Hq, n_sel) of D for the CUDA-core path;
 // fp16 rows of D, G8 per selected slot and (layer, KV head), for the tensor
 // cores.  The region holds either.
@@ -536,6 +593,7 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H *
                            decode_tc_g8(Hq / f->shape.H) * D);              // packed fp16 queries
     at = align_up(at + sizeof(float4) * slots * 16 * (HALF / 2));      // per-slot rotation tables
+    at += 2 * shadow_bytes_per_kind(f);                                 // INT8: fp16 factors
     return at;
 }
 
@@ -575,6 +633,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     __half *qpack = (__half *)(w + at);
     at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H * decode_tc_g8(Hq / f->shape.H) * D);
     float4 *rot_slot = (float4 *)(w + at);
+    at = align_up(at + sizeof(float4) * slots * 16 * (HALF / 2));
+    __half *shadow0 = (__half *)(w + at);
+    __half *shadow1 = (__half *)(w + at + shadow_bytes_per_kind(f));
 
     DecodeArgs a{};
     a.kv[0] = f->kv[0];
@@ -592,6 +653,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.qpack = qpack;
     a.rot_slot = rot_slot;
     a.pmap = nullptr;   // the CUDA-core path's partials are indexed directly
+    a.f16 = 0;
     {   // a test-injected fault applies to this call only
         std::lock_guard<std::mutex> lk(g_inject_mu);
         a.wait_ns = g_inject_wait_ns ? g_inject_wait_ns : kWaitNs;
@@ -604,6 +666,7 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ((n_b + 1) * 3 + 1), s);
     if (e != cudaSuccess) return cuda_check(e, "memset");
     const int sg = (int)std::min<int64_t>((slots + 255) / 256, 1024);
+    cudaEvent_t t0 = tmark(s);
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
     k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, n_b);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
@@ -611,6 +674,12 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
         selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t, rope_lo, rope_hi);
     if (decode_tc_supported(a)) {
+        if (a.factor_dtype == MILO_INT8) {   // dequantised to fp16 for the tensor cores
+            k_dequant_selected<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, shadow0, shadow1);
+            a.kv[0].data = shadow0;
+            a.kv[1].data = shadow1;
+            a.f16 = 1;
+        }
         // items: each block's slots sorted by position (the fill order is not
         // deterministic), cut into runs of equal position; item starts per block
         k_blk_items<<<(n_b + 127) / 128, 128, 0, s>>>(selected, positions, n_b, f->shape.block_len, start, list,
@@ -622,13 +691,23 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
         const int64_t nrot = slots * 16 * (HALF / 2);
         k_rot_slots<<<(int)std::min<int64_t>((nrot + 255) / 256, 8192), 256, 0, s>>>(rope_q, rope_hi, (int)slots,
                                                                                     rot_slot);
+        tpush(MILO_TK_DECODE_PREP, t0, tmark(s));
+        t0 = tmark(s);
         a.pmap = pmap;
         st = cuda_check(launch_decode_tc(a, istart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
+        tpush(MILO_TK_DECODE, t0, tmark(s));
+        t0 = tmark(s);
         k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
+        tpush(MILO_TK_COMBINE, t0, tmark(s));
     } else {
+        tpush(MILO_TK_DECODE_PREP, t0, tmark(s));
+        t0 = tmark(s);
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
+        tpush(MILO_TK_DECODE, t0, tmark(s));
+        t0 = tmark(s);
         k_combine<float><<<(unsigned)rows, D, 0, s>>>(a, a.part_o);
+        tpush(MILO_TK_COMBINE, t0, tmark(s));
     }
     return cuda_check(cudaGetLastError(), "decode launch");
 }
@@ -730,6 +809,47 @@ milo_status milo_test_decode_inject(int32_t mode, uint64_t wait_ns) {
     std::lock_guard<std::mutex> lk(g_inject_mu);
     g_inject_mode = mode;
     g_inject_wait_ns = wait_ns;
+    return MILO_OK;
+}
+
+milo_status milo_timing_enable(int32_t on) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    if (on) timing_drop_locked();
+    g_timing.on = on != 0;
+    return MILO_OK;
+}
+
+milo_status milo_timing_read(double *ms, int64_t *count, int32_t n) {
+    if (n < 0 || n > MILO_TK_COUNT || (n > 0 && (!ms || !count))) return MILO_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    milo_status st = MILO_OK;
+    for (int k = 0; k < MILO_TK_COUNT; ++k) {
+        double sum = 0.0;
+        for (auto &p : g_timing.ev[k]) {
+            float t = 0.f;
+            cudaError_t e = cudaEventSynchronize(p.second);
+            if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.first, p.second);
+            if (e != cudaSuccess && st == MILO_OK) st = cuda_check(e, "timing events");
+            sum += t;
+        }
+        if (k < n) {
+            ms[k] = sum;
+            count[k] = (int64_t)g_timing.ev[k].size();
+        }
+    }
+    timing_drop_locked();
+    return st;
+}
+
+milo_status milo_jacobi_rounds(int64_t *rounds, milo_stream_t stream) {
+    if (!rounds) return MILO_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_check(e, "stream sync");
+    unsigned long long v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, g_jacobi_rounds, sizeof(v));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_jacobi_rounds, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_check(e, "counter read");
+    *rounds = (int64_t)v;
     return MILO_OK;
 }
 

@@ -53,8 +53,12 @@ EXPORTS = [
     "milo_compress", "milo_allocate_workspace_size", "milo_allocate", "milo_decode_workspace_size",
     "milo_decode_attn", "milo_factors_get", "milo_factors_wrap", "milo_factors_export",
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
-    "milo_allocate_noalloc", "milo_test_decode_inject",
+    "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
+    "milo_jacobi_rounds",
 ]
+
+# stages of milo_timing_read, in order (milo_timed_stage)
+TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine"]
 
 MILO_NOALLOC_MAX_BLOCKS = 65536
 
@@ -96,6 +100,9 @@ def lib():
         L.milo_version.argtypes = []; L.milo_version.restype = ctypes.c_char_p
         L.milo_test_decode_inject.argtypes = [I32, ctypes.c_uint64]
         L.milo_test_decode_inject.restype = ctypes.c_int
+        L.milo_timing_enable.argtypes = [I32]; L.milo_timing_enable.restype = ctypes.c_int
+        L.milo_timing_read.argtypes = [P, P, I32]; L.milo_timing_read.restype = ctypes.c_int
+        L.milo_jacobi_rounds.argtypes = [P, P]; L.milo_jacobi_rounds.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -307,6 +314,31 @@ def milo_test_decode_inject(mode: int, wait_ns: int = 0) -> int:
     """Test hook: arm (mode 1) a withheld copy and a wait limit of wait_ns for
     the next tensor-core decode call, or disarm (mode 0).  Returns the status."""
     return lib().milo_test_decode_inject(int(mode), int(wait_ns))
+
+
+def milo_timing_enable(on: bool = True) -> None:
+    """Start (dropping earlier records) or stop bracketing each stage's kernels
+    with CUDA events on their launch stream."""
+    _check(lib().milo_timing_enable(1 if on else 0), "milo_timing_enable")
+
+
+def milo_timing_read() -> dict:
+    """{stage: (summed ms, launches)} of the records since milo_timing_enable;
+    waits for the events and drops them."""
+    n = len(TIMED_STAGES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(lib().milo_timing_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n),
+           "milo_timing_read")
+    return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(TIMED_STAGES)}
+
+
+def milo_jacobi_rounds(stream=None) -> int:
+    """Jacobi rounds that applied rotations since the last read (synchronises)."""
+    v = ctypes.c_int64(0)
+    _check(lib().milo_jacobi_rounds(ctypes.cast(ctypes.byref(v), ctypes.c_void_p), _stream(stream)),
+           "milo_jacobi_rounds")
+    return int(v.value)
 
 
 def milo_version() -> str:

@@ -264,6 +264,42 @@ void milo_factors_destroy(milo_factors *f);
  */
 milo_status milo_test_decode_inject(int32_t mode, uint64_t wait_ns);
 
+/* ---------------------------------------------------------------- timing */
+
+/*
+ * Kernel timing (measurement; no counterpart on the pages).  While enabled,
+ * the library brackets the kernels of each stage below with CUDA events on
+ * the stream the stage is launched on, and sums their elapsed times.
+ */
+typedef enum {
+    MILO_TK_GRAM = 0,        /* Gram matrices (k_gram_tc or k_gram_simt) */
+    MILO_TK_JACOBI = 1,      /* one-sided Jacobi eigensolve (k_jacobi) */
+    MILO_TK_REFINE = 2,      /* singular values recomputed from the blocks (k_refine_sigma) */
+    MILO_TK_SELECT = 3,      /* eps and the global top-R rank selection */
+    MILO_TK_PROJECT = 4,     /* projection and packing of A and B (k_project_a, k_project_b) */
+    MILO_TK_DECODE_PREP = 5, /* decode index, table and query-packing kernels */
+    MILO_TK_DECODE = 6,      /* decode attention (k_decode_tc or k_decode_simt) */
+    MILO_TK_COMBINE = 7,     /* merge of the per-block partials (k_combine) */
+    MILO_TK_COUNT = 8
+} milo_timed_stage;
+
+/* on != 0: start recording (previous records are dropped); on == 0: stop.
+ * Host-side only; the events are created on the current device. */
+milo_status milo_timing_enable(int32_t on);
+
+/* Wait for every recorded event, then write per stage (n entries, stage
+ * order above; n <= MILO_TK_COUNT) the summed milliseconds into ms and the
+ * number of bracketed launches into count, and drop the records.  ms and
+ * count are host arrays.  MILO_ERR_INVALID_ARG for n outside 0 .. 8 or a NULL
+ * array; a CUDA error of the event queries is returned as MILO_ERR_CUDA. */
+milo_status milo_timing_read(double *ms, int64_t *count, int32_t n);
+
+/* Synchronise stream, then read and clear the count of Jacobi rounds that
+ * applied rotations, summed over every (block, kind) eigensolve since the
+ * last read (one round = the 64 disjoint plane rotations applied to the
+ * d x d Gram tile and to W).  The eigensolve's work for its throughput. */
+milo_status milo_jacobi_rounds(int64_t *rounds, milo_stream_t stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronise stream, then read and clear the current device's status word:

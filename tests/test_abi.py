@@ -142,3 +142,15 @@ def test_wrap_views_and_export_size(L):
     assert L.milo_factors_wrap(ctypes.byref(s), ctypes.byref(p), fake, n - 1, ctypes.byref(h)) == \
         milo.MILO_ERR_WORKSPACE
     L.milo_factors_destroy(h)
+
+
+def test_timing_hooks_on_host(L):
+    """Timing records need no device while nothing was launched: enabling,
+    reading (all zero) and argument checks run on the host."""
+    milo.milo_timing_enable(True)
+    t = milo.milo_timing_read()
+    assert set(t) == set(milo.TIMED_STAGES) and all(v == (0.0, 0) for v in t.values())
+    milo.milo_timing_enable(False)
+    assert L.milo_timing_read(None, None, 0) == milo.MILO_OK
+    assert L.milo_timing_read(None, None, 3) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_timing_read(None, None, 9) == milo.MILO_ERR_INVALID_ARG

@@ -69,3 +69,41 @@ def test_single_rank_needs_no_process_group():
     b = _bench()
     assert not dist.is_initialized()
     assert b.max_over_ranks([1.0, 2.0], 1, torch.device("cpu")) == [1.0, 2.0]
+
+
+def test_decode_traffic_follows_the_kernel_source(tmp_path):
+    """Traffic comes from the committed ncu counters only while the decode
+    kernel's code is the one they were taken on, for the same workload,
+    factor type and budget; it scales with the layer count."""
+    import json
+
+    b = _bench()
+    p = tmp_path / "t.json"
+    rec = dict(workload="qwen7b-128k", factor="bf16", budget=0.5, layers=4, dram_bytes_read=3_000_000,
+               dram_bytes_write=1_000_000, source_sha256_16=b.source_hash())
+    p.write_text(json.dumps(rec))
+    b.TRAFFIC_JSON = str(p)
+    w = b.synth.WORKLOADS["qwen7b-128k"]
+    assert b.decode_traffic(w, "bf16", 0.5) == 4_000_000 * w.L // 4
+    assert b.decode_traffic(w, "int8", 0.5) is None
+    assert b.decode_traffic(w, "bf16", 0.25) is None
+    assert b.decode_traffic(b.synth.WORKLOADS["qwen3b-32k"], "bf16", 0.5) is None
+    p.write_text(json.dumps(dict(rec, source_sha256_16="0" * 16)))
+    assert b.decode_traffic(w, "bf16", 0.5) is None
+
+
+def test_oracle_sample_uses_the_greedy_allocation():
+    """The CPU baseline's sample: the oracle's own SVD, eps and greedy top-R
+    ranks over the sampled blocks (sum of ranks = the sample's budget), and a
+    decode loop that counts the factor bytes per query."""
+    import oracle
+
+    b = _bench()
+    w = b.synth.WORKLOADS["toy"]
+    s = b.oracle_sample(w, 0.5, "f32")
+    nb = len(s["blocks"])
+    R = oracle.budget(1, 1, nb * w.block_len, w.block_len, w.d, 0.5)
+    assert sum(s["facs"][blk][0][0].shape[1] for blk in s["blocks"]) == R
+    assert sum(s["facs"][blk][1][0].shape[1] for blk in s["blocks"]) == R
+    nbytes, n, el = b._oracle_decode_loop(s, 0.0)
+    assert n == 1 and nbytes == s["bytes_per_query"] > 0
