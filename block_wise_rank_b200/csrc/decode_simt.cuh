@@ -30,51 +30,32 @@ struct DecodeArgs {
     const int32_t *slot_list;  // [S * n_sel] slot = s * n_sel + j
     const float2 *rope_q;      // [S * n_sel][64] (cos, sin)(p theta_i)
     const float2 *rope_t;      // [block_len][64] (cos, sin)(t theta_i)
-    const float2 *rope_lo;     // [32][64] (cos, sin)(u theta_i), u < 32: in-block angle, low five bits
-    const float4 *rope_hi;     // [16][32] (cos, sin)(32 v theta_i) of pairs (2k, 2k+1): (c0, c1, s0, s1)
-    float *part_o;             // [L][S][Hq][n_sel][D] (CUDA-core path)
-    __half *part_o16;          // tensor-core path: rows of D, one per (item, query column) (see pmap)
+    float *part_o;             // [L][S][Hq][n_sel][D]
     float2 *part_ml;           // [L][S][Hq][n_sel] (max, sum)
     float *out;                // [L][S][Hq][D]
     int32_t *claim;            // tensor-core path: next unclaimed work item (zeroed before the launch)
     uint64_t wait_ns;          // tensor-core path: limit of every wait on the device
     int inject;                // tensor-core path: 1 = withhold one copy (tests of the bounded waits)
-    int G8;                    // tensor-core path: GQA group padded to a multiple of 8
-    int spi;                   // tensor-core path: sessions per work item (64 / G8 queries, at most 8)
-    const __half *qpack;       // tensor-core path: [L][S][H][G8 x 128] packed fp16 queries (k_q_pack)
-    const float4 *rot_slot;    // tensor-core path: [S * n_sel][16][32] (cos, sin)((p + 32 v) theta_i) (k_rot_slots)
-    int32_t *pmap;             // tensor-core path: row of part_o16 holding each partial (written by k_dt_items)
     int f16;                   // tensor-core path: kv[].data holds fp16 factors (INT8 dequantised), else bf16
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
-// in-block token, angles in double, theta_i = base^(-2i/d).  The same
-// in-block angles split as t = 32 v + u (u < 32, v < 16) for the tensor-core
-// path: (u theta_i) per pair and (32 v theta_i) per pair of pairs.
+// in-block token, angles in double, theta_i = base^(-2i/d).
 __global__ void k_rope_tables(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int n_slots,
-                              int block_len, double base, float2 *__restrict__ rope_q, float2 *__restrict__ rope_t,
-                              float2 *__restrict__ rope_lo, float4 *__restrict__ rope_hi) {
-    const int64_t total = (int64_t)(n_slots + block_len + 32 + 16) * HALF;
+                              int block_len, double base, float2 *__restrict__ rope_q, float2 *__restrict__ rope_t) {
+    const int64_t total = (int64_t)(n_slots + block_len) * HALF;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int i = (int)(e % HALF);
         const int64_t row = e / HALF;
         const double theta = pow(base, -2.0 * (double)i / (double)D);
         double p;
         if (row < n_slots) p = pos ? (double)pos[row] : (double)sel[row] * (double)block_len;
-        else if (row < n_slots + block_len) p = (double)(row - n_slots);
-        else if (row < n_slots + block_len + 32) p = (double)(row - n_slots - block_len);
-        else p = 32.0 * (double)(row - n_slots - block_len - 32);
+        else p = (double)(row - n_slots);
         double sn, cs;
         sincos(p * theta, &sn, &cs);
         const float2 v = make_float2((float)cs, (float)sn);
         if (row < n_slots) rope_q[row * HALF + i] = v;
-        else if (row < n_slots + block_len) rope_t[(row - n_slots) * HALF + i] = v;
-        else if (row < n_slots + block_len + 32) rope_lo[(row - n_slots - block_len) * HALF + i] = v;
-        else {
-            float *h = reinterpret_cast<float *>(rope_hi + (row - n_slots - block_len - 32) * (HALF / 2) + i / 2);
-            h[i & 1] = v.x;
-            h[2 + (i & 1)] = v.y;
-        }
+        else rope_t[(row - n_slots) * HALF + i] = v;
     }
 }
 
@@ -135,44 +116,11 @@ __global__ void k_slot_fill(const int32_t *__restrict__ sel, int n_slots, int n_
     }
 }
 
-// Position of a selected slot: the caller's start position, or block id *
-// block_len.
-__device__ __forceinline__ int slot_pos(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int slot,
-                                        int block_len) {
-    return pos ? pos[slot] : sel[slot] * block_len;
-}
-
-// Tensor-core path: per block id, sort its slot list by (position, slot) in
-// place and count its work items: runs of equal position, up to `spi`
-// sessions each.  One thread per block id.
-__global__ void k_blk_items(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int n_b, int block_len,
-                            const int32_t *__restrict__ start, int32_t *__restrict__ list, int spi,
-                            int32_t *__restrict__ nitems) {
+// Tensor-core path: query passes of every block id, ceil(slots x G / pass_q).
+__global__ void k_pass_counts(const int32_t *__restrict__ start, int n_b, int G, int pass_q,
+                              int32_t *__restrict__ passes) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= n_b) return;
-    const int s0 = start[b], s1 = start[b + 1];
-    for (int i = s0 + 1; i < s1; ++i) {   // insertion sort by (position, slot)
-        const int x = list[i];
-        const int px = slot_pos(sel, pos, x, block_len);
-        int k = i - 1;
-        while (k >= s0) {
-            const int y = list[k];
-            const int py = slot_pos(sel, pos, y, block_len);
-            if (py < px || (py == px && y < x)) break;
-            list[k + 1] = y;
-            --k;
-        }
-        list[k + 1] = x;
-    }
-    int cnt = 0;
-    for (int i = s0; i < s1;) {
-        const int p = slot_pos(sel, pos, list[i], block_len);
-        int k = i;
-        while (k < s1 && slot_pos(sel, pos, list[k], block_len) == p) ++k;
-        cnt += (k - i + spi - 1) / spi;
-        i = k;
-    }
-    nitems[b] = cnt;
+    if (b < n_b) passes[b] = ((start[b + 1] - start[b]) * G + pass_q - 1) / pass_q;
 }
 
 // Exclusive prefix sum of n values (one CTA of 1024 threads): out[i] for i <=
@@ -207,36 +155,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) k_scan_counts(const int32_t *__r
         acc += in[b];
     }
     if (tid == SCAN_THREADS - 1) out[n] = wsum[31];
-}
-
-// Tensor-core path: the queries of every (layer, session, KV head) in fp16,
-// GQA heads padded to G8 = round_up(G, 8) with zeros, already in the tensor
-// cores' K-major operand layout [g/8][cg][g%8][8]: core-matrix column 2c holds
-// channels 8c .. 8c+7, column 2c+1 channels 64+8c .. 64+8c+7 (the order the
-// rotated keys are packed in).  One 16-byte chunk per thread.
-__global__ void k_q_pack(const float *__restrict__ q, int L, int S, int H, int G, int G8, __half *__restrict__ qp) {
-    const int64_t total = (int64_t)L * S * H * G8 * 16;
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int r = (int)(e & 7);
-        const int cg = (int)((e >> 3) & 15);
-        const int64_t rest = e >> 7;                  // (lsh, g / 8)
-        const int rg = (int)(rest % (G8 / 8));
-        const int64_t lsh = rest / (G8 / 8);
-        const int h = (int)(lsh % H);
-        const int64_t ls = lsh / H;                   // l * S + s
-        const int g = rg * 8 + r;
-        const int ch = (cg & 1) ? HALF + 8 * (cg >> 1) : 8 * (cg >> 1);
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (g < G) {
-            const float4 *src = reinterpret_cast<const float4 *>(q + (ls * (H * G) + h * G + g) * D + ch);
-            const float4 a = src[0], b = src[1];
-            const __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
-            const __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
-            out = make_uint4(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1),
-                             *reinterpret_cast<const uint32_t *>(&h2), *reinterpret_cast<const uint32_t *>(&h3));
-        }
-        *reinterpret_cast<uint4 *>(qp + lsh * (int64_t)G8 * D + rg * 1024 + cg * 64 + r * 8) = out;
-    }
 }
 
 constexpr int DS_QC = 16;   // queries per pass
@@ -414,8 +332,7 @@ __global__ void __launch_bounds__(128) k_combine(DecodeArgs a, const PT *__restr
         if (bid < 0 || bid >= a.n_b) continue;
         const float2 ml = a.part_ml[row * a.n_sel + u];
         const float w = __expf(ml.x - M) * ml.y;
-        const int64_t prow = a.pmap ? (int64_t)a.pmap[row * a.n_sel + u] : row * a.n_sel + u;
-        num = fmaf(w, part_elem(part_o, prow * D + j), num);
+        num = fmaf(w, part_elem(part_o, (row * a.n_sel + u) * D + j), num);
         den += w;
     }
     a.out[row * D + j] = den > 0.f ? num / den : 0.f;

@@ -568,31 +568,18 @@ static size_t shadow_bytes_per_kind(const milo_factors *f) {
                     (size_t)(round_up(f->shape.block_len, FTILE) + D));
 }
 
-// Partial outputs: fp32 rows (L, S, Hq, n_sel) of D for the CUDA-core path;
-// fp16 rows of D, G8 per selected slot and (layer, KV head), for the tensor
-// cores.  The region holds either.
-static size_t part_o_bytes(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
-    const int64_t slots = (int64_t)S * n_sel;
-    const size_t simt = sizeof(float) * (size_t)f->shape.L * S * Hq * n_sel * D;
-    const size_t tc = sizeof(__half) * (size_t)f->shape.L * f->shape.H * slots * decode_tc_g8(Hq / f->shape.H) * D;
-    return std::max(simt, tc);
-}
-
 size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
     if (!f || S <= 0 || Hq <= 0 || n_sel <= 0) return 0;
     const int64_t slots = (int64_t)S * n_sel;
     const int64_t rows = (int64_t)f->shape.L * S * Hq;
     size_t at = 0;
-    at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursors / item counts, slot starts, item starts, claim
+    at = align_up(at + sizeof(int32_t) * ((f->n_b + 1) * 3 + 1));      // counts / cursor / passes, starts, item starts, claim
     at = align_up(at + sizeof(int32_t) * slots);                       // slot list
-    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);  // rope tables
-    at = align_up(at + part_o_bytes(f, S, Hq, n_sel));                 // partial o
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);  // rope tables
+    at = align_up(at + sizeof(float) * rows * n_sel * D);              // partial o
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
-    at = align_up(at + sizeof(int32_t) * rows * n_sel);                // partial -> row of partial o (tensor cores)
-    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));  // tensor-core work items
-    at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H *
-                           decode_tc_g8(Hq / f->shape.H) * D);              // packed fp16 queries
-    at = align_up(at + sizeof(float4) * slots * 16 * (HALF / 2));      // per-slot rotation tables
+    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
+                                                            Hq / f->shape.H));  // tensor-core work items
     at += 2 * shadow_bytes_per_kind(f);                                 // INT8: fp16 factors
     return at;
 }
@@ -616,24 +603,18 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     size_t at = 0;
     int32_t *cnt = (int32_t *)(w + at);
     int32_t *start = cnt + (n_b + 1);
-    int32_t *istart = start + (n_b + 1);   // tensor-core work items of each block id, scanned
-    int32_t *claim = istart + (n_b + 1);   // next unclaimed tensor-core work item
+    int32_t *pstart = start + (n_b + 1);   // tensor-core work items of each block id, scanned
+    int32_t *claim = pstart + (n_b + 1);   // next unclaimed tensor-core work item
     at = align_up(at + sizeof(int32_t) * ((n_b + 1) * 3 + 1));
     int32_t *list = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * slots);
     float2 *rope_q = (float2 *)(w + at);
     float2 *rope_t = rope_q + slots * HALF;
-    float2 *rope_lo = rope_t + (int64_t)f->shape.block_len * HALF;
-    float4 *rope_hi = (float4 *)(rope_lo + 32 * HALF);
-    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len + 32 + 16) * HALF);
-    float *part_o = (float *)(w + at); at = align_up(at + part_o_bytes(f, S, Hq, n_sel));
+    at = align_up(at + sizeof(float2) * (slots + f->shape.block_len) * HALF);
+    float *part_o = (float *)(w + at); at = align_up(at + sizeof(float) * rows * n_sel * D);
     float2 *part_ml = (float2 *)(w + at); at = align_up(at + sizeof(float2) * rows * n_sel);
-    int32_t *pmap = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * rows * n_sel);
     DtItem *items = (DtItem *)(w + at);
-    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, slots));
-    __half *qpack = (__half *)(w + at);
-    at = align_up(at + sizeof(__half) * (size_t)f->shape.L * S * f->shape.H * decode_tc_g8(Hq / f->shape.H) * D);
-    float4 *rot_slot = (float4 *)(w + at);
-    at = align_up(at + sizeof(float4) * slots * 16 * (HALF / 2));
+    at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
+                                                            Hq / f->shape.H));
     __half *shadow0 = (__half *)(w + at);
     __half *shadow1 = (__half *)(w + at + shadow_bytes_per_kind(f));
 
@@ -645,14 +626,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     a.S = S; a.Hq = Hq; a.n_sel = n_sel;
     a.q = q; a.sel = selected; a.pos = positions;
     a.slot_start = start; a.slot_list = list;
-    a.rope_q = rope_q; a.rope_t = rope_t; a.rope_lo = rope_lo; a.rope_hi = rope_hi;
-    a.part_o = part_o; a.part_o16 = (__half *)part_o; a.part_ml = part_ml; a.out = out;
+    a.rope_q = rope_q; a.rope_t = rope_t;
+    a.part_o = part_o; a.part_ml = part_ml; a.out = out;
     a.claim = claim;
-    a.G8 = decode_tc_g8(a.G);
-    a.spi = decode_tc_spi(a.G);
-    a.qpack = qpack;
-    a.rot_slot = rot_slot;
-    a.pmap = nullptr;   // the CUDA-core path's partials are indexed directly
     a.f16 = 0;
     {   // a test-injected fault applies to this call only
         std::lock_guard<std::mutex> lk(g_inject_mu);
@@ -670,9 +646,9 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
     k_slot_count<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, cnt);
     k_slot_scan<<<1, SCAN_THREADS, 0, s>>>(cnt, start, n_b);
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
-    const int64_t rt = (slots + f->shape.block_len + 32 + 16) * HALF;
+    const int64_t rt = (slots + f->shape.block_len) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
-        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t, rope_lo, rope_hi);
+        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
     if (decode_tc_supported(a)) {
         if (a.factor_dtype == MILO_INT8) {   // dequantised to fp16 for the tensor cores
             k_dequant_selected<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, shadow0, shadow1);
@@ -680,35 +656,23 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
             a.kv[1].data = shadow1;
             a.f16 = 1;
         }
-        // items: each block's slots sorted by position (the fill order is not
-        // deterministic), cut into runs of equal position; item starts per block
-        k_blk_items<<<(n_b + 127) / 128, 128, 0, s>>>(selected, positions, n_b, f->shape.block_len, start, list,
-                                                     a.spi, cnt);
-        k_scan_counts<<<1, SCAN_THREADS, 0, s>>>(cnt, istart, n_b);
-        const int64_t qchunks = (int64_t)a.L * S * a.H * a.G8 * 16;
-        k_q_pack<<<(int)std::min<int64_t>((qchunks + 255) / 256, 8192), 256, 0, s>>>(q, a.L, S, a.H, a.G, a.G8,
-                                                                                     qpack);
-        const int64_t nrot = slots * 16 * (HALF / 2);
-        k_rot_slots<<<(int)std::min<int64_t>((nrot + 255) / 256, 8192), 256, 0, s>>>(rope_q, rope_hi, (int)slots,
-                                                                                    rot_slot);
+        // work items: passes of up to DT_NQ queries per block id (counts reuse cnt)
+        k_pass_counts<<<(n_b + 255) / 256, 256, 0, s>>>(start, n_b, a.G, DT_NQ, cnt);
+        k_scan_counts<<<1, SCAN_THREADS, 0, s>>>(cnt, pstart, n_b);
         tpush(MILO_TK_DECODE_PREP, t0, tmark(s));
         t0 = tmark(s);
-        a.pmap = pmap;
-        st = cuda_check(launch_decode_tc(a, istart, items, sm_count(), s), "decode (tensor cores) launch");
+        st = cuda_check(launch_decode_tc(a, pstart, items, sm_count(), s), "decode (tensor cores) launch");
         if (st != MILO_OK) return st;
         tpush(MILO_TK_DECODE, t0, tmark(s));
-        t0 = tmark(s);
-        k_combine<__half><<<(unsigned)rows, D, 0, s>>>(a, a.part_o16);
-        tpush(MILO_TK_COMBINE, t0, tmark(s));
     } else {
         tpush(MILO_TK_DECODE_PREP, t0, tmark(s));
         t0 = tmark(s);
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
         tpush(MILO_TK_DECODE, t0, tmark(s));
-        t0 = tmark(s);
-        k_combine<float><<<(unsigned)rows, D, 0, s>>>(a, a.part_o);
-        tpush(MILO_TK_COMBINE, t0, tmark(s));
     }
+    t0 = tmark(s);
+    k_combine<float><<<(unsigned)rows, D, 0, s>>>(a, a.part_o);
+    tpush(MILO_TK_COMBINE, t0, tmark(s));
     return cuda_check(cudaGetLastError(), "decode launch");
 }
 

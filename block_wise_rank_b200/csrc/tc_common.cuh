@@ -48,9 +48,9 @@ __device__ __forceinline__ uint64_t globaltimer() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the phase with this parity to complete.  Gives up after ~2 s of
-// wall time, raises ST_TIMEOUT and returns false, so that a broken pipeline
-// ends the kernel instead of hanging the GPU.
+// Wait for the phase with this parity to complete.  Gives up after limit_ns
+// of wall time (2 s by default), raises ST_TIMEOUT and returns false, so that
+// a broken pipeline ends the kernel instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -62,12 +62,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
     if (mbar_test_wait(bar, parity)) return true;   // already complete: no suspend round trip
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > 2000000000ull) {
+        if (globaltimer() - t0 > limit_ns) {
             raise_status(ST_TIMEOUT);
             return false;
         }
