@@ -504,13 +504,18 @@ constexpr int kMaxDevices = 64;
 void *g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device (looked up once
-// per device, with that device current); nullptr on failure.
-void *noalloc_scratch() {
+// Device address of the scratch array on the current device; nullptr on
+// failure.  Looked up again on every call made outside stream capture (a
+// context torn down by cudaDeviceReset and created anew may place the array
+// elsewhere); a call being captured into a graph reuses the address of the
+// last lookup on that device and looks it up only if there was none.
+void *noalloc_scratch(cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return nullptr;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_ptr[dev] || cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p) {
@@ -543,7 +548,7 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
     int64_t caps, floors;
     cap_sums(&shp, r_min, r_max, caps, floors);
     if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
-    void *scratch = noalloc_scratch();
+    void *scratch = noalloc_scratch((cudaStream_t)stream);
     if (!scratch) return MILO_ERR_CUDA;
     // the scratch layout for kNoAllocBlocks also holds any smaller problem
     AllocScratch as = alloc_scratch(scratch, kNoAllocBlocks);
