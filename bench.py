@@ -294,9 +294,10 @@ class Run:
         torch.cuda.synchronize()
         stages = milo.milo_timing_read()
         milo.milo_timing_enable(False)
-        rounds = milo.milo_jacobi_rounds()
+        rounds, rotations = milo.milo_jacobi_rounds()
         return dict(total_ms=t_begin.elapsed_time(t_end), comp_ms=sum(e[0].elapsed_time(e[1]) for e in evs),
                     dec_ms=sum(e[1].elapsed_time(e[2]) for e in evs), stages=stages, jacobi_rounds=rounds,
+                    jacobi_rotations=rotations,
                     status=milo.milo_get_status())
 
     def release(self):
@@ -341,6 +342,7 @@ def compression_roofline(run, t, steps, pk):
         flop = t["jacobi_rounds"] / steps * JACOBI_FLOP_PER_ROUND
         tfl = flop / sec / 1e12
         out["jacobi"] = dict(ms=round(ms / steps, 4), rounds_per_block=round(t["jacobi_rounds"] / steps / (2 * nblk), 1),
+                             rotations_per_round=round(t["jacobi_rotations"] / max(t["jacobi_rounds"], 1), 1),
                              tflops=round(tfl, 3), bound="alu", frac=round(tfl / pk["fp32"], 4),
                              peak=f"derived: {pk['sms']} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x "
                                   f"{pk['sm_mhz']:.0f} MHz = {pk['fp32']:.1f} TFLOP/s")

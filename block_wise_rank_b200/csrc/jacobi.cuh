@@ -87,7 +87,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
 
     bool converged = false;
     int sweeps_done = 0;
-    unsigned rounds_applied = 0;
+    unsigned rounds_applied = 0, rotations = 0;
     for (int sweep = 0; sweep < max_sweeps && !converged; ++sweep) {
         ++sweeps_done;
         int any = 0;
@@ -110,10 +110,12 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                 sm.p[tid] = p; sm.q[tid] = q;
                 sm.c[tid] = c; sm.s[tid] = s; sm.t[tid] = tn;
             }
-            rot = __syncthreads_or(rot);
+            const int nrot = __syncthreads_count(rot);   // rotating pairs of this round
+            rot = nrot > 0;
             any |= rot;
             if (!rot) continue;   // uniform across the CTA
             ++rounds_applied;
+            rotations += nrot;
             // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2 (upper triangle)
             for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
                 const int i = sm.tri[e][0], i2 = sm.tri[e][1];
@@ -164,7 +166,10 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
     }
     if (!converged && tid == 0) raise_status(ST_NOT_CONVERGED);
     MILO_TRACE_JACOBI(sweeps_done);
-    if (tid == 0) atomicAdd(&g_jacobi_rounds, (unsigned long long)rounds_applied);
+    if (tid == 0) {
+        atomicAdd(&g_jacobi_rounds, (unsigned long long)rounds_applied);
+        atomicAdd(&g_jacobi_rotations, (unsigned long long)rotations);
+    }
 
     // eigenvalues, stable descending order
     if (tid < D) sm.lam[tid] = sm.G[jac_g(tid, tid)];

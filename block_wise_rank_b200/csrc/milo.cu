@@ -810,15 +810,17 @@ milo_status milo_timing_read(double *ms, int64_t *count, int32_t n) {
     return st;
 }
 
-milo_status milo_jacobi_rounds(int64_t *rounds, milo_stream_t stream) {
-    if (!rounds) return MILO_ERR_INVALID_ARG;
+milo_status milo_jacobi_rounds(int64_t *rounds, int64_t *rotations, milo_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_check(e, "stream sync");
-    unsigned long long v = 0, zero = 0;
+    unsigned long long v = 0, w = 0, zero = 0;
     e = cudaMemcpyFromSymbol(&v, g_jacobi_rounds, sizeof(v));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&w, g_jacobi_rotations, sizeof(w));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_jacobi_rounds, &zero, sizeof(zero));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_jacobi_rotations, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_check(e, "counter read");
-    *rounds = (int64_t)v;
+    if (rounds) *rounds = (int64_t)v;
+    if (rotations) *rotations = (int64_t)w;
     return MILO_OK;
 }
 

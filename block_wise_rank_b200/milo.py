@@ -102,7 +102,7 @@ def lib():
         L.milo_test_decode_inject.restype = ctypes.c_int
         L.milo_timing_enable.argtypes = [I32]; L.milo_timing_enable.restype = ctypes.c_int
         L.milo_timing_read.argtypes = [P, P, I32]; L.milo_timing_read.restype = ctypes.c_int
-        L.milo_jacobi_rounds.argtypes = [P, P]; L.milo_jacobi_rounds.restype = ctypes.c_int
+        L.milo_jacobi_rounds.argtypes = [P, P, P]; L.milo_jacobi_rounds.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -333,12 +333,15 @@ def milo_timing_read() -> dict:
     return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(TIMED_STAGES)}
 
 
-def milo_jacobi_rounds(stream=None) -> int:
-    """Jacobi rounds that applied rotations since the last read (synchronises)."""
+def milo_jacobi_rounds(stream=None) -> tuple:
+    """(rounds that applied rotations, rotations applied) of the Jacobi
+    eigensolves since the last read (synchronises)."""
     v = ctypes.c_int64(0)
-    _check(lib().milo_jacobi_rounds(ctypes.cast(ctypes.byref(v), ctypes.c_void_p), _stream(stream)),
+    w = ctypes.c_int64(0)
+    _check(lib().milo_jacobi_rounds(ctypes.cast(ctypes.byref(v), ctypes.c_void_p),
+                                    ctypes.cast(ctypes.byref(w), ctypes.c_void_p), _stream(stream)),
            "milo_jacobi_rounds")
-    return int(v.value)
+    return int(v.value), int(w.value)
 
 
 def milo_version() -> str:

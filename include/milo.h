@@ -294,11 +294,12 @@ milo_status milo_timing_enable(int32_t on);
  * array; a CUDA error of the event queries is returned as MILO_ERR_CUDA. */
 milo_status milo_timing_read(double *ms, int64_t *count, int32_t n);
 
-/* Synchronise stream, then read and clear the count of Jacobi rounds that
- * applied rotations, summed over every (block, kind) eigensolve since the
- * last read (one round = the 64 disjoint plane rotations applied to the
- * d x d Gram tile and to W).  The eigensolve's work for its throughput. */
-milo_status milo_jacobi_rounds(int64_t *rounds, milo_stream_t stream);
+/* Synchronise stream, then read and clear the Jacobi work counters, summed
+ * over every (block, kind) eigensolve since the last read: *rounds = rounds
+ * that applied rotations (one round updates the d x d Gram tile and W for up
+ * to 64 disjoint plane rotations), *rotations = plane rotations applied.
+ * Either pointer may be NULL.  The eigensolve's work for its throughput. */
+milo_status milo_jacobi_rounds(int64_t *rounds, int64_t *rotations, milo_stream_t stream);
 
 /* ---------------------------------------------------------------- status */
 
