@@ -28,8 +28,6 @@ __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status
 // Jacobi rounds that applied rotations, summed over all (block, kind) solves
 // since the last read (work counter for the eigensolve's throughput).
 __device__ unsigned long long g_jacobi_rounds;
-// plane rotations applied in those rounds (at most 64 per round)
-__device__ unsigned long long g_jacobi_rotations;
 
 __host__ __device__ __forceinline__ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 

@@ -24,6 +24,9 @@
 
 namespace milo {
 
+// plane rotations applied in the counted rounds (at most 64 per round)
+__device__ unsigned long long g_jacobi_rotations;
+
 constexpr int JAC_THREADS = 512;
 constexpr int JAC_NPAIR = D / 2;                       // 64 pairs per round
 constexpr int JAC_NTRI = JAC_NPAIR * (JAC_NPAIR + 1) / 2;  // 2080 pair blocks (i <= i2)
