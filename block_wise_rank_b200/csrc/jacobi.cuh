@@ -45,8 +45,8 @@ __device__ __forceinline__ int jac_g(int x, int y) {
 struct JacobiSmem {
     float G[JAC_GT];
     float W[D * JAC_LD];
-    float c[JAC_NPAIR], s[JAC_NPAIR], t[JAC_NPAIR];
-    int p[JAC_NPAIR], q[JAC_NPAIR];
+    float4 rot[JAC_NPAIR];   // per pair of the round: (c, s, p, q), p and q as int bits
+    float t[JAC_NPAIR];
     unsigned short tri[JAC_NTRI][2];
     float lam[D];
     int rank[D];
@@ -110,8 +110,8 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                     s = c * tn;
                     rot = 1;
                 }
-                sm.p[tid] = p; sm.q[tid] = q;
-                sm.c[tid] = c; sm.s[tid] = s; sm.t[tid] = tn;
+                sm.rot[tid] = make_float4(c, s, __int_as_float(p), __int_as_float(q));
+                sm.t[tid] = tn;
             }
             const int nrot = __syncthreads_count(rot);   // rotating pairs of this round
             rot = nrot > 0;
@@ -122,8 +122,9 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
             // G <- J^T G J on every 2x2 pair block (i, i2), i <= i2 (upper triangle)
             for (int e = tid; e < JAC_NTRI; e += JAC_THREADS) {
                 const int i = sm.tri[e][0], i2 = sm.tri[e][1];
-                const int p = sm.p[i], q = sm.q[i];
-                const float c1 = sm.c[i], s1 = sm.s[i];
+                const float4 r1 = sm.rot[i];
+                const int p = __float_as_int(r1.z), q = __float_as_int(r1.w);
+                const float c1 = r1.x, s1 = r1.y;
                 if (i == i2) {
                     if (s1 != 0.f) {
                         const float tn = sm.t[i];
@@ -135,9 +136,10 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
                     }
                     continue;
                 }
-                const float c2 = sm.c[i2], s2 = sm.s[i2];
+                const float4 r2 = sm.rot[i2];
+                const float c2 = r2.x, s2 = r2.y;
                 if (s1 == 0.f && s2 == 0.f) continue;   // neither pair rotates: block unchanged
-                const int p2 = sm.p[i2], q2 = sm.q[i2];
+                const int p2 = __float_as_int(r2.z), q2 = __float_as_int(r2.w);
                 const int ia = jac_g(p, p2), ib = jac_g(p, q2), ic = jac_g(q, p2), ie = jac_g(q, q2);
                 const float a = sm.G[ia], bb = sm.G[ib];
                 const float cc = sm.G[ic], ee = sm.G[ie];
@@ -155,10 +157,11 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
             // consecutive rows of one pair (row stride 129: no bank conflicts)
             for (int e = tid; e < D * JAC_NPAIR; e += JAC_THREADS) {
                 const int j = e % D, i = e / D;
-                const float s1 = sm.s[i];
+                const float4 r1 = sm.rot[i];
+                const float s1 = r1.y;
                 if (s1 == 0.f) continue;
-                const float c1 = sm.c[i];
-                const int p = sm.p[i], q = sm.q[i];
+                const float c1 = r1.x;
+                const int p = __float_as_int(r1.z), q = __float_as_int(r1.w);
                 const float wp = sm.W[j * JAC_LD + p], wq = sm.W[j * JAC_LD + q];
                 sm.W[j * JAC_LD + p] = c1 * wp - s1 * wq;
                 sm.W[j * JAC_LD + q] = s1 * wp + c1 * wq;
