@@ -12,8 +12,10 @@
 // K-hat nor V-hat is written to memory.  Each (query, selected slot) gets a
 // partial (max, sum, unnormalised output) merged by k_combine.
 //
-// This kernel is the FP32 path: it serves f32 and int8 factors; the tensor
-// core kernel in decode_tc.cuh serves bf16 factors.
+// This kernel is the FP32 path: it serves f32 factors (and bf16 / INT8
+// factors of blocks longer than 512 tokens, or when MILO_FORCE_SIMT is set,
+// as the tests' cross-check); the tensor-core kernel in decode_tc.cuh serves
+// bf16 factors, and INT8 factors dequantised to fp16.
 #pragma once
 #include "common.cuh"
 
