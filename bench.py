@@ -595,6 +595,22 @@ def _worker(args):
         return _oracle_decode_loop(sample, seconds)
 
 
+def _all_cores(pool, ncores, sample, secs):
+    """The decode loop on every core at once: (bytes, queries, seconds)."""
+    parts = pool.map(_worker, [(sample, secs)] * ncores)
+    return sum(p[0] for p in parts), sum(p[1] for p in parts), max(p[2] for p in parts)
+
+
+def _baseline_record(w, factor, budget, sample, secs, one, allc, ncores):
+    return dict(value=allc["value"], unit=UNIT, cores=ncores, kind="oracle",
+                sample=f"1 (layer, KV head) of {w.name}: oracle SVD of the {len(sample['blocks'])} blocks "
+                       f"session 0 selects (K and V), eps, greedy top-R at {int(budget * 100)}%; then fp64 "
+                       f"decode of that KV head's {w.G} query heads over them, ~{secs:.0f} s per measurement; "
+                       f"bytes = the {factor} factor bytes each query reads",
+                single_thread=one, all_cores=allc, cpu_model=cpu_model(), nproc=ncores,
+                compress_blocks_per_s=round(sample["comp_blocks"] / sample["comp_s"], 3))
+
+
 def cpu_baseline(args, w, factor):
     """The fp64 oracle, as it stands, on this host: one thread, then every
     core (a spawned process per core running the same decode loop)."""
@@ -607,35 +623,38 @@ def cpu_baseline(args, w, factor):
         b1, n1, e1 = _oracle_decode_loop(sample, secs)
     ncores = os.cpu_count() or 1
     with mp.get_context("spawn").Pool(ncores) as pool:
-        parts = pool.map(_worker, [(sample, secs)] * ncores)
-    ball = sum(p[0] for p in parts)
-    eall = max(p[2] for p in parts)
+        ball, nall, eall = _all_cores(pool, ncores, sample, secs)
     one = dict(value=round(b1 / e1 / 1e9, 6), queries=n1, seconds=round(e1, 2))
-    allc = dict(value=round(ball / eall / 1e9, 6), queries=sum(p[1] for p in parts), seconds=round(eall, 2))
-    return dict(value=allc["value"], unit=UNIT, cores=ncores, kind="oracle",
-                sample=f"1 (layer, KV head) of {w.name}: oracle SVD of the {len(sample['blocks'])} blocks "
-                       f"session 0 selects (K and V), eps, greedy top-R at {int(args.budget * 100)}%; then fp64 "
-                       f"decode of that KV head's {w.G} query heads over them, ~{secs:.0f} s per variant; "
-                       f"bytes = the {factor} factor bytes each query reads",
-                single_thread=one, all_cores=allc, cpu_model=cpu_model(), nproc=ncores,
-                compress_blocks_per_s=round(sample["comp_blocks"] / sample["comp_s"], 3))
+    allc = dict(value=round(ball / eall / 1e9, 6), queries=nall, seconds=round(eall, 2))
+    return _baseline_record(w, factor, args.budget, sample, secs, one, allc, ncores)
 
 
 def run_reference(args):
     """The fp64 CPU oracle, as it stands, on a bounded sample of the workload
-    (this host's cores)."""
+    (this host's cores): the sample is compressed once, then each step is
+    ~6 s of decode on every core."""
+    import multiprocessing as mp
+
+    from threadpoolctl import threadpool_limits
     w = workload_of(args.workload, args.layers)
     factor = args.factor or ("f32" if w.dtype == "f32" else "bf16")
-    vals = []
-    cb = None
-    for i in range(args.warmup + args.steps):
-        a = argparse.Namespace(**vars(args))
-        a.cpu_sample_s = min(args.cpu_sample_s, 6.0)
-        cb = cpu_baseline(a, w, factor)
-        if i >= args.warmup:
-            vals.append(cb["value"])
+    sample = oracle_sample(w, args.budget, factor)
+    secs = min(args.cpu_sample_s, 6.0)
+    with threadpool_limits(1):
+        b1, n1, e1 = _oracle_decode_loop(sample, secs)
+    ncores = os.cpu_count() or 1
+    vals, nq, el = [], 0, 0.0
+    with mp.get_context("spawn").Pool(ncores) as pool:
+        for i in range(args.warmup + args.steps):
+            b, n, e = _all_cores(pool, ncores, sample, secs)
+            if i >= args.warmup:
+                vals.append(b / e / 1e9)
+                nq += n
+                el += e
     v = statistics.median(vals)
-    cb = dict(cb, value=round(v, 6))
+    one = dict(value=round(b1 / e1 / 1e9, 6), queries=n1, seconds=round(e1, 2))
+    allc = dict(value=round(v, 6), queries=nq, seconds=round(el, 2))
+    cb = _baseline_record(w, factor, args.budget, sample, secs, one, allc, ncores)
     return dict(impl="reference", metric=METRIC, value=round(v, 6), unit=UNIT, n_gpus=1, steps=args.steps,
                 warmup=args.warmup, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic",
