@@ -22,6 +22,8 @@ inputs), timing is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import bisect
+import ctypes
 import dataclasses
 import hashlib
 import json
@@ -77,6 +79,8 @@ def parse():
     ap.add_argument("--row-steps", type=int, default=2, help="timed steps per row (one warm-up step each)")
     ap.add_argument("--profile", action="store_true",
                     help="only the warm-up and timed steps (for ncu launch lists): no profiler, e2e or CPU legs")
+    ap.add_argument("--timeline", type=int, default=-1, metavar="CTA",
+                    help="decode timeline of one CTA of k_decode_tc from the tracing build; prints a summary, no JSON")
     return ap.parse_args()
 
 
@@ -414,6 +418,144 @@ def decode_traffic(w, factor, budget):
     return int((d["dram_bytes_read"] + d["dram_bytes_write"]) * w.L / d["layers"])
 
 
+# ------------------------------------------------------------------ timeline
+# k_decode_tc's warps: 0 producer, 1 MMA issuer, 2-9 RoPE, 10-17 softmax
+# (two groups of four), 18-19 helpers; the tracing build records lane 0 of each.
+TL_ROLE_WARPS = dict(producer=0, mma=1, rope=2, softmax0=10, softmax1=14, helper=18)
+
+
+def timeline_events():
+    """Event names in the order of k_decode_tc's TlEvent list (its values start at 1)."""
+    text = open(os.path.join(ROOT, "block_wise_rank_b200", "csrc", "decode_tc.cuh")).read()
+    body = re.search(r"enum TlEvent[^{]*\{(.*?)\};", text, flags=re.S).group(1)
+    return [m.group(1) for m in re.finditer(r"^\s*TL_(\w+)", body, flags=re.M)]
+
+
+def timeline_summary(rec, cnt, cta, skip=2):
+    """Per-item busy and wait times (median over the CTA's steady items, SM
+    cycles) of each role, from the tracing build's records."""
+    names = timeline_events()
+    ev = {}     # (warp, name, n, t) -> first clock
+    rets = []   # clocks of the MMA thread's returns from an issue
+    for wi in range(rec.shape[0]):
+        for r in rec[wi, :int(cnt[wi])]:
+            code = int(r["code"])
+            key = (wi, names[(code & 0xFF) - 1], int(r["n"]), code >> 8)
+            ev.setdefault(key, int(r["t"]))
+            if key[1] == "M_RET" and wi == TL_ROLE_WARPS["mma"]:
+                rets.append(int(r["t"]))
+    rets.sort()
+    W = TL_ROLE_WARPS
+
+    def at(role, name, n, t=0):
+        return ev.get((W[role], name, n, t))
+
+    items = sorted({k[2] for k in ev if k[0] == W["mma"] and k[1] == "M_REB" and k[3] == 0})
+    steady = items[skip:-skip - 1] if len(items) > 2 * skip + 2 else items[:-1]
+    rows = {}
+
+    def add(key, v):
+        if v is not None:
+            rows.setdefault(key, []).append(v)
+
+    for n in steady:
+        nt = 1 + max(k[3] for k in ev if k[0] == W["softmax0"] and k[1] == "S_END" and k[2] == n)
+        p0, p1 = at("mma", "M_REB", n), at("mma", "M_REB", n + 1)
+        add("item period (rebuild of tile 0 to the next item's)", p1 - p0)
+        for g in ("softmax0", "softmax1"):
+            busy = sum(at(g, "S_END", n, t) - at(g, "S_START", n, t) for t in range(nt))
+            wait = sum(at(g, "S_START", n, t) - at(g, "S_END", n, t - 1) for t in range(1, nt))
+            add(f"{g}: softmax of the {nt} tiles (busy)", busy)
+            ph = [("S_START", "S_LOADED", "load of the first slab from TMEM"),
+                  ("S_LOADED", "S_MADE", "first slab's p and the group's rare-path vote"),
+                  ("S_MADE", "S_PFREE", "wait for the P buffer (previous PV done)"),
+                  ("S_PFREE", "S_END", "P stores and the remaining slabs")]
+            for e0, e1, what in ph:
+                vals = [at(g, e1, n, t) - at(g, e0, n, t) for t in range(nt)
+                        if at(g, e1, n, t) is not None and at(g, e0, n, t) is not None]
+                if len(vals) == nt:
+                    add(f"{g}:   of which {what}", sum(vals))
+            add(f"{g}: waiting for the next tile's scores", wait)
+            add(f"{g}: after the last tile: O_A wait + denominators + staging",
+                at(g, "S_DONE", n) - at(g, "S_END", n, nt - 1))
+            prev = at(g, "S_DONE", n - 1)
+            if prev is not None:
+                add(f"{g}: item start to the first tile's scores", at(g, "S_START", n, 0) - prev)
+        for g, w0 in (("softmax0", 10), ("softmax1", 14)):
+            # the same first-slab load, slowest and fastest of the group's four warps
+            spans = []
+            for t in range(nt):
+                d = [ev.get((w, "S_LOADED", n, t), 0) - ev.get((w, "S_START", n, t), 0) for w in range(w0, w0 + 4)]
+                spans.append((max(d), min(d)))
+            add(f"{g}: first-slab load, slowest (fastest) warp, sum over tiles",
+                (sum(x[0] for x in spans), sum(x[1] for x in spans)))
+        add("rope: rotation of the tiles (busy)",
+            sum(at("rope", "R_END", n, t) - at("rope", "R_START", n, t) for t in range(nt)))
+        if at("rope", "R_OUT", n) is not None:
+            add("rope: read-out of the output (of which waiting for it)",
+                (at("rope", "R_OUT_END", n) - at("rope", "R_OUT", n), at("rope", "R_OUT_GOT", n) - at("rope", "R_OUT", n)))
+        mma = W["mma"]
+        iss = [(k, v) for k, v in ev.items() if k[0] == mma and k[2] == n and k[1] in ("M_REB", "M_SCO", "M_PV", "M_O")]
+        kind = {"M_REB": 0, "M_SCO": 1, "M_PV": 2, "M_O": 3}
+        busy = 0
+        for k, v in iss:
+            j = bisect.bisect_left(rets, v)
+            if j < len(rets):
+                busy += rets[j] - v
+        add(f"mma: issuing the item's {len(iss)} MMA groups (thread busy)", busy)
+        for t in range(1, nt):
+            free, issued = at("softmax0", "S_END", n, t - 1), at("mma", "M_SCO", n, t)
+            add("mma: softmax done -> next scores issued", issued - free)
+            add("mma: scores issued -> softmax sees them", at("softmax0", "S_START", n, t) - issued)
+        req = [(k[3], v) for k, v in ev.items() if k[0] == W["producer"] and k[1] == "P_REQ" and k[2] == n]
+        add("producer: waiting for ring space",
+            sum(at("producer", "P_PLACED", n, t) - v for t, v in req if at("producer", "P_PLACED", n, t) is not None))
+        if at("helper", "H_Q_START", n) is not None:
+            add("helper: query rotation of the item", at("helper", "H_Q_END", n) - at("helper", "H_Q_START", n))
+            last = at("softmax0", "S_END", n - 1, nt - 1) if n > 0 else None
+            if last is not None:
+                add("helper: queries ready minus previous item's last softmax", at("helper", "H_Q_END", n) - last)
+    out = [f"CTA {cta}: {len(items)} items, {len(steady)} steady items summarised (median, SM cycles)", "",
+           "| per item | cycles | share of period |", "|---|---|---|"]
+    per = statistics.median(rows["item period (rebuild of tile 0 to the next item's)"])
+    for k, vs in rows.items():
+        if isinstance(vs[0], tuple):
+            a, b = statistics.median(v[0] for v in vs), statistics.median(v[1] for v in vs)
+            out.append(f"| {k} | {a:.0f} ({b:.0f}) | {a / per:.2f} |")
+        else:
+            m = statistics.median(vs)
+            out.append(f"| {k} | {m:.0f} | {m / per:.2f} |")
+    return "\n".join(out)
+
+
+def run_timeline(args):
+    """Decode timeline of CTA args.timeline from the tracing build of the library."""
+    import numpy as np
+    from block_wise_rank_b200 import build
+    milo.LIB_PATH = build.build(trace=True)
+    L = milo.lib()
+    L.milo_timeline_select.argtypes = [ctypes.c_int32]
+    L.milo_timeline_read.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload_of(args.workload, args.layers)
+    factor = args.factor or ("f32" if w.dtype == "f32" else "bf16")
+    run = Run(w, args.budget, factor, dev, args.decode_steps)
+    for _ in range(max(args.warmup, 1)):
+        run.step()
+    torch.cuda.synchronize()
+    assert L.milo_timeline_select(args.timeline) == 0
+    run.step()
+    torch.cuda.synchronize()
+    rec = np.zeros((20, 4096), dtype=[("t", "<i8"), ("code", "<u4"), ("n", "<u4")])
+    cnt = np.zeros(20, dtype=np.uint32)
+    assert L.milo_timeline_read(rec.ctypes.data, cnt.ctypes.data) == 0
+    L.milo_timeline_select(-1)
+    print(f"workload {w.name}, {w.L} layers, budget {args.budget}, {factor} factors, "
+          f"status {milo.status_string(milo.milo_get_status())}")
+    print(timeline_summary(rec, cnt, args.timeline))
+
+
 # ------------------------------------------------------------------ the arm
 def run_e2e(run, steps, world, dev):
     """Decode GB/s with per-step H2D of q/ids/positions from pinned host
@@ -669,6 +811,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)))
+        return
+    if args.timeline >= 0:
+        if rank == 0:
+            run_timeline(args)
         return
     if world > 1:
         import datetime

@@ -11,6 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmilo.so")
+TRACE_LIB = os.path.join(PKG, "libmilo_trace.so")   # decode timeline build (-DMILO_DECODE_TRACE)
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -25,21 +26,24 @@ def sources():
                   [os.path.join(INCLUDE, "milo.h")])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra=(), trace: bool = False) -> str:
+    """Build libmilo.so (or, with `trace`, libmilo_trace.so: the same library
+    whose decode kernel records a per-warp timeline) if a source is newer."""
+    lib = TRACE_LIB if trace else LIB
     newest = max(os.path.getmtime(p) for p in sources())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not extra:
-        return LIB
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= newest and not extra:
+        return lib
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
-           os.path.join(CSRC, "milo.cu"), "-lcudart"]
+    tmp = lib + f".tmp{os.getpid()}"
+    flags = [*NVCC_FLAGS, *(["-DMILO_DECODE_TRACE"] if trace else []), *extra]
+    cmd = [nvcc, *flags, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "milo.cu"), "-lcudart"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv,
                 extra=["-Xptxas", "-v"] if "--ptxas" in sys.argv else []))

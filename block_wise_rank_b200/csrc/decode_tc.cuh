@@ -42,21 +42,47 @@
 #include "decode_simt.cuh"
 #include "tc_common.cuh"
 
-// Timeline hooks: empty unless a tracing build defines them.
-#ifndef MILO_TRACE_EVENT
-#define MILO_TRACE_EVENT(grp, id)
-#endif
-#ifndef MILO_TRACE_MMA
-#define MILO_TRACE_MMA(n, id)
-#endif
-#ifndef MILO_TRACE_WARP
-#define MILO_TRACE_WARP(id)
-#endif
-#ifndef MILO_TRACE_WAIT
-#define MILO_TRACE_WAIT(dist, reuse, overlap)
-#endif
-#ifndef MILO_TRACE_TILE
-#define MILO_TRACE_TILE(role, n, k)
+namespace milo {
+// Timeline events of k_decode_tc (argument: the CTA's item n and a tile or
+// ring position t).  Recorded only by the tracing build (decode_trace.cuh);
+// elsewhere the hooks compile to nothing.
+enum TlEvent : uint32_t {
+    TL_P_CLAIM = 1,    // producer: item claimed
+    TL_P_REQ,          // producer: ring position t wanted
+    TL_P_PLACED,       // producer: ring space for t found
+    TL_P_ISSUED,       // producer: copy of t issued (t = 31: B_K)
+    TL_M_REB,          // MMA thread: rebuild of tile t issued
+    TL_M_SCO,          // MMA thread: scores of tile t issued
+    TL_M_PV,           // MMA thread: PV of tile t issued
+    TL_M_O,            // MMA thread: output product issued
+    TL_M_RET,          // MMA thread: back from an issue (t = the kind: 0 rebuild, 1 scores, 2 PV, 3 O)
+    TL_R_START,        // RoPE: rebuilt keys of tile t in TMEM, rotation starts
+    TL_R_END,          // RoPE: rotated keys of tile t handed to the scores
+    TL_R_OUT,          // RoPE: read-out of item n's output starts
+    TL_R_OUT_GOT,      // RoPE: item n's output product complete
+    TL_R_OUT_END,      // RoPE: item n's output written
+    TL_S_START,        // softmax: scores of tile t in TMEM
+    TL_S_LOADED,       // softmax: first slab of tile t loaded from TMEM
+    TL_S_MADE,         // softmax: first slab's p made and the group agreed on the rare path
+    TL_S_PFREE,        // softmax: P buffer of tile t free
+    TL_S_RESCALE,      // softmax: rare path taken in tile t
+    TL_S_END,          // softmax: P of tile t handed over
+    TL_S_OA,           // softmax: O_A of item n complete
+    TL_S_DONE,         // softmax: item n's denominators and staging done
+    TL_H_CONV,         // helpers: ring position t converted / passed
+    TL_H_Q_START,      // helpers: queries of item n start
+    TL_H_Q_END,        // helpers: queries of item n staged
+};
+}  // namespace milo
+#ifdef MILO_DECODE_TRACE
+#include "decode_trace.cuh"
+#else
+#define MILO_TL_LOCALS
+#define MILO_TL(ev, n, t) \
+    do {                  \
+        (void)(n);        \
+        (void)(t);        \
+    } while (0)
 #endif
 
 
@@ -311,6 +337,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_items = (int64_t)a.L * a.H * pstart[a.n_b];
     const uint64_t lim = a.wait_ns;   // limit of every wait (ns of %globaltimer)
+    MILO_TL_LOCALS
     // Items are claimed dynamically: the producer takes the next unclaimed one
     // from a global counter and publishes it in the item table; every role
     // walks the same sequence n = 0, 1, ... of this CTA's items.  (The factor
@@ -374,10 +401,8 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // is the oldest tile not yet seen released.
         uint32_t head = 0, seq = 0, tail = 0;
         bool withheld = false;   // the first B_K copy never issued (tests of the bounded waits)
-        uint32_t trace_n = 0;
+        uint32_t trace_n = 0;   // item and ring position of the tile being placed (timeline only)
         int trace_k = 0;
-        (void)trace_n;
-        (void)trace_k;
         bool ok = true;
         // room for a tile of `bytes`: lane 0 releases tiles from the tail
         // (all older than the new tile, so all released without it) until the
@@ -392,7 +417,6 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     const bool room = t0 < head ? (off == head || off + bytes <= t0)
                                                 : (off >= head && off + bytes <= t0);
                     if (room && seq - tail < DT_NBAR) break;
-                    MILO_TRACE_WAIT(seq - tail, 0, 1);
                     if (!tc::mbar_wait(&sm.empty[tail % DT_NBAR], (tail / DT_NBAR) & 1u, lim)) { ok = false; break; }
                     ++tail;
                 }
@@ -418,7 +442,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         auto ring_tile = [&](const uint8_t *src, int rows, int copy, bool ones) {
             const uint32_t off = place((uint32_t)rows * 256u);
             if (!ok) return;
-            if (lane == 0) MILO_TRACE_TILE(3, trace_n, trace_k);
+            if (lane == 0) MILO_TL(TL_P_PLACED, trace_n, trace_k);
             uint8_t *dst = sm.ring + off;
             if (rows > copy) fill_rows(dst, copy, rows, ones);
             if (lane == 0) {
@@ -442,11 +466,16 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
             const int64_t i = __shfl_sync(0xffffffffu, claimed, 0);
             if (i < 0) break;
+            if (lane == 0) MILO_TL(TL_P_CLAIM, n, 0);
             const DtItem it = items[i];
             const DtGeo g = dt_geo(it.Tb, it.rK, it.rV, it.nq);
             const uint8_t *bK = dataK + 2 * it.offK, *bV = dataV + 2 * it.offV;
             const int64_t tileK = (int64_t)g.R8K * 256, tileV = (int64_t)g.R8V * 256;
+            trace_n = n;
+            trace_k = 0;
+            if (lane == 0) MILO_TL(TL_P_REQ, n, 0);
             ring_tile(bK, g.R16K, g.R8K, false);                               // A_K tile 0 (position 0)
+            if (lane == 0) MILO_TL(TL_P_ISSUED, n, 0);
             if (!ok) break;
             // B_K into its own buffer once the previous item's rebuilds are done
             if (lane == 0) ok = tc::mbar_wait(&sm.bk_empty, (n & 1u) ^ 1u, lim);
@@ -458,19 +487,18 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             } else if (lane == 0) {
                 tc::mbar_arrive_expect_tx(&sm.bk_full, (uint32_t)tileK);
                 if (tileK) tc::bulk_g2s(sm.bk, bK + g.nt * tileK, (uint32_t)tileK, &sm.bk_full);
-                MILO_TRACE_TILE(0, n, 15);
+                MILO_TL(TL_P_ISSUED, n, 31);
             }
-            MILO_TRACE_TILE(0, n, 0);
             for (int k = 1; k <= 2 * g.nt && ok; ++k) {
                 int t;
                 const int kind = dt_tile_at(g.nt, k, &t);
-                if (lane == 0) MILO_TRACE_TILE(2, n, k);
+                if (lane == 0) MILO_TL(TL_P_REQ, n, k);
                 trace_n = n;
                 trace_k = k;
                 if (kind == 0) ring_tile(bK + t * tileK, g.R16K, g.R8K, false);          // A_K(t)
                 else if (kind == 1) ring_tile(bV + t * tileV, g.rowsV, g.R8V, g.ones);   // A_V(t)
                 else ring_tile(bV + g.nt * tileV, g.R16V, g.R8V, false);                // B_V
-                if (lane == 0) MILO_TRACE_TILE(0, n, k);
+                if (lane == 0) MILO_TL(TL_P_ISSUED, n, k);
             }
         }
         if (!ok && lane == 0) sm.abort = 1;
@@ -525,7 +553,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     const uint32_t k = seqR + dt_pos_k(tR), s = k % DT_NBAR, b = rc & 1u;
                     if (mbar_test(&sm.full[s], (k / DT_NBAR) & 1u) && (tR > 0 || mbar_test(&sm.bk_full, nR & 1u)) &&
                         mbar_test(&sm.d1_empty[b], ((rc >> 1) & 1u) ^ 1u)) {
-                        MILO_TRACE_MMA(nR, tR);
+                        MILO_TL(TL_M_REB, nR, tR);
                         tc::tc_fence_after();
                         const uint32_t sa = sring + sm.toff[s];
                         for (int ks = 0; ks < gR.R16K / 16; ++ks)
@@ -535,6 +563,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         tc::mma_commit(&sm.d1_full[b]);
                         tc::mma_commit(&sm.empty[s]);
                         if ((int)tR == gR.nt - 1) tc::mma_commit(&sm.bk_empty);
+                        MILO_TL(TL_M_RET, nR, 0);
                         ++rc;
                         if ((int)++tR == gR.nt) {
                             seqR += dt_ring_tiles(gR);
@@ -553,7 +582,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     if (mbar_test(&sm.kt_full[b], (rcS >> 1) & 1u) && (tS > 0 || mbar_test(&sm.q_full, nS & 1u)) &&
                         mbar_test(&sm.d2_empty[d2b], (u2[d2b] & 1u) ^ 1u) &&
                         (gS.dbl || mbar_test(&sm.d2_empty[1], (u2[1] & 1u) ^ 1u))) {
-                        MILO_TRACE_MMA(nS, 4 + tS);
+                        MILO_TL(TL_M_SCO, nS, tS);
                         tc::tc_fence_after();
                         const uint32_t id_sc = tc::idesc_f16(128, gS.nq16, 0, 0, 0);   // fp16, A tmem, B K-major
                         const uint32_t kt = tmem + DT_COL_D1 + 128 * b;
@@ -567,6 +596,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         tc::mma_commit(&sm.d2_full[d2b]);
                         tc::mma_commit(&sm.d1_empty[b]);
                         if ((int)tS == gS.nt - 1) tc::mma_commit(&sm.q_empty);
+                        MILO_TL(TL_M_RET, nS, 1);
                         u2.inc(d2b);
                         ++rcS;
                         if ((int)++tS == gS.nt) {
@@ -588,7 +618,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         (tP > 0 || mbar_test(&sm.oa_free, (nP & 1u) ^ 1u))) {
                         tc::tc_fence_after();
                         if ((int)tP < gP.nt) {   // O_A^T += A_V(tile)^T P
-                            MILO_TRACE_MMA(nP, 8 + tP);
+                            MILO_TL(TL_M_PV, nP, tP);
                             const uint32_t k = kv, s = k % DT_NBAR;
                             const uint32_t sa = sring + sm.toff[s];
                             const uint32_t id_pv = tc::idesc_f16(128, gP.nq16, 0, 0, 1);   // fp16, A K-major, B MN-major
@@ -599,10 +629,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             tc::mma_commit(&sm.p_empty[pb]);
                             tc::mma_commit(&sm.empty[s]);
                             if ((int)tP == gP.nt - 1) tc::mma_commit(&sm.oa_full);
+                            MILO_TL(TL_M_RET, nP, 2);
                             pu.inc(pb);
                             ++tP;
                         } else {                 // O = B_V^T (O_A / l), over O_A's columns
-                            MILO_TRACE_MMA(nP, 12);
+                            MILO_TL(TL_M_O, nP, tP);
                             const uint32_t k = kv, s = k % DT_NBAR;
                             const uint32_t sa = sring + sm.toff[s];
                             const uint32_t id_o = tc::idesc_f16(128, gP.nq16, 0, 1, 1);    // fp16, A/B MN-major
@@ -613,6 +644,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                             tc::mma_commit(&sm.p_empty[pb]);
                             tc::mma_commit(&sm.empty[s]);
                             tc::mma_commit(&sm.o_full);
+                            MILO_TL(TL_M_RET, nP, 3);
                             pu.inc(pb);
                             seqP += dt_ring_tiles(gP);
                             tP = 0;
@@ -656,7 +688,9 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         int pend_nq = -1;   // queries of the item whose O is still to be read, or -1
         uint32_t pend_n = 0;
         auto readout = [&]() -> bool {
+            MILO_TL(TL_R_OUT, pend_n, 0);
             if (!grp_and<DT_BAR_R, DT_RGROUP>(tc::mbar_wait(&sm.o_full, pend_n & 1u, lim) && !sm.abort)) return false;
+            MILO_TL(TL_R_OUT_GOT, pend_n, 0);
             tc::tc_fence_after();
             const int *qp = sm.qpidx[pend_n & 3u];
             const int nq = pend_nq, nq16 = (nq + 15) & ~15;
@@ -672,6 +706,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.oa_free);
+            MILO_TL(TL_R_OUT_END, pend_n, 0);
             pend_nq = -1;
             return true;
         };
@@ -685,7 +720,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 const uint32_t b = rc & 1u;
                 ok = grp_and<DT_BAR_R, DT_RGROUP>(tc::mbar_wait(&sm.d1_full[b], (rc >> 1) & 1u, lim) && !sm.abort);
                 if (!ok) break;
-                MILO_TRACE_EVENT(0, 2 * t);
+                MILO_TL(TL_R_START, n, t);
                 tc::tc_fence_after();
                 const uint32_t base = tmem + DT_COL_D1 + 128 * b + lane_off;
                 const int tok = t * FTILE + row;   // in-block token of this lane
@@ -730,7 +765,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 tc::tc_fence_before();
                 tc::mbar_arrive(&sm.kt_full[b]);
                 ++rc;
-                MILO_TRACE_EVENT(0, 2 * t + 1);
+                MILO_TL(TL_R_END, n, t);
                 // the previous item's output, once this item's first two tiles
                 // are rotated (the softmax group has work queued meanwhile)
                 if (t == min(1, nt - 1) && pend_nq >= 0 && !(ok = readout())) break;
@@ -749,7 +784,6 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // groups only meet at the counted arrivals.
         const int sg = (warp - DT_W_S) >> 2;
         const int gt = threadIdx.x - 32 * DT_W_S - DT_GROUP * sg;   // thread within the group
-        const int et = gt + DT_GROUP * sg;                 // trace hooks: thread 0 of group 0
         const int bar_id = sg == 0 ? DT_BAR_S : DT_BAR_S2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;                  // TMEM lane of this thread
@@ -778,7 +812,6 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             const int nq = g.nq, nq16 = g.nq16;
             const uint32_t lbo_p = (uint32_t)(nq16 / 8) * 128u;
             int pv_issued = 0;
-            MILO_TRACE_EVENT(1, 0);
 
             // ---- P tile tt to the PV product (its A_V tile is converted by the helpers)
             auto handoff = [&](int tt) {
@@ -870,7 +903,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                 const uint32_t dcol = tmem + DT_COL_D2 + 64 * d2b + lane_off;
                 if (!grp_and_rt(bar_id, tc::mbar_wait(&sm.d2_full[d2b], u2[d2b] & 1u, lim))) return false;
                 u2.inc(d2b);
-                MILO_TRACE_EVENT(1, 2 + 2 * t);
+                MILO_TL(TL_S_START, n, t);
                 tc::tc_fence_after();
                 const int tok = t * FTILE + row;
                 const bool valid = tok < Tb;
@@ -909,7 +942,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
                     if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
                     tc::tmem_wait_ld();
-                    if (c0 == 0) MILO_TRACE_EVENT(1, 17 + 8 * t);
+                    if (c0 == 32 * sg) MILO_TL(TL_S_LOADED, n, t);
                     auto make_p = [&](float &pmax) {
                         const float2 *c2 = reinterpret_cast<const float2 *>(sm.cref + c0);
 #pragma unroll
@@ -928,9 +961,9 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     float pmax = 0.f;
                     make_p(pmax);
                     const bool any_over = grp_or_rt(bar_id, !(pmax <= 256.f));
-                    if (c0 == 0) MILO_TRACE_EVENT(1, 18 + 8 * t);
+                    if (c0 == 32 * sg) MILO_TL(TL_S_MADE, n, t);
                     if (any_over) {
-                        MILO_TRACE_EVENT(1, 23 + 8 * t);
+                        MILO_TL(TL_S_RESCALE, n, t);
                         if (!rescale(c0, w, dcol, lim)) return false;
                         tc::tmem_ld16(dcol + c0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
                         if (w == 32) tc::tmem_ld16(dcol + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
@@ -941,7 +974,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                     if (!p_ready) {
                         if (!drain()) return false;
                         p_ready = true;
-                        MILO_TRACE_EVENT(1, 19 + 8 * t);
+                        MILO_TL(TL_S_PFREE, n, t);
                     }
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -953,14 +986,13 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(q8[4], q8[5], q8[6], q8[7]);
                         if (!g.ones) colsum(q8, ch);
                     }
-                    if (c0 == 0) MILO_TRACE_EVENT(1, 20 + 8 * t);
                 }
                 // every score of the tile this thread needed has been read
                 tc::tc_fence_before();
                 tc::mbar_arrive(&sm.d2_empty[d2b]);
                 // a group without slabs keeps the same drain sequence
                 if (!p_ready && !drain()) return false;
-                MILO_TRACE_EVENT(1, 3 + 2 * t);
+                MILO_TL(TL_S_END, n, t);
                 return true;
             };
 
@@ -974,7 +1006,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             // group's columns); the last product and its read-out are the RoPE group's
             ok = grp_and_rt(bar_id, tc::mbar_wait(&sm.oa_full, n & 1u, lim));
             if (!ok) break;
-            MILO_TRACE_EVENT(1, 12);
+            MILO_TL(TL_S_OA, n, 0);
             tc::tc_fence_after();
             if (g.ones && quad == (g.R8V >> 5)) {   // the ones row holds sum_t p
                 for (int c0 = 32 * sg; c0 < nq16; c0 += 64)
@@ -1029,7 +1061,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             // one group-wide decision per item (also orders this item's reads of
             // cref / lsum before the next item's writes)
             ok = grp_and_rt(bar_id, !sm.abort);
-            MILO_TRACE_EVENT(1, 14);
+            MILO_TL(TL_S_DONE, n, 0);
         }
         if (!ok) sm.abort = 1;
     } else {
@@ -1040,6 +1072,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
         // four threads per query, 16 pairs each
         auto qprep = [&](int64_t j, uint32_t nj) -> bool {
             if (!grp_and<DT_BAR_H, DT_HELP>(tc::mbar_wait(&sm.q_empty, (nj & 1u) ^ 1u, lim))) return false;
+            MILO_TL(TL_H_Q_START, nj, 0);
             const int nq = __ldg(&items[j].nq), nq16 = (nq + 15) & ~15;
             const int jl = __ldg(&items[j].l), jh = __ldg(&items[j].h), jq0 = __ldg(&items[j].q0);
             const int jslot0 = __ldg(&items[j].slot0);
@@ -1124,7 +1157,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
                         grp_sync<DT_BAR_H, DT_HELP>();
                     }
                     if (et == 0) tc::mbar_arrive(&sm.conv[s]);
-                    if (et == 0) MILO_TRACE_TILE(1, nc, kc);
+                    MILO_TL(TL_H_CONV, nc, kc);
                     if (++kc == dt_ring_tiles(gc)) {
                         seqC += dt_ring_tiles(gc);
                         kc = 0;
@@ -1136,7 +1169,7 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
             }
             if (iq >= 0 && grp_and<DT_BAR_H, DT_HELP>(mbar_test(&sm.q_empty, (nqp & 1u) ^ 1u))) {
                 ok = qprep(iq, nqp);
-                if (et == 0) MILO_TRACE_TILE(1, nqp, 14);
+                MILO_TL(TL_H_Q_END, nqp, 0);
                 ++nqp;
                 iq = kPend;
                 did = true;

@@ -839,4 +839,24 @@ milo_status milo_get_status(milo_stream_t stream) {
     return MILO_OK;
 }
 
+#ifdef MILO_DECODE_TRACE
+// Tracing build only (not part of milo.h): pick the CTA of k_decode_tc whose
+// warps record the timeline, clearing earlier records (cta < 0: none), and
+// copy the records out: TL_WARPS x TL_CAP TlRec rows and TL_WARPS counts.
+static_assert(TL_WARPS * 32 == DT_THREADS, "one timeline row per decode warp");
+milo_status milo_timeline_select(int32_t cta) {
+    static uint32_t zeros[TL_WARPS];
+    cudaError_t e = cudaMemcpyToSymbol(g_tl_cnt, zeros, sizeof(zeros));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tl_cta, &cta, sizeof(cta));
+    return e == cudaSuccess ? MILO_OK : cuda_check(e, "timeline select");
+}
+milo_status milo_timeline_read(void *records, uint32_t *counts) {
+    if (!records || !counts) return MILO_ERR_INVALID_ARG;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(records, g_tl, sizeof(g_tl));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(counts, g_tl_cnt, sizeof(g_tl_cnt));
+    return e == cudaSuccess ? MILO_OK : cuda_check(e, "timeline read");
+}
+#endif
+
 }  // extern "C"

@@ -107,3 +107,51 @@ def test_oracle_sample_uses_the_greedy_allocation():
     assert sum(s["facs"][blk][1][0].shape[1] for blk in s["blocks"]) == R
     nbytes, n, el = b._oracle_decode_loop(s, 0.0)
     assert n == 1 and nbytes == s["bytes_per_query"] > 0
+
+
+def test_timeline_summary_on_planted_records():
+    """The decode timeline summary reads the tracing build's records: planted
+    per-warp events of ten items (four tiles each) give back the planted
+    period, busy and wait figures, and the event names follow the kernel's
+    TlEvent list."""
+    import numpy as np
+
+    b = _bench()
+    names = b.timeline_events()
+    assert names[0] == "P_CLAIM" and "S_END" in names and "H_Q_END" in names
+    code = {nm: i + 1 for i, nm in enumerate(names)}
+    rec = np.zeros((20, 4096), dtype=[("t", "<i8"), ("code", "<u4"), ("n", "<u4")])
+    cnt = np.zeros(20, np.uint32)
+
+    def put(w, nm, n, t, clk):
+        rec[w, cnt[w]] = (clk, code[nm] | (t << 8), n)
+        cnt[w] += 1
+
+    for n in range(10):
+        base = n * 10000
+        for t in range(4):
+            put(1, "M_REB", n, t, base + 100 + 2000 * t)
+            put(1, "M_RET", n, 0, base + 150 + 2000 * t)
+            put(1, "M_SCO", n, t, base + 600 + 2000 * t)
+            put(1, "M_RET", n, 1, base + 650 + 2000 * t)
+            put(2, "R_START", n, t, base + 200 + 2000 * t)
+            put(2, "R_END", n, t, base + 500 + 2000 * t)
+            for w in range(10, 18):
+                put(w, "S_START", n, t, base + 700 + 2000 * t)
+                put(w, "S_END", n, t, base + 1700 + 2000 * t)
+            put(1, "M_PV", n, t, base + 1800 + 2000 * t)
+            put(1, "M_RET", n, 2, base + 1850 + 2000 * t)
+        for w in (10, 14):
+            put(w, "S_OA", n, 0, base + 8000)
+            put(w, "S_DONE", n, 0, base + 8500)
+        put(1, "M_O", n, 4, base + 8600)
+        put(1, "M_RET", n, 3, base + 8650)
+    text = b.timeline_summary(rec, cnt, 5)
+    rows = {line.split(" | ")[0].strip("| "): line.split(" | ")[1] for line in text.splitlines() if line.startswith("| ")}
+    assert rows["item period (rebuild of tile 0 to the next item's)"] == "10000"
+    assert rows["softmax0: softmax of the 4 tiles (busy)"] == "4000"
+    assert rows["softmax0: waiting for the next tile's scores"] == "3000"
+    assert rows["softmax0: after the last tile: O_A wait + denominators + staging"] == "800"
+    assert rows["rope: rotation of the tiles (busy)"] == "1200"
+    assert rows["mma: issuing the item's 13 MMA groups (thread busy)"] == "650"
+    assert rows["mma: softmax done -> next scores issued"] == "900"
