@@ -272,7 +272,7 @@ def compress(K, V, block_len: int, budget_frac: float = 0.5, budget_abs: int = 0
     return out
 
 
-def decode_one(AK, BK, AV, BV, q, blocks, positions, rope_base: float):
+def decode_one(AK, BK, AV, BV, q, blocks, positions, rope_base: float, k_tail=None, v_tail=None):
     """Attention output of one query vector (post-RoPE, length d).
 
     AK/BK/AV/BV: callables or nested lookups giving, for a block id, the
@@ -280,6 +280,14 @@ def decode_one(AK, BK, AV, BV, q, blocks, positions, rope_base: float):
     blocks/positions: the selected block ids and their start positions.
     Keys are rebuilt (A B), rotated to absolute positions p + t, values are
     rebuilt, and dense softmax attention runs over all their tokens.
+
+    k_tail/v_tail (n x d, optional): the recent tokens that follow the
+    compressed demonstrations -- the question and the tokens generated so
+    far -- which stay uncompressed (evolve.pub review, Summary and FAQ "What
+    is MILO": the compressed cache holds the demonstrations; a query rebuilds
+    the blocks it retrieves and attends sparsely).  Reading: they join the
+    same softmax as the rebuilt tokens, their keys taken as given (already
+    rotated to their positions, like q).
     """
     keys_, vals = [], []
     for b, p in zip(blocks, positions):
@@ -289,6 +297,12 @@ def decode_one(AK, BK, AV, BV, q, blocks, positions, rope_base: float):
             kh[t] = rope(kh[t], p + t, rope_base)
         keys_.append(kh)
         vals.append(vh)
-    Kc = np.concatenate(keys_, axis=0)
-    Vc = np.concatenate(vals, axis=0)
+    if k_tail is not None and len(k_tail) > 0:
+        keys_.append(np.asarray(k_tail, dtype=np.float64))
+        vals.append(np.asarray(v_tail, dtype=np.float64))
+    d = len(q)
+    Kc = np.concatenate(keys_, axis=0) if keys_ else np.zeros((0, d))
+    Vc = np.concatenate(vals, axis=0) if vals else np.zeros((0, d))
+    if Kc.shape[0] == 0:
+        return np.zeros(d)
     return attention(np.asarray(q, dtype=np.float64)[None, :], Kc, Vc)[0]

@@ -361,6 +361,41 @@ def test_decode_invariances(oracle_mod):
     assert np.allclose(o_zero, AV[0].mean(axis=0) @ BV[0], atol=1e-14)
 
 
+def test_decode_recent_tail(oracle_mod):
+    """Recent uncompressed tokens join the blocks' softmax: checked against
+    scipy's softmax over the union of the rebuilt (rotated) block tokens and
+    the tail as given, against the tail alone, and by moving a block's rebuilt
+    tokens from the selection into the tail."""
+    rng = np.random.default_rng(23)
+    T, d, bl, base = 128, 16, 64, 1e4
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    AK, BK = _full_rank_factors(oracle_mod, K, bl)
+    AV, BV = _full_rank_factors(oracle_mod, V, bl)
+    f = (lambda b: AK[b], lambda b: BK[b], lambda b: AV[b], lambda b: BV[b])
+    q = rng.standard_normal(d) * 2
+    Kt = rng.standard_normal((19, d)) * 1.5   # tail keys, already rotated
+    Vt = rng.standard_normal((19, d))
+    Kr = np.stack([oracle_mod.rope(K[t], t, base) for t in range(T)])
+    out = oracle_mod.decode_one(*f, q, [0, 1], [0, bl], base, k_tail=Kt, v_tail=Vt)
+    ref = scipy.special.softmax(np.r_[Kr, Kt] @ q / math.sqrt(d)) @ np.r_[V, Vt]
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+    # the tail alone
+    out_t = oracle_mod.decode_one(*f, q, [], [], base, k_tail=Kt, v_tail=Vt)
+    ref_t = scipy.special.softmax(Kt @ q / math.sqrt(d)) @ Vt
+    assert np.abs(out_t - ref_t).max() <= 1e-13 * np.abs(ref_t).max()
+    # block 1's rebuilt, rotated tokens given as the tail instead of selected
+    kb1 = oracle_mod.reconstruct(AK[1], BK[1])
+    kb1 = np.stack([oracle_mod.rope(kb1[t], bl + t, base) for t in range(bl)])
+    vb1 = oracle_mod.reconstruct(AV[1], BV[1])
+    moved = oracle_mod.decode_one(*f, q, [0], [0], base, k_tail=kb1, v_tail=vb1)
+    both = oracle_mod.decode_one(*f, q, [0, 1], [0, bl], base)
+    assert np.abs(moved - both).max() <= 1e-13 * np.abs(both).max()
+    # an empty tail changes nothing
+    empty = oracle_mod.decode_one(*f, q, [0, 1], [0, bl], base, k_tail=np.zeros((0, d)), v_tail=np.zeros((0, d)))
+    assert np.array_equal(empty, both)
+
+
 def test_compress_end_to_end_small(oracle_mod):
     from block_wise_rank_b200 import synth
     import torch
