@@ -58,8 +58,8 @@ TRAFFIC_JSON = os.path.join("profiles", "decode_tc_traffic.json")
 DECODE_SOURCES = ("block_wise_rank_b200/csrc/decode_tc.cuh", "block_wise_rank_b200/csrc/tc_common.cuh",
                   "block_wise_rank_b200/csrc/common.cuh")
 # the other rows: (workload, rank budget, factor dtype)
-ROWS = [("qwen7b-128k", 0.25, "bf16"), ("qwen7b-128k", 0.75, "bf16"), ("qwen7b-128k", 0.5, "int8"),
-        ("qwen7b-64k", 0.5, "bf16"), ("qwen3b-32k", 0.5, "bf16")]
+ROWS = [("qwen7b-128k", 0.25, "bf16", 0), ("qwen7b-128k", 0.75, "bf16", 0), ("qwen7b-128k", 0.5, "int8", 0),
+        ("qwen7b-128k", 0.5, "bf16", 512), ("qwen7b-64k", 0.5, "bf16", 0), ("qwen3b-32k", 0.5, "bf16", 0)]
 
 
 def parse():
@@ -242,8 +242,8 @@ class Run:
     """One workload at one budget and factor type on one GPU: the synthetic
     cache, the compressed factors, the decode inputs, and a step."""
 
-    def __init__(self, w, budget, factor, dev, n_dec=0):
-        self.w, self.budget, self.factor, self.dev = w, budget, factor, dev
+    def __init__(self, w, budget, factor, dev, n_dec=0, tail=0):
+        self.w, self.budget, self.factor, self.dev, self.tail = w, budget, factor, dev, tail
         self.params = milo.default_params(factor_dtype=factor, budget_frac=budget)
         gen_dtype = torch.float64 if w.T * w.L * w.H <= 1 << 16 else torch.float32
         self.K, self.V = synth.workload_cache(w, device=dev, gen_dtype=gen_dtype)
@@ -256,8 +256,10 @@ class Run:
         # per-step decode inputs (different seeded queries / selections per decode step)
         self.dec_inputs = [synth.decode_inputs(w, step=i, device=dev) for i in range(self.n_dec)]
         self.f = milo.milo_compress(self.K, self.V, w.block_len, self.params, workspace=self.ws, arena=self.arena)
-        self.dws = torch.empty(milo.milo_decode_workspace_size(self.f, w.sessions, w.Hq, w.n_sel),
-                               dtype=torch.uint8, device=dev)
+        wsz = (milo.milo_decode_tail_workspace_size if tail else milo.milo_decode_workspace_size)
+        self.dws = torch.empty(wsz(self.f, w.sessions, w.Hq, w.n_sel), dtype=torch.uint8, device=dev)
+        # recent uncompressed tokens of every session, in the cache's element type
+        self.kt, self.vt, self.tl = synth.recent_tail(w, tail, dev, self.K.dtype) if tail else (None, None, None)
         self.out = torch.empty(w.L, w.sessions, w.Hq, w.d, dtype=torch.float32, device=dev)
 
     def step(self, ev=None):
@@ -269,14 +271,23 @@ class Run:
         if ev:
             ev[1].record(self.stream)
         for (q, sel, pos) in self.dec_inputs:
-            milo.milo_decode_attn(self.f, q, sel, pos, rope_base=w.rope_base, out=self.out, workspace=self.dws)
+            if self.tail:
+                milo.milo_decode_attn_tail(self.f, q, sel, self.kt, self.vt, self.tl, pos, rope_base=w.rope_base,
+                                           out=self.out, workspace=self.dws)
+            else:
+                milo.milo_decode_attn(self.f, q, sel, pos, rope_base=w.rope_base, out=self.out, workspace=self.dws)
         if ev:
             ev[2].record(self.stream)
+
+    def tail_bytes(self):
+        """K and V bytes of the recent tokens read per decode step."""
+        return 2 * self.kt.numel() * self.kt.element_size() if self.tail else 0
 
     def decode_bytes(self):
         ranks = read_ranks(self.f)
         w = self.w
-        return sum(decode_bytes(ranks, w, sel, self.factor, w.sessions, w.Hq) for (_, sel, _) in self.dec_inputs)
+        return sum(decode_bytes(ranks, w, sel, self.factor, w.sessions, w.Hq) + self.tail_bytes()
+                   for (_, sel, _) in self.dec_inputs)
 
     def timed(self, steps, warmup):
         """Warm-up, then `steps` timed steps with the library's per-stage
@@ -306,7 +317,7 @@ class Run:
 
     def release(self):
         self.f.close()
-        for name in ("K", "V", "ws", "arena", "dws", "out", "dec_inputs"):
+        for name in ("K", "V", "ws", "arena", "dws", "out", "dec_inputs", "kt", "vt", "tl"):
             setattr(self, name, None)
         torch.cuda.empty_cache()
 
@@ -376,9 +387,16 @@ def row_of(run, t, steps, pk):
     kgbs = (dbytes / run.n_dec) / (kms / kn / 1e3) / 1e9 if kn else None
     stages, dom = compression_roofline(run, t, steps, pk)
     nblk = 2 * w.L * w.H * w.n_b
+    tail = None
+    if run.tail:
+        tms, tn = stage_ms(t, "tail")
+        tgbs = run.tail_bytes() / (tms / tn / 1e3) / 1e9 if tn else None
+        tail = dict(tokens_per_session=run.tail, bytes_per_decode_step=run.tail_bytes(),
+                    kernel_gbs=round(tgbs, 2) if tgbs else None,
+                    kernel_frac_hbm=round(tgbs / pk["hbm"], 4) if tgbs else None)
     return dict(workload=w.name, layers=w.L, kv_heads=w.H, gqa=w.G, tokens=w.T, block_len=w.block_len,
                 sessions=w.sessions, selected=f"{w.n_sel}/{w.n_b}", decode_steps=run.n_dec,
-                budget=run.budget, factor=run.factor,
+                budget=run.budget, factor=run.factor, recent_tail=tail,
                 decode=dict(gbs=round(gbs, 2), frac_hbm=round(gbs / pk["hbm"], 4),
                             kernel_gbs=round(kgbs, 2) if kgbs else None,
                             kernel_frac_hbm=round(kgbs / pk["hbm"], 4) if kgbs else None,
@@ -652,10 +670,10 @@ def run_ours(args, rank, world):
     if world == 1 and not args.no_rows:
         rows = [row_of(run, t, args.steps, pk)]
         run.release()
-        for (name, budget, fac) in ROWS:
-            if name == w.name and budget == args.budget and fac == factor:
+        for (name, budget, fac, tail) in ROWS:
+            if name == w.name and budget == args.budget and fac == factor and tail == 0:
                 continue
-            r = Run(workload_of(name), budget, fac, dev)
+            r = Run(workload_of(name), budget, fac, dev, tail=tail)
             tr = r.timed(args.row_steps, 1)
             rows.append(row_of(r, tr, args.row_steps, pk))
             r.release()

@@ -39,6 +39,8 @@ struct DecodeArgs {
     uint64_t wait_ns;          // tensor-core path: limit of every wait on the device
     int inject;                // tensor-core path: 1 = withhold one copy (tests of the bounded waits)
     int f16;                   // tensor-core path: kv[].data holds fp16 factors (INT8 dequantised), else bf16
+    const float *tail_o;       // [L][S][Hq][D] partial of the recent uncompressed tokens, or null
+    const float2 *tail_ml;     // [L][S][Hq] its (max, sum), or null
 };
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
@@ -308,7 +310,8 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
 
 // out[l][s][hq] = sum_j w_j l_j o_j / sum_j w_j l_j, w_j = exp(m_j - max m),
 // with o_j the normalised output of slot j (fp32 from the CUDA-core path,
-// fp16 from the tensor-core path).
+// fp16 from the tensor-core path), and the recent-token partial as one more
+// term when there is one (an empty tail has sum 0 and adds nothing).
 // grid (L * S * Hq), 128 threads.  Slots with an out-of-range block id
 // contribute nothing.
 template <typename PT> __device__ __forceinline__ float part_elem(const PT *p, int64_t i);
@@ -328,7 +331,17 @@ __global__ void __launch_bounds__(128) k_combine(DecodeArgs a, const PT *__restr
         if (bid < 0 || bid >= a.n_b) continue;
         M = fmaxf(M, a.part_ml[row * a.n_sel + u].x);
     }
+    float2 tml = make_float2(-INFINITY, 0.f);
+    if (a.tail_ml) {
+        tml = a.tail_ml[row];
+        if (tml.y > 0.f) M = fmaxf(M, tml.x);
+    }
     float num = 0.f, den = 0.f;
+    if (tml.y > 0.f) {
+        const float w = __expf(tml.x - M) * tml.y;
+        num = w * a.tail_o[row * D + j];
+        den = w;
+    }
     for (int u = 0; u < a.n_sel; ++u) {
         const int bid = a.sel[(int64_t)s * a.n_sel + u];
         if (bid < 0 || bid >= a.n_b) continue;

@@ -26,6 +26,7 @@
 #include "project_simt.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "decode_tail.cuh"
 
 using namespace milo;
 
@@ -589,15 +590,32 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     return at;
 }
 
-milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
-                             const int32_t *selected, const int32_t *positions, int32_t n_sel, double rope_base,
-                             float *out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// the recent uncompressed tokens of a decode call (k == nullptr: none)
+struct TailIn {
+    const void *k = nullptr, *v = nullptr;
+    milo_dtype dtype = MILO_F32;
+    int32_t cap = 0;
+    const int32_t *len = nullptr;
+};
+
+size_t tail_workspace_bytes(const milo_factors *f, int32_t S, int32_t Hq) {
+    const int64_t rows = (int64_t)f->shape.L * S * Hq;
+    return align_up(sizeof(float) * rows * D) + align_up(sizeof(float2) * rows);
+}
+
+milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_t Hq, const int32_t *selected,
+                        const int32_t *positions, int32_t n_sel, double rope_base, const TailIn &tail, float *out,
+                        void *workspace, size_t ws_bytes, milo_stream_t stream) {
     if (!f || !q || !selected || !out || !workspace || S <= 0 || Hq <= 0 || n_sel <= 0)
         return MILO_ERR_INVALID_ARG;
     if (Hq % f->shape.H != 0 || !(rope_base > 0.0)) return MILO_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, kAlign) || !aligned(selected, 4))
         return MILO_ERR_INVALID_ARG;
-    if (ws_bytes < milo_decode_workspace_size(f, S, Hq, n_sel)) return MILO_ERR_WORKSPACE;
+    const size_t ws_dec = milo_decode_workspace_size(f, S, Hq, n_sel);
+    if (ws_bytes < ws_dec + (tail.k ? tail_workspace_bytes(f, S, Hq) : 0)) return MILO_ERR_WORKSPACE;
     milo_status st = set_smem_attrs();
     if (st != MILO_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
@@ -675,10 +693,58 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
         k_decode_simt<<<dim3(n_b, f->shape.H, f->shape.L), 256, sizeof(DecodeSimtSmem), s>>>(a);
         tpush(MILO_TK_DECODE, t0, tmark(s));
     }
+    if (tail.k) {   // the recent tokens' partial, then merged with the blocks'
+        float *tail_o = (float *)(w + ws_dec);
+        float2 *tail_ml = (float2 *)(w + ws_dec + align_up(sizeof(float) * rows * D));
+        t0 = tmark(s);
+        const dim3 grid((unsigned)f->shape.H, (unsigned)S, (unsigned)f->shape.L);
+        if (tail.dtype == MILO_BF16)
+            k_tail_attn<__nv_bfloat16><<<grid, D, 0, s>>>(a, (const __nv_bfloat16 *)tail.k,
+                                                          (const __nv_bfloat16 *)tail.v, tail.cap, tail.len,
+                                                          tail_o, tail_ml);
+        else
+            k_tail_attn<float><<<grid, D, 0, s>>>(a, (const float *)tail.k, (const float *)tail.v, tail.cap,
+                                                  tail.len, tail_o, tail_ml);
+        tpush(MILO_TK_TAIL, t0, tmark(s));
+        a.tail_o = tail_o;
+        a.tail_ml = tail_ml;
+    }
     t0 = tmark(s);
     k_combine<float><<<(unsigned)rows, D, 0, s>>>(a, a.part_o);
     tpush(MILO_TK_COMBINE, t0, tmark(s));
     return cuda_check(cudaGetLastError(), "decode launch");
+}
+}  // namespace
+
+extern "C" {
+
+milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                             const int32_t *selected, const int32_t *positions, int32_t n_sel, double rope_base,
+                             float *out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
+    return decode_impl(f, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_bytes,
+                       stream);
+}
+
+size_t milo_decode_tail_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    const size_t base = milo_decode_workspace_size(f, S, Hq, n_sel);
+    return base ? base + tail_workspace_bytes(f, S, Hq) : 0;
+}
+
+milo_status milo_decode_attn_tail(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                  const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                  double rope_base, const void *k_tail, const void *v_tail, milo_dtype tail_dtype,
+                                  int32_t tail_cap, const int32_t *tail_len, float *out, void *workspace,
+                                  size_t ws_bytes, milo_stream_t stream) {
+    if (!k_tail || !v_tail || !tail_len || tail_cap < 0) return MILO_ERR_INVALID_ARG;
+    if (tail_dtype != MILO_F32 && tail_dtype != MILO_BF16) return MILO_ERR_UNSUPPORTED;
+    if (!aligned(k_tail, 4) || !aligned(v_tail, 4) || !aligned(tail_len, 4)) return MILO_ERR_INVALID_ARG;
+    TailIn t;
+    t.k = k_tail;
+    t.v = v_tail;
+    t.dtype = tail_dtype;
+    t.cap = tail_cap;
+    t.len = tail_len;
+    return decode_impl(f, q, S, Hq, selected, positions, n_sel, rope_base, t, out, workspace, ws_bytes, stream);
 }
 
 milo_status milo_factors_get(const milo_factors *f, int32_t kind, int32_t **ranks, int64_t **offsets,

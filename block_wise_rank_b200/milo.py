@@ -54,11 +54,11 @@ EXPORTS = [
     "milo_decode_attn", "milo_factors_get", "milo_factors_wrap", "milo_factors_export",
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
     "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
-    "milo_jacobi_rounds",
+    "milo_jacobi_rounds", "milo_decode_tail_workspace_size", "milo_decode_attn_tail",
 ]
 
 # stages of milo_timing_read, in order (milo_timed_stage)
-TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine"]
+TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine", "tail"]
 
 MILO_NOALLOC_MAX_BLOCKS = 65536
 
@@ -85,6 +85,11 @@ def lib():
         L.milo_allocate_noalloc.restype = ctypes.c_int
         L.milo_decode_workspace_size.argtypes = [P, I32, I32, I32]; L.milo_decode_workspace_size.restype = SZ
         L.milo_decode_attn.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
+        L.milo_decode_tail_workspace_size.argtypes = [P, I32, I32, I32]
+        L.milo_decode_tail_workspace_size.restype = SZ
+        L.milo_decode_attn_tail.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, I32, I32, P, P, P,
+                                            SZ, P]
+        L.milo_decode_attn_tail.restype = ctypes.c_int
         L.milo_decode_attn.restype = ctypes.c_int
         L.milo_factors_get.argtypes = [P, I32, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
                                        ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
@@ -276,6 +281,39 @@ def milo_decode_attn(f: Factors, q: torch.Tensor, selected: torch.Tensor, positi
     s = lib().milo_decode_attn(f.handle, _ptr(q), S, Hq, _ptr(selected), _ptr(positions), n_sel, float(rope_base),
                                _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(s, "milo_decode_attn")
+    return out
+
+
+def milo_decode_tail_workspace_size(f: Factors, S: int, Hq: int, n_sel: int) -> int:
+    return lib().milo_decode_tail_workspace_size(f.handle, S, Hq, n_sel)
+
+
+def milo_decode_attn_tail(f: Factors, q: torch.Tensor, selected: torch.Tensor, k_tail: torch.Tensor,
+                          v_tail: torch.Tensor, tail_len: torch.Tensor, positions=None, rope_base=1e6, out=None,
+                          workspace=None, stream=None):
+    """Decode attention over the selected compressed blocks and each session's
+    recent uncompressed tokens: k_tail / v_tail [L][S][H][tail_cap][d] (fp32 or
+    bf16, keys already rotated), tail_len int32 [S]."""
+    assert q.dtype == torch.float32 and q.is_contiguous() and q.is_cuda
+    L, S, Hq, d = q.shape
+    n_sel = selected.shape[1]
+    assert selected.dtype == torch.int32 and selected.shape[0] == S and selected.is_contiguous()
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.shape == selected.shape and positions.is_contiguous()
+    assert k_tail.dtype == v_tail.dtype and k_tail.dtype in (torch.float32, torch.bfloat16)
+    assert k_tail.shape == v_tail.shape and k_tail.dim() == 5 and k_tail.shape[:2] == (L, S) and k_tail.shape[4] == d
+    assert k_tail.shape[2] == f.shape.H
+    assert k_tail.is_contiguous() and v_tail.is_contiguous()
+    assert tail_len.dtype == torch.int32 and tail_len.shape == (S,) and tail_len.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = _bytes(milo_decode_tail_workspace_size(f, S, Hq, n_sel), q.device)
+    dt = MILO_BF16 if k_tail.dtype == torch.bfloat16 else MILO_F32
+    s = lib().milo_decode_attn_tail(f.handle, _ptr(q), S, Hq, _ptr(selected), _ptr(positions), n_sel,
+                                    float(rope_base), _ptr(k_tail), _ptr(v_tail), dt, k_tail.shape[3],
+                                    _ptr(tail_len), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(s, "milo_decode_attn_tail")
     return out
 
 

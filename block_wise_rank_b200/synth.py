@@ -182,3 +182,17 @@ def decode_inputs(w: Workload, step: int = 0, device="cpu"):
     sel = retrieval_standin(w.n_b, w.sessions, w.n_sel, w.seed * 1000 + 200 + step, device)
     pos = (sel.to(torch.int64) * w.block_len).to(torch.int32)
     return q, sel, pos
+
+
+def recent_tail(w: Workload, n_tail: int, device="cpu", dtype=torch.float32):
+    """Recent uncompressed tokens of every session (the question and the
+    tokens generated so far): keys and values [L][S][H][n_tail][d] ~ N(0, 1)
+    in the cache's element type, every session's tail n_tail tokens long.
+    Returns (k_tail, v_tail, tail_len int32 [S])."""
+    g = _gen(w.seed * 1000 + 300 + n_tail, "cpu")
+    shape = (w.L, w.sessions, w.H, n_tail, w.d)
+    k = torch.randn(*shape, generator=g, dtype=torch.float32).to(dtype).to(device)
+    v = torch.randn(*shape, generator=g, dtype=torch.float32).to(dtype).to(device)
+    n = torch.full((w.sessions,), n_tail, dtype=torch.int32, device=device)
+    return k, v, n
+

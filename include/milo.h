@@ -224,6 +224,37 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
                              double rope_base, float *out, void *workspace, size_t ws_bytes,
                              milo_stream_t stream);
 
+/* Bytes of scratch milo_decode_attn_tail needs (milo_decode_workspace_size
+ * plus one partial per query row). */
+size_t milo_decode_tail_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel);
+
+/*
+ * milo_decode_attn plus each session's recent, uncompressed tokens in the
+ * same softmax: a complete decode step.  "MILO ... Block-wise Low-rank
+ * Compression" (evolve.pub review), Summary and FAQ "What is MILO": the
+ * compressed cache holds the many-shot demonstrations, a query rebuilds the
+ * blocks it retrieves and attends sparsely; the tokens that follow the
+ * demonstrations (the question, the tokens generated so far) stay
+ * uncompressed and are attended densely.  For (l, s, hq) the output is
+ * softmax over the selected blocks' tokens (as in milo_decode_attn) and the
+ * tail tokens i < tail_len[s] with s_i = q . k_tail[l][s][hq / G][i] / sqrt(d),
+ * times v_tail[l][s][hq / G][i].
+ *   k_tail, v_tail: device, [L][S][H][tail_cap][d] of tail_dtype (MILO_F32 or
+ *             MILO_BF16; else MILO_ERR_UNSUPPORTED); keys already rotated to
+ *             their own positions (as a model caches them), values plain
+ *   tail_len: device, int32 [S], 0 <= tail_len[s] <= tail_cap; a length
+ *             outside that range sets MILO_ERR_BOUNDS in the status word and
+ *             counts as an empty tail
+ * Other arguments, errors and the workspace rule as milo_decode_attn, with
+ * ws_bytes >= milo_decode_tail_workspace_size.  An empty tail for every
+ * session gives milo_decode_attn's output bit for bit.
+ */
+milo_status milo_decode_attn_tail(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                  const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                  double rope_base, const void *k_tail, const void *v_tail, milo_dtype tail_dtype,
+                                  int32_t tail_cap, const int32_t *tail_len, float *out, void *workspace,
+                                  size_t ws_bytes, milo_stream_t stream);
+
 /* ------------------------------------------------------ factor handles */
 
 /* Views (device pointers into the arena) of one kind (0 = K, 1 = V).  Any
@@ -280,7 +311,8 @@ typedef enum {
     MILO_TK_DECODE_PREP = 5, /* decode index, table and query-packing kernels */
     MILO_TK_DECODE = 6,      /* decode attention (k_decode_tc or k_decode_simt) */
     MILO_TK_COMBINE = 7,     /* merge of the per-block partials (k_combine) */
-    MILO_TK_COUNT = 8
+    MILO_TK_TAIL = 8,        /* attention over the recent uncompressed tokens (k_tail_attn) */
+    MILO_TK_COUNT = 9
 } milo_timed_stage;
 
 /* on != 0: start recording (previous records are dropped); on == 0: stop.

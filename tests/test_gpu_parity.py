@@ -438,3 +438,55 @@ def test_decode_bounded_wait_runs_out(oracle_mod):
             ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // G, 2, q[0, s, hq].double().cpu().numpy(), blocks,
                               [b * bl for b in blocks], 1e6)
             assert _rel_inf(out[0, s, hq], ref) <= DEC_TOL
+
+
+@pytest.mark.parametrize("factor,tail_dtype", [("bf16", torch.bfloat16), ("f32", torch.float32)])
+def test_decode_recent_tail(oracle_mod, factor, tail_dtype):
+    """milo_decode_attn_tail: the selected blocks plus each session's recent
+    uncompressed tokens in one softmax.  Ragged tails (0, 1, 33, 64, 70 = the
+    capacity, 5 tokens), bf16 factors (tensor-core decode) and f32 factors
+    (CUDA-core decode), fp32 and bf16 tails.  Checked against the oracle on
+    the same factors and the same tail values; an all-empty tail gives
+    milo_decode_attn's output bit for bit; a length past the capacity sets
+    MILO_ERR_BOUNDS and counts as empty."""
+    L, H, G, T, bl, S, cap = 2, 2, 4, 1000, 512, 6, 70
+    K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=61, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=62, out_dtype=torch.bfloat16)
+    if factor == "f32":
+        K, V = K.float(), V.float()
+    f = milo.milo_compress(K.cuda(), V.cuda(), bl, milo.default_params(factor_dtype=factor, budget_frac=0.5))
+    g = torch.Generator().manual_seed(63)
+    q = torch.randn(L, S, H * G, 128, generator=g)
+    sel = torch.stack([torch.randperm(2, generator=g) for _ in range(S)]).to(torch.int32)
+    pos = torch.randint(0, 120000, (S, 2), generator=g, dtype=torch.int32)
+    kt = (torch.randn(L, S, H, cap, 128, generator=g) * 1.5).to(tail_dtype)
+    vt = (torch.randn(L, S, H, cap, 128, generator=g) * 40.0).to(tail_dtype)
+    tl = torch.tensor([0, 1, 33, 70, 64, 5], dtype=torch.int32)
+    qd, seld, posd, ktd, vtd = q.cuda(), sel.cuda(), pos.cuda(), kt.cuda(), vt.cuda()
+    out = milo.milo_decode_attn_tail(f, qd, seld, ktd, vtd, tl.cuda(), posd, rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    U = [A.unpack(f, 0), A.unpack(f, 1)]
+    for u in U:
+        u["H"] = H
+    ktn, vtn = kt.double().numpy(), vt.double().numpy()
+    for s in range(S):
+        for (l, hq) in [(0, 0), (1, 5), (0, 7), (1, 2)]:
+            n, h = int(tl[s]), hq // G
+            ref = oracle_mod.decode_one(
+                lambda b: U[0]["A"][(l * H + h) * 2 + b], lambda b: U[0]["B"][(l * H + h) * 2 + b],
+                lambda b: U[1]["A"][(l * H + h) * 2 + b], lambda b: U[1]["B"][(l * H + h) * 2 + b],
+                q[l, s, hq].double().numpy(), sel[s].tolist(), pos[s].tolist(), 1e6,
+                k_tail=ktn[l, s, h, :n], v_tail=vtn[l, s, h, :n])
+            assert _rel_inf(out[l, s, hq], ref) <= DEC_TOL, (s, l, hq, _rel_inf(out[l, s, hq], ref))
+    # every tail empty: the blocks-only call, bit for bit
+    base = milo.milo_decode_attn(f, qd, seld, posd, rope_base=1e6).cpu().numpy()
+    zero = milo.milo_decode_attn_tail(f, qd, seld, ktd, vtd, torch.zeros(S, dtype=torch.int32).cuda(), posd,
+                                      rope_base=1e6).cpu().numpy()
+    assert np.array_equal(zero, base)
+    # a length past the capacity: status bounds, that session as if empty
+    bad = tl.clone()
+    bad[2] = cap + 1
+    o_bad = milo.milo_decode_attn_tail(f, qd, seld, ktd, vtd, bad.cuda(), posd, rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_ERR_BOUNDS
+    assert np.array_equal(o_bad[:, 2], base[:, 2])
+    assert np.array_equal(o_bad[:, 3], out[:, 3])
