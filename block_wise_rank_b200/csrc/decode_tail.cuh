@@ -22,36 +22,65 @@
 
 namespace milo {
 
-constexpr int TAIL_CHUNK = 32;   // tail tokens staged per round
-constexpr int TAIL_GSUB = 16;    // query heads of one KV head per pass over the tail
+constexpr int TAIL_CHUNK = 32;   // tail tokens per round
+constexpr int TAIL_GSUB = 8;     // query heads of one KV head per pass over the tail (static smem < 48 KB)
 
-struct TailSmem {
+struct alignas(16) TailSmem {
     float q[TAIL_GSUB][D];
-    float k[TAIL_CHUNK][D + 1];   // padded rows: thread-per-token reads are conflict-free
+    float k[TAIL_CHUNK][D + 4];              // padded rows: 16-byte reads of 32 different rows are conflict-free
     float v[TAIL_CHUNK][D];
     float p[TAIL_GSUB][TAIL_CHUNK];
+    float part[4][TAIL_GSUB][TAIL_CHUNK];    // score partials of the four quarters of d
     float m[TAIL_GSUB], l[TAIL_GSUB], f[TAIL_GSUB];
 };
 
-template <typename T> __device__ __forceinline__ float tail_elem(const T *p, int64_t i);
-template <> __device__ __forceinline__ float tail_elem<float>(const float *p, int64_t i) { return __ldg(p + i); }
-template <> __device__ __forceinline__ float tail_elem<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-    return __bfloat162float(p[i]);
-}
+// one 16-byte vector of tail elements as fp32
+template <typename T> struct TailVec;
+template <> struct TailVec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void get(uint4 u, float (&x)[4]) {
+        x[0] = __uint_as_float(u.x);
+        x[1] = __uint_as_float(u.y);
+        x[2] = __uint_as_float(u.z);
+        x[3] = __uint_as_float(u.w);
+    }
+};
+template <> struct TailVec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void get(uint4 u, float (&x)[8]) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+            x[2 * i] = t.x;
+            x[2 * i + 1] = t.y;
+        }
+    }
+};
 
-// grid (H, S, L), 128 threads (thread j = output channel j).
-//   k_tail, v_tail: [L][S][H][tail_cap][D]; tail_len[S] tokens of each session
-//   are live (a length outside [0, tail_cap] raises ST_BOUNDS and counts as 0).
+// grid (H, S, L), 128 threads.
+//   k_tail, v_tail: [L][S][H][tail_cap][D], 16-byte aligned; tail_len[S] tokens
+//   of each session are live (a length outside [0, tail_cap] raises ST_BOUNDS
+//   and counts as 0).
 //   tail_o: [L][S][Hq][D] normalised outputs; tail_ml: [L][S][Hq] (max score,
 //   sum of exp(score - max)); an empty tail leaves (-inf, 0) and zeros.
+// Each round loads a 32-token chunk of K and V as 16-byte vectors, all issued
+// before the first is used, and stages both in shared memory as fp32; thread
+// j then accumulates output channel j of every query head.
 template <typename T>
 __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__restrict__ k_tail,
                                                    const T *__restrict__ v_tail, int tail_cap,
                                                    const int32_t *__restrict__ tail_len, float *__restrict__ tail_o,
                                                    float2 *__restrict__ tail_ml) {
+    constexpr int EPV = TailVec<T>::N;                 // elements per vector
+    constexpr int VPR = D / EPV;                       // vectors per row
+    constexpr int NV = TAIL_CHUNK * VPR / 128;         // vectors per thread and array (rows per thread)
+    constexpr int NGRP = 128 / VPR;                    // threads loading the same channels of different rows
+    static_assert(NV * NGRP == TAIL_CHUNK, "row groups");
     __shared__ TailSmem sm;
     const int h = blockIdx.x, s = blockIdx.y, l = blockIdx.z;
     const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    const int cgrp = j % VPR, rgrp = j / VPR;          // channels [EPV cgrp, +EPV), rows rgrp + NGRP i
     int n = tail_len[s];
     if (n < 0 || n > tail_cap) {
         if (j == 0 && h == 0 && l == 0) raise_status(ST_BOUNDS);
@@ -72,30 +101,62 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
         for (int g = 0; g < TAIL_GSUB; ++g) acc[g] = 0.f;
         for (int c0 = 0; c0 < n; c0 += TAIL_CHUNK) {
             const int cn = min(TAIL_CHUNK, n - c0);
-            __syncthreads();   // previous round's k, v, p and f fully used; q, m, l written
-#pragma unroll 8
-            for (int t = 0; t < TAIL_CHUNK; ++t) {
-                const bool live = t < cn;
-                const int64_t e = (kv0 + c0 + t) * D + j;
-                sm.k[t][j] = live ? tail_elem(k_tail, e) : 0.f;
-                sm.v[t][j] = live ? tail_elem(v_tail, e) : 0.f;
+            uint4 kr[NV], vr[NV];
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int r = rgrp + NGRP * i;
+                kr[i] = vr[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (r < cn) {
+                    const int64_t row = (kv0 + c0 + r) * D;
+                    kr[i] = __ldg(reinterpret_cast<const uint4 *>(k_tail + row) + cgrp);
+                    vr[i] = __ldg(reinterpret_cast<const uint4 *>(v_tail + row) + cgrp);
+                }
+            }
+            __syncthreads();   // previous round's k, p and f used; q, m, l written
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                float x[EPV], y[EPV];
+                TailVec<T>::get(kr[i], x);
+                TailVec<T>::get(vr[i], y);
+                float4 *dk = reinterpret_cast<float4 *>(&sm.k[rgrp + NGRP * i][cgrp * EPV]);
+                float4 *dv = reinterpret_cast<float4 *>(&sm.v[rgrp + NGRP * i][cgrp * EPV]);
+#pragma unroll
+                for (int e = 0; e < EPV / 4; ++e) {
+                    dk[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                    dv[e] = make_float4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3]);
+                }
             }
             __syncthreads();
-            // scores: pair (g, t) = (u / 32, u % 32), one lane per token
+            // scores: warp w dots dims [32w, 32w + 32) of key t = lane with every
+            // query head (each key element read once, q broadcast), then the four
+            // quarters are added per (query head, token)
+            {
+                float sp[TAIL_GSUB];
+#pragma unroll
+                for (int g = 0; g < TAIL_GSUB; ++g) sp[g] = 0.f;
+                const float4 *kt = reinterpret_cast<const float4 *>(sm.k[lane]) + 8 * warp;
+#pragma unroll
+                for (int d4 = 0; d4 < 8; ++d4) {
+                    const float4 b4 = kt[d4];
+#pragma unroll
+                    for (int g = 0; g < TAIL_GSUB; ++g) {
+                        if (g >= gn) break;
+                        const float4 a4 = reinterpret_cast<const float4 *>(sm.q[g])[8 * warp + d4];
+                        sp[g] = fmaf(a4.w, b4.w, fmaf(a4.z, b4.z, fmaf(a4.y, b4.y, fmaf(a4.x, b4.x, sp[g]))));
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < TAIL_GSUB; ++g)
+                    if (g < gn) sm.part[warp][g][lane] = sp[g];
+            }
+            __syncthreads();
             for (int u = j; u < gn * TAIL_CHUNK; u += blockDim.x) {
                 const int g = u / TAIL_CHUNK, t = u % TAIL_CHUNK;
-                float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;   // four chains for the FMA latency
-#pragma unroll 4
-                for (int dd = 0; dd < D; dd += 4) {
-                    x0 = fmaf(sm.q[g][dd], sm.k[t][dd], x0);
-                    x1 = fmaf(sm.q[g][dd + 1], sm.k[t][dd + 1], x1);
-                    x2 = fmaf(sm.q[g][dd + 2], sm.k[t][dd + 2], x2);
-                    x3 = fmaf(sm.q[g][dd + 3], sm.k[t][dd + 3], x3);
-                }
-                sm.p[g][t] = t < cn ? ((x0 + x1) + (x2 + x3)) * scale : -INFINITY;
+                const float x = (sm.part[0][g][t] + sm.part[1][g][t]) + (sm.part[2][g][t] + sm.part[3][g][t]);
+                sm.p[g][t] = t < cn ? x * scale : -INFINITY;
             }
             __syncthreads();
-            // online softmax: warp w takes query heads w, w + 4, ...; lane = token
+            // online softmax: warp w takes query heads w, w + 4; lane = token
             for (int g = warp; g < gn; g += 4) {
                 const float x = sm.p[g][lane];
                 float cm = x;
@@ -105,7 +166,6 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
                 const float pe = __expf(x - m_new);
                 float ps = pe;
                 for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-                __syncwarp();
                 sm.p[g][lane] = pe;
                 if (lane == 0) {
                     const float fct = m_old == -INFINITY ? 0.f : __expf(m_old - m_new);
@@ -115,13 +175,21 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
                 }
             }
             __syncthreads();
+            // o_g[j] = f_g o_g[j] + sum_t p_g[t] v[t][j]: each v[t][j] read once for
+            // every query head, p read four tokens at a time (broadcast)
 #pragma unroll
-            for (int g = 0; g < TAIL_GSUB; ++g) {
-                if (g >= gn) break;
-                float x = acc[g] * sm.f[g];
-#pragma unroll 8
-                for (int t = 0; t < TAIL_CHUNK; ++t) x = fmaf(sm.p[g][t], sm.v[t][j], x);
-                acc[g] = x;
+            for (int g = 0; g < TAIL_GSUB; ++g)
+                if (g < gn) acc[g] *= sm.f[g];
+#pragma unroll 2
+            for (int t4 = 0; t4 < TAIL_CHUNK / 4; ++t4) {
+                const float v0 = sm.v[4 * t4][j], v1 = sm.v[4 * t4 + 1][j];
+                const float v2 = sm.v[4 * t4 + 2][j], v3 = sm.v[4 * t4 + 3][j];
+#pragma unroll
+                for (int g = 0; g < TAIL_GSUB; ++g) {
+                    if (g >= gn) break;
+                    const float4 p4 = reinterpret_cast<const float4 *>(sm.p[g])[t4];
+                    acc[g] = fmaf(p4.w, v3, fmaf(p4.z, v2, fmaf(p4.y, v1, fmaf(p4.x, v0, acc[g]))));
+                }
             }
         }
         __syncthreads();
@@ -132,7 +200,7 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
             tail_o[(row0 + g) * D + j] = lg > 0.f ? acc[g] / lg : 0.f;
             if (j == 0) tail_ml[row0 + g] = make_float2(sm.m[g], lg);
         }
-        __syncthreads();   // m and l are reset for the next group of query heads
+        __syncthreads();   // m and l read before the next pass resets them
     }
 }
 

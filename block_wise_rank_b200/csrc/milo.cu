@@ -737,7 +737,7 @@ milo_status milo_decode_attn_tail(const milo_factors *f, const float *q, int32_t
                                   size_t ws_bytes, milo_stream_t stream) {
     if (!k_tail || !v_tail || !tail_len || tail_cap < 0) return MILO_ERR_INVALID_ARG;
     if (tail_dtype != MILO_F32 && tail_dtype != MILO_BF16) return MILO_ERR_UNSUPPORTED;
-    if (!aligned(k_tail, 4) || !aligned(v_tail, 4) || !aligned(tail_len, 4)) return MILO_ERR_INVALID_ARG;
+    if (!aligned(k_tail, 16) || !aligned(v_tail, 16) || !aligned(tail_len, 4)) return MILO_ERR_INVALID_ARG;
     TailIn t;
     t.k = k_tail;
     t.v = v_tail;

@@ -239,9 +239,10 @@ size_t milo_decode_tail_workspace_size(const milo_factors *f, int32_t S, int32_t
  * softmax over the selected blocks' tokens (as in milo_decode_attn) and the
  * tail tokens i < tail_len[s] with s_i = q . k_tail[l][s][hq / G][i] / sqrt(d),
  * times v_tail[l][s][hq / G][i].
- *   k_tail, v_tail: device, [L][S][H][tail_cap][d] of tail_dtype (MILO_F32 or
- *             MILO_BF16; else MILO_ERR_UNSUPPORTED); keys already rotated to
- *             their own positions (as a model caches them), values plain
+ *   k_tail, v_tail: device, 16-byte aligned, [L][S][H][tail_cap][d] of
+ *             tail_dtype (MILO_F32 or MILO_BF16; else MILO_ERR_UNSUPPORTED);
+ *             keys already rotated to their own positions (as a model caches
+ *             them), values plain
  *   tail_len: device, int32 [S], 0 <= tail_len[s] <= tail_cap; a length
  *             outside that range sets MILO_ERR_BOUNDS in the status word and
  *             counts as an empty tail

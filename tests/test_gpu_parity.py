@@ -440,16 +440,18 @@ def test_decode_bounded_wait_runs_out(oracle_mod):
             assert _rel_inf(out[0, s, hq], ref) <= DEC_TOL
 
 
-@pytest.mark.parametrize("factor,tail_dtype", [("bf16", torch.bfloat16), ("f32", torch.float32)])
-def test_decode_recent_tail(oracle_mod, factor, tail_dtype):
+@pytest.mark.parametrize("factor,tail_dtype,G", [("bf16", torch.bfloat16, 4), ("f32", torch.float32, 4),
+                                                  ("bf16", torch.float32, 12)])
+def test_decode_recent_tail(oracle_mod, factor, tail_dtype, G):
     """milo_decode_attn_tail: the selected blocks plus each session's recent
     uncompressed tokens in one softmax.  Ragged tails (0, 1, 33, 64, 70 = the
     capacity, 5 tokens), bf16 factors (tensor-core decode) and f32 factors
-    (CUDA-core decode), fp32 and bf16 tails.  Checked against the oracle on
+    (CUDA-core decode), fp32 and bf16 tails, GQA 4 and 12 (more query heads
+    than one pass over the tail takes).  Checked against the oracle on
     the same factors and the same tail values; an all-empty tail gives
     milo_decode_attn's output bit for bit; a length past the capacity sets
     MILO_ERR_BOUNDS and counts as empty."""
-    L, H, G, T, bl, S, cap = 2, 2, 4, 1000, 512, 6, 70
+    L, H, T, bl, S, cap = 2, 2, 1000, 512, 6, 70
     K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=61, out_dtype=torch.bfloat16)
     V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=62, out_dtype=torch.bfloat16)
     if factor == "f32":
@@ -470,7 +472,7 @@ def test_decode_recent_tail(oracle_mod, factor, tail_dtype):
         u["H"] = H
     ktn, vtn = kt.double().numpy(), vt.double().numpy()
     for s in range(S):
-        for (l, hq) in [(0, 0), (1, 5), (0, 7), (1, 2)]:
+        for (l, hq) in [(0, 0), (1, 5), (0, 2 * G - 1), (1, G + 1), (0, 2 * G - 3)]:
             n, h = int(tl[s]), hq // G
             ref = oracle_mod.decode_one(
                 lambda b: U[0]["A"][(l * H + h) * 2 + b], lambda b: U[0]["B"][(l * H + h) * 2 + b],
