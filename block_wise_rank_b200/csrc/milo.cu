@@ -27,6 +27,7 @@
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
 #include "decode_tail.cuh"
+#include "decode_offload.cuh"
 
 using namespace milo;
 
@@ -722,6 +723,103 @@ milo_status milo_decode_attn(const milo_factors *f, const float *q, int32_t S, i
                              const int32_t *selected, const int32_t *positions, int32_t n_sel, double rope_base,
                              float *out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
     return decode_impl(f, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_bytes,
+                       stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- offload
+namespace {
+struct OffloadLayout {
+    size_t used, sizes[2], ranks[2], scaleA[2], scaleB[2], data[2], bytes;
+};
+// the staging area after the decode's own scratch
+OffloadLayout offload_layout(const milo_factors *f, size_t at) {
+    OffloadLayout o{};
+    const SectionLayout sec = section_layout(&f->shape, &f->params, f->R);
+    const bool i8 = f->params.factor_dtype == MILO_INT8;
+    o.used = at; at = align_up(at + sizeof(int32_t) * (f->n_b + 1));
+    for (int k = 0; k < 2; ++k) {
+        o.sizes[k] = at; at = align_up(at + sizeof(int64_t) * (f->n_blk + 1));
+        o.ranks[k] = at; at = align_up(at + sizeof(int32_t) * f->n_blk);
+        o.scaleA[k] = at; at = align_up(at + (i8 ? sizeof(float) * f->n_blk * D : 0));
+        o.scaleB[k] = at; at = align_up(at + (i8 ? sizeof(float) * f->n_blk * D : 0));
+        o.data[k] = at; at = align_up(at + (sec.bytes - sec.data));   // every block selected at most
+    }
+    o.bytes = at;
+    return o;
+}
+
+// the device address of p, a pointer into f's arena (null stays null), given
+// the device address of the arena
+template <typename P> P *on_device(const milo_factors *f, P *p, char *dev_arena) {
+    return p ? (P *)(dev_arena + ((const char *)p - (const char *)f->arena)) : nullptr;
+}
+}  // namespace
+
+extern "C" {
+
+size_t milo_decode_offload_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    const size_t base = milo_decode_workspace_size(f, S, Hq, n_sel);
+    return base ? offload_layout(f, align_up(base)).bytes : 0;
+}
+
+milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                     const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                     double rope_base, float *out, void *workspace, size_t ws_bytes,
+                                     milo_stream_t stream) {
+    if (!f || !f->arena || !q || !selected || !out || !workspace || S <= 0 || Hq <= 0 || n_sel <= 0)
+        return MILO_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign)) return MILO_ERR_INVALID_ARG;
+    const size_t ws_dec = align_up(milo_decode_workspace_size(f, S, Hq, n_sel));
+    const OffloadLayout o = offload_layout(f, ws_dec);
+    if (ws_bytes < o.bytes) return MILO_ERR_WORKSPACE;
+    // the arena must be reachable from the device: pinned, mapped host memory
+    // (or device memory); pageable memory is refused before any launch
+    cudaPointerAttributes attr{};
+    cudaError_t e = cudaPointerGetAttributes(&attr, f->arena);
+    if (e != cudaSuccess) return cuda_check(e, "arena attributes");
+    if ((attr.type != cudaMemoryTypeHost && attr.type != cudaMemoryTypeDevice &&
+         attr.type != cudaMemoryTypeManaged) || !attr.devicePointer)
+        return MILO_ERR_INVALID_ARG;
+    char *dev_arena = (char *)attr.devicePointer;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = (char *)workspace;
+    int32_t *used = (int32_t *)(w + o.used);
+    milo_factors st = *f;   // the staged copy: same shape, params and block ids
+    st.arena = nullptr;
+    st.arena_bytes = 0;
+    cudaEvent_t t0 = tmark(s);
+    e = cudaMemsetAsync(used, 0, sizeof(int32_t) * (f->n_b + 1), s);
+    if (e != cudaSuccess) return cuda_check(e, "memset");
+    const int64_t slots = (int64_t)S * n_sel;
+    k_flag_selected<<<(int)std::min<int64_t>((slots + 255) / 256, 1024), 256, 0, s>>>(selected, (int)slots, f->n_b,
+                                                                                      used);
+    const int esize = dtype_bytes(f->params.factor_dtype);
+    for (int k = 0; k < 2; ++k) {
+        KindView host = f->kv[k];
+        host.ranks = on_device(f, host.ranks, dev_arena);
+        host.offsets = on_device(f, host.offsets, dev_arena);
+        host.scaleA = on_device(f, host.scaleA, dev_arena);
+        host.scaleB = on_device(f, host.scaleB, dev_arena);
+        host.data = on_device(f, (char *)host.data, dev_arena);
+        KindView &sv = st.kv[k];
+        sv.sigma = nullptr;
+        sv.eps = nullptr;
+        sv.ranks = (int32_t *)(w + o.ranks[k]);
+        sv.offsets = (int64_t *)(w + o.sizes[k]);
+        sv.scaleA = host.scaleA ? (float *)(w + o.scaleA[k]) : nullptr;
+        sv.scaleB = host.scaleB ? (float *)(w + o.scaleB[k]) : nullptr;
+        sv.data = w + o.data[k];
+        k_stage_sizes<<<(int)std::min<int64_t>((f->n_blk + 255) / 256, 4096), 256, 0, s>>>(
+            host.ranks, used, f->n_blk, f->n_b, f->shape.T, f->shape.block_len, sv.offsets, sv.ranks);
+        k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(sv.offsets, f->n_blk);
+        k_stage_copy<<<(unsigned)f->n_blk, 256, 0, s>>>(host, sv, used, f->n_b, esize);
+    }
+    tpush(MILO_TK_STAGE, t0, tmark(s));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_check(e, "staging launch");
+    return decode_impl(&st, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_dec,
                        stream);
 }
 

@@ -55,10 +55,12 @@ EXPORTS = [
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
     "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
     "milo_jacobi_rounds", "milo_decode_tail_workspace_size", "milo_decode_attn_tail",
+    "milo_decode_offload_workspace_size", "milo_decode_attn_offload",
 ]
 
 # stages of milo_timing_read, in order (milo_timed_stage)
-TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine", "tail"]
+TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine", "tail",
+                "stage"]
 
 MILO_NOALLOC_MAX_BLOCKS = 65536
 
@@ -90,6 +92,10 @@ def lib():
         L.milo_decode_attn_tail.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, I32, I32, P, P, P,
                                             SZ, P]
         L.milo_decode_attn_tail.restype = ctypes.c_int
+        L.milo_decode_offload_workspace_size.argtypes = [P, I32, I32, I32]
+        L.milo_decode_offload_workspace_size.restype = SZ
+        L.milo_decode_attn_offload.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
+        L.milo_decode_attn_offload.restype = ctypes.c_int
         L.milo_decode_attn.restype = ctypes.c_int
         L.milo_factors_get.argtypes = [P, I32, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
                                        ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
@@ -314,6 +320,40 @@ def milo_decode_attn_tail(f: Factors, q: torch.Tensor, selected: torch.Tensor, k
                                     float(rope_base), _ptr(k_tail), _ptr(v_tail), dt, k_tail.shape[3],
                                     _ptr(tail_len), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(s, "milo_decode_attn_tail")
+    return out
+
+
+def factors_to_host(f: Factors) -> Factors:
+    """A handle over a pinned host copy of f's arena (for milo_decode_attn_offload)."""
+    n = f.arena.numel()
+    raw = torch.empty(n + 256, dtype=torch.uint8, pin_memory=True)
+    host = raw[(-raw.data_ptr()) % 256:][:n]   # the arena's 256-byte alignment
+    host.copy_(f.arena)
+    return milo_factors_wrap(f.shape, f.params, host)
+
+
+def milo_decode_offload_workspace_size(f: Factors, S: int, Hq: int, n_sel: int) -> int:
+    return lib().milo_decode_offload_workspace_size(f.handle, S, Hq, n_sel)
+
+
+def milo_decode_attn_offload(f: Factors, q: torch.Tensor, selected: torch.Tensor, positions=None, rope_base=1e6,
+                             out=None, workspace=None, stream=None):
+    """milo_decode_attn for a handle whose arena is in pinned host memory: the
+    selected blocks' factors are staged on the device each call."""
+    assert q.dtype == torch.float32 and q.is_contiguous() and q.is_cuda
+    L, S, Hq, d = q.shape
+    n_sel = selected.shape[1]
+    assert selected.dtype == torch.int32 and selected.shape[0] == S and selected.is_contiguous()
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.shape == selected.shape and positions.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = _bytes(milo_decode_offload_workspace_size(f, S, Hq, n_sel), q.device)
+    s = lib().milo_decode_attn_offload(f.handle, _ptr(q), S, Hq, _ptr(selected), _ptr(positions), n_sel,
+                                       float(rope_base), _ptr(out), _ptr(workspace), workspace.numel(),
+                                       _stream(stream))
+    _check(s, "milo_decode_attn_offload")
     return out
 
 

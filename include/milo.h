@@ -256,6 +256,29 @@ milo_status milo_decode_attn_tail(const milo_factors *f, const float *q, int32_t
                                   int32_t tail_cap, const int32_t *tail_len, float *out, void *workspace,
                                   size_t ws_bytes, milo_stream_t stream);
 
+/* Bytes of scratch milo_decode_attn_offload needs: milo_decode_workspace_size
+ * plus a staging area that holds every block's factors at most. */
+size_t milo_decode_offload_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel);
+
+/*
+ * milo_decode_attn for factors kept in host memory: the handle's arena
+ * (from milo_factors_wrap over a copy of a compressed arena) lives in pinned,
+ * device-mapped host memory.  Each call copies the factors (and INT8 scales)
+ * of the blocks some session selected into the workspace's staging area over
+ * the host link, then decodes there; the output equals milo_decode_attn on a
+ * device copy of the same arena bit for bit.  "MILO ... Block-wise Low-rank
+ * Compression" (evolve.pub review), Summary and FAQ "How much memory saving
+ * and speedup does MILO achieve?": the pages measure MILO against offloading
+ * the full KV cache to CPU memory; only the retrieved blocks' factors move.
+ * Arguments, errors and the result as milo_decode_attn, with ws_bytes >=
+ * milo_decode_offload_workspace_size; an arena in pageable host memory gives
+ * MILO_ERR_INVALID_ARG before any launch.
+ */
+milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                     const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                     double rope_base, float *out, void *workspace, size_t ws_bytes,
+                                     milo_stream_t stream);
+
 /* ------------------------------------------------------ factor handles */
 
 /* Views (device pointers into the arena) of one kind (0 = K, 1 = V).  Any
@@ -313,7 +336,8 @@ typedef enum {
     MILO_TK_DECODE = 6,      /* decode attention (k_decode_tc or k_decode_simt) */
     MILO_TK_COMBINE = 7,     /* merge of the per-block partials (k_combine) */
     MILO_TK_TAIL = 8,        /* attention over the recent uncompressed tokens (k_tail_attn) */
-    MILO_TK_COUNT = 9
+    MILO_TK_STAGE = 9,       /* host-resident factors of the selected blocks staged on the device */
+    MILO_TK_COUNT = 10
 } milo_timed_stage;
 
 /* on != 0: start recording (previous records are dropped); on == 0: stop.

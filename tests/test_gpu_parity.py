@@ -492,3 +492,44 @@ def test_decode_recent_tail(oracle_mod, factor, tail_dtype, G):
     assert milo.milo_get_status() == milo.MILO_ERR_BOUNDS
     assert np.array_equal(o_bad[:, 2], base[:, 2])
     assert np.array_equal(o_bad[:, 3], out[:, 3])
+
+
+@pytest.mark.parametrize("factor", ["bf16", "int8", "f32"])
+def test_decode_offloaded_factors(factor):
+    """milo_decode_attn_offload on a pinned host copy of the arena stages the
+    selected blocks' factors and gives milo_decode_attn's output bit for bit:
+    bf16 (tensor cores), INT8 (scales staged too) and f32 (CUDA cores), with
+    blocks no session selects (the staging offsets skip them) and a ragged
+    last block.  An arena in pageable host memory is refused before any
+    launch."""
+    L, H, G, T, bl, S = 2, 2, 4, 3900, 512, 3
+    K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=71, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=72, out_dtype=torch.bfloat16)
+    if factor == "f32":
+        K, V = K.float(), V.float()
+    f = milo.milo_compress(K.cuda(), V.cuda(), bl, milo.default_params(factor_dtype=factor, budget_frac=0.5))
+    g = torch.Generator().manual_seed(73)
+    q = torch.randn(L, S, H * G, 128, generator=g).cuda()
+    sel = torch.tensor([[1, 7], [7, 4], [4, 1]], dtype=torch.int32).cuda()   # blocks 0, 2, 3, 5, 6 unused
+    pos = (sel * bl).to(torch.int32)
+    ref = milo.milo_decode_attn(f, q, sel, pos, rope_base=1e6).cpu()
+    assert milo.milo_get_status() == milo.MILO_OK
+    fh = milo.factors_to_host(f)
+    out = milo.milo_decode_attn_offload(fh, q, sel, pos, rope_base=1e6).cpu()
+    assert milo.milo_get_status() == milo.MILO_OK
+    assert torch.equal(out, ref)
+    # a second call with another selection reuses nothing stale
+    sel2 = torch.tensor([[0, 3], [6, 3], [5, 0]], dtype=torch.int32).cuda()
+    pos2 = (sel2 * bl).to(torch.int32)
+    ws = torch.empty(milo.milo_decode_offload_workspace_size(fh, S, H * G, 2), dtype=torch.uint8, device="cuda")
+    milo.milo_decode_attn_offload(fh, q, sel, pos, rope_base=1e6, workspace=ws)
+    out2 = milo.milo_decode_attn_offload(fh, q, sel2, pos2, rope_base=1e6, workspace=ws).cpu()
+    assert torch.equal(out2, milo.milo_decode_attn(f, q, sel2, pos2, rope_base=1e6).cpu())
+    # pageable host memory: refused, nothing launched
+    raw = torch.empty(f.arena.numel() + 256, dtype=torch.uint8)
+    pageable = raw[(-raw.data_ptr()) % 256:][:f.arena.numel()]
+    pageable.copy_(f.arena)
+    fp = milo.milo_factors_wrap(f.shape, f.params, pageable)
+    with pytest.raises(milo.MiloError):
+        milo.milo_decode_attn_offload(fp, q, sel, pos, rope_base=1e6)
+    assert milo.milo_get_status() == milo.MILO_OK
