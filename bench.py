@@ -409,6 +409,67 @@ def row_of(run, t, steps, pk):
                 status=milo.status_string(t["status"]))
 
 
+# ------------------------------------------------------------------ offloaded factors
+def h2d_copy_gbs(dev, nbytes=1 << 30, reps=3):
+    """Host-to-device copy bandwidth of this machine: one pinned buffer copied with
+    cudaMemcpyAsync, CUDA events around `reps` copies after one warm-up."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst.copy_(src, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        dst.copy_(src, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    return nbytes * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
+
+
+def offload_measure(run, reps=3):
+    """The pages' offloaded setting on this workload: the factor arena in
+    pinned host memory and each decode step staging the selected blocks'
+    factors over the host link (milo_decode_attn_offload), against the
+    transfer that offloading the full KV cache of the same blocks needs at this
+    box's measured host-to-device copy bandwidth (a lower bound of that
+    baseline's step time, so the speed-up is a lower bound too)."""
+    w = run.w
+    fh = milo.factors_to_host(run.f)
+    q, sel, pos = run.dec_inputs[0]
+    ws = torch.empty(milo.milo_decode_offload_workspace_size(fh, w.sessions, w.Hq, w.n_sel), dtype=torch.uint8,
+                     device=run.dev)
+    out = torch.empty_like(run.out)
+    milo.milo_decode_attn_offload(fh, q, sel, pos, rope_base=w.rope_base, out=out, workspace=ws)
+    same = bool(torch.equal(out, milo.milo_decode_attn(run.f, q, sel, pos, rope_base=w.rope_base)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    milo.milo_timing_enable(True)
+    e0.record()
+    for _ in range(reps):
+        milo.milo_decode_attn_offload(fh, q, sel, pos, rope_base=w.rope_base, out=out, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    stages = milo.milo_timing_read()
+    milo.milo_timing_enable(False)
+    status = milo.milo_get_status()
+    ms = e0.elapsed_time(e1) / reps
+    sms, sn = stages["stage"]
+    stage_ms = sms / sn if sn else None
+    fbytes = decode_bytes(read_ranks(run.f), w, sel, run.factor, w.sessions, w.Hq) - \
+        (2 * w.L * w.sessions * w.Hq * w.d * 4 + 2 * sel.numel() * 4)
+    uniq = sorted(set(sel.reshape(-1).tolist()))
+    kv_tokens = sum(min(w.block_len, w.T - b * w.block_len) for b in uniq)
+    kv_bytes = 2 * w.L * w.H * kv_tokens * w.d * run.K.element_size()
+    del ws, out
+    fh.close()
+    torch.cuda.empty_cache()
+    h2d = h2d_copy_gbs(run.dev)
+    kv_ms = kv_bytes / (h2d * 1e9) * 1e3
+    return dict(decode_ms=round(ms, 3), stage_ms=round(stage_ms, 3) if stage_ms else None,
+                staged_factor_bytes=int(fbytes), link_gbs=round(fbytes / (stage_ms / 1e3) / 1e9, 2) if stage_ms else None,
+                h2d_copy_gbs=round(h2d, 2), full_kv_bytes=int(kv_bytes), full_kv_transfer_ms_at_least=round(kv_ms, 3),
+                speedup_vs_full_kv_offload_at_least=round(kv_ms / ms, 3), tokens_per_s=round(w.sessions / (ms / 1e3), 1),
+                bit_identical_to_resident=same, status=milo.status_string(status))
+
+
 # ------------------------------------------------------------------ traffic
 def source_hash():
     """Hash of the decode kernel's code (comments and blank space removed)."""
@@ -668,6 +729,7 @@ def run_ours(args, rank, world):
         status=milo.status_string(t["status"]),
     )
     if world == 1 and not args.no_rows:
+        res["offload"] = offload_measure(run)
         rows = [row_of(run, t, args.steps, pk)]
         run.release()
         for (name, budget, fac, tail) in ROWS:
