@@ -306,3 +306,52 @@ def decode_one(AK, BK, AV, BV, q, blocks, positions, rope_base: float, k_tail=No
     if Kc.shape[0] == 0:
         return np.zeros(d)
     return attention(np.asarray(q, dtype=np.float64)[None, :], Kc, Vc)[0]
+
+
+# --------------------------------------------------------------------------
+# block retrieval
+# --------------------------------------------------------------------------
+def bm25_scores(blocks, block_len, queries, k1: float = 1.2, beta: float = 0.75):
+    """Okapi BM25 score of every block for every query, fp64.
+
+    evolve.pub review, Summary: a query retrieves its relevant blocks with
+    BM25.  The function is the textbook Okapi BM25 (Robertson and Zaragoza,
+    "The Probabilistic Relevance Framework: BM25 and Beyond", 2009):
+    idf(t) = ln(1 + (N - n_t + 0.5) / (n_t + 0.5)) over N blocks, n_t of them
+    holding t; a block's score adds, over its terms t that the query holds,
+    qtf(t) idf(t) tf (k1 + 1) / (tf + k1 (1 - beta + beta len / avgdl)).
+    blocks / queries: lists of (terms, counts) rows, each term once per row;
+    block_len: tokens per block.  Returns scores [n_queries][n_blocks].
+    """
+    N = len(blocks)
+    df = {}
+    for terms, _ in blocks:
+        for t in terms:
+            df[int(t)] = df.get(int(t), 0) + 1
+    total = 0.0
+    for n in block_len:
+        total += float(n)
+    avgdl = total / N
+    out = np.zeros((len(queries), N))
+    for s, (qt, qc) in enumerate(queries):
+        w = {}
+        for t, c in zip(qt, qc):
+            n = float(df.get(int(t), 0))
+            w[int(t)] = float(c) * math.log1p(((N - n) + 0.5) / (n + 0.5))
+        for b, (terms, counts) in enumerate(blocks):
+            norm = k1 * ((1.0 - beta) + (beta * float(block_len[b])) / avgdl)
+            sc = 0.0
+            for t, c in zip(terms, counts):
+                if int(t) in w:
+                    tf = float(c)
+                    sc += ((w[int(t)] * tf) * (k1 + 1.0)) / (tf + norm)
+            out[s, b] = sc
+    return out
+
+
+def bm25_select(scores, n_sel: int):
+    """The n_sel highest-scoring block ids of each row, by score descending and
+    block id ascending among equal scores."""
+    return np.array([sorted(range(len(row)), key=lambda b: (-row[b], b))[:n_sel] for row in scores],
+                    dtype=np.int32)
+

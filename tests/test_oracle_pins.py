@@ -416,3 +416,69 @@ def test_compress_end_to_end_small(oracle_mod):
                 Xh = oracle_mod.reconstruct(r["A"][0][h][b], r["B"][0][h][b]) if rb else np.zeros_like(Xb)
                 tail = np.sum(r["sigma"][0, h, b, rb:] ** 2)
                 assert abs(np.sum((Xb - Xh) ** 2) - tail) <= 1e-9 * tail + 1e-20
+
+
+# ---------------------------------------------------------------- BM25 retrieval
+def test_bm25_closed_forms(oracle_mod):
+    """Special cases of Okapi BM25 with known values: one query term held by
+    one of three equal-length blocks with tf = 1 scores idf = ln(8/3); blocks
+    without a query term score 0; k1 = 0 reduces the score to the sum of the
+    held terms' qtf idf; a term in every block has idf ln(1 + 0.5 / (N + 0.5))."""
+    blocks = [([1, 4], [1, 2]), ([2, 4], [1, 1]), ([3, 4], [1, 5])]
+    lens = [10, 10, 10]
+    sc = oracle_mod.bm25_scores(blocks, lens, [([1], [1])])
+    assert abs(sc[0, 0] - math.log(8 / 3)) <= 1e-15 and sc[0, 1] == 0.0 and sc[0, 2] == 0.0
+    # k1 = 0: presence only, qtf times idf
+    sc0 = oracle_mod.bm25_scores(blocks, lens, [([1, 4], [2, 3])], k1=0.0)
+    idf4 = math.log(1 + 0.5 / 3.5)
+    assert abs(sc0[0, 0] - (2 * math.log(8 / 3) + 3 * idf4)) <= 1e-14
+    assert abs(sc0[0, 1] - 3 * idf4) <= 1e-15
+    # saturation: a huge tf approaches idf (k1 + 1)
+    big = oracle_mod.bm25_scores([([7], [10 ** 9]), ([8], [1])], [5, 5], [([7], [1])], k1=1.2)
+    assert abs(big[0, 0] - math.log(1 + 1.5 / 1.5) * 2.2) <= 1e-8
+
+
+def test_bm25_invariances(oracle_mod):
+    """Scores rise with tf and fall with block length (beta > 0); with beta = 0
+    the lengths do not matter; relabelling terms changes nothing; an extra
+    block holding a term lowers that term's idf."""
+    rng = np.random.default_rng(31)
+    blocks = []
+    for _ in range(12):
+        t = rng.choice(60, size=15, replace=False)
+        blocks.append((t.tolist(), rng.integers(1, 6, size=15).tolist()))
+    lens = rng.integers(100, 600, size=12).tolist()
+    q = [(rng.choice(60, size=6, replace=False).tolist(), [1] * 6)]
+    sc = oracle_mod.bm25_scores(blocks, lens, q)
+    # tf up in one block, for a query term it holds: its score rises, others unchanged
+    b0 = next(b for b in range(12) if set(blocks[b][0]) & set(q[0][0]))
+    t = next(x for x in blocks[b0][0] if x in q[0][0])
+    i = blocks[b0][0].index(t)
+    more = [list(r) for r in blocks]
+    more[b0] = (blocks[b0][0], [c + (3 if k == i else 0) for k, c in enumerate(blocks[b0][1])])
+    sc_more = oracle_mod.bm25_scores(more, lens, q)
+    assert sc_more[0, b0] > sc[0, b0] and np.array_equal(np.delete(sc_more, b0, 1), np.delete(sc, b0, 1))
+    # a longer block scores lower (beta > 0); beta = 0 ignores lengths
+    longer = list(lens)
+    longer[b0] += 500
+    assert oracle_mod.bm25_scores(blocks, longer, q)[0, b0] < sc[0, b0]
+    flat = oracle_mod.bm25_scores(blocks, lens, q, beta=0.0)
+    assert np.allclose(oracle_mod.bm25_scores(blocks, longer, q, beta=0.0), flat, rtol=0, atol=1e-15)
+    # term relabelling
+    perm = rng.permutation(60)
+    rb = [([int(perm[x]) for x in tt], cc) for tt, cc in blocks]
+    rq = [([int(perm[x]) for x in q[0][0]], q[0][1])]
+    assert np.array_equal(oracle_mod.bm25_scores(rb, lens, rq), sc)
+    # one more block holding t: t's idf falls, so b0's score falls
+    extra = blocks + [([t], [1])]
+    assert oracle_mod.bm25_scores(extra, lens + [300], q)[0, b0] < sc[0, b0]
+
+
+def test_bm25_select_brute_force(oracle_mod):
+    """Top-n selection against numpy's lexsort on (id, -score), with planted
+    ties (equal scores go to the lower block id)."""
+    rng = np.random.default_rng(32)
+    scores = rng.integers(0, 5, size=(6, 40)).astype(float) * 0.25   # many exact ties
+    for n in (1, 7, 40):
+        ref = np.stack([np.lexsort((np.arange(40), -row))[:n] for row in scores]).astype(np.int32)
+        assert np.array_equal(oracle_mod.bm25_select(scores, n), ref)
