@@ -409,6 +409,32 @@ def row_of(run, t, steps, pk):
                 status=milo.status_string(t["status"]))
 
 
+# ------------------------------------------------------------------ retrieval
+BM25_VOCAB = 8192
+
+
+def retrieval_measure(run, reps=20):
+    """GPU BM25 block retrieval for this workload's sessions over synthetic
+    term-count tables (milo_bm25_select): device time per call and the
+    selection it makes.  The decode rows keep the seeded uniform selection so
+    that their bytes stay comparable across changes."""
+    w = run.w
+    tables = [x.to(run.dev) for x in synth.bm25_tables(w, vocab=BM25_VOCAB)]
+    ws = torch.empty(milo.lib().milo_bm25_workspace_size(w.n_b, BM25_VOCAB, w.sessions), dtype=torch.uint8,
+                     device=run.dev)
+    sel, _ = milo.milo_bm25_select(tables, BM25_VOCAB, w.n_sel, device=run.dev, workspace=ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        milo.milo_bm25_select(tables, BM25_VOCAB, w.n_sel, device=run.dev, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    return dict(scorer="Okapi BM25 (k1 1.2, beta 0.75), fp64", vocab=BM25_VOCAB, sessions=w.sessions, blocks=w.n_b,
+                n_sel=w.n_sel, ms_per_call=round(e0.elapsed_time(e1) / reps, 4),
+                unique_blocks_selected=int(torch.unique(sel).numel()),
+                status=milo.status_string(milo.milo_get_status()))
+
+
 # ------------------------------------------------------------------ offloaded factors
 def h2d_copy_gbs(dev, nbytes=1 << 30, reps=3):
     """Host-to-device copy bandwidth of this machine: one pinned buffer copied with
@@ -729,6 +755,7 @@ def run_ours(args, rank, world):
         status=milo.status_string(t["status"]),
     )
     if world == 1 and not args.no_rows:
+        res["retrieval"] = retrieval_measure(run)
         res["offload"] = offload_measure(run)
         rows = [row_of(run, t, args.steps, pk)]
         run.release()

@@ -28,6 +28,7 @@
 #include "decode_tc.cuh"
 #include "decode_tail.cuh"
 #include "decode_offload.cuh"
+#include "bm25.cuh"
 
 using namespace milo;
 
@@ -821,6 +822,49 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
     if (e != cudaSuccess) return cuda_check(e, "staging launch");
     return decode_impl(&st, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_dec,
                        stream);
+}
+
+// ---------------------------------------------------------------- retrieval
+size_t milo_bm25_workspace_size(int32_t n_b, int32_t V, int32_t S) {
+    if (n_b <= 0 || V <= 0 || S <= 0) return 0;
+    return align_up(sizeof(int32_t) * V) + align_up(sizeof(double) * (size_t)S * V) + align_up(sizeof(double)) +
+           align_up(sizeof(double) * (size_t)S * n_b);
+}
+
+milo_status milo_bm25_select(const int32_t *blk_ptr, const int32_t *blk_term, const int32_t *blk_tf,
+                             const int32_t *blk_len, int32_t n_b, int32_t nnz_b, int32_t V, const int32_t *q_ptr,
+                             const int32_t *q_term, const int32_t *q_tf, int32_t S, int32_t nnz_q, double k1,
+                             double beta, int32_t n_sel, int32_t *selected, double *scores, void *workspace,
+                             size_t ws_bytes, milo_stream_t stream) {
+    if (!blk_ptr || !blk_len || !q_ptr || !selected || !workspace) return MILO_ERR_INVALID_ARG;
+    if (n_b <= 0 || V <= 0 || S <= 0 || nnz_b < 0 || nnz_q < 0 || n_sel < 1 || n_sel > n_b) return MILO_ERR_INVALID_ARG;
+    if ((nnz_b > 0 && (!blk_term || !blk_tf)) || (nnz_q > 0 && (!q_term || !q_tf))) return MILO_ERR_INVALID_ARG;
+    if (!(k1 >= 0.0) || !(beta >= 0.0 && beta <= 1.0) || !aligned(workspace, kAlign)) return MILO_ERR_INVALID_ARG;
+    if (ws_bytes < milo_bm25_workspace_size(n_b, V, S)) return MILO_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = (char *)workspace;
+    size_t at = 0;
+    Bm25Args a{};
+    a.blk_ptr = blk_ptr; a.blk_term = blk_term; a.blk_tf = blk_tf; a.blk_len = blk_len;
+    a.q_ptr = q_ptr; a.q_term = q_term; a.q_tf = q_tf;
+    a.n_b = n_b; a.V = V; a.S = S; a.n_sel = n_sel; a.nnz_b = nnz_b; a.nnz_q = nnz_q;
+    a.k1 = k1; a.beta = beta;
+    a.df = (int32_t *)(w + at); at = align_up(at + sizeof(int32_t) * V);
+    a.qw = (double *)(w + at); at = align_up(at + sizeof(double) * (size_t)S * V);
+    a.avgdl = (double *)(w + at); at = align_up(at + sizeof(double));
+    a.scores = scores ? scores : (double *)(w + at);
+    a.selected = selected;
+    cudaEvent_t t0 = tmark(s);
+    cudaError_t e = cudaMemsetAsync(a.df, 0, sizeof(int32_t) * V, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.qw, 0, sizeof(double) * (size_t)S * V, s);
+    if (e != cudaSuccess) return cuda_check(e, "memset");
+    k_bm25_df<<<(int)std::min<int64_t>(((int64_t)nnz_b + 255) / 256 + 1, 1024), 256, 0, s>>>(a);
+    k_bm25_avgdl<<<1, 32, 0, s>>>(a);
+    k_bm25_qweights<<<S, 128, 0, s>>>(a);
+    k_bm25_scores<<<(unsigned)(((int64_t)S * n_b + 255) / 256), 256, 0, s>>>(a);
+    k_bm25_topk<<<S, 256, 0, s>>>(a);
+    tpush(MILO_TK_RETRIEVE, t0, tmark(s));
+    return cuda_check(cudaGetLastError(), "retrieval launch");
 }
 
 size_t milo_decode_tail_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {

@@ -55,12 +55,13 @@ EXPORTS = [
     "milo_factors_import", "milo_factors_destroy", "milo_get_status", "milo_status_string", "milo_version",
     "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
     "milo_jacobi_rounds", "milo_decode_tail_workspace_size", "milo_decode_attn_tail",
-    "milo_decode_offload_workspace_size", "milo_decode_attn_offload",
+    "milo_decode_offload_workspace_size", "milo_decode_attn_offload", "milo_bm25_workspace_size",
+    "milo_bm25_select",
 ]
 
 # stages of milo_timing_read, in order (milo_timed_stage)
 TIMED_STAGES = ["gram", "jacobi", "refine", "select", "project", "decode_prep", "decode", "combine", "tail",
-                "stage"]
+                "stage", "retrieve"]
 
 MILO_NOALLOC_MAX_BLOCKS = 65536
 
@@ -96,6 +97,11 @@ def lib():
         L.milo_decode_offload_workspace_size.restype = SZ
         L.milo_decode_attn_offload.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
         L.milo_decode_attn_offload.restype = ctypes.c_int
+        L.milo_bm25_workspace_size.argtypes = [I32, I32, I32]
+        L.milo_bm25_workspace_size.restype = SZ
+        L.milo_bm25_select.argtypes = [P, P, P, P, I32, I32, I32, P, P, P, I32, I32, ctypes.c_double,
+                                       ctypes.c_double, I32, P, P, P, SZ, P]
+        L.milo_bm25_select.restype = ctypes.c_int
         L.milo_decode_attn.restype = ctypes.c_int
         L.milo_factors_get.argtypes = [P, I32, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
                                        ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
@@ -355,6 +361,26 @@ def milo_decode_attn_offload(f: Factors, q: torch.Tensor, selected: torch.Tensor
                                        _stream(stream))
     _check(s, "milo_decode_attn_offload")
     return out
+
+
+def milo_bm25_select(tables, vocab: int, n_sel: int, k1: float = 1.2, beta: float = 0.75, device="cuda",
+                     workspace=None, stream=None):
+    """BM25 block retrieval on the GPU.  tables = (blk_ptr, blk_term, blk_tf,
+    blk_len, q_ptr, q_term, q_tf), int32 (any device).  Returns (selected
+    int32 [S][n_sel], scores fp64 [S][n_b]) on `device`."""
+    t = [x.to(device=device, dtype=torch.int32).contiguous() for x in tables]
+    blk_ptr, blk_term, blk_tf, blk_len, q_ptr, q_term, q_tf = t
+    n_b, S = blk_len.numel(), q_ptr.numel() - 1
+    selected = torch.empty(S, n_sel, dtype=torch.int32, device=device)
+    scores = torch.empty(S, n_b, dtype=torch.float64, device=device)
+    if workspace is None:
+        workspace = _bytes(lib().milo_bm25_workspace_size(n_b, vocab, S), device)
+    s = lib().milo_bm25_select(_ptr(blk_ptr), _ptr(blk_term), _ptr(blk_tf), _ptr(blk_len), n_b, blk_term.numel(),
+                               vocab, _ptr(q_ptr), _ptr(q_term), _ptr(q_tf), S, q_term.numel(), float(k1),
+                               float(beta), n_sel, _ptr(selected), _ptr(scores), _ptr(workspace), workspace.numel(),
+                               _stream(stream))
+    _check(s, "milo_bm25_select")
+    return selected, scores
 
 
 def milo_factors_wrap(shape, params, arena: torch.Tensor) -> Factors:

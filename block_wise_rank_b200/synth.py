@@ -196,3 +196,39 @@ def recent_tail(w: Workload, n_tail: int, device="cpu", dtype=torch.float32):
     n = torch.full((w.sessions,), n_tail, dtype=torch.int32, device=device)
     return k, v, n
 
+
+def bm25_tables(w: Workload, vocab: int = 8192, terms_per_block: int = 160, query_terms: int = 16, step: int = 0):
+    """Synthetic term-count tables for the BM25 retriever, seeded.
+
+    Blocks: `terms_per_block` distinct terms each, drawn without replacement
+    with Zipf-like weights 1 / (rank + 10) over `vocab` terms; counts
+    1 + Poisson(1.5).  Lengths: each block's tokens.  Queries (one per
+    session): half of the terms from one block the session is about (drawn
+    uniformly), half from the Zipf vocabulary, distinct, count 1.
+    Returns int32 CPU tensors (blk_ptr, blk_term, blk_tf, blk_len, q_ptr,
+    q_term, q_tf).
+    """
+    g = _gen(w.seed * 1000 + 400 + step, "cpu")
+    zipf = 1.0 / (torch.arange(vocab, dtype=torch.float64) + 10.0)
+    terms, tfs, ptr = [], [], [0]
+    for _ in range(w.n_b):
+        t = torch.multinomial(zipf, terms_per_block, replacement=False, generator=g)
+        terms.append(t)
+        tfs.append(1 + torch.poisson(torch.full((terms_per_block,), 1.5, dtype=torch.float64), generator=g).long())
+        ptr.append(ptr[-1] + terms_per_block)
+    blk_len = torch.tensor([min(w.block_len, w.T - b * w.block_len) for b in range(w.n_b)], dtype=torch.int32)
+    q_terms, q_ptr = [], [0]
+    for _ in range(w.sessions):
+        topic = int(torch.randint(0, w.n_b, (1,), generator=g))
+        own = terms[topic][torch.randperm(terms_per_block, generator=g)[:query_terms // 2]]
+        pick = set(own.tolist())
+        while len(pick) < query_terms:
+            pick.add(int(torch.multinomial(zipf, 1, generator=g)))
+        q = torch.tensor(sorted(pick), dtype=torch.int64)
+        q_terms.append(q)
+        q_ptr.append(q_ptr[-1] + len(q))
+    q_term = torch.cat(q_terms)
+    return (torch.tensor(ptr, dtype=torch.int32), torch.cat(terms).to(torch.int32), torch.cat(tfs).to(torch.int32),
+            blk_len, torch.tensor(q_ptr, dtype=torch.int32), q_term.to(torch.int32),
+            torch.ones(len(q_term), dtype=torch.int32))
+

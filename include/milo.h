@@ -279,6 +279,38 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
                                      double rope_base, float *out, void *workspace, size_t ws_bytes,
                                      milo_stream_t stream);
 
+/* ---------------------------------------------------------------- retrieval */
+
+/* Bytes of scratch milo_bm25_select needs. */
+size_t milo_bm25_workspace_size(int32_t n_b, int32_t V, int32_t S);
+
+/*
+ * Block retrieval: Okapi BM25 scores of every block for every session's query
+ * and each session's top n_sel blocks.  "MILO ... Block-wise Low-rank
+ * Compression" (evolve.pub review), Summary: a query retrieves its relevant
+ * blocks with BM25 and only those are rebuilt.  Scoring (Robertson and
+ * Zaragoza 2009): idf(t) = ln(1 + (N - n_t + 0.5) / (n_t + 0.5)) over the
+ * n_b blocks, and score(s, b) = sum over the block's terms t of
+ * qtf_s(t) idf(t) tf(t,b) (k1 + 1) / (tf(t,b) + k1 (1 - beta + beta len_b / avgdl)),
+ * fp64 with every operation rounded separately, terms added in row order.
+ *   blk_ptr [n_b + 1], blk_term / blk_tf [nnz_b]: device, the blocks' term
+ *             counts in CSR form (term ids in [0, V), each once per row,
+ *             counts >= 1); blk_len [n_b]: tokens of each block
+ *   q_ptr [S + 1], q_term / q_tf [nnz_q]: device, each session's query terms
+ *             (each once per row, with its count)
+ *   selected: device, int32 [S][n_sel] out: block ids by score descending,
+ *             ties to the lower id (usable as milo_decode_attn's selection)
+ *   scores:   device, fp64 [S][n_b] out, or NULL
+ * 1 <= n_sel <= n_b, k1 >= 0, 0 <= beta <= 1.  Row pointers outside
+ * [0, nnz] and term ids outside [0, V) set MILO_ERR_BOUNDS in the status word
+ * and are clamped or skipped.
+ */
+milo_status milo_bm25_select(const int32_t *blk_ptr, const int32_t *blk_term, const int32_t *blk_tf,
+                             const int32_t *blk_len, int32_t n_b, int32_t nnz_b, int32_t V, const int32_t *q_ptr,
+                             const int32_t *q_term, const int32_t *q_tf, int32_t S, int32_t nnz_q, double k1,
+                             double beta, int32_t n_sel, int32_t *selected, double *scores, void *workspace,
+                             size_t ws_bytes, milo_stream_t stream);
+
 /* ------------------------------------------------------ factor handles */
 
 /* Views (device pointers into the arena) of one kind (0 = K, 1 = V).  Any
@@ -337,7 +369,8 @@ typedef enum {
     MILO_TK_COMBINE = 7,     /* merge of the per-block partials (k_combine) */
     MILO_TK_TAIL = 8,        /* attention over the recent uncompressed tokens (k_tail_attn) */
     MILO_TK_STAGE = 9,       /* host-resident factors of the selected blocks staged on the device */
-    MILO_TK_COUNT = 10
+    MILO_TK_RETRIEVE = 10,   /* BM25 block scores and the per-session top blocks */
+    MILO_TK_COUNT = 11
 } milo_timed_stage;
 
 /* on != 0: start recording (previous records are dropped); on == 0: stop.

@@ -533,3 +533,59 @@ def test_decode_offloaded_factors(factor):
     with pytest.raises(milo.MiloError):
         milo.milo_decode_attn_offload(fp, q, sel, pos, rope_base=1e6)
     assert milo.milo_get_status() == milo.MILO_OK
+
+
+def _bm25_rows(tables):
+    blk_ptr, blk_term, blk_tf, blk_len, q_ptr, q_term, q_tf = [x.tolist() for x in tables]
+    blocks = [(blk_term[blk_ptr[b]:blk_ptr[b + 1]], blk_tf[blk_ptr[b]:blk_ptr[b + 1]]) for b in range(len(blk_len))]
+    queries = [(q_term[q_ptr[s]:q_ptr[s + 1]], q_tf[q_ptr[s]:q_ptr[s + 1]]) for s in range(len(q_ptr) - 1)]
+    return blocks, blk_len, queries
+
+
+@pytest.mark.parametrize("name", ["qwen7b-128k", "qwen3b-32k"])
+def test_bm25_select(oracle_mod, name):
+    """GPU BM25 scores against the oracle's (fp64 on both sides; they may
+    differ only through the logarithm's last bit: 1e-13 relative) and the
+    selection: equal to the oracle's wherever the scores leave no near-tie,
+    and always valid (no unselected block scores above a selected one)."""
+    w = synth.WORKLOADS[name]
+    tables = synth.bm25_tables(w)
+    sel, sc = milo.milo_bm25_select(tables, 8192, w.n_sel)
+    assert milo.milo_get_status() == milo.MILO_OK
+    sel, sc = sel.cpu().numpy(), sc.cpu().numpy()
+    blocks, lens, queries = _bm25_rows(tables)
+    ref = oracle_mod.bm25_scores(blocks, lens, queries)
+    assert np.all(np.abs(sc - ref) <= 1e-13 * np.abs(ref).max())
+    ref_sel = oracle_mod.bm25_select(ref, w.n_sel)
+    for s in range(len(queries)):
+        row = ref[s]
+        kth = np.sort(row)[::-1][w.n_sel - 1]
+        near = np.abs(row - kth) <= 1e-12 * np.abs(row).max()
+        if near.sum() == 1:
+            assert sorted(sel[s].tolist()) == sorted(ref_sel[s].tolist())
+        assert len(set(sel[s].tolist())) == w.n_sel
+        unsel = np.setdiff1d(np.arange(len(row)), sel[s])
+        assert row[sel[s]].min() >= row[unsel].max() - 1e-12 * np.abs(row).max()
+
+
+def test_bm25_ties_and_bounds(oracle_mod):
+    """Identical blocks tie exactly and go by the lower id (the oracle's
+    order, bit for bit); a term id out of range sets MILO_ERR_BOUNDS."""
+    blocks = [([1, 2], [1, 3]), ([5], [2]), ([1, 2], [1, 3]), ([7, 1], [4, 1]), ([1, 2], [1, 3])]
+    lens = [40, 40, 40, 40, 40]
+    queries = [([1, 2], [1, 1]), ([5, 7], [1, 2])]
+    flat = lambda rows: torch.tensor([x for r in rows for x in r], dtype=torch.int32)
+    ptr = lambda rows: torch.tensor(np.cumsum([0] + [len(r[0]) for r in rows]).tolist(), dtype=torch.int32)
+    tables = (ptr(blocks), flat([r[0] for r in blocks]), flat([r[1] for r in blocks]),
+              torch.tensor(lens, dtype=torch.int32), ptr(queries), flat([r[0] for r in queries]),
+              flat([r[1] for r in queries]))
+    sel, sc = milo.milo_bm25_select(tables, 16, 3)
+    assert milo.milo_get_status() == milo.MILO_OK
+    ref = oracle_mod.bm25_scores(blocks, lens, queries)
+    assert np.array_equal(sel.cpu().numpy(), oracle_mod.bm25_select(ref, 3))
+    assert np.allclose(sc.cpu().numpy(), ref, rtol=1e-14, atol=0)
+    bad = list(tables)
+    bad[1] = bad[1].clone()
+    bad[1][0] = 99
+    milo.milo_bm25_select(bad, 16, 3)
+    assert milo.milo_get_status() == milo.MILO_ERR_BOUNDS
