@@ -151,6 +151,52 @@ def quant_int8_cols(X):
     return Q, s
 
 
+INT2_GROUP = 32
+
+
+def quant_int2_groups(A, group: int = INT2_GROUP):
+    """2-bit asymmetric codes of a factor A (T_b x r): each rank column in
+    groups of `group` consecutive tokens, zero = the group's min and scale =
+    (max - min) / 3, both stored in fp16, code = clamp(rint((a - zero) /
+    scale), 0, 3) computed with the stored parameters (scale 0: code 0).
+
+    evolve.pub review, Summary and Key claims: MILO composes with INT8 and
+    with KIVI-style low-bit codes.  Reading (KIVI: asymmetric 2-bit, per-channel
+    groups along the tokens): the channels of A are its rank columns.  The
+    arithmetic is fp32 with every operation rounded (the precision in which
+    the codes are decided), parameters rounded to fp16 to nearest even.
+    Returns (codes uint8 [T_b][r], scale fp16 [n_groups][r], zero fp16 [n_groups][r]).
+    """
+    A = np.asarray(A, dtype=np.float32)
+    T, r = A.shape
+    ng = (T + group - 1) // group
+    codes = np.zeros((T, r), dtype=np.uint8)
+    scale = np.zeros((ng, r), dtype=np.float16)
+    zero = np.zeros((ng, r), dtype=np.float16)
+    three = np.float32(3.0)
+    for g in range(ng):
+        rows = A[g * group:min((g + 1) * group, T)]
+        for k in range(r):
+            col = rows[:, k]
+            lo, hi = col.min(), col.max()
+            s16 = np.float16(np.float32(hi - lo) / three)
+            z16 = np.float16(lo)
+            scale[g, k], zero[g, k] = s16, z16
+            s32, z32 = np.float32(s16), np.float32(z16)
+            for i, a in enumerate(col):
+                if s32 > 0:
+                    q = np.rint(np.float32(np.float32(a - z32) / s32))
+                    codes[g * group + i, k] = int(min(max(q, 0.0), 3.0))
+    return codes, scale, zero
+
+
+def dequant_int2_groups(codes, scale, zero, group: int = INT2_GROUP):
+    """zero + code * scale per element (fp64, the fp16 parameters exact)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    g = np.arange(codes.shape[0]) // group
+    return np.asarray(zero, np.float64)[g] + codes * np.asarray(scale, np.float64)[g]
+
+
 def rope(x, pos: float, base: float):
     """RoPE (rotate-half pairs, theta_i = base^(-2i/d)) of one d-vector at pos."""
     y = np.array(x, dtype=np.float64, copy=True)

@@ -482,3 +482,52 @@ def test_bm25_select_brute_force(oracle_mod):
     for n in (1, 7, 40):
         ref = np.stack([np.lexsort((np.arange(40), -row))[:n] for row in scores]).astype(np.int32)
         assert np.array_equal(oracle_mod.bm25_select(scores, n), ref)
+
+
+# ---------------------------------------------------------------- 2-bit codes
+def test_int2_groups_exact_levels_and_constants(oracle_mod):
+    """Groups whose values are exactly the four levels zero + q scale (fp16
+    zero and scale, q = 0..3) come back exactly with those codes; a constant
+    group has scale 0, codes 0 and comes back exactly; a ragged last group
+    uses only its own rows."""
+    rng = np.random.default_rng(41)
+    z, s = np.float16(-1.5), np.float16(0.25)
+    q = rng.integers(0, 4, size=(70, 3))
+    q[0, :] = 0
+    q[1, :] = 3          # every group spans all four levels
+    q[32, :] = 0
+    q[33, :] = 3
+    q[64, :] = 0
+    q[65, :] = 3
+    A = (np.float64(z) + q * np.float64(s)).astype(np.float32)
+    codes, sc, ze = oracle_mod.quant_int2_groups(A)
+    assert sc.shape == (3, 3) and np.all(sc == s) and np.all(ze == z)
+    assert np.array_equal(codes, q.astype(np.uint8))
+    assert np.array_equal(oracle_mod.dequant_int2_groups(codes, sc, ze), A.astype(np.float64))
+    C = np.full((40, 2), 0.375, dtype=np.float32)
+    c2, s2, z2 = oracle_mod.quant_int2_groups(C)
+    assert np.all(c2 == 0) and np.all(s2 == 0) and np.all(oracle_mod.dequant_int2_groups(c2, s2, z2) == 0.375)
+
+
+def test_int2_groups_nearest_level_brute_force(oracle_mod):
+    """Every code is the nearest of the four levels of its group's stored
+    parameters (brute force over q = 0..3, within fp32 rounding of the
+    division), the group's min takes code 0 and its max code 3, and the error
+    is at most half a step plus the fp16 rounding of the parameters."""
+    rng = np.random.default_rng(42)
+    A = (rng.standard_normal((200, 5)) * np.array([0.01, 1.0, 30.0, 300.0, 5.0])).astype(np.float32)
+    codes, sc, ze = oracle_mod.quant_int2_groups(A)
+    deq = oracle_mod.dequant_int2_groups(codes, sc, ze)
+    for t in range(200):
+        g = t // 32
+        for k in range(5):
+            s, z = float(sc[g, k]), float(ze[g, k])
+            levels = z + np.arange(4) * s
+            best = np.abs(levels - float(A[t, k])).min()
+            assert abs(deq[t, k] - float(A[t, k])) <= best + 1e-6 * s
+    for g in range(7):
+        rows = slice(32 * g, min(32 * g + 32, 200))
+        for k in range(5):
+            assert codes[rows, k][np.argmin(A[rows, k])] == 0 and codes[rows, k][np.argmax(A[rows, k])] == 3
+            rng_ = float(A[rows, k].max() - A[rows, k].min())
+            assert np.abs(deq[rows, k] - A[rows, k]).max() <= rng_ / 6 * (1 + 2e-3) + abs(float(ze[g, k]) - float(A[rows, k].min()))
