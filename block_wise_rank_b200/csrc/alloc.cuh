@@ -74,6 +74,7 @@ struct SelArgs {
 struct SelShape {
     int n_b, T, block_len, r_min, r_max;
     int64_t n_blk;
+    int dtype;   // factor type of the offsets written (their unit: block_units)
 };
 
 // key bits of component k of block blk ((sigma/eps)^2 as a double, 0 if eps <= 0)
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
         const int r = k0 + a.gt[i] + (int)take;
         a.ranks[i] = r;
         const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
-        elems += block_elems(r, tb);
+        elems += block_units(sh.dtype, r, tb);
     }
     if (a.offsets == nullptr) return;
     sB[tid] = elems;
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
     for (int64_t i = lo; i < hi; ++i) {
         a.offsets[i] = off;
         const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
-        off += block_elems(a.ranks[i], tb);
+        off += block_units(sh.dtype, a.ranks[i], tb);
     }
     if (hi == n && lo < hi) a.offsets[n] = off;
     if (n == 0 && tid == 0) a.offsets[0] = 0;

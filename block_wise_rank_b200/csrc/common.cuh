@@ -58,6 +58,7 @@ __device__ __forceinline__ float load_elem(const void *base, int64_t i, int dtyp
     }
 }
 
+// bytes of one offset unit of the factor data (elements; bytes for 2-bit codes)
 __host__ __device__ __forceinline__ int dtype_bytes(int dtype) {
     return dtype == MILO_F32 ? 4 : (dtype == MILO_BF16 ? 2 : 1);
 }
@@ -84,6 +85,24 @@ __host__ __device__ __forceinline__ int64_t a_index(int R8, int t, int k) {
 // B_b[k][j] (rank k, channel j)
 __host__ __device__ __forceinline__ int64_t b_index(int R8, int n_tiles, int k, int j) {
     return (int64_t)n_tiles * R8 * FTILE + (k >> 3) * (8 * D) + (j >> 3) * 64 + (k & 7) * 8 + (j & 7);
+}
+
+// 2-bit factors (MILO_INT2), byte offsets from the block start: A_b's codes
+// four tokens per byte at a_index / 4 (token u at bits 2 (u % 4)); B_b's
+// INT8 codes after them at b_index - nt R8 FTILE; then A_b's (scale, zero)
+// fp16 pairs per rank k and group of INT2_GROUP tokens, [k][t / INT2_GROUP].
+constexpr int INT2_GROUP = 32;
+__host__ __device__ __forceinline__ int64_t int2_b_off(int R8, int nt) { return (int64_t)nt * R8 * (FTILE / 4); }
+__host__ __device__ __forceinline__ int64_t int2_param_off(int R8, int nt) {
+    return int2_b_off(R8, nt) + (int64_t)R8 * D;
+}
+__host__ __device__ __forceinline__ int64_t int2_block_bytes(int r, int Tb) {
+    const int R8 = rank_pad(r), nt = token_tiles(Tb);
+    return int2_param_off(R8, nt) + (int64_t)R8 * nt * (FTILE / INT2_GROUP) * 4;
+}
+// a block's size in offset units of its factor type
+__host__ __device__ __forceinline__ int64_t block_units(int dtype, int r, int Tb) {
+    return dtype == MILO_INT2 ? int2_block_bytes(r, Tb) : block_elems(r, Tb);
 }
 
 // One kind's section of the factor arena (device pointers).

@@ -10,9 +10,9 @@
 //
 // The arena keeps its layout (ranks, offsets, scales, data per kind) in pinned,
 // device-mapped host memory.  Per call: flag the block ids some session
-// selected; size each (layer, head, block) of those in elements (0 for the
-// rest) and scan the sizes into staging offsets; copy the flagged blocks'
-// factors (and INT8 scales) from host memory into the staging area with
+// selected; size each (layer, head, block) of those in offset units (0 for
+// the rest) and scan the sizes into staging offsets; copy the flagged blocks'
+// factors (and the INT8 / 2-bit scales) from host memory into the staging area with
 // 16-byte loads (one CTA per block).  The staged copy is indexed by the
 // original block ids, so the decode kernels run on it unchanged.
 #pragma once
@@ -29,59 +29,26 @@ __global__ void k_flag_selected(const int32_t *__restrict__ sel, int n_slots, in
     }
 }
 
-// elements of every (layer, head, block) of one kind in the staging area:
-// the block's factors when its id is flagged, else 0; the ranks are copied
-// for every block.  grid over nblk.
+// size (offset units of the factor type) of every (layer, head, block) of one
+// kind in the staging area: the block's factors when its id is flagged, else
+// 0; the ranks are copied for every block.  grid over nblk.
 __global__ void k_stage_sizes(const int32_t *__restrict__ host_ranks, const int32_t *__restrict__ used, int64_t nblk,
-                              int n_b, int T, int block_len, int64_t *__restrict__ sizes,
+                              int n_b, int T, int block_len, int dtype, int64_t *__restrict__ sizes,
                               int32_t *__restrict__ ranks) {
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
          blk += (int64_t)gridDim.x * blockDim.x) {
         const int b = (int)(blk % n_b);
         const int r = host_ranks[blk];
         ranks[blk] = r;
-        sizes[blk] = used[b] ? block_elems(r, block_tokens(T, block_len, b)) : 0;
+        sizes[blk] = used[b] ? block_units(dtype, r, block_tokens(T, block_len, b)) : 0;
     }
-}
-
-// Exclusive prefix sum of n int64 values in place (one CTA of 1024 threads);
-// v[n] receives the total.
-__global__ void __launch_bounds__(SCAN_THREADS) k_scan_i64(int64_t *__restrict__ v, int64_t n) {
-    __shared__ long long wsum[SCAN_THREADS / 32];
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int64_t chunk = (n + SCAN_THREADS - 1) / SCAN_THREADS;
-    const int64_t b0 = min(n, (int64_t)tid * chunk), b1 = min(n, b0 + chunk);
-    long long mine = 0;
-    for (int64_t b = b0; b < b1; ++b) mine += v[b];
-    long long inc = mine;
-    for (int o = 1; o < 32; o <<= 1) {
-        const long long x = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += x;
-    }
-    if (lane == 31) wsum[wid] = inc;
-    __syncthreads();
-    if (wid == 0) {
-        long long w = wsum[lane];
-        for (int o = 1; o < 32; o <<= 1) {
-            const long long x = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += x;
-        }
-        wsum[lane] = w;
-    }
-    __syncthreads();
-    long long acc = inc - mine + (wid > 0 ? wsum[wid - 1] : 0);
-    for (int64_t b = b0; b < b1; ++b) {
-        const long long c = v[b];
-        v[b] = acc;
-        acc += c;
-    }
-    if (tid == SCAN_THREADS - 1) v[n] = wsum[31];
 }
 
 // One CTA per (layer, head, block): the flagged blocks' factors from the
-// host arena (device-mapped pointers) to the staging area, and their INT8
-// scales.  Offsets are in elements; every block starts on a multiple of
-// 1024 elements, so 16-byte vectors tile it exactly.
+// host arena (device-mapped pointers) to the staging area, and their scales.
+// Offsets count offset units of esize bytes; every block's size is a
+// multiple of 16 bytes (1024 elements, or 16 bytes of 2-bit codes), so
+// 16-byte vectors tile it exactly.
 __global__ void __launch_bounds__(256) k_stage_copy(KindView host, KindView stage, const int32_t *__restrict__ used,
                                                     int n_b, int esize) {
     const int64_t blk = blockIdx.x;
@@ -98,9 +65,9 @@ __global__ void __launch_bounds__(256) k_stage_copy(KindView host, KindView stag
         dst[e + 768] = a3;
     }
     for (; e < n16; e += 256) dst[e] = __ldg(src + e);
-    if (host.scaleA && threadIdx.x < D) {
-        stage.scaleA[blk * D + threadIdx.x] = host.scaleA[blk * D + threadIdx.x];
-        stage.scaleB[blk * D + threadIdx.x] = host.scaleB[blk * D + threadIdx.x];
+    if (threadIdx.x < D) {
+        if (host.scaleA) stage.scaleA[blk * D + threadIdx.x] = host.scaleA[blk * D + threadIdx.x];
+        if (host.scaleB) stage.scaleB[blk * D + threadIdx.x] = host.scaleB[blk * D + threadIdx.x];
     }
 }
 

@@ -120,6 +120,40 @@ __global__ void k_slot_fill(const int32_t *__restrict__ sel, int n_slots, int n_
     }
 }
 
+// Exclusive prefix sum of n int64 values in place (one CTA of 1024 threads);
+// v[n] receives the total.
+__global__ void __launch_bounds__(SCAN_THREADS) k_scan_i64(int64_t *__restrict__ v, int64_t n) {
+    __shared__ long long wsum[SCAN_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t chunk = (n + SCAN_THREADS - 1) / SCAN_THREADS;
+    const int64_t b0 = min(n, (int64_t)tid * chunk), b1 = min(n, b0 + chunk);
+    long long mine = 0;
+    for (int64_t b = b0; b < b1; ++b) mine += v[b];
+    long long inc = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+    }
+    if (lane == 31) wsum[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        long long w = wsum[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long x = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += x;
+        }
+        wsum[lane] = w;
+    }
+    __syncthreads();
+    long long acc = inc - mine + (wid > 0 ? wsum[wid - 1] : 0);
+    for (int64_t b = b0; b < b1; ++b) {
+        const long long c = v[b];
+        v[b] = acc;
+        acc += c;
+    }
+    if (tid == SCAN_THREADS - 1) v[n] = wsum[31];
+}
+
 // Tensor-core path: query passes of every block id, ceil(slots x G / pass_q).
 __global__ void k_pass_counts(const int32_t *__restrict__ start, int n_b, int G, int pass_q,
                               int32_t *__restrict__ passes) {

@@ -1195,11 +1195,71 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
     if (warp == 1) tc::tmem_dealloc(tmem, DT_TMEM_COLS);
 }
 
+// Element sizes (the bf16 layout of common.cuh) of every block, for the fp16
+// copy of 2-bit factors; scanned into its element offsets.  grid over nblk.
+__global__ void k_elem_sizes(const int32_t *__restrict__ ranks, int64_t nblk, int n_b, int T, int block_len,
+                             int64_t *__restrict__ sizes) {
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
+         blk += (int64_t)gridDim.x * blockDim.x)
+        sizes[blk] = block_elems(ranks[blk], block_tokens(T, block_len, (int)(blk % n_b)));
+}
+
+// 2-bit factors for the tensor cores: the selected blocks' A codes as zero +
+// code * scale of their (rank, 32-token group) and B's INT8 codes times the
+// channel scale, rounded to fp16, written at the element offsets eoff of the
+// bf16 layout into `out` (one section per kind).  Grid (L*H*n_b, 2); blocks no
+// slot selected are skipped.
+__global__ void __launch_bounds__(256) k_dequant_int2(DecodeArgs a, const int64_t *__restrict__ eoff0,
+                                                      const int64_t *__restrict__ eoff1, __half *out0,
+                                                      __half *out1) {
+    const int64_t blk = blockIdx.x;
+    const int kind = blockIdx.y;
+    const int b = (int)(blk % a.n_b);
+    if (a.slot_start[b + 1] == a.slot_start[b]) return;
+    const KindView &kv = a.kv[kind];
+    const int R8 = rank_pad(kv.ranks[blk]);
+    if (R8 == 0) return;
+    const int nt = token_tiles(block_tokens(a.T, a.block_len, b));
+    const int64_t nA = (int64_t)nt * R8 * FTILE, nAll = nA + (int64_t)R8 * D;
+    const uint8_t *src = (const uint8_t *)kv.data + kv.offsets[blk];
+    __half *dst = (kind ? out1 : out0) + (kind ? eoff1 : eoff0)[blk];
+    const __half2 *prm = reinterpret_cast<const __half2 *>(src + int2_param_off(R8, nt));
+    const float *sB = kv.scaleB + blk * D;
+    for (int64_t e = (int64_t)threadIdx.x * 8; e < nAll; e += 256 * 8) {   // one core-matrix row
+        float v[8];
+        if (e < nA) {   // A tile: [k/8][u/8][k%8][u%8], eight tokens of rank k
+            const int tau = (int)(e / (R8 * FTILE));
+            const int r = (int)(e % (R8 * FTILE));
+            const int k = (r >> 10) * 8 + ((r >> 3) & 7), t0 = tau * FTILE + ((r >> 6) & 15) * 8;
+            const float2 sz = __half22float2(prm[(int64_t)k * (4 * nt) + t0 / INT2_GROUP]);   // (scale, zero)
+            const uint32_t codes = *reinterpret_cast<const uint16_t *>(src + (e >> 2));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = fmaf((float)((codes >> (2 * i)) & 3u), sz.x, sz.y);
+        } else {        // B: [k/8][j/8][k%8][j%8], INT8 codes of eight channels
+            const int64_t r = e - nA;
+            const int j0 = (int)((r & 1023) >> 6) * 8;
+            const uint2 q8 = *reinterpret_cast<const uint2 *>(src + int2_b_off(R8, nt) + r);
+            const int8_t *c = reinterpret_cast<const int8_t *>(&q8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = (float)c[i] * sB[j0 + i];
+        }
+        uint4 o;
+        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+            ow[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(dst + e) = o;
+    }
+}
+
 inline size_t decode_tc_smem_bytes() { return sizeof(DecTcSmem) + 128; }
 
 inline bool decode_tc_supported(const DecodeArgs &a) {
-    if (getenv("MILO_FORCE_SIMT")) return false;
-    return (a.factor_dtype == MILO_BF16 || a.factor_dtype == MILO_INT8) && a.block_len <= 512;
+    if (getenv("MILO_FORCE_SIMT") && a.factor_dtype != MILO_INT2) return false;   // 2-bit: no CUDA-core path
+    return (a.factor_dtype == MILO_BF16 || a.factor_dtype == MILO_INT8 || a.factor_dtype == MILO_INT2) &&
+           a.block_len <= 512;
 }
 
 // INT8 factors for the tensor cores: the selected blocks' factors of both

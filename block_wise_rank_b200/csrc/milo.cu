@@ -121,11 +121,17 @@ SectionLayout section_layout(const milo_cache_shape *s, const milo_compress_para
         at = align_up(at + sizeof(float) * nblk * D);
         o.scaleB = at;
         at = align_up(at + sizeof(float) * nblk * D);
+    } else if (p->factor_dtype == MILO_INT2) {   // B's scales only (A's travel with its codes)
+        at = align_up(at + sizeof(float) * nblk * D);
     }
     o.data = at;
     // sum_b round_up(r_b, 8) (128 ceil(T_b/128) + d) <= (R + 7 N_blk) (128 ceil(block_len/128) + d)
-    at = align_up(at + (size_t)(R + 7 * nblk) * (size_t)(round_up(s->block_len, FTILE) + D) *
-                           dtype_bytes(p->factor_dtype));
+    // elements; 2-bit: sum_b R8 (48 ceil(T_b/128) + d) bytes
+    if (p->factor_dtype == MILO_INT2)
+        at = align_up(at + (size_t)(R + 7 * nblk) * (size_t)(48 * (round_up(s->block_len, FTILE) / FTILE) + D));
+    else
+        at = align_up(at + (size_t)(R + 7 * nblk) * (size_t)(round_up(s->block_len, FTILE) + D) *
+                               dtype_bytes(p->factor_dtype));
     o.bytes = at;
     return o;
 }
@@ -138,8 +144,9 @@ void fill_views(milo_factors *f) {
         f->kv[k].offsets = (int64_t *)(base + o.offsets);
         f->kv[k].sigma = (float *)(base + o.sigma);
         f->kv[k].eps = (double *)(base + o.eps);
-        f->kv[k].scaleA = f->params.factor_dtype == MILO_INT8 ? (float *)(base + o.scaleA) : nullptr;
-        f->kv[k].scaleB = f->params.factor_dtype == MILO_INT8 ? (float *)(base + o.scaleB) : nullptr;
+        const int dt = f->params.factor_dtype;
+        f->kv[k].scaleA = dt == MILO_INT8 ? (float *)(base + o.scaleA) : nullptr;
+        f->kv[k].scaleB = dt == MILO_INT8 || dt == MILO_INT2 ? (float *)(base + o.scaleB) : nullptr;
         f->kv[k].data = base + o.data;
     }
 }
@@ -147,7 +154,8 @@ void fill_views(milo_factors *f) {
 milo_status params_ok(const milo_cache_shape *s, const milo_compress_params *p, int64_t *R_out) {
     if (!shape_ok(s) || !p) return MILO_ERR_INVALID_ARG;
     if (s->d != D) return MILO_ERR_UNSUPPORTED;
-    if (p->factor_dtype != MILO_F32 && p->factor_dtype != MILO_BF16 && p->factor_dtype != MILO_INT8)
+    if (p->factor_dtype != MILO_F32 && p->factor_dtype != MILO_BF16 && p->factor_dtype != MILO_INT8 &&
+        p->factor_dtype != MILO_INT2)
         return MILO_ERR_INVALID_ARG;
     if (p->r_min < 0 || p->r_max < 0 || p->eps_scope < 0 || p->eps_scope > 1 || !(p->eps_rel >= 0.0))
         return MILO_ERR_INVALID_ARG;
@@ -404,7 +412,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     // 4. global top-R selection, ranks and packed offsets
     int64_t caps, floors;
     cap_sums(shape, p.r_min, p.r_max, caps, floors);
-    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk};
+    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk, (int)p.factor_dtype};
     SelArgs a[2];
     for (int k = 0; k < 2; ++k) {
         a[k].sigma = f->kv[k].sigma;
@@ -468,7 +476,7 @@ milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_group
     cap_sums(&shp, r_min, r_max, caps, floors);
     if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
     AllocScratch as = alloc_scratch(workspace, nblk);
-    SelShape sh{n_b, T, block_len, r_min, r_max, nblk};
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32};
     SelArgs a{};
     a.sigma = sigma;
     a.eps = eps;
@@ -555,7 +563,7 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
     if (!scratch) return MILO_ERR_CUDA;
     // the scratch layout for kNoAllocBlocks also holds any smaller problem
     AllocScratch as = alloc_scratch(scratch, kNoAllocBlocks);
-    SelShape sh{n_b, T, block_len, r_min, r_max, nblk};
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32};
     SelArgs a{};
     a.sigma = sigma;
     a.eps = eps;
@@ -571,7 +579,7 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
 // INT8 factors on the tensor cores: an fp16 copy of each kind's data section
 // (the selected blocks' elements are written, at the INT8 element offsets).
 static size_t shadow_bytes_per_kind(const milo_factors *f) {
-    if (f->params.factor_dtype != MILO_INT8) return 0;
+    if (f->params.factor_dtype != MILO_INT8 && f->params.factor_dtype != MILO_INT2) return 0;
     return align_up(sizeof(__half) * (size_t)(f->R + 7 * f->n_blk) *
                     (size_t)(round_up(f->shape.block_len, FTILE) + D));
 }
@@ -588,7 +596,9 @@ size_t milo_decode_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, 
     at = align_up(at + sizeof(float2) * rows * n_sel);                 // partial (m, l)
     at = align_up(at + sizeof(DtItem) * decode_tc_max_items(f->shape.L, f->shape.H, f->n_b, slots,
                                                             Hq / f->shape.H));  // tensor-core work items
-    at += 2 * shadow_bytes_per_kind(f);                                 // INT8: fp16 factors
+    at += 2 * shadow_bytes_per_kind(f);                                 // INT8 / 2-bit: fp16 factors
+    if (f->params.factor_dtype == MILO_INT2)                           // 2-bit: element offsets of the fp16 copy
+        at += 2 * align_up(sizeof(int64_t) * (f->n_blk + 1));
     return at;
 }
 
@@ -616,6 +626,8 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
     if (Hq % f->shape.H != 0 || !(rope_base > 0.0)) return MILO_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, kAlign) || !aligned(selected, 4))
         return MILO_ERR_INVALID_ARG;
+    // 2-bit factors decode on the tensor cores only (blocks of at most 512 tokens)
+    if (f->params.factor_dtype == MILO_INT2 && f->shape.block_len > 512) return MILO_ERR_UNSUPPORTED;
     const size_t ws_dec = milo_decode_workspace_size(f, S, Hq, n_sel);
     if (ws_bytes < ws_dec + (tail.k ? tail_workspace_bytes(f, S, Hq) : 0)) return MILO_ERR_WORKSPACE;
     milo_status st = set_smem_attrs();
@@ -642,6 +654,8 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
                                                             Hq / f->shape.H));
     __half *shadow0 = (__half *)(w + at);
     __half *shadow1 = (__half *)(w + at + shadow_bytes_per_kind(f));
+    int64_t *eoff0 = (int64_t *)(w + at + 2 * shadow_bytes_per_kind(f));
+    int64_t *eoff1 = (int64_t *)((char *)eoff0 + align_up(sizeof(int64_t) * (f->n_blk + 1)));
 
     DecodeArgs a{};
     a.kv[0] = f->kv[0];
@@ -679,6 +693,18 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
             k_dequant_selected<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, shadow0, shadow1);
             a.kv[0].data = shadow0;
             a.kv[1].data = shadow1;
+            a.f16 = 1;
+        } else if (a.factor_dtype == MILO_INT2) {   // the same, into the bf16 layout's element offsets
+            const int eg = (int)std::min<int64_t>((f->n_blk + 255) / 256, 4096);
+            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[0].ranks, f->n_blk, n_b, f->shape.T, f->shape.block_len, eoff0);
+            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[1].ranks, f->n_blk, n_b, f->shape.T, f->shape.block_len, eoff1);
+            k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(eoff0, f->n_blk);
+            k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(eoff1, f->n_blk);
+            k_dequant_int2<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, eoff0, eoff1, shadow0, shadow1);
+            a.kv[0].data = shadow0;
+            a.kv[1].data = shadow1;
+            a.kv[0].offsets = eoff0;
+            a.kv[1].offsets = eoff1;
             a.f16 = 1;
         }
         // work items: passes of up to DT_NQ queries per block id (counts reuse cnt)
@@ -739,12 +765,13 @@ OffloadLayout offload_layout(const milo_factors *f, size_t at) {
     OffloadLayout o{};
     const SectionLayout sec = section_layout(&f->shape, &f->params, f->R);
     const bool i8 = f->params.factor_dtype == MILO_INT8;
+    const bool sB = i8 || f->params.factor_dtype == MILO_INT2;   // B's scales
     o.used = at; at = align_up(at + sizeof(int32_t) * (f->n_b + 1));
     for (int k = 0; k < 2; ++k) {
         o.sizes[k] = at; at = align_up(at + sizeof(int64_t) * (f->n_blk + 1));
         o.ranks[k] = at; at = align_up(at + sizeof(int32_t) * f->n_blk);
         o.scaleA[k] = at; at = align_up(at + (i8 ? sizeof(float) * f->n_blk * D : 0));
-        o.scaleB[k] = at; at = align_up(at + (i8 ? sizeof(float) * f->n_blk * D : 0));
+        o.scaleB[k] = at; at = align_up(at + (sB ? sizeof(float) * f->n_blk * D : 0));
         o.data[k] = at; at = align_up(at + (sec.bytes - sec.data));   // every block selected at most
     }
     o.bytes = at;
@@ -813,7 +840,8 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
         sv.scaleB = host.scaleB ? (float *)(w + o.scaleB[k]) : nullptr;
         sv.data = w + o.data[k];
         k_stage_sizes<<<(int)std::min<int64_t>((f->n_blk + 255) / 256, 4096), 256, 0, s>>>(
-            host.ranks, used, f->n_blk, f->n_b, f->shape.T, f->shape.block_len, sv.offsets, sv.ranks);
+            host.ranks, used, f->n_blk, f->n_b, f->shape.T, f->shape.block_len, f->params.factor_dtype, sv.offsets,
+            sv.ranks);
         k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(sv.offsets, f->n_blk);
         k_stage_copy<<<(unsigned)f->n_blk, 256, 0, s>>>(host, sv, used, f->n_b, esize);
     }

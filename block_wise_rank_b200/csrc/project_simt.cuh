@@ -7,6 +7,10 @@
 // arena in the tiled layout of common.cuh (A_b^T tiles, then B_b).  INT8 composition
 // (same page, Summary: combined with INT8 quantisation): symmetric per-column
 // absmax codes, scale = absmax / 127, round half to even, clamp to +-127.
+// 2-bit composition (same page, Key claims: KIVI-style low-bit codes): A_b's
+// rank columns in groups of INT2_GROUP tokens, zero = min, scale = (max -
+// min) / 3 in fp16, code = clamp(rint((a - zero) / scale), 0, 3) decided in
+// fp32 with the stored parameters; B_b in INT8.
 #pragma once
 #include "common.cuh"
 
@@ -76,6 +80,35 @@ __global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
                     if (c < kc) atomicMax((int *)&amax[c], __float_as_int(fabsf(acc[c])));
+            } else if (pa.out_dtype == MILO_INT2) {
+                // a warp holds the 32 consecutive tokens of one group (ldT is a
+                // multiple of 128 and t = 32 w + lane + 256 i)
+                uint8_t *blkp = (uint8_t *)kv.data + base;
+                const int lane = threadIdx.x & 31, g = t / INT2_GROUP, nt = ldT / FTILE;
+                for (int c = 0; c < kw; ++c) {
+                    const bool live = t < Tb && c < kc;
+                    const float a = acc[c];
+                    float lo = live ? a : INFINITY, hi = live ? a : -INFINITY;
+                    for (int o = 16; o; o >>= 1) {
+                        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                    }
+                    __half sh = __float2half_rn(0.f), zh = sh;   // no live token: 0, 0
+                    if (lo <= hi) {
+                        sh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 3.f));
+                        zh = __float2half_rn(lo);
+                    }
+                    const float s32 = __half2float(sh), z32 = __half2float(zh);
+                    int q = 0;
+                    if (live && s32 > 0.f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(a, z32), s32)), 0.f), 3.f);
+                    int byte = q << (2 * (lane & 3));   // four consecutive tokens per byte
+                    byte |= __shfl_xor_sync(0xffffffffu, byte, 1);
+                    byte |= __shfl_xor_sync(0xffffffffu, byte, 2);
+                    if ((lane & 3) == 0) blkp[a_index(R8, t, k0 + c) >> 2] = (uint8_t)byte;
+                    if (lane == 0)
+                        *reinterpret_cast<__half2 *>(blkp + int2_param_off(R8, nt) +
+                                                     4 * ((int64_t)(k0 + c) * (4 * nt) + g)) = __halves2half2(sh, zh);
+                }
             } else {
                 for (int c = 0; c < kw; ++c) {
                     const int64_t o = base + a_index(R8, t, k0 + c);
@@ -105,7 +138,8 @@ __global__ void __launch_bounds__(128) k_project_b(ProjArgs pa) {
     const int64_t base = kv.offsets[blk];
     const float *Wb = pa.W[kind] + (int64_t)blk * D * D + (int64_t)j * D;
     float s = 0.f;
-    if (pa.out_dtype == MILO_INT8) {
+    const bool i8 = pa.out_dtype == MILO_INT8 || pa.out_dtype == MILO_INT2;   // B is INT8 in both
+    if (i8) {
         float m = 0.f;
         for (int k = 0; k < r; ++k) m = fmaxf(m, fabsf(Wb[k]));
         s = __fdiv_rn(m, 127.f);
@@ -113,8 +147,10 @@ __global__ void __launch_bounds__(128) k_project_b(ProjArgs pa) {
     }
     for (int k = 0; k < R8; ++k) {
         const float w = k < r ? Wb[k] : 0.f;
-        const int64_t o = base + b_index(R8, nt, k, j);
-        if (pa.out_dtype == MILO_INT8) ((int8_t *)kv.data)[o] = quant_i8(w, s);
+        const int64_t o = pa.out_dtype == MILO_INT2
+                              ? base + int2_b_off(R8, nt) + (b_index(R8, nt, k, j) - (int64_t)nt * R8 * FTILE)
+                              : base + b_index(R8, nt, k, j);
+        if (i8) ((int8_t *)kv.data)[o] = quant_i8(w, s);
         else if (pa.out_dtype == MILO_BF16) ((__nv_bfloat16 *)kv.data)[o] = __float2bfloat16_rn(w);
         else ((float *)kv.data)[o] = w;
     }

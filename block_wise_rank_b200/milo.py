@@ -26,8 +26,8 @@ MILO_ERR_NONFINITE = -5
 MILO_ERR_BOUNDS = -6
 MILO_ERR_TIMEOUT = -7
 
-MILO_F32, MILO_BF16, MILO_INT8 = 0, 1, 2
-DTYPES = {"f32": MILO_F32, "bf16": MILO_BF16, "int8": MILO_INT8}
+MILO_F32, MILO_BF16, MILO_INT8, MILO_INT2 = 0, 1, 2, 3
+DTYPES = {"f32": MILO_F32, "bf16": MILO_BF16, "int8": MILO_INT8, "int2": MILO_INT2}
 
 
 class milo_cache_shape(ctypes.Structure):

@@ -59,7 +59,9 @@ typedef enum {
     MILO_ERR_TIMEOUT = -7          /* a bounded wait on the device ran out    */
 } milo_status;
 
-typedef enum { MILO_F32 = 0, MILO_BF16 = 1, MILO_INT8 = 2 } milo_dtype;
+/* MILO_INT2: factor codes only (A_b in 2 bits per element, B_b in INT8; see
+ * the arena layout below). */
+typedef enum { MILO_F32 = 0, MILO_BF16 = 1, MILO_INT8 = 2, MILO_INT2 = 3 } milo_dtype;
 
 /* A KV cache of one kind: [L][H][T][d] row-major (d contiguous). */
 typedef struct {
@@ -84,7 +86,7 @@ typedef struct {
     /* Rank bounds per block: r_min <= r_b <= min(T_b, d, r_max or d). */
     int32_t r_min;
     int32_t r_max;                /* 0 means no cap beyond min(T_b, d) */
-    milo_dtype factor_dtype;      /* MILO_F32, MILO_BF16 or MILO_INT8  */
+    milo_dtype factor_dtype;      /* MILO_F32, MILO_BF16, MILO_INT8 or MILO_INT2 */
     int32_t max_sweeps;           /* Jacobi sweep cap (0 -> 24)        */
     float jacobi_tol;             /* rotate while |g_pq| > tol*sqrt(g_pp g_qq) (0 -> 1e-7) */
 } milo_compress_params;
@@ -97,11 +99,11 @@ typedef struct milo_factors milo_factors;
  * each section start 256-byte aligned; N_blk = L*H*n_b, n_b = ceil(T /
  * block_len)):
  *   int32  ranks  [N_blk]
- *   int64  offsets[N_blk + 1]   element offset of block b in data
+ *   int64  offsets[N_blk + 1]   element offset of block b in data (bytes for MILO_INT2)
  *   float  sigma  [N_blk][d]    singular values, descending
  *   double eps    [L*H]
  *   float  scaleA [N_blk][d]    INT8 only: scale of column k of A_b
- *   float  scaleB [N_blk][d]    INT8 only: scale of column j of B_b
+ *   float  scaleB [N_blk][d]    INT8 and INT2: scale of column j of B_b
  *   elem   data   [...]         elem = factor dtype
  * A_b = U_r Sigma_r (T_b x r_b) and B_b = V_r^T (r_b x d), so X_b ~ A_b B_b.
  * Block b occupies R8 * (128 * nt + d) elements at data + offsets[b], with
@@ -114,6 +116,16 @@ typedef struct milo_factors milo_factors;
  * layout, so that each 128-token tile of A_b and the whole of B_b are single
  * contiguous copies.  The data section holds at most
  * (R + 7 N_blk) * (128 * ceil(block_len / 128) + d) elements.
+ *
+ * MILO_INT2 (evolve.pub review, Summary and Key claims: MILO composes with
+ * KIVI-style low-bit codes): A_b in 2-bit asymmetric codes per rank column k
+ * and group of 32 tokens g -- zero z = the group's min, scale s = (max - min)
+ * / 3, both fp16, code = clamp(rint((a - z) / s), 0, 3) in fp32 (0 when s =
+ * 0), a = z + code * s -- and B_b in INT8 as above.  Block b occupies
+ * R8 * (48 * nt + d) bytes: the codes of A_b at byte (index of A_b[t][k]
+ * above) / 4, bits 2*(u%4) (four consecutive tokens per byte); B_b's INT8
+ * codes at byte nt*R8*32 + (index of B_b[k][j] above) - nt*R8*128; then the
+ * (s, z) fp16 pairs at byte nt*R8*32 + R8*d + 4 * (k * 4*nt + t / 32).
  */
 
 /* ----------------------------------------------------------------- sizes */

@@ -67,7 +67,7 @@ def unpack(f: milo.Factors, kind: int):
 
     Returns dict(ranks [n_blk], offsets [n_blk+1], sigma [n_blk][d],
     eps [L*H], A[blk] (T_b x r fp64), B[blk] (r x d fp64), Aq/Bq raw codes and
-    scales for INT8).
+    scales for INT8; for 2-bit factors also A_scale / A_zero [n_groups][r]).
     """
     (p_r, p_o, p_s, p_e, p_d, p_sa, p_sb), R = f.view(kind)
     sh, pr = f.shape, f.params
@@ -79,24 +79,48 @@ def unpack(f: milo.Factors, kind: int):
     sigma = arena_tensor(f, p_s, 4 * nblk * d).view(torch.float32).cpu().numpy().reshape(nblk, d).copy()
     eps = arena_tensor(f, p_e, 8 * L * H).view(torch.float64).cpu().numpy().copy()
     dt = pr.factor_dtype
-    es = {milo.MILO_F32: 4, milo.MILO_BF16: 2, milo.MILO_INT8: 1}[dt]
+    es = {milo.MILO_F32: 4, milo.MILO_BF16: 2, milo.MILO_INT8: 1, milo.MILO_INT2: 1}[dt]
     total = int(offs[-1])
     raw = arena_tensor(f, p_d, es * total) if total else torch.zeros(0, dtype=torch.uint8, device=f.arena.device)
     if dt == milo.MILO_F32:
         data = raw.view(torch.float32).cpu().numpy().astype(np.float64)
     elif dt == milo.MILO_BF16:
         data = raw.view(torch.bfloat16).float().cpu().numpy().astype(np.float64)
-    else:
+    elif dt == milo.MILO_INT8:
         data = raw.view(torch.int8).cpu().numpy().astype(np.float64)
+    else:
+        data = raw.cpu().numpy()
     sA = sB = None
     if dt == milo.MILO_INT8:
         sA = arena_tensor(f, p_sa, 4 * nblk * d).view(torch.float32).cpu().numpy().reshape(nblk, d).copy()
+    if dt in (milo.MILO_INT8, milo.MILO_INT2):
         sB = arena_tensor(f, p_sb, 4 * nblk * d).view(torch.float32).cpu().numpy().reshape(nblk, d).copy()
-    A, B, Aq, Bq = [], [], [], []
+    A, B, Aq, Bq, A_scale, A_zero = [], [], [], [], [], []
     for blk in range(nblk):
         b = blk % nb
         tb = min(bl, T - b * bl)
         r = int(ranks[blk])
+        if dt == milo.MILO_INT2:
+            # codes four per byte (token u%4 at bits 2(u%4)), then B's INT8
+            # codes, then (scale, zero) fp16 per rank and 32-token group
+            R8, nt = padded_rank(r), tiles(tb)
+            reg = data[int(offs[blk]):int(offs[blk + 1])]
+            assert reg.size == R8 * (48 * nt + d)
+            nc = nt * R8 * 32
+            codes = ((reg[:nc, None] >> (2 * np.arange(4))[None, :]) & 3).reshape(-1).astype(np.float64)
+            b8 = reg[nc:nc + R8 * d].view(np.int8).astype(np.float64)
+            prm = reg[nc + R8 * d:].view(np.float16).astype(np.float64).reshape(R8, 4 * nt, 2)
+            At, Bm = untile(np.concatenate([codes, b8]), r, tb, d)
+            grp = np.arange(tb) // 32
+            Aq.append(At[:r, :tb].T.copy())
+            Bq.append(Bm[:r].copy())
+            A_scale.append(prm[:r, :, 0].T.copy())
+            A_zero.append(prm[:r, :, 1].T.copy())
+            A.append(prm[:r, grp, 1].T + At[:r, :tb].T * prm[:r, grp, 0].T)
+            B.append(Bm[:r] * sB[blk].astype(np.float64)[None, :])
+            assert np.all(At[r:] == 0) and np.all(At[:, tb:] == 0), "code padding must be zero"
+            assert np.all(Bm[r:] == 0), "B padding rows must be zero"
+            continue
         At, Bm = untile(data[int(offs[blk]):int(offs[blk + 1])], r, tb, d)
         Aq.append(At[:r, :tb].T.copy())
         Bq.append(Bm[:r].copy())
@@ -109,7 +133,7 @@ def unpack(f: milo.Factors, kind: int):
         assert np.all(At[r:] == 0) and np.all(At[:, tb:] == 0), "A padding must be zero"
         assert np.all(Bm[r:] == 0), "B padding rows must be zero"
     return dict(ranks=ranks, offsets=offs, sigma=sigma, eps=eps, A=A, B=B, Aq=Aq, Bq=Bq, sA=sA, sB=sB, R=R,
-                nb=nb, nblk=nblk)
+                nb=nb, nblk=nblk, A_scale=A_scale, A_zero=A_zero)
 
 
 def pack(shape, params, A_lists, B_lists, sigma_lists=None, eps_lists=None, device="cuda"):

@@ -494,11 +494,12 @@ def test_decode_recent_tail(oracle_mod, factor, tail_dtype, G):
     assert np.array_equal(o_bad[:, 3], out[:, 3])
 
 
-@pytest.mark.parametrize("factor", ["bf16", "int8", "f32"])
+@pytest.mark.parametrize("factor", ["bf16", "int8", "f32", "int2"])
 def test_decode_offloaded_factors(factor):
     """milo_decode_attn_offload on a pinned host copy of the arena stages the
     selected blocks' factors and gives milo_decode_attn's output bit for bit:
-    bf16 (tensor cores), INT8 (scales staged too) and f32 (CUDA cores), with
+    bf16 (tensor cores), INT8 and 2-bit (scales staged too) and f32 (CUDA
+    cores), with
     blocks no session selects (the staging offsets skip them) and a ragged
     last block.  An arena in pageable host memory is refused before any
     launch."""
@@ -589,3 +590,42 @@ def test_bm25_ties_and_bounds(oracle_mod):
     bad[1][0] = 99
     milo.milo_bm25_select(bad, 16, 3)
     assert milo.milo_get_status() == milo.MILO_ERR_BOUNDS
+
+
+def test_int2_codes_and_decode(oracle_mod):
+    """2-bit factors: A's codes and fp16 (scale, zero) per 32-token group equal
+    the oracle's quantiser applied to the same fp32 A (the f32 compression of
+    the same cache; the codes are decided in fp32 on both sides), B's INT8
+    codes are within half a step of the fp32 B, and the decode (tensor cores
+    on an fp16 copy) matches the oracle on the same dequantised factors.  A
+    ragged last block (1000 = 3 x 256 + 232 tokens) and rank-0 padding are
+    included."""
+    K = synth.planted_cache(1, 2, 1000, 128, 256, (4.0, 32.0), seed=33, out_dtype=torch.bfloat16)
+    V = synth.planted_cache(1, 2, 1000, 128, 256, (16.0, 64.0), seed=34, out_dtype=torch.bfloat16)
+    f32 = milo.milo_compress(K.cuda(), V.cuda(), 256, milo.default_params(factor_dtype="f32"))
+    f2 = milo.milo_compress(K.cuda(), V.cuda(), 256, milo.default_params(factor_dtype="int2"))
+    assert milo.milo_get_status() == milo.MILO_OK
+    for kind in range(2):
+        u32, u2 = A.unpack(f32, kind), A.unpack(f2, kind)
+        assert np.array_equal(u32["ranks"], u2["ranks"])
+        for blk in range(u2["nblk"]):
+            r = int(u2["ranks"][blk])
+            if r == 0:
+                continue
+            codes, sc, ze = oracle_mod.quant_int2_groups(u32["A"][blk].astype(np.float32))
+            assert np.array_equal(codes.astype(np.float64), u2["Aq"][blk])
+            assert np.array_equal(sc.astype(np.float64), u2["A_scale"][blk])
+            assert np.array_equal(ze.astype(np.float64), u2["A_zero"][blk])
+            sB = u2["sB"][blk].astype(np.float64)
+            assert np.all(np.abs(u2["B"][blk] - u32["B"][blk]) <= 0.5 * sB[None, :] * (1 + 1e-6) + 1e-12)
+    U = [A.unpack(f2, 0), A.unpack(f2, 1)]
+    for u in U:
+        u["H"] = 2
+    q = torch.randn(1, 1, 8, 128, generator=torch.Generator().manual_seed(4))
+    sel = torch.tensor([[0, 1, 3]], dtype=torch.int32)
+    out = milo.milo_decode_attn(f2, q.cuda(), sel.cuda(), None, rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    for hq in range(8):
+        ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // 4, 4, q[0, 0, hq].double().numpy(), [0, 1, 3],
+                          [0, 256, 768], 1e6)
+        assert _rel_inf(out[0, 0, hq], ref) <= DEC_TOL, (hq, _rel_inf(out[0, 0, hq], ref))
