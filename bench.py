@@ -59,6 +59,7 @@ DECODE_SOURCES = ("block_wise_rank_b200/csrc/decode_tc.cuh", "block_wise_rank_b2
                   "block_wise_rank_b200/csrc/common.cuh")
 # the other rows: (workload, rank budget, factor dtype)
 ROWS = [("qwen7b-128k", 0.25, "bf16", 0), ("qwen7b-128k", 0.75, "bf16", 0), ("qwen7b-128k", 0.5, "int8", 0),
+        ("qwen7b-128k", 0.5, "int2", 0),
         ("qwen7b-128k", 0.5, "bf16", 512), ("qwen7b-64k", 0.5, "bf16", 0), ("qwen3b-32k", 0.5, "bf16", 0)]
 
 
@@ -70,7 +71,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen7b-128k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget", type=float, default=0.5)
-    ap.add_argument("--factor", default=None, choices=["bf16", "int8", "f32"])
+    ap.add_argument("--factor", default=None, choices=["bf16", "int8", "int2", "f32"])
     ap.add_argument("--decode-steps", type=int, default=0, help="decode steps per step (0: the workload's)")
     ap.add_argument("--cpu-sample-s", type=float, default=12.0, help="seconds of CPU oracle work per variant")
     ap.add_argument("--layers", type=int, default=0,
@@ -156,25 +157,33 @@ def factor_bytes_per_elem(factor):
     return {"bf16": 2, "f32": 4, "int8": 1}[factor]
 
 
+def block_factor_bytes(rk, rv, tb, d, factor):
+    """Bytes of a block's factors (both kinds) at its true ranks: A and B
+    elements at the factor width, INT8 scales (r + d per kind), or for 2-bit
+    codes A at 2 bits plus an fp16 (scale, zero) per rank and 32-token group
+    and B in INT8 with its d channel scales."""
+    r = rk + rv
+    if factor == "int2":
+        return r * tb / 4 + r * ((tb + 31) // 32) * 4 + r * d + 2 * d * 4
+    b = r * (tb + d) * factor_bytes_per_elem(factor)
+    return b + ((r + 2 * d) * 4 if factor == "int8" else 0)
+
+
 def decode_bytes(ranks, w, sel, factor, S, Hq):
     """Algorithmic bytes of one decode step (all layers).
 
-    Unique selected (l, h, b): r_b^K (T_b + d) + r_b^V (T_b + d) factor
-    elements (+ int8 scales r_b + d per kind), plus q and out (fp32) and the
-    ids/positions.
+    Unique selected (l, h, b): its factors' bytes (block_factor_bytes), plus
+    q and out (fp32) and the ids/positions.
     """
     rk, rv = ranks
-    es = factor_bytes_per_elem(factor)
     nb = w.n_b
     uniq = torch.zeros(nb, dtype=torch.bool)
     uniq[sel.reshape(-1).long().cpu()] = True
     tb = torch.tensor([min(w.block_len, w.T - b * w.block_len) for b in range(nb)], dtype=torch.float64)
     mask = uniq.to(torch.float64)
-    per = ((rk + rv).to(torch.float64).reshape(w.L * w.H, nb) * (tb + w.d)[None, :]) * es
+    per = block_factor_bytes(rk.to(torch.float64).reshape(w.L * w.H, nb), rv.to(torch.float64).reshape(w.L * w.H, nb),
+                             tb[None, :], w.d, factor)
     total = float((per * mask[None, :]).sum())
-    if factor == "int8":
-        sc = ((rk + rv).to(torch.float64).reshape(w.L * w.H, nb) + 2 * w.d) * 4
-        total += float((sc * mask[None, :]).sum())
     total += 2 * w.L * S * Hq * w.d * 4          # q in, out
     total += 2 * sel.numel() * 4                 # ids, positions
     return total
@@ -814,9 +823,8 @@ def oracle_sample(w, budget, factor):
     comp_s = time.perf_counter() - t0
     q, sel, pos = synth.decode_inputs(w)
     queries = [q[0, 0, g].double().numpy() for g in range(w.G)]
-    es = factor_bytes_per_elem(factor)
-    bytes_per_query = sum(facs[b][k][0].shape[1] * (facs[b][k][0].shape[0] + w.d) * es
-                          for b in blocks for k in (0, 1)) + 2 * w.d * 4
+    bytes_per_query = sum(block_factor_bytes(facs[b][0][0].shape[1], facs[b][1][0].shape[1], facs[b][0][0].shape[0],
+                                             w.d, factor) for b in blocks) + 2 * w.d * 4
     return dict(facs=facs, blocks=blocks, positions=[b * w.block_len for b in blocks], queries=queries,
                 bytes_per_query=bytes_per_query, comp_s=comp_s, comp_blocks=2 * len(blocks), rope_base=w.rope_base)
 
