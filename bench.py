@@ -376,9 +376,12 @@ def compression_roofline(run, t, steps, pk):
             out[name] = dict(ms=round(ms / steps, 4))
     ms, n = stage_ms(t, "project")
     if n:
+        # bytes written: every block's padded factors (R8 rank rows, whole 128-token tiles)
         ranks = read_ranks(run.f)
-        es = factor_bytes_per_elem(run.factor)
-        fac = float(sum(((r.to(torch.float64) + 7) // 8 * 8).sum() for r in ranks)) * (128 + w.d) * es
+        nt = torch.tensor([-(-min(w.block_len, w.T - b * w.block_len) // 128) for b in range(w.n_b)],
+                          dtype=torch.float64).repeat(w.L * w.H)
+        per_r8 = 48 * nt + w.d if run.factor == "int2" else (128 * nt + w.d) * factor_bytes_per_elem(run.factor)
+        fac = float(sum((((r.to(torch.float64) + 7) // 8 * 8) * per_r8).sum() for r in ranks))
         nbytes = 2 * w.L * w.H * w.T * w.d * es_in + fac
         gbs = nbytes / (ms / 1e3 / steps) / 1e9
         out["project"].update(gbs=round(gbs, 1), bound="hbm", frac=round(gbs / pk["hbm"], 4))
