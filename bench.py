@@ -777,6 +777,8 @@ def run_ours(args, rank, world):
             r = Run(workload_of(name), budget, fac, dev, tail=tail)
             tr = r.timed(args.row_steps, 1)
             rows.append(row_of(r, tr, args.row_steps, pk))
+            if fac in ("int8", "int2"):   # the codes' point: fewer bytes over the host link
+                rows[-1]["offload"] = offload_measure(r)
             r.release()
         res["rows"] = rows
     return res
