@@ -154,3 +154,57 @@ def test_timing_hooks_on_host(L):
     assert L.milo_timing_read(None, None, 0) == milo.MILO_OK
     assert L.milo_timing_read(None, None, 3) == milo.MILO_ERR_INVALID_ARG
     assert L.milo_timing_read(None, None, 9) == milo.MILO_ERR_INVALID_ARG
+
+
+def test_next_entry_points_reject_bad_arguments_on_host(L):
+    """The recent-token, offloaded-factor and BM25 entry points refuse bad
+    arguments before any device work (so these run without a GPU), their
+    size queries return 0 on a null handle, and 2-bit factors size the arena
+    by the documented formula."""
+    P = ctypes.c_void_p(256)
+    BIG = 1 << 30
+    # recent tokens: null tail, unsupported tail type, tail not 16-byte aligned
+    assert L.milo_decode_attn_tail(None, P, 1, 1, P, None, 1, 1e6, None, P, milo.MILO_BF16, 4, P, P, P, BIG,
+                                   None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_attn_tail(None, P, 1, 1, P, None, 1, 1e6, P, P, milo.MILO_INT8, 4, P, P, P, BIG,
+                                   None) == milo.MILO_ERR_UNSUPPORTED
+    assert L.milo_decode_attn_tail(None, P, 1, 1, P, None, 1, 1e6, ctypes.c_void_p(264), P, milo.MILO_BF16, 4, P,
+                                   P, P, BIG, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_attn_tail(None, P, 1, 1, P, None, 1, 1e6, P, P, milo.MILO_BF16, -1, P, P, P, BIG,
+                                   None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_tail_workspace_size(None, 1, 1, 1) == 0
+    # offloaded factors: null handle
+    assert L.milo_decode_attn_offload(None, P, 1, 1, P, None, 1, 1e6, P, P, BIG, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_offload_workspace_size(None, 1, 1, 1) == 0
+    # BM25: n_sel outside [1, n_b], beta outside [0, 1], negative k1, null
+    # outputs, entries without their arrays, small workspace
+    ws = L.milo_bm25_workspace_size(8, 100, 2)
+    assert ws > 0 and L.milo_bm25_workspace_size(0, 100, 2) == 0
+    ok = dict(bp=P, bt=P, bf=P, bl=P, nb=8, nnzb=10, V=100, qp=P, qt=P, qf=P, S=2, nnzq=4, k1=1.2, beta=0.75,
+              nsel=3, sel=P, sc=None, ws=P, wsb=ws)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.milo_bm25_select(a["bp"], a["bt"], a["bf"], a["bl"], a["nb"], a["nnzb"], a["V"], a["qp"], a["qt"],
+                                  a["qf"], a["S"], a["nnzq"], a["k1"], a["beta"], a["nsel"], a["sel"], a["sc"],
+                                  a["ws"], a["wsb"], None)
+    assert call(nsel=0) == milo.MILO_ERR_INVALID_ARG
+    assert call(nsel=9) == milo.MILO_ERR_INVALID_ARG
+    assert call(beta=1.5) == milo.MILO_ERR_INVALID_ARG
+    assert call(k1=-0.1) == milo.MILO_ERR_INVALID_ARG
+    assert call(sel=None) == milo.MILO_ERR_INVALID_ARG
+    assert call(bt=None) == milo.MILO_ERR_INVALID_ARG
+    assert call(qf=None) == milo.MILO_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(264)) == milo.MILO_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == milo.MILO_ERR_WORKSPACE
+    # 2-bit factors: the data section holds (R + 7 N_blk) R8-rows of 48 nt + d bytes
+    s = _shape()
+    p2, p16 = milo.default_params(factor_dtype="int2"), milo.default_params(factor_dtype="bf16")
+    R = milo.milo_rank_budget(s, p2)
+    assert R == milo.milo_rank_budget(s, p16) > 0
+    n_b = -(-s.T // s.block_len)
+    nblk = s.L * s.H * n_b
+    nt = -(-s.block_len // 128)
+    data = (R + 7 * nblk) * (48 * nt + 128)
+    assert milo.milo_factor_arena_size(s, p2) >= 2 * data
+    assert milo.milo_factor_arena_size(s, p2) < milo.milo_factor_arena_size(s, p16)
