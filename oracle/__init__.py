@@ -231,24 +231,37 @@ def attention(Q, K, V):
 # --------------------------------------------------------------------------
 # the path, step by step
 # --------------------------------------------------------------------------
-def block_lengths(T: int, block_len: int):
-    """Blocking: block b covers tokens [b*block_len, min((b+1)*block_len, T))."""
-    return [min(block_len, T - b * block_len) for b in range(math.ceil(T / block_len))]
+def block_bounds(T: int, block_len: int, starts=None):
+    """Blocking: (first token, end) of every block.  Fixed length: block b
+    covers tokens [b*block_len, min((b+1)*block_len, T)).  With `starts`
+    (ascending token offsets, starts[0] = 0, starts[-1] = T) block b covers
+    [starts[b], starts[b+1]): variable-length blocks that each hold whole
+    demonstrations (shd-paper mirror, original abstract: each block holds
+    several many-shot examples)."""
+    if starts is not None:
+        return [(int(starts[b]), int(starts[b + 1])) for b in range(len(starts) - 1)]
+    return [(b * block_len, min((b + 1) * block_len, T)) for b in range(math.ceil(T / block_len))]
 
 
-def rank_caps(T: int, block_len: int, d: int, r_max: int = 0):
+def block_lengths(T: int, block_len: int, starts=None):
+    """Tokens of every block (block_bounds)."""
+    return [e - s for s, e in block_bounds(T, block_len, starts)]
+
+
+def rank_caps(T: int, block_len: int, d: int, r_max: int = 0, starts=None):
     """Largest rank of each block: min(T_b, d), lowered to r_max when r_max > 0."""
-    caps = [min(tb, d) for tb in block_lengths(T, block_len)]
+    caps = [min(tb, d) for tb in block_lengths(T, block_len, starts)]
     if r_max > 0:
         caps = [min(c, r_max) for c in caps]
     return caps
 
 
-def budget(L: int, H: int, T: int, block_len: int, d: int, frac: float = 0.5, absolute: int = 0) -> int:
+def budget(L: int, H: int, T: int, block_len: int, d: int, frac: float = 0.5, absolute: int = 0,
+           starts=None) -> int:
     """Global rank budget per kind: absolute if > 0, else floor(frac * sum_b min(T_b, d))."""
     if absolute > 0:
         return int(absolute)
-    total = L * H * sum(min(tb, d) for tb in block_lengths(T, block_len))
+    total = L * H * sum(min(tb, d) for tb in block_lengths(T, block_len, starts))
     return int(math.floor(frac * total))
 
 
@@ -263,31 +276,32 @@ def eps_of(sigma_lhb, eps_rel: float, scope: int = 0):
     return eps_rel * top
 
 
-def svd_blocks(X_lhtd, block_len: int):
+def svd_blocks(X_lhtd, block_len: int, starts=None):
     """SVD of every block of one kind.  X: [L][H][T][d] -> per-block results."""
     X = np.asarray(X_lhtd, dtype=np.float64)
     L, H, T, d = X.shape
-    nb = math.ceil(T / block_len)
+    bounds = block_bounds(T, block_len, starts)
+    nb = len(bounds)
     sigma = np.zeros((L, H, nb, d))
     Vr = np.zeros((L, H, nb, d, d))
     US = [[[None] * nb for _ in range(H)] for _ in range(L)]
     for l in range(L):
         for h in range(H):
             for b in range(nb):
-                s, v, us, _ = svd(X[l, h, b * block_len:min((b + 1) * block_len, T)])
+                s, v, us, _ = svd(X[l, h, bounds[b][0]:bounds[b][1]])
                 sigma[l, h, b] = s
                 Vr[l, h, b] = v
                 US[l][h][b] = us
     return sigma, Vr, US
 
 
-def allocate(sigma_lhb, eps_lh, T: int, block_len: int, R: int, r_min: int = 0, r_max: int = 0):
+def allocate(sigma_lhb, eps_lh, T: int, block_len: int, R: int, r_min: int = 0, r_max: int = 0, starts=None):
     """Ranks [L][H][n_b] for one kind; greedy and sort forms must agree."""
     sigma = np.asarray(sigma_lhb, dtype=np.float64)
     L, H, nb, d = sigma.shape
     group = np.repeat(np.arange(L * H, dtype=np.int32), nb)
     key = keys(sigma.reshape(L * H * nb, d), np.asarray(eps_lh, dtype=np.float64).reshape(-1), group)
-    caps = np.tile(np.asarray(rank_caps(T, block_len, d, r_max), dtype=np.int32), L * H)
+    caps = np.tile(np.asarray(rank_caps(T, block_len, d, r_max, starts), dtype=np.int32), L * H)
     g = allocate_greedy(key, caps, R, r_min)
     s = allocate_sort(key, caps, R, r_min)
     if not np.array_equal(g, s):
@@ -296,7 +310,7 @@ def allocate(sigma_lhb, eps_lh, T: int, block_len: int, R: int, r_min: int = 0, 
 
 
 def compress(K, V, block_len: int, budget_frac: float = 0.5, budget_abs: int = 0,
-             eps_rel: float = 1e-2, eps_scope: int = 0, r_min: int = 0, r_max: int = 0):
+             eps_rel: float = 1e-2, eps_scope: int = 0, r_min: int = 0, r_max: int = 0, starts=None):
     """Whole compression of one cache: per kind (0 = K pre-RoPE, 1 = V).
 
     Returns a list of two dicts with sigma [L][H][nb][d], eps [L][H],
@@ -307,10 +321,10 @@ def compress(K, V, block_len: int, budget_frac: float = 0.5, budget_abs: int = 0
     for X in (K, V):
         X = np.asarray(X, dtype=np.float64)
         L, H, T, d = X.shape
-        sigma, Vr, US = svd_blocks(X, block_len)
+        sigma, Vr, US = svd_blocks(X, block_len, starts)
         eps = eps_of(sigma, eps_rel, eps_scope)
-        R = budget(L, H, T, block_len, d, budget_frac, budget_abs)
-        ranks = allocate(sigma, eps, T, block_len, R, r_min, r_max)
+        R = budget(L, H, T, block_len, d, budget_frac, budget_abs, starts)
+        ranks = allocate(sigma, eps, T, block_len, R, r_min, r_max, starts)
         nb = sigma.shape[2]
         A = [[[US[l][h][b][:, :ranks[l, h, b]].copy() for b in range(nb)] for h in range(H)] for l in range(L)]
         B = [[[Vr[l, h, b][:, :ranks[l, h, b]].T.copy() for b in range(nb)] for h in range(H)] for l in range(L)]

@@ -531,3 +531,61 @@ def test_int2_groups_nearest_level_brute_force(oracle_mod):
             assert codes[rows, k][np.argmin(A[rows, k])] == 0 and codes[rows, k][np.argmax(A[rows, k])] == 3
             rng_ = float(A[rows, k].max() - A[rows, k].min())
             assert np.abs(deq[rows, k] - A[rows, k]).max() <= rng_ / 6 * (1 + 2e-3) + abs(float(ze[g, k]) - float(A[rows, k].min()))
+
+
+# ---------------------------------------------------------------- variable-length blocks
+def test_variable_blocks_budget_caps_and_dense_decode(oracle_mod):
+    """Blocks given by their starts: the budget is floor(frac * sum min(T_b, d))
+    over the given lengths (hand values), short blocks cap the rank at their
+    length, and full-rank factors of irregular blocks decode to dense
+    attention over exactly the selected tokens at their own positions
+    (scipy softmax)."""
+    starts = [0, 100, 300, 307, 500, 650]          # lengths 100, 200, 7, 193, 150
+    assert oracle_mod.block_lengths(650, 0, starts) == [100, 200, 7, 193, 150]
+    assert oracle_mod.budget(2, 3, 650, 0, 128, 0.5, starts=starts) == (2 * 3 * (100 + 128 + 7 + 128 + 128)) // 2
+    assert oracle_mod.rank_caps(650, 0, 128, 0, starts) == [100, 128, 7, 128, 128]
+    assert oracle_mod.rank_caps(650, 0, 128, 50, starts) == [50, 50, 7, 50, 50]
+    rng = np.random.default_rng(24)
+    d, base = 16, 1e4
+    K = rng.standard_normal((650, d))
+    V = rng.standard_normal((650, d))
+    bounds = oracle_mod.block_bounds(650, 0, starts)
+    AK, BK = _full_rank_factors_bounds(oracle_mod, K, bounds)
+    AV, BV = _full_rank_factors_bounds(oracle_mod, V, bounds)
+    q = rng.standard_normal(d)
+    sel = [1, 2, 4]
+    out = oracle_mod.decode_one(lambda b: AK[b], lambda b: BK[b], lambda b: AV[b], lambda b: BV[b],
+                                q, sel, [starts[b] for b in sel], base)
+    idx = np.r_[100:300, 300:307, 500:650]
+    Kr = np.stack([oracle_mod.rope(K[t], t, base) for t in idx])
+    ref = scipy.special.softmax(Kr @ q / math.sqrt(d)) @ V[idx]
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def _full_rank_factors_bounds(oracle_mod, X, bounds):
+    A, B = [], []
+    for s, e in bounds:
+        sv, Vr, US, _ = oracle_mod.svd(X[s:e])
+        m = min(e - s, X.shape[1])
+        A.append(US[:, :m])
+        B.append(Vr[:, :m].T)
+    return A, B
+
+
+def test_variable_blocks_compress_equals_per_block(oracle_mod):
+    """compress with starts runs every step on exactly the given token ranges:
+    its sigma equal LAPACK's singular values of each slice, and starts that
+    spell out a fixed block length reproduce the fixed-length compression."""
+    rng = np.random.default_rng(25)
+    K = rng.standard_normal((1, 1, 300, 16))
+    V = rng.standard_normal((1, 1, 300, 16))
+    starts = [0, 40, 41, 200, 300]
+    out = oracle_mod.compress(K, V, 0, 0.5, starts=starts)
+    for b, (s, e) in enumerate(oracle_mod.block_bounds(300, 0, starts)):
+        ref = scipy.linalg.svd(K[0, 0, s:e], compute_uv=False)
+        assert np.allclose(out[0]["sigma"][0, 0, b, :len(ref)], ref, rtol=1e-12, atol=1e-12)
+    fixed = oracle_mod.compress(K, V, 64, 0.5)
+    spelled = oracle_mod.compress(K, V, 0, 0.5, starts=[0, 64, 128, 192, 256, 300])
+    for k in range(2):
+        assert np.array_equal(fixed[k]["ranks"], spelled[k]["ranks"]) and fixed[k]["R"] == spelled[k]["R"]
+        assert np.array_equal(fixed[k]["sigma"], spelled[k]["sigma"])
