@@ -74,7 +74,9 @@ struct SelArgs {
 struct SelShape {
     int n_b, T, block_len, r_min, r_max;
     int64_t n_blk;
-    int dtype;   // factor type of the offsets written (their unit: block_units)
+    int dtype;              // factor type of the offsets written (their unit: block_units)
+    const int32_t *starts;  // variable-length blocks' starts, or null (BlockGeo)
+    __device__ __forceinline__ int len(int b) const { return BlockGeo{T, block_len, starts}.len(b); }
 };
 
 // key bits of component k of block blk ((sigma/eps)^2 as a double, 0 if eps <= 0)
@@ -87,7 +89,7 @@ __device__ __forceinline__ unsigned long long key_bits(const SelArgs &a, int64_t
 
 __device__ __forceinline__ void elig_range(const SelShape &sh, int64_t blk, int &k0, int &k1) {
     const int b = (int)(blk % sh.n_b);
-    const int cap = block_cap(block_tokens(sh.T, sh.block_len, b), sh.r_max);
+    const int cap = block_cap(sh.len(b), sh.r_max);
     k0 = sh.r_min < cap ? sh.r_min : cap;
     k1 = cap;
 }
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
         elig_range(sh, i, k0, k1);
         const int r = k0 + a.gt[i] + (int)take;
         a.ranks[i] = r;
-        const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
+        const int tb = sh.len((int)(i % sh.n_b));
         elems += block_units(sh.dtype, r, tb);
     }
     if (a.offsets == nullptr) return;
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(1024) k_sel_ranks(SelArgs a0, SelArgs a1, SelS
     long long off = sB[tid] - elems;
     for (int64_t i = lo; i < hi; ++i) {
         a.offsets[i] = off;
-        const int tb = block_tokens(sh.T, sh.block_len, (int)(i % sh.n_b));
+        const int tb = sh.len((int)(i % sh.n_b));
         off += block_units(sh.dtype, a.ranks[i], tb);
     }
     if (hi == n && lo < hi) a.offsets[n] = off;

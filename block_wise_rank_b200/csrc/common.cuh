@@ -37,6 +37,19 @@ __host__ __device__ __forceinline__ int block_tokens(int T, int block_len, int b
     return r < block_len ? r : block_len;
 }
 
+// Block b of every (layer, head) covers tokens [start(b), start(b) + len(b)):
+// a fixed length block_len (the last block may be short), or given starts
+// (variable-length blocks: starts[0] = 0, ascending, starts[n_b] = T, every
+// length in [1, block_len]; `starts` is then device-readable).
+struct BlockGeo {
+    int T, block_len;
+    const int32_t *starts;   // [n_b + 1] or null
+    __device__ __forceinline__ int start(int b) const { return starts ? starts[b] : b * block_len; }
+    __device__ __forceinline__ int len(int b) const {
+        return starts ? starts[b + 1] - starts[b] : block_tokens(T, block_len, b);
+    }
+};
+
 // largest admissible rank of a block: min(T_b, d, r_max if > 0)
 __host__ __device__ __forceinline__ int block_cap(int Tb, int r_max) {
     int c = Tb < D ? Tb : D;

@@ -33,14 +33,14 @@ __global__ void k_flag_selected(const int32_t *__restrict__ sel, int n_slots, in
 // kind in the staging area: the block's factors when its id is flagged, else
 // 0; the ranks are copied for every block.  grid over nblk.
 __global__ void k_stage_sizes(const int32_t *__restrict__ host_ranks, const int32_t *__restrict__ used, int64_t nblk,
-                              int n_b, int T, int block_len, int dtype, int64_t *__restrict__ sizes,
+                              int n_b, BlockGeo geo, int dtype, int64_t *__restrict__ sizes,
                               int32_t *__restrict__ ranks) {
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
          blk += (int64_t)gridDim.x * blockDim.x) {
         const int b = (int)(blk % n_b);
         const int r = host_ranks[blk];
         ranks[blk] = r;
-        sizes[blk] = used[b] ? block_units(dtype, r, block_tokens(T, block_len, b)) : 0;
+        sizes[blk] = used[b] ? block_units(dtype, r, geo.len(b)) : 0;
     }
 }
 

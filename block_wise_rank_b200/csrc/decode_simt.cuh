@@ -28,6 +28,7 @@ struct DecodeArgs {
     const float *q;            // [L][S][Hq][D]
     const int32_t *sel;        // [S][n_sel]
     const int32_t *pos;        // [S][n_sel] or null
+    const int32_t *starts;     // variable-length blocks' starts [n_b + 1], or null (BlockGeo)
     const int32_t *slot_start; // [n_b + 1] slots of each block id
     const int32_t *slot_list;  // [S * n_sel] slot = s * n_sel + j
     const float2 *rope_q;      // [S * n_sel][64] (cos, sin)(p theta_i)
@@ -45,15 +46,20 @@ struct DecodeArgs {
 
 // (cos, sin)(p theta_i) for every selected slot and (t theta_i) for every
 // in-block token, angles in double, theta_i = base^(-2i/d).
-__global__ void k_rope_tables(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos, int n_slots,
-                              int block_len, double base, float2 *__restrict__ rope_q, float2 *__restrict__ rope_t) {
+__global__ void k_rope_tables(const int32_t *__restrict__ sel, const int32_t *__restrict__ pos,
+                              const int32_t *__restrict__ starts, int n_b, int n_slots, int block_len, double base,
+                              float2 *__restrict__ rope_q, float2 *__restrict__ rope_t) {
     const int64_t total = (int64_t)(n_slots + block_len) * HALF;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int i = (int)(e % HALF);
         const int64_t row = e / HALF;
         const double theta = pow(base, -2.0 * (double)i / (double)D);
         double p;
-        if (row < n_slots) p = pos ? (double)pos[row] : (double)sel[row] * (double)block_len;
+        if (row < n_slots) {   // a selected block's start: given, else where the block starts
+            const int b = sel[row];
+            p = pos ? (double)pos[row]
+                    : (starts ? (b >= 0 && b < n_b ? (double)starts[b] : 0.0) : (double)b * (double)block_len);
+        }
         else p = (double)(row - n_slots);
         double sn, cs;
         sincos(p * theta, &sn, &cs);
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeArgs a) {
     const int64_t blk = ((int64_t)l * a.H + h) * a.n_b + b;
     const KindView &K = a.kv[0], &V = a.kv[1];
     const int rK = K.ranks[blk], rV = V.ranks[blk];
-    const int Tb = block_tokens(a.T, a.block_len, b);
+    const int Tb = BlockGeo{a.T, a.block_len, a.starts}.len(b);
     const int nt = token_tiles(Tb);
     const int R8K = rank_pad(rK), R8V = rank_pad(rV);
     const int64_t baseK = K.offsets[blk], baseV = V.offsets[blk];

@@ -161,7 +161,7 @@ __global__ void k_dt_items(DecodeArgs a, const int32_t *__restrict__ pstart, DtI
     it.l = (int)(lh / a.H);
     it.h = (int)(lh % a.H);
     it.b = b;
-    it.Tb = block_tokens(a.T, a.block_len, b);
+    it.Tb = BlockGeo{a.T, a.block_len, a.starts}.len(b);
     it.rK = a.kv[0].ranks[blk];
     it.rV = a.kv[1].ranks[blk];
     it.offK = a.kv[0].offsets[blk];
@@ -1197,11 +1197,11 @@ k_decode_tc(DecodeArgs a, const int32_t *__restrict__ pstart, const DtItem *__re
 
 // Element sizes (the bf16 layout of common.cuh) of every block, for the fp16
 // copy of 2-bit factors; scanned into its element offsets.  grid over nblk.
-__global__ void k_elem_sizes(const int32_t *__restrict__ ranks, int64_t nblk, int n_b, int T, int block_len,
+__global__ void k_elem_sizes(const int32_t *__restrict__ ranks, int64_t nblk, int n_b, BlockGeo geo,
                              int64_t *__restrict__ sizes) {
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
          blk += (int64_t)gridDim.x * blockDim.x)
-        sizes[blk] = block_elems(ranks[blk], block_tokens(T, block_len, (int)(blk % n_b)));
+        sizes[blk] = block_elems(ranks[blk], geo.len((int)(blk % n_b)));
 }
 
 // 2-bit factors for the tensor cores: the selected blocks' A codes as zero +
@@ -1219,7 +1219,7 @@ __global__ void __launch_bounds__(256) k_dequant_int2(DecodeArgs a, const int64_
     const KindView &kv = a.kv[kind];
     const int R8 = rank_pad(kv.ranks[blk]);
     if (R8 == 0) return;
-    const int nt = token_tiles(block_tokens(a.T, a.block_len, b));
+    const int nt = token_tiles(BlockGeo{a.T, a.block_len, a.starts}.len(b));
     const int64_t nA = (int64_t)nt * R8 * FTILE, nAll = nA + (int64_t)R8 * D;
     const uint8_t *src = (const uint8_t *)kv.data + kv.offsets[blk];
     __half *dst = (kind ? out1 : out0) + (kind ? eoff1 : eoff0)[blk];
@@ -1275,7 +1275,7 @@ __global__ void __launch_bounds__(256) k_dequant_selected(DecodeArgs a, __half *
     const KindView &kv = a.kv[kind];
     const int R8 = rank_pad(kv.ranks[blk]);
     if (R8 == 0) return;
-    const int Tb = block_tokens(a.T, a.block_len, b);
+    const int Tb = BlockGeo{a.T, a.block_len, a.starts}.len(b);
     const int nt = token_tiles(Tb);
     const int64_t base = kv.offsets[blk];
     const int64_t nA = (int64_t)nt * R8 * FTILE, nAll = nA + (int64_t)R8 * D;

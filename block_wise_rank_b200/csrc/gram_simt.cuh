@@ -16,15 +16,15 @@ namespace milo {
 // chunks of 32 rows.  G is written row-major to G_out[kind][blk][128][128].
 template <typename T>
 __global__ void __launch_bounds__(256) k_gram_simt(const T *__restrict__ K, const T *__restrict__ V,
-                                                    int H, int Tn, int block_len, int n_b,
+                                                    int H, BlockGeo geo, int n_b,
                                                     float *__restrict__ G_out, int64_t n_blk) {
     __shared__ __align__(16) float xs[32][D + 4];
     const int blk = blockIdx.x;
     const int kind = blockIdx.y;
     const T *X = kind == 0 ? K : V;
     const int lh = blk / n_b, b = blk % n_b;
-    const int Tb = block_tokens(Tn, block_len, b);
-    const T *Xb = X + ((int64_t)lh * Tn + (int64_t)b * block_len) * D;
+    const int Tb = geo.len(b);
+    const T *Xb = X + ((int64_t)lh * geo.T + geo.start(b)) * D;
     const int tid = threadIdx.x;
     const int ti = tid / 16, tj = tid % 16;
     float acc[8][8];

@@ -59,7 +59,7 @@ struct JacobiSmem {
 // min(T_b, d) are set to 0 (the rank of a T_b x d block).
 __global__ void __launch_bounds__(JAC_THREADS, 2)
 k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restrict__ sigma_V,
-         int64_t n_blk, int Tn, int block_len, int n_b, int max_sweeps, float tol) {
+         int64_t n_blk, BlockGeo geo, int n_b, int max_sweeps, float tol) {
     extern __shared__ __align__(16) unsigned char jac_raw[];
     JacobiSmem &sm = *reinterpret_cast<JacobiSmem *>(jac_raw);
     const int tid = threadIdx.x;
@@ -191,7 +191,7 @@ k_jacobi(float *__restrict__ G_io, float *__restrict__ sigma_K, float *__restric
         if (!isfinite(lk)) raise_status(ST_NONFINITE);
         float *sig = (kind == 0 ? sigma_K : sigma_V) + (int64_t)blk * D;
         // X_b has rank <= T_b: singular values past min(T_b, d) are exactly 0
-        const int Tb = block_tokens(Tn, block_len, blk % n_b);
+        const int Tb = geo.len(blk % n_b);
         sig[rk] = rk < Tb ? sqrtf(fmaxf(lk, 0.f)) : 0.f;
     }
     __syncthreads();

@@ -33,7 +33,7 @@
 using namespace milo;
 
 struct milo_factors {
-    milo_cache_shape shape;
+    milo_cache_shape shape;        // shape.block_starts points at starts_host (or is null)
     milo_compress_params params;
     void *arena;
     size_t arena_bytes;
@@ -41,6 +41,8 @@ struct milo_factors {
     int64_t n_blk;
     int64_t R;
     KindView kv[2];
+    int32_t *starts;               // variable-length blocks: the arena's starts (else null)
+    std::vector<int32_t> starts_host;
 };
 
 namespace {
@@ -69,12 +71,28 @@ milo_compress_params effective(const milo_compress_params *p) {
     return q;
 }
 
-bool shape_ok(const milo_cache_shape *s) {
-    return s && s->L > 0 && s->H > 0 && s->T > 0 && s->block_len > 0 &&
-           (s->in_dtype == MILO_F32 || s->in_dtype == MILO_BF16);
+int n_blocks(const milo_cache_shape *s) {
+    return s->block_starts ? s->n_blocks : (s->T + s->block_len - 1) / s->block_len;
 }
 
-int n_blocks(const milo_cache_shape *s) { return (s->T + s->block_len - 1) / s->block_len; }
+// tokens of block b (host side)
+int host_block_tokens(const milo_cache_shape *s, int b) {
+    return s->block_starts ? s->block_starts[b + 1] - s->block_starts[b] : block_tokens(s->T, s->block_len, b);
+}
+
+bool shape_ok(const milo_cache_shape *s) {
+    if (!(s && s->L > 0 && s->H > 0 && s->T > 0 && s->block_len > 0 &&
+          (s->in_dtype == MILO_F32 || s->in_dtype == MILO_BF16)))
+        return false;
+    if (!s->block_starts) return true;
+    // variable-length blocks: from 0 to T, ascending, each of 1 .. block_len tokens
+    if (s->n_blocks <= 0 || s->block_starts[0] != 0 || s->block_starts[s->n_blocks] != s->T) return false;
+    for (int b = 0; b < s->n_blocks; ++b) {
+        const int n = s->block_starts[b + 1] - s->block_starts[b];
+        if (n < 1 || n > s->block_len) return false;
+    }
+    return true;
+}
 
 // sum over one (layer, head) row of the rank caps and of the r_min floors
 void cap_sums(const milo_cache_shape *s, int r_min, int r_max, int64_t &caps, int64_t &floors) {
@@ -82,7 +100,7 @@ void cap_sums(const milo_cache_shape *s, int r_min, int r_max, int64_t &caps, in
     floors = 0;
     const int nb = n_blocks(s);
     for (int b = 0; b < nb; ++b) {
-        const int c = block_cap(block_tokens(s->T, s->block_len, b), r_max);
+        const int c = block_cap(host_block_tokens(s, b), r_max);
         caps += c;
         floors += r_min < c ? r_min : c;
     }
@@ -95,7 +113,7 @@ int64_t budget_of(const milo_cache_shape *s, const milo_compress_params *p) {
     int64_t total = 0;
     const int nb = n_blocks(s);
     for (int b = 0; b < nb; ++b) {
-        const int tb = block_tokens(s->T, s->block_len, b);
+        const int tb = host_block_tokens(s, b);
         total += tb < D ? tb : D;
     }
     total *= (int64_t)s->L * s->H;
@@ -104,13 +122,14 @@ int64_t budget_of(const milo_cache_shape *s, const milo_compress_params *p) {
 
 // Byte offsets of one kind's arrays inside its arena section.
 struct SectionLayout {
-    size_t ranks, offsets, sigma, eps, scaleA, scaleB, data, bytes;
+    size_t starts, ranks, offsets, sigma, eps, scaleA, scaleB, data, bytes;
 };
 
 SectionLayout section_layout(const milo_cache_shape *s, const milo_compress_params *p, int64_t R) {
     SectionLayout o{};
     const int64_t nblk = (int64_t)s->L * s->H * n_blocks(s);
     size_t at = 0;
+    o.starts = at;  at = align_up(at + sizeof(int32_t) * (n_blocks(s) + 1));
     o.ranks = at;   at = align_up(at + sizeof(int32_t) * nblk);
     o.offsets = at; at = align_up(at + sizeof(int64_t) * (nblk + 1));
     o.sigma = at;   at = align_up(at + sizeof(float) * nblk * D);
@@ -136,8 +155,21 @@ SectionLayout section_layout(const milo_cache_shape *s, const milo_compress_para
     return o;
 }
 
+// the handle's shape with its own copy of the variable blocks' starts
+void set_shape(milo_factors *f, const milo_cache_shape *s) {
+    f->shape = *s;
+    f->starts_host.clear();
+    if (s->block_starts) {
+        f->starts_host.assign(s->block_starts, s->block_starts + s->n_blocks + 1);
+        f->shape.block_starts = f->starts_host.data();
+    } else {
+        f->shape.n_blocks = 0;
+    }
+}
+
 void fill_views(milo_factors *f) {
     const SectionLayout o = section_layout(&f->shape, &f->params, f->R);
+    f->starts = f->shape.block_starts ? (int32_t *)((char *)f->arena + o.starts) : nullptr;
     for (int k = 0; k < 2; ++k) {
         char *base = (char *)f->arena + (size_t)k * o.bytes;
         f->kv[k].ranks = (int32_t *)(base + o.ranks);
@@ -357,7 +389,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     const milo_compress_params p = effective(params_in);
     milo_factors *f = new (std::nothrow) milo_factors();
     if (!f) return MILO_ERR_INVALID_ARG;
-    f->shape = *shape;
+    set_shape(f, shape);
     f->params = p;
     f->arena = arena;
     f->arena_bytes = arena_bytes;
@@ -368,40 +400,45 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t nblk = f->n_blk;
     float *GW = (float *)workspace;
+    const BlockGeo geo{shape->T, shape->block_len, f->starts};
+    if (f->starts) {   // the variable blocks' starts into the arena, for every kernel
+        cudaError_t e = cudaMemcpyAsync(f->starts, f->starts_host.data(), sizeof(int32_t) * (f->n_b + 1),
+                                        cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) { delete f; return cuda_check(e, "block starts copy"); }
+    }
     AllocScratch as = alloc_scratch((char *)workspace + align_up(sizeof(float) * 2 * (size_t)nblk * D * D), nblk);
 
     // 1. Gram matrices of every block of K and V
     const dim3 grid2((unsigned)nblk, 2);
     cudaEvent_t t0 = tmark(s);
-    if (shape->in_dtype == MILO_BF16 && gram_tc_supported(shape->T, shape->block_len)) {
+    if (shape->in_dtype == MILO_BF16 && !f->starts && gram_tc_supported(shape->T, shape->block_len)) {
         st = cuda_check(launch_gram_tc((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, shape->L * shape->H,
                                        shape->T, shape->block_len, f->n_b, GW, nblk, sm_count(), s),
                         "Gram (tensor cores) launch");
         if (st != MILO_OK) { delete f; return st; }
     } else if (shape->in_dtype == MILO_BF16) {
         k_gram_simt<__nv_bfloat16><<<grid2, 256, 0, s>>>((const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
-                                                          shape->H, shape->T, shape->block_len, f->n_b, GW, nblk);
+                                                          shape->H, geo, f->n_b, GW, nblk);
     } else {
-        k_gram_simt<float><<<grid2, 256, 0, s>>>((const float *)K, (const float *)V, shape->H, shape->T,
-                                                  shape->block_len, f->n_b, GW, nblk);
+        k_gram_simt<float><<<grid2, 256, 0, s>>>((const float *)K, (const float *)V, shape->H, geo, f->n_b, GW,
+                                                  nblk);
     }
     cudaEvent_t t1 = tmark(s);
     tpush(MILO_TK_GRAM, t0, t1);
     // 2. eigensolve: sigma into the arena, sorted eigenvectors back into GW
     t0 = tmark(s);
-    k_jacobi<<<grid2, JAC_THREADS, jacobi_smem_bytes(), s>>>(GW, f->kv[0].sigma, f->kv[1].sigma, nblk, shape->T,
-                                                             shape->block_len, f->n_b, p.max_sweeps, p.jacobi_tol);
+    k_jacobi<<<grid2, JAC_THREADS, jacobi_smem_bytes(), s>>>(GW, f->kv[0].sigma, f->kv[1].sigma, nblk, geo,
+                                                             f->n_b, p.max_sweeps, p.jacobi_tol);
     tpush(MILO_TK_JACOBI, t0, tmark(s));
     // 2b. singular values recomputed from the blocks, sigma / W re-sorted
     t0 = tmark(s);
     if (shape->in_dtype == MILO_BF16)
         k_refine_sigma<__nv_bfloat16><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
-            (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T,
-            shape->block_len, f->n_b, nblk);
+            (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, GW, f->kv[0].sigma, f->kv[1].sigma, geo, f->n_b,
+            nblk);
     else
         k_refine_sigma<float><<<grid2, RF_THREADS, refine_smem_bytes(), s>>>(
-            (const float *)K, (const float *)V, GW, f->kv[0].sigma, f->kv[1].sigma, shape->T, shape->block_len,
-            f->n_b, nblk);
+            (const float *)K, (const float *)V, GW, f->kv[0].sigma, f->kv[1].sigma, geo, f->n_b, nblk);
     tpush(MILO_TK_REFINE, t0, tmark(s));
     // 3. eps per (layer, head, kind)
     const int ngroups = shape->L * shape->H;
@@ -412,7 +449,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     // 4. global top-R selection, ranks and packed offsets
     int64_t caps, floors;
     cap_sums(shape, p.r_min, p.r_max, caps, floors);
-    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk, (int)p.factor_dtype};
+    SelShape sh{f->n_b, shape->T, shape->block_len, p.r_min, p.r_max, nblk, (int)p.factor_dtype, f->starts};
     SelArgs a[2];
     for (int k = 0; k < 2; ++k) {
         a[k].sigma = f->kv[k].sigma;
@@ -440,6 +477,7 @@ milo_status milo_compress(const milo_cache_shape *shape, const void *K, const vo
     pa.in_dtype = shape->in_dtype;
     pa.out_dtype = p.factor_dtype;
     pa.n_blk = nblk;
+    pa.starts = f->starts;
     t0 = tmark(s);
     if (shape->in_dtype == MILO_BF16)
         k_project_a<__nv_bfloat16><<<dim3((unsigned)nblk, D / 32, 2), 256, 0, s>>>(pa);
@@ -476,7 +514,7 @@ milo_status milo_allocate(const float *sigma, const double *eps, int32_t n_group
     cap_sums(&shp, r_min, r_max, caps, floors);
     if (R < floors * n_groups || R > caps * n_groups) return MILO_ERR_INVALID_ARG;
     AllocScratch as = alloc_scratch(workspace, nblk);
-    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32};
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32, nullptr};
     SelArgs a{};
     a.sigma = sigma;
     a.eps = eps;
@@ -563,7 +601,7 @@ milo_status milo_allocate_noalloc(const float *sigma, const double *eps, int32_t
     if (!scratch) return MILO_ERR_CUDA;
     // the scratch layout for kNoAllocBlocks also holds any smaller problem
     AllocScratch as = alloc_scratch(scratch, kNoAllocBlocks);
-    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32};
+    SelShape sh{n_b, T, block_len, r_min, r_max, nblk, MILO_F32, nullptr};
     SelArgs a{};
     a.sigma = sigma;
     a.eps = eps;
@@ -663,7 +701,7 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
     a.L = f->shape.L; a.H = f->shape.H; a.G = Hq / f->shape.H; a.T = f->shape.T;
     a.block_len = f->shape.block_len; a.n_b = n_b; a.factor_dtype = f->params.factor_dtype;
     a.S = S; a.Hq = Hq; a.n_sel = n_sel;
-    a.q = q; a.sel = selected; a.pos = positions;
+    a.q = q; a.sel = selected; a.pos = positions; a.starts = f->starts;
     a.slot_start = start; a.slot_list = list;
     a.rope_q = rope_q; a.rope_t = rope_t;
     a.part_o = part_o; a.part_ml = part_ml; a.out = out;
@@ -687,7 +725,7 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
     k_slot_fill<<<sg, 256, 0, s>>>(selected, (int)slots, n_b, start, cnt, list);
     const int64_t rt = (slots + f->shape.block_len) * HALF;
     k_rope_tables<<<(int)std::min<int64_t>((rt + 255) / 256, 4096), 256, 0, s>>>(
-        selected, positions, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
+        selected, positions, f->starts, n_b, (int)slots, f->shape.block_len, rope_base, rope_q, rope_t);
     if (decode_tc_supported(a)) {
         if (a.factor_dtype == MILO_INT8) {   // dequantised to fp16 for the tensor cores
             k_dequant_selected<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, shadow0, shadow1);
@@ -696,8 +734,9 @@ milo_status decode_impl(const milo_factors *f, const float *q, int32_t S, int32_
             a.f16 = 1;
         } else if (a.factor_dtype == MILO_INT2) {   // the same, into the bf16 layout's element offsets
             const int eg = (int)std::min<int64_t>((f->n_blk + 255) / 256, 4096);
-            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[0].ranks, f->n_blk, n_b, f->shape.T, f->shape.block_len, eoff0);
-            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[1].ranks, f->n_blk, n_b, f->shape.T, f->shape.block_len, eoff1);
+            const BlockGeo geo{f->shape.T, f->shape.block_len, f->starts};
+            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[0].ranks, f->n_blk, n_b, geo, eoff0);
+            k_elem_sizes<<<eg, 256, 0, s>>>(f->kv[1].ranks, f->n_blk, n_b, geo, eoff1);
             k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(eoff0, f->n_blk);
             k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(eoff1, f->n_blk);
             k_dequant_int2<<<dim3((unsigned)f->n_blk, 2), 256, 0, s>>>(a, eoff0, eoff1, shadow0, shadow1);
@@ -817,6 +856,7 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
     milo_factors st = *f;   // the staged copy: same shape, params and block ids
     st.arena = nullptr;
     st.arena_bytes = 0;
+    st.starts = on_device(f, f->starts, dev_arena);   // read in place over the host link (a few words)
     cudaEvent_t t0 = tmark(s);
     e = cudaMemsetAsync(used, 0, sizeof(int32_t) * (f->n_b + 1), s);
     if (e != cudaSuccess) return cuda_check(e, "memset");
@@ -840,8 +880,8 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
         sv.scaleB = host.scaleB ? (float *)(w + o.scaleB[k]) : nullptr;
         sv.data = w + o.data[k];
         k_stage_sizes<<<(int)std::min<int64_t>((f->n_blk + 255) / 256, 4096), 256, 0, s>>>(
-            host.ranks, used, f->n_blk, f->n_b, f->shape.T, f->shape.block_len, f->params.factor_dtype, sv.offsets,
-            sv.ranks);
+            host.ranks, used, f->n_blk, f->n_b, BlockGeo{f->shape.T, f->shape.block_len, st.starts},
+            f->params.factor_dtype, sv.offsets, sv.ranks);
         k_scan_i64<<<1, SCAN_THREADS, 0, s>>>(sv.offsets, f->n_blk);
         k_stage_copy<<<(unsigned)f->n_blk, 256, 0, s>>>(host, sv, used, f->n_b, esize);
     }
@@ -944,7 +984,7 @@ milo_status milo_factors_wrap(const milo_cache_shape *shape, const milo_compress
     if (arena_bytes < milo_factor_arena_size(shape, params)) return MILO_ERR_WORKSPACE;
     milo_factors *f = new (std::nothrow) milo_factors();
     if (!f) return MILO_ERR_INVALID_ARG;
-    f->shape = *shape;
+    set_shape(f, shape);
     f->params = effective(params);
     f->arena = arena;
     f->arena_bytes = arena_bytes;
@@ -967,20 +1007,27 @@ struct BlobHeader {
 };
 }  // namespace
 
+// Blob: the header, the variable blocks' starts (n_blocks + 1 int32, only
+// when the shape has them; the header's pointer is cleared), then the arena.
 milo_status milo_factors_export(const milo_factors *f, void *host_buf, size_t *bytes, milo_stream_t stream) {
     if (!f || !bytes) return MILO_ERR_INVALID_ARG;
-    const size_t need = sizeof(BlobHeader) + milo_factor_arena_size(&f->shape, &f->params);
+    const size_t nst = f->starts_host.size() * sizeof(int32_t);
+    const size_t arena = milo_factor_arena_size(&f->shape, &f->params);
+    const size_t need = sizeof(BlobHeader) + nst + arena;
     if (!host_buf) { *bytes = need; return MILO_OK; }
     if (*bytes < need) { *bytes = need; return MILO_ERR_WORKSPACE; }
     BlobHeader h{};
     memcpy(h.magic, "MILOFAC1", 8);
     h.version = 1;
     h.shape = f->shape;
+    h.shape.block_starts = nullptr;
     h.params = f->params;
-    h.arena_bytes = need - sizeof(BlobHeader);
+    h.arena_bytes = arena;
     memcpy(host_buf, &h, sizeof(h));
+    if (nst) memcpy((char *)host_buf + sizeof(h), f->starts_host.data(), nst);
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = cudaMemcpyAsync((char *)host_buf + sizeof(h), f->arena, h.arena_bytes, cudaMemcpyDeviceToHost, s);
+    cudaError_t e = cudaMemcpyAsync((char *)host_buf + sizeof(h) + nst, f->arena, h.arena_bytes,
+                                    cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     *bytes = need;
     return cuda_check(e, "export copy");
@@ -994,16 +1041,30 @@ milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena,
     BlobHeader h;
     memcpy(&h, host_buf, sizeof(h));
     if (memcmp(h.magic, "MILOFAC1", 8) != 0 || h.version != 1) return MILO_ERR_INVALID_ARG;
-    if (bytes < sizeof(h) + h.arena_bytes) return MILO_ERR_INVALID_ARG;
+    if (h.shape.n_blocks < 0 || h.shape.n_blocks > (1 << 28)) return MILO_ERR_INVALID_ARG;
+    const size_t nst = h.shape.n_blocks > 0 ? sizeof(int32_t) * (size_t)(h.shape.n_blocks + 1) : 0;
+    if (bytes < sizeof(h) + nst) return MILO_ERR_INVALID_ARG;
+    std::vector<int32_t> starts(nst / sizeof(int32_t));
+    if (nst) memcpy(starts.data(), (const char *)host_buf + sizeof(h), nst);
+    h.shape.block_starts = nst ? starts.data() : nullptr;
+    if (bytes < sizeof(h) + nst + h.arena_bytes) return MILO_ERR_INVALID_ARG;
     if (h.arena_bytes != milo_factor_arena_size(&h.shape, &h.params)) return MILO_ERR_INVALID_ARG;
     milo_factors *f = nullptr;
     milo_status st = milo_factors_wrap(&h.shape, &h.params, arena, arena_bytes, &f);
     if (st != MILO_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = cudaMemcpyAsync(arena, (const char *)host_buf + sizeof(h), h.arena_bytes, cudaMemcpyHostToDevice, s);
+    cudaError_t e = cudaMemcpyAsync(arena, (const char *)host_buf + sizeof(h) + nst, h.arena_bytes,
+                                    cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) { delete f; return cuda_check(e, "import copy"); }
     *out = f;
+    return MILO_OK;
+}
+
+milo_status milo_factors_shape(const milo_factors *f, milo_cache_shape *shape, milo_compress_params *params) {
+    if (!f) return MILO_ERR_INVALID_ARG;
+    if (shape) *shape = f->shape;
+    if (params) *params = f->params;
     return MILO_OK;
 }
 

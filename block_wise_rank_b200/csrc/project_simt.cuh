@@ -33,6 +33,7 @@ struct ProjArgs {
     KindView kv[2];
     int T, block_len, n_b, in_dtype, out_dtype;
     int64_t n_blk;
+    const int32_t *starts;     // variable-length blocks' starts, or null (BlockGeo)
 };
 
 // grid (n_blk, D/32 rank chunks, 2 kinds), 256 threads.  Writes the rank
@@ -51,9 +52,10 @@ __global__ void __launch_bounds__(256) k_project_a(ProjArgs pa) {
     const int kw = min(32, R8 - k0);          // rows written (incl. zero padding)
     const int kc = max(0, min(32, r - k0));   // rows with data
     const int b = blk % pa.n_b, lh = blk / pa.n_b;
-    const int Tb = block_tokens(pa.T, pa.block_len, b);
+    const BlockGeo geo{pa.T, pa.block_len, pa.starts};
+    const int Tb = geo.len(b);
     const int ldT = token_tiles(Tb) * FTILE;
-    const TI *Xb = (const TI *)pa.X[kind] + ((int64_t)lh * pa.T + (int64_t)b * pa.block_len) * D;
+    const TI *Xb = (const TI *)pa.X[kind] + ((int64_t)lh * pa.T + geo.start(b)) * D;
     const float *Wb = pa.W[kind] + (int64_t)blk * D * D;
     for (int e = threadIdx.x; e < D * 32; e += 256) {
         const int j = e / 32, c = e % 32;
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(128) k_project_b(ProjArgs pa) {
     const int r = kv.ranks[blk];
     const int R8 = rank_pad(r);
     const int b = blk % pa.n_b;
-    const int nt = token_tiles(block_tokens(pa.T, pa.block_len, b));
+    const int nt = token_tiles(BlockGeo{pa.T, pa.block_len, pa.starts}.len(b));
     const int64_t base = kv.offsets[blk];
     const float *Wb = pa.W[kind] + (int64_t)blk * D * D + (int64_t)j * D;
     float s = 0.f;

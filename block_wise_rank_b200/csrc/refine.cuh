@@ -31,14 +31,14 @@ struct RefineSmem {
 template <typename T>
 __global__ void __launch_bounds__(RF_THREADS) k_refine_sigma(const T *__restrict__ K, const T *__restrict__ V,
                                                              float *__restrict__ W_io, float *__restrict__ sigma_K,
-                                                             float *__restrict__ sigma_V, int Tn, int block_len,
-                                                             int n_b, int64_t n_blk) {
+                                                             float *__restrict__ sigma_V, BlockGeo geo, int n_b,
+                                                             int64_t n_blk) {
     extern __shared__ __align__(16) unsigned char rf_raw[];
     RefineSmem &sm = *reinterpret_cast<RefineSmem *>(rf_raw);
     const int blk = blockIdx.x, kind = blockIdx.y, tid = threadIdx.x;
     const int lh = blk / n_b, b = blk % n_b;
-    const int Tb = block_tokens(Tn, block_len, b);
-    const T *Xb = (kind == 0 ? K : V) + ((int64_t)lh * Tn + (int64_t)b * block_len) * D;
+    const int Tb = geo.len(b);
+    const T *Xb = (kind == 0 ? K : V) + ((int64_t)lh * geo.T + geo.start(b)) * D;
     float *Wg = W_io + ((int64_t)kind * n_blk + blk) * D * D;
     for (int e = tid; e < D * D; e += RF_THREADS) sm.W[e / D][e % D] = Wg[e];
     __syncthreads();

@@ -32,7 +32,8 @@ DTYPES = {"f32": MILO_F32, "bf16": MILO_BF16, "int8": MILO_INT8, "int2": MILO_IN
 
 class milo_cache_shape(ctypes.Structure):
     _fields_ = [("L", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("d", ctypes.c_int32),
-                ("block_len", ctypes.c_int32), ("in_dtype", ctypes.c_int)]
+                ("block_len", ctypes.c_int32), ("in_dtype", ctypes.c_int), ("n_blocks", ctypes.c_int32),
+                ("block_starts", ctypes.c_void_p)]
 
 
 class milo_compress_params(ctypes.Structure):
@@ -56,7 +57,7 @@ EXPORTS = [
     "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
     "milo_jacobi_rounds", "milo_decode_tail_workspace_size", "milo_decode_attn_tail",
     "milo_decode_offload_workspace_size", "milo_decode_attn_offload", "milo_bm25_workspace_size",
-    "milo_bm25_select",
+    "milo_bm25_select", "milo_factors_shape",
 ]
 
 # stages of milo_timing_read, in order (milo_timed_stage)
@@ -112,6 +113,8 @@ def lib():
         L.milo_factors_import.argtypes = [P, SZ, P, SZ, ctypes.POINTER(P), P]
         L.milo_factors_import.restype = ctypes.c_int
         L.milo_factors_destroy.argtypes = [P]; L.milo_factors_destroy.restype = None
+        L.milo_factors_shape.argtypes = [P, ctypes.POINTER(milo_cache_shape), ctypes.POINTER(milo_compress_params)]
+        L.milo_factors_shape.restype = ctypes.c_int
         L.milo_get_status.argtypes = [P]; L.milo_get_status.restype = ctypes.c_int
         L.milo_status_string.argtypes = [ctypes.c_int]; L.milo_status_string.restype = ctypes.c_char_p
         L.milo_version.argtypes = []; L.milo_version.restype = ctypes.c_char_p
@@ -164,10 +167,24 @@ def default_params(**kw) -> milo_compress_params:
     return p
 
 
-def cache_shape(L, H, T, d, block_len, in_dtype) -> milo_cache_shape:
+def cache_shape(L, H, T, d, block_len, in_dtype, starts=None) -> milo_cache_shape:
+    """The C shape; `starts` (token offsets of variable-length blocks, n_b + 1
+    values from 0 to T) is kept alive on the returned object."""
     if isinstance(in_dtype, torch.dtype):
         in_dtype = _dtype_code(in_dtype)
-    return milo_cache_shape(L, H, T, d, block_len, in_dtype)
+    if starts is None:
+        return milo_cache_shape(L, H, T, d, block_len, in_dtype, 0, None)
+    arr = (ctypes.c_int32 * len(starts))(*[int(x) for x in starts])
+    s = milo_cache_shape(L, H, T, d, block_len, in_dtype, len(starts) - 1, ctypes.cast(arr, ctypes.c_void_p))
+    s._starts = arr
+    return s
+
+
+def block_starts(shape: milo_cache_shape):
+    """The variable blocks' starts of a shape (a list), or None."""
+    if not shape.n_blocks or not shape.block_starts:
+        return None
+    return list((ctypes.c_int32 * (shape.n_blocks + 1)).from_address(shape.block_starts))
 
 
 def milo_factor_arena_size(shape, params) -> int:
@@ -217,12 +234,14 @@ class Factors:
 
 
 def milo_compress(K: torch.Tensor, V: torch.Tensor, block_len: int, params=None, workspace=None,
-                  arena=None, stream=None) -> Factors:
-    """Compress caches K (pre-RoPE) and V, [L][H][T][d] device tensors."""
+                  arena=None, stream=None, starts=None) -> Factors:
+    """Compress caches K (pre-RoPE) and V, [L][H][T][d] device tensors.  With
+    `starts` (n_b + 1 token offsets) the blocks have variable lengths and
+    block_len is the longest."""
     assert K.shape == V.shape and K.dtype == V.dtype and K.is_cuda and V.is_cuda
     assert K.is_contiguous() and V.is_contiguous()
     L, H, T, d = K.shape
-    shape = cache_shape(L, H, T, d, block_len, K.dtype)
+    shape = cache_shape(L, H, T, d, block_len, K.dtype, starts)
     params = params or default_params()
     ws_n = milo_compress_workspace_size(shape, params)
     ar_n = milo_factor_arena_size(shape, params)
@@ -402,11 +421,9 @@ def milo_factors_import(blob: bytes, arena: torch.Tensor, stream=None) -> Factor
     h = ctypes.c_void_p()
     _check(lib().milo_factors_import(blob, len(blob), _ptr(arena), arena.numel() * arena.element_size(),
                                      ctypes.byref(h), _stream(stream)), "milo_factors_import")
-    # recover shape/params from the blob header fields
-    shape = milo_cache_shape.from_buffer_copy(blob[16:16 + ctypes.sizeof(milo_cache_shape)])
-    off = 16 + ctypes.sizeof(milo_cache_shape)
-    off = (off + 7) // 8 * 8
-    params = milo_compress_params.from_buffer_copy(blob[off:off + ctypes.sizeof(milo_compress_params)])
+    # shape and params from the new handle (its block starts stay valid while it lives)
+    shape, params = milo_cache_shape(), milo_compress_params()
+    _check(lib().milo_factors_shape(h, ctypes.byref(shape), ctypes.byref(params)), "milo_factors_shape")
     return Factors(h, arena, shape, params)
 
 

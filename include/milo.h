@@ -69,8 +69,21 @@ typedef struct {
     int32_t H;          /* KV heads per layer                            */
     int32_t T;          /* tokens per (layer, head)                      */
     int32_t d;          /* head dimension; must be 128                   */
-    int32_t block_len;  /* tokens per block (>= 1); the last may be short */
+    int32_t block_len;  /* tokens per block (>= 1); the last may be short;
+                           with block_starts: the longest block's tokens */
     milo_dtype in_dtype;/* MILO_F32 or MILO_BF16                         */
+    /* Variable-length blocks, or 0 / NULL for fixed block_len.  Host array of
+     * n_blocks + 1 token offsets shared by every (layer, head): block b =
+     * tokens [block_starts[b], block_starts[b+1]); block_starts[0] = 0,
+     * block_starts[n_blocks] = T, every length in [1, block_len].  Blocks
+     * that each hold whole demonstrations ("MILO ... Block-wise Low-rank
+     * Compression", shd-paper mirror, original abstract: each block holds
+     * several many-shot examples).  The handle keeps its own copy, and the
+     * arena a device copy (its `starts` array below).  With variable blocks
+     * the Gram runs on CUDA cores (the tensor-core Gram needs whole
+     * fixed-length blocks). */
+    int32_t n_blocks;
+    const int32_t *block_starts;
 } milo_cache_shape;
 
 typedef struct {
@@ -98,6 +111,7 @@ typedef struct milo_factors milo_factors;
  * Factor arena layout (device, caller-owned, one section per kind: K then V,
  * each section start 256-byte aligned; N_blk = L*H*n_b, n_b = ceil(T /
  * block_len)):
+ *   int32  starts [n_b + 1]     variable-length blocks: their token starts (unused otherwise)
  *   int32  ranks  [N_blk]
  *   int64  offsets[N_blk + 1]   element offset of block b in data (bytes for MILO_INT2)
  *   float  sigma  [N_blk][d]    singular values, descending
@@ -332,7 +346,9 @@ milo_status milo_factors_get(const milo_factors *f, int32_t kind, int32_t **rank
                              float **scaleB, int64_t *R);
 
 /* Wrap an arena already filled in the documented layout (for instance by
- * the caller) in a new handle.  No device access. */
+ * the caller; with variable blocks its starts array holds shape's
+ * block_starts, as milo_compress writes it) in a new handle.  No device
+ * access. */
 milo_status milo_factors_wrap(const milo_cache_shape *shape, const milo_compress_params *params,
                               void *arena, size_t arena_bytes, milo_factors **out);
 
@@ -345,6 +361,11 @@ milo_status milo_factors_export(const milo_factors *f, void *host_buf, size_t *b
  * recorded in the blob) and return a handle over it.  Synchronises stream. */
 milo_status milo_factors_import(const void *host_buf, size_t bytes, void *arena, size_t arena_bytes,
                                 milo_factors **out, milo_stream_t stream);
+
+/* The handle's shape and params.  A variable-block shape's block_starts
+ * points at the handle's own copy, valid while the handle lives.  Any
+ * output may be NULL. */
+milo_status milo_factors_shape(const milo_factors *f, milo_cache_shape *shape, milo_compress_params *params);
 
 /* Free the handle only; the arena stays the caller's. */
 void milo_factors_destroy(milo_factors *f);

@@ -72,7 +72,8 @@ def unpack(f: milo.Factors, kind: int):
     (p_r, p_o, p_s, p_e, p_d, p_sa, p_sb), R = f.view(kind)
     sh, pr = f.shape, f.params
     L, H, T, d, bl = sh.L, sh.H, sh.T, sh.d, sh.block_len
-    nb = math.ceil(T / bl)
+    starts = milo.block_starts(sh)
+    nb = len(starts) - 1 if starts else math.ceil(T / bl)
     nblk = L * H * nb
     ranks = arena_tensor(f, p_r, 4 * nblk).view(torch.int32).cpu().numpy().copy()
     offs = arena_tensor(f, p_o, 8 * (nblk + 1)).view(torch.int64).cpu().numpy().copy()
@@ -98,7 +99,7 @@ def unpack(f: milo.Factors, kind: int):
     A, B, Aq, Bq, A_scale, A_zero = [], [], [], [], [], []
     for blk in range(nblk):
         b = blk % nb
-        tb = min(bl, T - b * bl)
+        tb = starts[b + 1] - starts[b] if starts else min(bl, T - b * bl)
         r = int(ranks[blk])
         if dt == milo.MILO_INT2:
             # codes four per byte (token u%4 at bits 2(u%4)), then B's INT8

@@ -56,7 +56,7 @@ def test_budget_matches_oracle_formula(L, oracle_mod):
 
 
 def test_arena_size_layout(L):
-    # section = ranks | offsets | sigma | eps | [scaleA | scaleB] | data, each 256-byte aligned
+    # section = starts | ranks | offsets | sigma | eps | [scaleA | scaleB] | data, each 256-byte aligned
     def al(x):
         return (x + 255) // 256 * 256
     for dt, es in ((milo.MILO_F32, 4), (milo.MILO_BF16, 2), (milo.MILO_INT8, 1)):
@@ -66,7 +66,7 @@ def test_arena_size_layout(L):
             nb = math.ceil(T / bl)
             nblk = Ln * H * nb
             R = milo.milo_rank_budget(s, p)
-            sec = al(4 * nblk) + al(8 * (nblk + 1)) + al(4 * nblk * 128) + al(8 * Ln * H)
+            sec = al(4 * (nb + 1)) + al(4 * nblk) + al(8 * (nblk + 1)) + al(4 * nblk * 128) + al(8 * Ln * H)
             if dt == milo.MILO_INT8:
                 sec += 2 * al(4 * nblk * 128)
             sec += al((R + 7 * nblk) * ((bl + 127) // 128 * 128 + 128) * es)
@@ -129,7 +129,7 @@ def test_wrap_views_and_export_size(L):
     ptrs = [P() for _ in range(7)]
     R = ctypes.c_int64()
     assert L.milo_factors_get(h, 0, *[ctypes.byref(x) for x in ptrs], ctypes.byref(R)) == 0
-    assert ptrs[0].value == (1 << 20)
+    assert ptrs[0].value == (1 << 20) + 256   # ranks after the (256-byte aligned) block-starts array
     assert R.value == milo.milo_rank_budget(s, p)
     k1 = [P() for _ in range(7)]
     assert L.milo_factors_get(h, 1, *[ctypes.byref(x) for x in k1], ctypes.byref(R)) == 0

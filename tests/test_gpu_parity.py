@@ -36,13 +36,12 @@ def _lib():
     assert torch.cuda.is_available()
 
 
-def _oracle_block_svds(oracle_mod, X, block_len, blocks):
+def _oracle_block_svds(oracle_mod, X, block_len, blocks, starts=None):
     """Oracle SVD of the listed (l, h, b) blocks of one kind."""
     out = {}
-    T = X.shape[2]
+    bounds = oracle_mod.block_bounds(X.shape[2], block_len, starts)
     for (l, h, b) in blocks:
-        Xb = X[l, h, b * block_len:min((b + 1) * block_len, T)]
-        out[(l, h, b)] = oracle_mod.svd(Xb)
+        out[(l, h, b)] = oracle_mod.svd(X[l, h, bounds[b][0]:bounds[b][1]])
     return out
 
 
@@ -67,17 +66,18 @@ def _rel_inf(a, b):
     return np.abs(a - b).max() / np.abs(b).max()
 
 
-def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None):
+def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None, starts=None):
     """Run milo_compress, check sigma/eps/ranks/offsets/reconstruction; return unpacked factors."""
     Kd, Vd = K.cuda(), V.cuda()
-    f = milo.milo_compress(Kd, Vd, block_len, params)
+    f = milo.milo_compress(Kd, Vd, block_len, params, starts=starts)
     st = milo.milo_get_status()
     assert st == milo.MILO_OK, milo.status_string(st)
     L, H, T, d = K.shape
-    nb = math.ceil(T / block_len)
+    bounds = oracle_mod.block_bounds(T, block_len, starts)
+    nb = len(bounds)
     Kn = K.double().numpy() if K.dtype != torch.bfloat16 else K.float().double().numpy()
     Vn = V.double().numpy() if V.dtype != torch.bfloat16 else V.float().double().numpy()
-    R = oracle_mod.budget(L, H, T, block_len, d, params.budget_frac, params.budget_abs)
+    R = oracle_mod.budget(L, H, T, block_len, d, params.budget_frac, params.budget_abs, starts=starts)
     if sample_blocks is None:
         sample_blocks = [(l, h, b) for l in range(L) for h in range(H) for b in range(nb)]
     U = []
@@ -92,20 +92,22 @@ def _compress_and_check(oracle_mod, K, V, block_len, params, sample_blocks=None)
         assert np.array_equal(u["eps"], eps_ref.reshape(-1))
         # ranks: bit-exact against the oracle allocator on the same sigma and eps
         r_ref = oracle_mod.allocate(u["sigma"].astype(np.float64).reshape(L, H, nb, d), u["eps"].reshape(L, H),
-                                    T, block_len, R, params.r_min, params.r_max)
+                                    T, block_len, R, params.r_min, params.r_max, starts=starts)
         assert np.array_equal(u["ranks"], r_ref.reshape(-1))
-        # offsets: exclusive scan of round_up(r_b, 8) (128 ceil(T_b / 128) + d)
-        lens = oracle_mod.block_lengths(T, block_len) * (L * H)
-        sizes = np.array([(r + 7) // 8 * 8 * ((tb + 127) // 128 * 128 + d) for r, tb in zip(u["ranks"], lens)],
+        # offsets: exclusive scan of round_up(r_b, 8) (128 ceil(T_b / 128) + d) elements,
+        # or of round_up(r_b, 8) (48 ceil(T_b / 128) + d) bytes for 2-bit codes
+        lens = oracle_mod.block_lengths(T, block_len, starts) * (L * H)
+        per = (lambda nt: 48 * nt + d) if params.factor_dtype == milo.MILO_INT2 else (lambda nt: 128 * nt + d)
+        sizes = np.array([(r + 7) // 8 * 8 * per((tb + 127) // 128) for r, tb in zip(u["ranks"], lens)],
                          dtype=np.int64)
         assert np.array_equal(u["offsets"], np.concatenate([[0], np.cumsum(sizes)]))
         # sigma and reconstruction against the oracle SVD on sampled blocks
-        ref = _oracle_block_svds(oracle_mod, X, block_len, sample_blocks)
+        ref = _oracle_block_svds(oracle_mod, X, block_len, sample_blocks, starts)
         for (l, h, b), (s_ref, _, _, _) in ref.items():
             blk = (l * H + h) * nb + b
             _check_sigma(u["sigma"][blk].astype(np.float64), s_ref)
             rb = int(u["ranks"][blk])
-            Xb = X[l, h, b * block_len:min((b + 1) * block_len, T)]
+            Xb = X[l, h, bounds[b][0]:bounds[b][1]]
             Xh = u["A"][blk] @ u["B"][blk] if rb else np.zeros_like(Xb)
             err = np.sum((Xb - Xh) ** 2)
             tail = np.sum(s_ref[rb:] ** 2)
@@ -629,3 +631,36 @@ def test_int2_codes_and_decode(oracle_mod):
         ref = _decode_ref(oracle_mod, U[0], U[1], 0, hq // 4, 4, q[0, 0, hq].double().numpy(), [0, 1, 3],
                           [0, 256, 768], 1e6)
         assert _rel_inf(out[0, 0, hq], ref) <= DEC_TOL, (hq, _rel_inf(out[0, 0, hq], ref))
+
+
+@pytest.mark.parametrize("factor", ["bf16", "f32", "int8", "int2"])
+def test_variable_length_blocks(oracle_mod, factor):
+    """Shot-aligned blocks given by their starts (lengths 100, 250, 7, 243,
+    400, 100, 400 of a 1500-token cache; the longest 400): sigma, eps, ranks,
+    offsets and reconstruction against the oracle on the same slices, then
+    decode at the blocks' own start positions against the oracle on the same
+    factors, and an export/import round trip that keeps the starts."""
+    starts = [0, 100, 350, 357, 600, 1000, 1100, 1500]
+    L, H, G, T, bl = 2, 2, 4, 1500, 400
+    dt = torch.float32 if factor == "f32" else torch.bfloat16
+    K = synth.planted_cache(L, H, T, 128, 300, (3.0, 30.0), seed=81, out_dtype=dt)
+    V = synth.planted_cache(L, H, T, 128, 300, (8.0, 60.0), seed=82, out_dtype=dt)
+    f, U = _compress_and_check(oracle_mod, K, V, bl, milo.default_params(factor_dtype=factor, budget_frac=0.4),
+                               starts=starts)
+    g = torch.Generator().manual_seed(83)
+    S = 3
+    q = torch.randn(L, S, H * G, 128, generator=g)
+    sel = torch.tensor([[1, 2, 6], [0, 3, 4], [2, 5, 1]], dtype=torch.int32)
+    out = milo.milo_decode_attn(f, q.cuda(), sel.cuda(), None, rope_base=1e6).cpu().numpy()
+    assert milo.milo_get_status() == milo.MILO_OK
+    nb = len(starts) - 1
+    for (l, s, hq) in [(0, 0, 0), (1, 1, 5), (0, 2, 7), (1, 0, 3)]:
+        ref = _decode_ref(oracle_mod, U[0], U[1], l, hq // G, nb, q[l, s, hq].double().numpy(), sel[s].tolist(),
+                          [starts[b] for b in sel[s].tolist()], 1e6)
+        assert _rel_inf(out[l, s, hq], ref) <= DEC_TOL, (l, s, hq, _rel_inf(out[l, s, hq], ref))
+    blob = milo.milo_factors_export(f)
+    arena2 = torch.empty_like(f.arena)
+    f2 = milo.milo_factors_import(blob, arena2)
+    assert milo.block_starts(f2.shape) == starts
+    out2 = milo.milo_decode_attn(f2, q.cuda(), sel.cuda(), None, rope_base=1e6).cpu().numpy()
+    assert np.array_equal(out, out2)
