@@ -59,7 +59,7 @@ DECODE_SOURCES = ("block_wise_rank_b200/csrc/decode_tc.cuh", "block_wise_rank_b2
                   "block_wise_rank_b200/csrc/common.cuh")
 # the other rows: (workload, rank budget, factor dtype)
 ROWS = [("qwen7b-128k", 0.25, "bf16", 0), ("qwen7b-128k", 0.75, "bf16", 0), ("qwen7b-128k", 0.5, "int8", 0),
-        ("qwen7b-128k", 0.5, "int2", 0),
+        ("qwen7b-128k", 0.5, "int2", 0), ("qwen7b-128k-shots", 0.5, "bf16", 0),
         ("qwen7b-128k", 0.5, "bf16", 512), ("qwen7b-64k", 0.5, "bf16", 0), ("qwen3b-32k", 0.5, "bf16", 0)]
 
 
@@ -179,7 +179,7 @@ def decode_bytes(ranks, w, sel, factor, S, Hq):
     nb = w.n_b
     uniq = torch.zeros(nb, dtype=torch.bool)
     uniq[sel.reshape(-1).long().cpu()] = True
-    tb = torch.tensor([min(w.block_len, w.T - b * w.block_len) for b in range(nb)], dtype=torch.float64)
+    tb = torch.tensor([w.block_tokens(b) for b in range(nb)], dtype=torch.float64)
     mask = uniq.to(torch.float64)
     per = block_factor_bytes(rk.to(torch.float64).reshape(w.L * w.H, nb), rv.to(torch.float64).reshape(w.L * w.H, nb),
                              tb[None, :], w.d, factor)
@@ -193,7 +193,7 @@ def read_ranks(f):
     out = []
     for kind in range(2):
         (p_r, *_), _ = f.view(kind)
-        n = f.shape.L * f.shape.H * math.ceil(f.shape.T / f.shape.block_len)
+        n = f.shape.L * f.shape.H * (f.shape.n_blocks or math.ceil(f.shape.T / f.shape.block_len))
         base = f.arena.data_ptr()
         out.append(f.arena[p_r - base:p_r - base + 4 * n].view(torch.int32).cpu())
     return out
@@ -259,12 +259,13 @@ class Run:
         torch.cuda.synchronize()
         self.n_dec = n_dec or w.steps
         self.stream = torch.cuda.current_stream()
-        shape = milo.cache_shape(w.L, w.H, w.T, w.d, w.block_len, self.K.dtype)
+        shape = milo.cache_shape(w.L, w.H, w.T, w.d, w.block_len, self.K.dtype, w.starts)
         self.ws = torch.empty(milo.milo_compress_workspace_size(shape, self.params), dtype=torch.uint8, device=dev)
         self.arena = torch.empty(milo.milo_factor_arena_size(shape, self.params), dtype=torch.uint8, device=dev)
         # per-step decode inputs (different seeded queries / selections per decode step)
         self.dec_inputs = [synth.decode_inputs(w, step=i, device=dev) for i in range(self.n_dec)]
-        self.f = milo.milo_compress(self.K, self.V, w.block_len, self.params, workspace=self.ws, arena=self.arena)
+        self.f = milo.milo_compress(self.K, self.V, w.block_len, self.params, workspace=self.ws, arena=self.arena,
+                                    starts=w.starts)
         wsz = (milo.milo_decode_tail_workspace_size if tail else milo.milo_decode_workspace_size)
         self.dws = torch.empty(wsz(self.f, w.sessions, w.Hq, w.n_sel), dtype=torch.uint8, device=dev)
         # recent uncompressed tokens of every session, in the cache's element type
@@ -276,7 +277,8 @@ class Run:
         if ev:
             ev[0].record(self.stream)
         self.f.close()
-        self.f = milo.milo_compress(self.K, self.V, w.block_len, self.params, workspace=self.ws, arena=self.arena)
+        self.f = milo.milo_compress(self.K, self.V, w.block_len, self.params, workspace=self.ws, arena=self.arena,
+                                    starts=w.starts)
         if ev:
             ev[1].record(self.stream)
         for (q, sel, pos) in self.dec_inputs:
@@ -378,7 +380,7 @@ def compression_roofline(run, t, steps, pk):
     if n:
         # bytes written: every block's padded factors (R8 rank rows, whole 128-token tiles)
         ranks = read_ranks(run.f)
-        nt = torch.tensor([-(-min(w.block_len, w.T - b * w.block_len) // 128) for b in range(w.n_b)],
+        nt = torch.tensor([-(-w.block_tokens(b) // 128) for b in range(w.n_b)],
                           dtype=torch.float64).repeat(w.L * w.H)
         per_r8 = 48 * nt + w.d if run.factor == "int2" else (128 * nt + w.d) * factor_bytes_per_elem(run.factor)
         fac = float(sum((((r.to(torch.float64) + 7) // 8 * 8) * per_r8).sum() for r in ranks))
@@ -408,6 +410,7 @@ def row_of(run, t, steps, pk):
                     kernel_frac_hbm=round(tgbs / pk["hbm"], 4) if tgbs else None)
     return dict(workload=w.name, layers=w.L, kv_heads=w.H, gqa=w.G, tokens=w.T, block_len=w.block_len,
                 sessions=w.sessions, selected=f"{w.n_sel}/{w.n_b}", decode_steps=run.n_dec,
+                blocks="shot-aligned, variable length" if w.starts else "fixed length",
                 budget=run.budget, factor=run.factor, recent_tail=tail,
                 decode=dict(gbs=round(gbs, 2), frac_hbm=round(gbs / pk["hbm"], 4),
                             kernel_gbs=round(kgbs, 2) if kgbs else None,
@@ -494,7 +497,7 @@ def offload_measure(run, reps=3):
     fbytes = decode_bytes(read_ranks(run.f), w, sel, run.factor, w.sessions, w.Hq) - \
         (2 * w.L * w.sessions * w.Hq * w.d * 4 + 2 * sel.numel() * 4)
     uniq = sorted(set(sel.reshape(-1).tolist()))
-    kv_tokens = sum(min(w.block_len, w.T - b * w.block_len) for b in uniq)
+    kv_tokens = sum(w.block_tokens(b) for b in uniq)
     kv_bytes = 2 * w.L * w.H * kv_tokens * w.d * run.K.element_size()
     del ws, out
     fh.close()

@@ -45,14 +45,39 @@ class Workload:
     noise: float = 1e-3
     rope_base: float = 1e6
     factor_dtypes: tuple = field(default=("same",))
+    starts: tuple = None     # variable-length blocks' token starts (block_len = the longest), or None
 
     @property
     def n_b(self) -> int:
-        return math.ceil(self.T / self.block_len)
+        return len(self.starts) - 1 if self.starts else math.ceil(self.T / self.block_len)
+
+    def block_start(self, b: int) -> int:
+        return self.starts[b] if self.starts else b * self.block_len
+
+    def block_tokens(self, b: int) -> int:
+        return self.starts[b + 1] - self.starts[b] if self.starts else min(self.block_len, self.T - b * self.block_len)
 
     @property
     def Hq(self) -> int:
         return self.H * self.G
+
+
+def shot_starts(T: int, max_len: int, seed: int, shot_range=(48, 160)):
+    """Shot-aligned block starts: demonstrations of uniform random length in
+    `shot_range` tokens packed whole into blocks of at most `max_len` tokens
+    (a demonstration that does not fit opens the next block); the last
+    demonstration ends at T."""
+    g = torch.Generator().manual_seed(seed)
+    starts, cur, pos = [0], 0, 0
+    while pos < T:
+        n = min(int(torch.randint(shot_range[0], shot_range[1] + 1, (1,), generator=g)), T - pos)
+        if cur + n > max_len:
+            starts.append(pos)
+            cur = 0
+        cur += n
+        pos += n
+    starts.append(T)
+    return tuple(starts)
 
 
 # The five workloads: a toy fp32 case, a one-layer Qwen2.5-3B-shaped case,
@@ -76,6 +101,11 @@ WORKLOADS = {
                             sessions=32, n_sel=64, steps=1, seed=5,
                             factor_dtypes=("bf16", "int8")),
 }
+# the 131072-token cache in shot-aligned blocks of at most 512 tokens
+WORKLOADS["qwen7b-128k-shots"] = Workload(
+    "qwen7b-128k-shots", L=28, H=4, G=7, T=131072, block_len=512, dtype="bf16", tau_k=(2.0, 48.0),
+    tau_v=(8.0, 96.0), budgets=(0.5,), sessions=32, n_sel=64, steps=1, seed=6,
+    starts=shot_starts(131072, 512, 6 * 1000 + 500))
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -180,7 +210,10 @@ def decode_inputs(w: Workload, step: int = 0, device="cpu"):
     g = _gen(w.seed * 1000 + 100 + step, "cpu")
     q = torch.randn(w.L, w.sessions, w.Hq, w.d, generator=g, dtype=torch.float32).to(device)
     sel = retrieval_standin(w.n_b, w.sessions, w.n_sel, w.seed * 1000 + 200 + step, device)
-    pos = (sel.to(torch.int64) * w.block_len).to(torch.int32)
+    if w.starts:
+        pos = torch.tensor(w.starts, dtype=torch.int32, device=sel.device)[sel.long()]
+    else:
+        pos = (sel.to(torch.int64) * w.block_len).to(torch.int32)
     return q, sel, pos
 
 
