@@ -80,6 +80,8 @@ def parse():
     ap.add_argument("--row-steps", type=int, default=2, help="timed steps per row (one warm-up step each)")
     ap.add_argument("--profile", action="store_true",
                     help="only the warm-up and timed steps (for ncu launch lists): no profiler, e2e or CPU legs")
+    ap.add_argument("--tail", type=int, default=0, metavar="N",
+                    help="profiling: each session's N recent uncompressed tokens in every decode (milo_decode_attn_tail)")
     ap.add_argument("--timeline", type=int, default=-1, metavar="CTA",
                     help="decode timeline of one CTA of k_decode_tc from the tracing build; prints a summary, no JSON")
     return ap.parse_args()
@@ -710,7 +712,7 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     w = workload_of(args.workload, args.layers)
     factor = args.factor or ("f32" if w.dtype == "f32" else "bf16")
-    run = Run(w, args.budget, factor, dev, args.decode_steps)
+    run = Run(w, args.budget, factor, dev, args.decode_steps, tail=args.tail)
     S, Hq = w.sessions, w.Hq
     if args.profile:
         for _ in range(args.warmup + args.steps):
