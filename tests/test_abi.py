@@ -208,3 +208,21 @@ def test_next_entry_points_reject_bad_arguments_on_host(L):
     data = (R + 7 * nblk) * (48 * nt + 128)
     assert milo.milo_factor_arena_size(s, p2) >= 2 * data
     assert milo.milo_factor_arena_size(s, p2) < milo.milo_factor_arena_size(s, p16)
+
+
+def test_block_starts_validated_and_budget_on_host(L, oracle_mod):
+    """Variable-length blocks: the rank budget follows the oracle's formula
+    over the given lengths; starts that do not run from 0 to T, that go
+    backwards, or that make a block longer than block_len (the longest) are
+    refused by every size query (0 / -1) before any device work; the arena
+    grows by the starts array only."""
+    starts = [0, 100, 350, 357, 600, 1000, 1100, 1500]
+    p = milo.default_params(budget_frac=0.4)
+    s = milo.cache_shape(2, 2, 1500, 128, 400, milo.MILO_BF16, starts)
+    assert milo.milo_rank_budget(s, p) == oracle_mod.budget(2, 2, 1500, 400, 128, 0.4, starts=starts)
+    assert milo.milo_factor_arena_size(s, p) > 0 and milo.milo_compress_workspace_size(s, p) > 0
+    for bad in ([0, 100, 90, 1500], [5, 100, 1500], [0, 100, 1499], [0, 100, 600, 1500]):
+        sb = milo.cache_shape(2, 2, 1500, 128, 400, milo.MILO_BF16, bad)
+        assert milo.milo_factor_arena_size(sb, p) == 0, bad
+        assert milo.milo_rank_budget(sb, p) == -1, bad
+    assert milo.block_starts(s) == starts and milo.block_starts(milo.cache_shape(1, 1, 10, 128, 5, 0)) is None
