@@ -11,12 +11,12 @@
 // cached them: already rotated to their own positions, like q.
 //
 // One CTA per (KV head, session, layer) reads that head's tail once for all
-// of its G query heads: 32-token chunks of K and V staged in shared memory,
-// scores by thread-per-(query, token) dot products, an online softmax per
-// query head, and thread j accumulating output channel j.  The result is one
-// more partial (max, sum, normalised output) per query row, which k_combine
-// merges with the block partials.  The work is a few MACs per byte; the
-// kernel streams K and V once (HBM-bound).
+// of its G query heads: 32-token rounds of K and V staged in shared memory,
+// score dot products split over the four warps by quarters of d, an online
+// softmax per query head, and thread j accumulating output channel j.  The
+// result is one more partial (max, sum, normalised output) per query row,
+// which k_combine merges with the block partials.  The work is a few MACs per
+// byte; the kernel streams K and V once (HBM-bound).
 #pragma once
 #include "decode_simt.cuh"
 
