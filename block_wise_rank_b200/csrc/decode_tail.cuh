@@ -25,10 +25,12 @@ namespace milo {
 constexpr int TAIL_CHUNK = 32;   // tail tokens per round
 constexpr int TAIL_GSUB = 8;     // query heads of one KV head per pass over the tail (static smem < 48 KB)
 
-struct alignas(16) TailSmem {
+// K and V are staged in their own element type (bf16 rows take half the
+// shared-memory traffic of fp32 ones) and widened as they are read.
+template <typename T> struct alignas(16) TailSmem {
     float q[TAIL_GSUB][D];
-    float k[TAIL_CHUNK][D + 4];              // padded rows: 16-byte reads of 32 different rows are conflict-free
-    float v[TAIL_CHUNK][D];
+    T k[TAIL_CHUNK][D + 16 / sizeof(T)];     // padded rows: 16-byte reads of 32 different rows are conflict-free
+    T v[TAIL_CHUNK][D];
     float p[TAIL_GSUB][TAIL_CHUNK];
     float part[4][TAIL_GSUB][TAIL_CHUNK];    // score partials of the four quarters of d
     float m[TAIL_GSUB], l[TAIL_GSUB], f[TAIL_GSUB];
@@ -65,8 +67,8 @@ template <> struct TailVec<__nv_bfloat16> {
 //   tail_o: [L][S][Hq][D] normalised outputs; tail_ml: [L][S][Hq] (max score,
 //   sum of exp(score - max)); an empty tail leaves (-inf, 0) and zeros.
 // Each round loads a 32-token chunk of K and V as 16-byte vectors, all issued
-// before the first is used, and stages both in shared memory as fp32; thread
-// j then accumulates output channel j of every query head.
+// before the first is used, and stages both in shared memory as they came;
+// thread j then accumulates output channel j of every query head.
 template <typename T>
 __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__restrict__ k_tail,
                                                    const T *__restrict__ v_tail, int tail_cap,
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
     constexpr int NV = TAIL_CHUNK * VPR / 128;         // vectors per thread and array (rows per thread)
     constexpr int NGRP = 128 / VPR;                    // threads loading the same channels of different rows
     static_assert(NV * NGRP == TAIL_CHUNK, "row groups");
-    __shared__ TailSmem sm;
+    __shared__ TailSmem<T> sm;
     const int h = blockIdx.x, s = blockIdx.y, l = blockIdx.z;
     const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
     const int cgrp = j % VPR, rgrp = j / VPR;          // channels [EPV cgrp, +EPV), rows rgrp + NGRP i
@@ -115,16 +117,8 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
             __syncthreads();   // previous round's k, p and f used; q, m, l written
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                float x[EPV], y[EPV];
-                TailVec<T>::get(kr[i], x);
-                TailVec<T>::get(vr[i], y);
-                float4 *dk = reinterpret_cast<float4 *>(&sm.k[rgrp + NGRP * i][cgrp * EPV]);
-                float4 *dv = reinterpret_cast<float4 *>(&sm.v[rgrp + NGRP * i][cgrp * EPV]);
-#pragma unroll
-                for (int e = 0; e < EPV / 4; ++e) {
-                    dk[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
-                    dv[e] = make_float4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3]);
-                }
+                *reinterpret_cast<uint4 *>(&sm.k[rgrp + NGRP * i][cgrp * EPV]) = kr[i];
+                *reinterpret_cast<uint4 *>(&sm.v[rgrp + NGRP * i][cgrp * EPV]) = vr[i];
             }
             __syncthreads();
             // scores: warp w dots dims [32w, 32w + 32) of key t = lane with every
@@ -134,15 +128,22 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
                 float sp[TAIL_GSUB];
 #pragma unroll
                 for (int g = 0; g < TAIL_GSUB; ++g) sp[g] = 0.f;
-                const float4 *kt = reinterpret_cast<const float4 *>(sm.k[lane]) + 8 * warp;
+                // dims [32 warp, 32 warp + 32) of key `lane`: 32 / EPV vectors
+                const uint4 *kt = reinterpret_cast<const uint4 *>(&sm.k[lane][32 * warp]);
 #pragma unroll
-                for (int d4 = 0; d4 < 8; ++d4) {
-                    const float4 b4 = kt[d4];
+                for (int vi = 0; vi < 32 / EPV; ++vi) {
+                    float x[EPV];
+                    TailVec<T>::get(kt[vi], x);
 #pragma unroll
-                    for (int g = 0; g < TAIL_GSUB; ++g) {
-                        if (g >= gn) break;
-                        const float4 a4 = reinterpret_cast<const float4 *>(sm.q[g])[8 * warp + d4];
-                        sp[g] = fmaf(a4.w, b4.w, fmaf(a4.z, b4.z, fmaf(a4.y, b4.y, fmaf(a4.x, b4.x, sp[g]))));
+                    for (int e4 = 0; e4 < EPV / 4; ++e4) {
+                        const int d4 = 8 * warp + vi * (EPV / 4) + e4;   // float4 index into q
+#pragma unroll
+                        for (int g = 0; g < TAIL_GSUB; ++g) {
+                            if (g >= gn) break;
+                            const float4 a4 = reinterpret_cast<const float4 *>(sm.q[g])[d4];
+                            sp[g] = fmaf(a4.w, x[4 * e4 + 3],
+                                         fmaf(a4.z, x[4 * e4 + 2], fmaf(a4.y, x[4 * e4 + 1], fmaf(a4.x, x[4 * e4], sp[g]))));
+                        }
                     }
                 }
 #pragma unroll
@@ -182,8 +183,8 @@ __global__ void __launch_bounds__(128) k_tail_attn(DecodeArgs a, const T *__rest
                 if (g < gn) acc[g] *= sm.f[g];
 #pragma unroll 2
             for (int t4 = 0; t4 < TAIL_CHUNK / 4; ++t4) {
-                const float v0 = sm.v[4 * t4][j], v1 = sm.v[4 * t4 + 1][j];
-                const float v2 = sm.v[4 * t4 + 2][j], v3 = sm.v[4 * t4 + 3][j];
+                const float v0 = to_f32(sm.v[4 * t4][j]), v1 = to_f32(sm.v[4 * t4 + 1][j]);
+                const float v2 = to_f32(sm.v[4 * t4 + 2][j]), v3 = to_f32(sm.v[4 * t4 + 3][j]);
 #pragma unroll
                 for (int g = 0; g < TAIL_GSUB; ++g) {
                     if (g >= gn) break;
