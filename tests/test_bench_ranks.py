@@ -155,3 +155,22 @@ def test_timeline_summary_on_planted_records():
     assert rows["rope: rotation of the tiles (busy)"] == "1200"
     assert rows["mma: issuing the item's 13 MMA groups (thread busy)"] == "650"
     assert rows["mma: softmax done -> next scores issued"] == "900"
+
+
+def test_shot_aligned_starts_and_workload():
+    """Shot-aligned blocks: starts run from 0 to T, every block holds at most
+    the longest allowed tokens, demonstrations (48..160 tokens) are never split
+    (each block but the last ends where its next demonstration would overflow
+    it), and the workload's block geometry and decode positions follow them."""
+    from block_wise_rank_b200 import synth
+
+    st = synth.shot_starts(20000, 512, 7)
+    lens = [b - a for a, b in zip(st, st[1:])]
+    assert st[0] == 0 and st[-1] == 20000 and all(0 < n <= 512 for n in lens)
+    assert all(n > 512 - 160 for n in lens[:-1])   # a block closes only when the next shot does not fit
+    w = synth.WORKLOADS["qwen7b-128k-shots"]
+    assert w.n_b == len(w.starts) - 1 and w.starts[-1] == w.T
+    assert all(w.block_tokens(b) <= w.block_len for b in range(w.n_b))
+    import dataclasses
+    q, sel, pos = synth.decode_inputs(dataclasses.replace(w, L=1))
+    assert all(int(p) == w.starts[int(s)] for p, s in zip(pos.reshape(-1), sel.reshape(-1)))
