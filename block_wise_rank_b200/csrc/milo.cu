@@ -824,22 +824,20 @@ template <typename P> P *on_device(const milo_factors *f, P *p, char *dev_arena)
 }
 }  // namespace
 
-extern "C" {
-
-size_t milo_decode_offload_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
-    const size_t base = milo_decode_workspace_size(f, S, Hq, n_sel);
-    return base ? offload_layout(f, align_up(base)).bytes : 0;
+namespace {
+// workspace: the decode's own scratch, the recent-token partials, the staging area
+size_t offload_front(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    return milo_decode_workspace_size(f, S, Hq, n_sel) + tail_workspace_bytes(f, S, Hq);
 }
 
-milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
-                                     const int32_t *selected, const int32_t *positions, int32_t n_sel,
-                                     double rope_base, float *out, void *workspace, size_t ws_bytes,
-                                     milo_stream_t stream) {
+milo_status offload_impl(const milo_factors *f, const float *q, int32_t S, int32_t Hq, const int32_t *selected,
+                         const int32_t *positions, int32_t n_sel, double rope_base, const TailIn &tail, float *out,
+                         void *workspace, size_t ws_bytes, milo_stream_t stream) {
     if (!f || !f->arena || !q || !selected || !out || !workspace || S <= 0 || Hq <= 0 || n_sel <= 0)
         return MILO_ERR_INVALID_ARG;
     if (!aligned(workspace, kAlign)) return MILO_ERR_INVALID_ARG;
-    const size_t ws_dec = align_up(milo_decode_workspace_size(f, S, Hq, n_sel));
-    const OffloadLayout o = offload_layout(f, ws_dec);
+    const size_t ws_front = offload_front(f, S, Hq, n_sel);
+    const OffloadLayout o = offload_layout(f, align_up(ws_front));
     if (ws_bytes < o.bytes) return MILO_ERR_WORKSPACE;
     // the arena must be reachable from the device: pinned, mapped host memory
     // (or device memory); pageable memory is refused before any launch
@@ -888,8 +886,41 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
     tpush(MILO_TK_STAGE, t0, tmark(s));
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "staging launch");
-    return decode_impl(&st, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_dec,
+    return decode_impl(&st, q, S, Hq, selected, positions, n_sel, rope_base, tail, out, workspace, ws_front,
                        stream);
+}
+}  // namespace
+
+extern "C" {
+
+size_t milo_decode_offload_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel) {
+    return milo_decode_workspace_size(f, S, Hq, n_sel) ? offload_layout(f, align_up(offload_front(f, S, Hq, n_sel))).bytes
+                                                       : 0;
+}
+
+milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                     const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                     double rope_base, float *out, void *workspace, size_t ws_bytes,
+                                     milo_stream_t stream) {
+    return offload_impl(f, q, S, Hq, selected, positions, n_sel, rope_base, TailIn{}, out, workspace, ws_bytes,
+                        stream);
+}
+
+milo_status milo_decode_attn_offload_tail(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                          const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                          double rope_base, const void *k_tail, const void *v_tail,
+                                          milo_dtype tail_dtype, int32_t tail_cap, const int32_t *tail_len,
+                                          float *out, void *workspace, size_t ws_bytes, milo_stream_t stream) {
+    if (!k_tail || !v_tail || !tail_len || tail_cap < 0) return MILO_ERR_INVALID_ARG;
+    if (tail_dtype != MILO_F32 && tail_dtype != MILO_BF16) return MILO_ERR_UNSUPPORTED;
+    if (!aligned(k_tail, 16) || !aligned(v_tail, 16) || !aligned(tail_len, 4)) return MILO_ERR_INVALID_ARG;
+    TailIn t;
+    t.k = k_tail;
+    t.v = v_tail;
+    t.dtype = tail_dtype;
+    t.cap = tail_cap;
+    t.len = tail_len;
+    return offload_impl(f, q, S, Hq, selected, positions, n_sel, rope_base, t, out, workspace, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------- retrieval

@@ -57,7 +57,7 @@ EXPORTS = [
     "milo_allocate_noalloc", "milo_test_decode_inject", "milo_timing_enable", "milo_timing_read",
     "milo_jacobi_rounds", "milo_decode_tail_workspace_size", "milo_decode_attn_tail",
     "milo_decode_offload_workspace_size", "milo_decode_attn_offload", "milo_bm25_workspace_size",
-    "milo_bm25_select", "milo_factors_shape",
+    "milo_bm25_select", "milo_factors_shape", "milo_decode_attn_offload_tail",
 ]
 
 # stages of milo_timing_read, in order (milo_timed_stage)
@@ -98,6 +98,9 @@ def lib():
         L.milo_decode_offload_workspace_size.restype = SZ
         L.milo_decode_attn_offload.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, SZ, P]
         L.milo_decode_attn_offload.restype = ctypes.c_int
+        L.milo_decode_attn_offload_tail.argtypes = [P, P, I32, I32, P, P, I32, ctypes.c_double, P, P, I32, I32, P,
+                                                    P, P, SZ, P]
+        L.milo_decode_attn_offload_tail.restype = ctypes.c_int
         L.milo_bm25_workspace_size.argtypes = [I32, I32, I32]
         L.milo_bm25_workspace_size.restype = SZ
         L.milo_bm25_select.argtypes = [P, P, P, P, I32, I32, I32, P, P, P, I32, I32, ctypes.c_double,
@@ -400,6 +403,31 @@ def milo_bm25_select(tables, vocab: int, n_sel: int, k1: float = 1.2, beta: floa
                                _stream(stream))
     _check(s, "milo_bm25_select")
     return selected, scores
+
+
+def milo_decode_attn_offload_tail(f: Factors, q: torch.Tensor, selected: torch.Tensor, k_tail: torch.Tensor,
+                                  v_tail: torch.Tensor, tail_len: torch.Tensor, positions=None, rope_base=1e6,
+                                  out=None, workspace=None, stream=None):
+    """milo_decode_attn_offload with each session's recent uncompressed tokens
+    (device tensors, as milo_decode_attn_tail) in the same softmax."""
+    assert q.dtype == torch.float32 and q.is_contiguous() and q.is_cuda
+    L, S, Hq, d = q.shape
+    n_sel = selected.shape[1]
+    assert selected.dtype == torch.int32 and selected.shape[0] == S and selected.is_contiguous()
+    assert k_tail.dtype == v_tail.dtype and k_tail.dtype in (torch.float32, torch.bfloat16)
+    assert k_tail.shape == v_tail.shape and k_tail.is_contiguous() and v_tail.is_contiguous()
+    assert tail_len.dtype == torch.int32 and tail_len.shape == (S,)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = _bytes(milo_decode_offload_workspace_size(f, S, Hq, n_sel), q.device)
+    dt = MILO_BF16 if k_tail.dtype == torch.bfloat16 else MILO_F32
+    s = lib().milo_decode_attn_offload_tail(f.handle, _ptr(q), S, Hq, _ptr(selected), _ptr(positions), n_sel,
+                                            float(rope_base), _ptr(k_tail), _ptr(v_tail), dt, k_tail.shape[3],
+                                            _ptr(tail_len), _ptr(out), _ptr(workspace), workspace.numel(),
+                                            _stream(stream))
+    _check(s, "milo_decode_attn_offload_tail")
+    return out
 
 
 def milo_factors_wrap(shape, params, arena: torch.Tensor) -> Factors:

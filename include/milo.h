@@ -282,8 +282,9 @@ milo_status milo_decode_attn_tail(const milo_factors *f, const float *q, int32_t
                                   int32_t tail_cap, const int32_t *tail_len, float *out, void *workspace,
                                   size_t ws_bytes, milo_stream_t stream);
 
-/* Bytes of scratch milo_decode_attn_offload needs: milo_decode_workspace_size
- * plus a staging area that holds every block's factors at most. */
+/* Bytes of scratch milo_decode_attn_offload and milo_decode_attn_offload_tail
+ * need: milo_decode_tail_workspace_size plus a staging area that holds every
+ * block's factors at most. */
 size_t milo_decode_offload_workspace_size(const milo_factors *f, int32_t S, int32_t Hq, int32_t n_sel);
 
 /*
@@ -304,6 +305,16 @@ milo_status milo_decode_attn_offload(const milo_factors *f, const float *q, int3
                                      const int32_t *selected, const int32_t *positions, int32_t n_sel,
                                      double rope_base, float *out, void *workspace, size_t ws_bytes,
                                      milo_stream_t stream);
+
+/* milo_decode_attn_offload plus each session's recent uncompressed tokens in
+ * the same softmax (their arguments as milo_decode_attn_tail; the tail stays in
+ * device memory), with ws_bytes >= milo_decode_offload_workspace_size: a
+ * complete decode step from host-resident factors. */
+milo_status milo_decode_attn_offload_tail(const milo_factors *f, const float *q, int32_t S, int32_t Hq,
+                                          const int32_t *selected, const int32_t *positions, int32_t n_sel,
+                                          double rope_base, const void *k_tail, const void *v_tail,
+                                          milo_dtype tail_dtype, int32_t tail_cap, const int32_t *tail_len,
+                                          float *out, void *workspace, size_t ws_bytes, milo_stream_t stream);
 
 /* ---------------------------------------------------------------- retrieval */
 

@@ -503,8 +503,8 @@ def test_decode_offloaded_factors(factor):
     bf16 (tensor cores), INT8 and 2-bit (scales staged too) and f32 (CUDA
     cores), with
     blocks no session selects (the staging offsets skip them) and a ragged
-    last block.  An arena in pageable host memory is refused before any
-    launch."""
+    last block; with recent tokens too (milo_decode_attn_offload_tail).  An
+    arena in pageable host memory is refused before any launch."""
     L, H, G, T, bl, S = 2, 2, 4, 3900, 512, 3
     K = synth.planted_cache(L, H, T, 128, bl, (3.0, 30.0), seed=71, out_dtype=torch.bfloat16)
     V = synth.planted_cache(L, H, T, 128, bl, (8.0, 60.0), seed=72, out_dtype=torch.bfloat16)
@@ -528,6 +528,16 @@ def test_decode_offloaded_factors(factor):
     milo.milo_decode_attn_offload(fh, q, sel, pos, rope_base=1e6, workspace=ws)
     out2 = milo.milo_decode_attn_offload(fh, q, sel2, pos2, rope_base=1e6, workspace=ws).cpu()
     assert torch.equal(out2, milo.milo_decode_attn(f, q, sel2, pos2, rope_base=1e6).cpu())
+    # with each session's recent tokens: the resident tail decode, bit for bit
+    kt, vt, tl = synth.recent_tail(synth.Workload("t", L=L, H=H, G=G, T=T, block_len=bl, dtype="bf16",
+                                                  tau_k=(1.0, 2.0), tau_v=(1.0, 2.0), budgets=(0.5,), sessions=S,
+                                                  n_sel=2, steps=1, seed=9), 37, "cuda",
+                                   torch.float32 if factor == "f32" else torch.bfloat16)
+    tl[1] = 0
+    ref_t = milo.milo_decode_attn_tail(f, q, sel, kt, vt, tl, pos, rope_base=1e6).cpu()
+    out_t = milo.milo_decode_attn_offload_tail(fh, q, sel, kt, vt, tl, pos, rope_base=1e6, workspace=ws).cpu()
+    assert milo.milo_get_status() == milo.MILO_OK
+    assert torch.equal(out_t, ref_t) and not torch.equal(out_t, out2)
     # pageable host memory: refused, nothing launched
     raw = torch.empty(f.arena.numel() + 256, dtype=torch.uint8)
     pageable = raw[(-raw.data_ptr()) % 256:][:f.arena.numel()]
