@@ -173,8 +173,13 @@ def test_next_entry_points_reject_bad_arguments_on_host(L):
     assert L.milo_decode_attn_tail(None, P, 1, 1, P, None, 1, 1e6, P, P, milo.MILO_BF16, -1, P, P, P, BIG,
                                    None) == milo.MILO_ERR_INVALID_ARG
     assert L.milo_decode_tail_workspace_size(None, 1, 1, 1) == 0
-    # offloaded factors: null handle
+    # offloaded factors: null handle; with recent tokens also the tail checks
     assert L.milo_decode_attn_offload(None, P, 1, 1, P, None, 1, 1e6, P, P, BIG, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_attn_offload_tail(None, P, 1, 1, P, None, 1, 1e6, P, P, milo.MILO_BF16, 4, P, P, P, BIG,
+                                           None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_decode_attn_offload_tail(None, P, 1, 1, P, None, 1, 1e6, P, P, milo.MILO_INT2, 4, P, P, P, BIG,
+                                           None) == milo.MILO_ERR_UNSUPPORTED
+    assert L.milo_factors_shape(None, None, None) == milo.MILO_ERR_INVALID_ARG
     assert L.milo_decode_offload_workspace_size(None, 1, 1, 1) == 0
     # BM25: n_sel outside [1, n_b], beta outside [0, 1], negative k1, null
     # outputs, entries without their arrays, small workspace
