@@ -81,7 +81,8 @@ typedef struct {
      * several many-shot examples).  The handle keeps its own copy, and the
      * arena a device copy (its `starts` array below).  With variable blocks
      * the Gram runs on CUDA cores (the tensor-core Gram needs whole
-     * fixed-length blocks). */
+     * fixed-length blocks), and milo_compress copies the starts to the device
+     * on its stream (a host-to-device copy from this array). */
     int32_t n_blocks;
     const int32_t *block_starts;
 } milo_cache_shape;
