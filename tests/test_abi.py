@@ -231,3 +231,24 @@ def test_block_starts_validated_and_budget_on_host(L, oracle_mod):
         assert milo.milo_factor_arena_size(sb, p) == 0, bad
         assert milo.milo_rank_budget(sb, p) == -1, bad
     assert milo.block_starts(s) == starts and milo.block_starts(milo.cache_shape(1, 1, 10, 128, 5, 0)) is None
+
+
+def test_workspace_sizes_nest_on_host(L):
+    """On a wrapped handle (no device access): the recent-token workspace is
+    the decode's plus one partial per query row, and the offload workspace
+    holds that plus a staging area for the factor data of every block."""
+    fake = ctypes.c_void_p(1 << 20)
+    for dt in (milo.MILO_BF16, milo.MILO_INT8, milo.MILO_INT2):
+        p = milo.default_params(factor_dtype=dt)
+        s = _shape(2, 2, 4096, 128, 512)
+        n = milo.milo_factor_arena_size(s, p)
+        h = ctypes.c_void_p()
+        assert L.milo_factors_wrap(ctypes.byref(s), ctypes.byref(p), fake, n, ctypes.byref(h)) == 0
+        S, Hq, n_sel = 4, 8, 3
+        dec = L.milo_decode_workspace_size(h, S, Hq, n_sel)
+        tail = L.milo_decode_tail_workspace_size(h, S, Hq, n_sel)
+        off = L.milo_decode_offload_workspace_size(h, S, Hq, n_sel)
+        rows = 2 * S * Hq
+        assert tail - dec == (rows * 128 * 4 + 255) // 256 * 256 + (rows * 8 + 255) // 256 * 256
+        assert off >= tail + n // 2   # staging: both kinds' data sections (most of the arena)
+        L.milo_factors_destroy(h)
